@@ -1,0 +1,310 @@
+/*
+ * nsa_oracle.c -- plain, slow, fp64 CPU oracle for the NSA compressed-attention
+ * path.  TEST INFRASTRUCTURE ONLY: tests, the smoke check and the benchmark's
+ * CPU-baseline leg call it; the product library never links, loads or calls it,
+ * and it shares no code, header or table with the CUDA path.
+ *
+ * Sources (web pages; cited by page title and the section/equation used):
+ *   [CMP]  "aclnnNsaCompress" (Ascend CANN API page) -- Formula section:
+ *          K~cmp_t = { phi(k_{id+1 : id+l}) | 0 <= i <= floor((t-l)/d) }.
+ *   [ATT]  "mindspore.ops.nsa_compress_attention" -- steps 1..7 of the
+ *          description, the note list (TND layout, prefix-sum lengths,
+ *          constraints) and the Returns list (output shapes).
+ *   [RFA]  "lite_boost.ops.rain_fusion_attention" -- select_idx parameter:
+ *          valid indices listed in ascending order first, then -1 padding.
+ *
+ * Readings taken where the pages are silent or garbled (each one is listed in
+ * the design notes of this repository):
+ *   phi     weighted sum over the window with weights w[j][n] (shape l x N2),
+ *           the same w for K and V; 0-based rows i*d .. i*d+l-1.
+ *   n_cmp   floor((S-l)/d)+1 when S >= l, else 0 (floor, not C truncation).
+ *   mask    compressed block i is visible to query position t iff i*d+l-1 <= t.
+ *   offset  query row t_loc of sequence b sits at position
+ *           t = t_loc + max(0, (n_cmp-1)*d + l - S_q) (bottom-right alignment;
+ *           0 when n_cmp == 0).
+ *   band    step 4 taken literally with out-of-range / invisible terms = 0;
+ *           a = l'/d and b = l/d must be integers.
+ *   group   step 5 sums over the query heads of one KV group (h / G == g).
+ *   top-k   candidates j < n_sel with j*l' <= t; k* = min(count, #candidates)
+ *           largest scores, ties to the smaller j, emitted ascending, then -1.
+ *           A row that sees no compressed block emits all -1, zero output,
+ *           max = -inf and sum = 0.
+ *   stats   softmax_max = max of the scaled scores, softmax_sum = sum of
+ *           exp(s - max) (natural exponent).
+ *
+ * Parity of the offset, candidate, ordering and empty-row readings is
+ * unpinned: no page gives an example for them.
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC (no fast-math: fp64 semantics kept).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------- */
+/* Rounding fp64 -> storage dtype, round-to-nearest-even, from the IEEE-754    */
+/* definition of binary16 (p = 11 bits, emin = -14) and bfloat16 (p = 8 bits, */
+/* emin = -126).  dtype 0 = bfloat16, 1 = float16.                            */
+/* ------------------------------------------------------------------------- */
+static double round_to_storage(double x, int dtype)
+{
+    int p = (dtype == 0) ? 8 : 11;          /* significand bits incl. implicit */
+    int emin = (dtype == 0) ? -126 : -14;   /* exponent of the smallest normal */
+    int emax = (dtype == 0) ? 127 : 15;     /* exponent of the largest normal  */
+    if (x == 0.0 || isnan(x) || isinf(x)) return x;
+    int e;
+    (void)frexp(x, &e);                     /* x = f * 2^e, 0.5 <= |f| < 1     */
+    int qexp = e - p;                       /* exponent of one unit in the last place */
+    if (qexp < emin - p + 1) qexp = emin - p + 1;  /* subnormal spacing */
+    double q = ldexp(1.0, qexp);
+    double y = nearbyint(x / q) * q;        /* default mode: ties to even      */
+    double maxfin = ldexp(2.0 - ldexp(1.0, 1 - p), emax);
+    if (fabs(y) > maxfin) y = (y > 0) ? INFINITY : -INFINITY;
+    return y;
+}
+
+void oracle_round(const double* in, int64_t n, int dtype, double* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = round_to_storage(in[i], dtype);
+}
+
+/* ------------------------------------------------------------------------- */
+/* [CMP] Formula: number of compressed blocks of a sequence of S tokens is    */
+/* floor((S-l)/d)+1 for S >= l (i runs 0..floor((S-l)/d)), 0 otherwise.       */
+/* cu_seqlens holds the cumulative end of each sequence (no leading 0).       */
+/* Writes cumulative ends of the compressed sequences.  Returns total.        */
+/* ------------------------------------------------------------------------- */
+int64_t oracle_compress_len(const int32_t* cu_seqlens, int batch, int l, int d,
+                            int32_t* cu_cmp)
+{
+    int64_t total = 0;
+    int32_t prev = 0;
+    for (int b = 0; b < batch; b++) {
+        int64_t S = (int64_t)cu_seqlens[b] - prev;
+        prev = cu_seqlens[b];
+        int64_t n = 0;
+        /* count the i with 0 <= i and i*d + l <= S, one by one */
+        for (int64_t i = 0; i * d + l <= S; i++) n++;
+        total += n;
+        cu_cmp[b] = (int32_t)total;
+    }
+    return total;
+}
+
+/* ------------------------------------------------------------------------- */
+/* [CMP] Formula with phi = weighted window sum (reading above):              */
+/*   out[c0+i][n][:] = sum_{j=0}^{l-1} w[j][n] * x[s0 + i*d + j][n][:]        */
+/* x: (T, N2, D) fp64; w: (l, N2) fp64; out: (Tc, N2, D) fp64, unrounded.     */
+/* ------------------------------------------------------------------------- */
+void oracle_compress(const double* x, const double* w, int l, int d,
+                     const int32_t* cu_seqlens, int batch, int n2, int dim,
+                     const int32_t* cu_cmp, double* out)
+{
+    for (int b = 0; b < batch; b++) {
+        int64_t s0 = (b == 0) ? 0 : cu_seqlens[b - 1];
+        int64_t c0 = (b == 0) ? 0 : cu_cmp[b - 1];
+        int64_t ncmp = cu_cmp[b] - c0;
+        #pragma omp parallel for schedule(static)
+        for (int64_t i = 0; i < ncmp; i++) {
+            for (int n = 0; n < n2; n++) {
+                for (int e = 0; e < dim; e++) {
+                    double acc = 0.0;
+                    for (int j = 0; j < l; j++) {
+                        double xv = x[((s0 + i * d + j) * n2 + n) * (int64_t)dim + e];
+                        acc += w[(int64_t)j * n2 + n] * xv;
+                    }
+                    out[((c0 + i) * n2 + n) * (int64_t)dim + e] = acc;
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* [ATT] step 4, taken literally:                                              */
+/*   P_slc[j] = sum_{m=0}^{a-1} sum_{n=0}^{b-1} P_cmp[a*j - m - n]             */
+/* with a = l'/d and b = l/d.  P_cmp[c] counts only for 0 <= c < n_vis (the    */
+/* visible compressed blocks); every other term is 0.  P holds n_vis values.  */
+/* ------------------------------------------------------------------------- */
+void oracle_importance(const double* P, int n_vis, int a, int b, int n_sel,
+                       double* pslc)
+{
+    for (int j = 0; j < n_sel; j++) {
+        double acc = 0.0;
+        for (int m = 0; m < a; m++) {
+            for (int n = 0; n < b; n++) {
+                int64_t c = (int64_t)a * j - m - n;
+                if (c >= 0 && c < n_vis) acc += P[c];
+            }
+        }
+        pslc[j] = acc;
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* [ATT] step 7 with the top-k reading above.  score has n_cand entries (the  */
+/* candidates j = 0..n_cand-1).  Picks k* = min(count, n_cand) indices by     */
+/* descending score, ties to the smaller j, then lists them ascending ([RFA]  */
+/* select_idx convention) and pads with -1 up to count.                       */
+/* ------------------------------------------------------------------------- */
+void oracle_topk(const double* score, int n_cand, int count, int32_t* idx)
+{
+    int kstar = (count < n_cand) ? count : n_cand;
+    char* taken = (char*)calloc((size_t)(n_cand > 0 ? n_cand : 1), 1);
+    for (int r = 0; r < kstar; r++) {
+        int best = -1;
+        for (int j = 0; j < n_cand; j++) {
+            if (taken[j]) continue;
+            if (best < 0 || score[j] > score[best]) best = j;   /* strict: earlier j wins ties */
+        }
+        taken[best] = 1;
+    }
+    int w = 0;
+    for (int j = 0; j < n_cand; j++)
+        if (taken[j]) idx[w++] = j;
+    for (; w < count; w++) idx[w] = -1;
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------- */
+/* [ATT] steps 1..7 for a list of query rows.                                  */
+/*  q  (T1, N1, D1), kc (Tc, N2, D1), vc (Tc, N2, D2): fp64 values of the      */
+/*     storage-dtype tensors (TND layout).                                     */
+/*  cu_q / cu_cmp / cu_sel: cumulative ends per sequence (no leading 0).      */
+/*  rows: global query-row indices to evaluate (nrows of them; NULL = all).   */
+/* Outputs, indexed by position r in the row list:                            */
+/*  out   (nrows, N1, D2)  fp64, unrounded                                     */
+/*  smax  (nrows, N1)      max of the scaled scores (-inf for empty rows)      */
+/*  ssum  (nrows, N1)      sum of exp(s - max) (0 for empty rows)              */
+/*  topk  (nrows, N2, count)                                                   */
+/*  score (nrows, N2, sel_cap) or NULL: P_slc' for j < min(n_sel, sel_cap)     */
+/*  ncand (nrows, N2) or NULL: number of top-k candidates of the row (0 when   */
+/*        the row sees no block)                                               */
+/* Returns 0, or -1 when l % d or l' % d is nonzero.                           */
+/* ------------------------------------------------------------------------- */
+int oracle_compress_attention(const double* q, const double* kc, const double* vc,
+                              double scale, int n1, int n2, int d1, int d2,
+                              int l, int d, int lp, int count,
+                              const int32_t* cu_q, const int32_t* cu_cmp,
+                              const int32_t* cu_sel, int batch,
+                              const int64_t* rows, int64_t nrows,
+                              double* out, double* smax, double* ssum,
+                              int32_t* topk, double* score, int sel_cap,
+                              int32_t* ncand)
+{
+    if (l % d != 0 || lp % d != 0) return -1;
+    const int a = lp / d, bb = l / d;
+    const int G = n1 / n2;
+    if (rows == NULL) nrows = cu_q[batch - 1];
+
+    #pragma omp parallel
+    {
+        int max_cmp = 0, max_sel = 0;
+        for (int s = 0; s < batch; s++) {
+            int nc = cu_cmp[s] - (s ? cu_cmp[s - 1] : 0);
+            int ns = cu_sel[s] - (s ? cu_sel[s - 1] : 0);
+            if (nc > max_cmp) max_cmp = nc;
+            if (ns > max_sel) max_sel = ns;
+        }
+        double* sc = (double*)malloc(sizeof(double) * (size_t)(max_cmp + 1));
+        double* P = (double*)malloc(sizeof(double) * (size_t)(max_cmp + 1));
+        double* pslc = (double*)malloc(sizeof(double) * (size_t)(max_sel + 1));
+        double* grp = (double*)malloc(sizeof(double) * (size_t)(max_sel + 1));
+
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < nrows; r++) {
+            int64_t t = rows ? rows[r] : r;
+            /* sequence that owns global row t (TND + prefix sums, [ATT] note) */
+            int s = 0;
+            while (cu_q[s] <= t) s++;
+            int64_t q0 = s ? cu_q[s - 1] : 0;
+            int64_t c0 = s ? cu_cmp[s - 1] : 0;
+            int64_t Sq = cu_q[s] - q0;
+            int n_cmp = (int)(cu_cmp[s] - c0);
+            int n_sel = (int)(cu_sel[s] - (s ? cu_sel[s - 1] : 0));
+            int64_t off = 0;
+            if (n_cmp > 0) {
+                off = (int64_t)(n_cmp - 1) * d + l - Sq;
+                if (off < 0) off = 0;
+            }
+            int64_t tpos = (t - q0) + off;
+
+            /* visible set: i < n_cmp with i*d + l - 1 <= tpos (counted one by one) */
+            int n_vis = 0;
+            for (int i = 0; i < n_cmp; i++)
+                if ((int64_t)i * d + l - 1 <= tpos) n_vis++;
+
+            /* candidates: j < n_sel with j*l' <= tpos */
+            int n_cand = 0;
+            for (int j = 0; j < n_sel; j++)
+                if ((int64_t)j * lp <= tpos) n_cand++;
+
+            for (int g = 0; g < n2; g++) {
+                for (int j = 0; j < n_sel; j++) grp[j] = 0.0;
+                for (int hh = 0; hh < G; hh++) {
+                    int h = g * G + hh;
+                    double* o = out + (r * n1 + h) * (int64_t)d2;
+                    for (int e = 0; e < d2; e++) o[e] = 0.0;
+                    if (n_vis == 0) {
+                        smax[r * n1 + h] = -INFINITY;
+                        ssum[r * n1 + h] = 0.0;
+                        continue;
+                    }
+                    /* step 1: QK = scale * query * key^T over the visible blocks */
+                    const double* qr = q + (t * n1 + h) * (int64_t)d1;
+                    for (int i = 0; i < n_vis; i++) {
+                        const double* kr = kc + ((c0 + i) * n2 + g) * (int64_t)d1;
+                        double acc = 0.0;
+                        for (int k = 0; k < d1; k++) acc += qr[k] * kr[k];
+                        sc[i] = scale * acc;
+                    }
+                    /* step 2: P_cmp = softmax(QK) */
+                    double m = sc[0];
+                    for (int i = 1; i < n_vis; i++) if (sc[i] > m) m = sc[i];
+                    double L = 0.0;
+                    for (int i = 0; i < n_vis; i++) L += exp(sc[i] - m);
+                    for (int i = 0; i < n_vis; i++) P[i] = exp(sc[i] - m) / L;
+                    smax[r * n1 + h] = m;
+                    ssum[r * n1 + h] = L;
+                    /* step 3: attentionOut = P_cmp * value */
+                    for (int i = 0; i < n_vis; i++) {
+                        const double* vr = vc + ((c0 + i) * n2 + g) * (int64_t)d2;
+                        for (int e = 0; e < d2; e++) o[e] += P[i] * vr[e];
+                    }
+                    /* step 4: importance score of this head */
+                    oracle_importance(P, n_vis, a, bb, n_sel, pslc);
+                    /* step 5: sum over the heads of the group */
+                    for (int j = 0; j < n_sel; j++) grp[j] += pslc[j];
+                }
+                if (score) {
+                    int lim = n_sel < sel_cap ? n_sel : sel_cap;
+                    double* dst = score + (r * n2 + g) * (int64_t)sel_cap;
+                    for (int j = 0; j < sel_cap; j++) dst[j] = (j < lim) ? grp[j] : 0.0;
+                }
+                if (ncand) ncand[r * n2 + g] = (n_vis == 0) ? 0 : n_cand;
+                /* steps 6-7: causal candidate set, then top-k */
+                int32_t* ti = topk + (r * n2 + g) * (int64_t)count;
+                if (n_vis == 0) {
+                    for (int k = 0; k < count; k++) ti[k] = -1;
+                } else {
+                    oracle_topk(grp, n_cand, count, ti);
+                }
+            }
+        }
+        free(sc); free(P); free(pslc); free(grp);
+    }
+    return 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,25 @@
+"""pytest configuration: the ``gpu`` marker and the repository root on sys.path."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA device (B200, sm_100a); parity tests of the CUDA path")
+
+
+def read_golden(name):
+    """Parse a tests/golden fixture: '# ...' comments, 'key: values' lines."""
+    out = {}
+    with open(os.path.join(ROOT, "tests", "golden", name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, val = line.partition(":")
+            out.setdefault(key.strip(), []).append(val.strip())
+    return out
