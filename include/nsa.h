@@ -1,0 +1,162 @@
+/*
+ * nsa.h -- C ABI of the B200 (sm_100a) NSA compressed-attention library.
+ *
+ * The library computes the compressed branch of Native Sparse Attention:
+ *   nsa_compress            sliding-window compression of raw K and V
+ *                           ("aclnnNsaCompress", Formula section);
+ *   nsa_compress_attention  causal GQA attention over the compressed blocks,
+ *                           importance scores, head-group sum and per-query
+ *                           top-k of selection blocks
+ *                           ("mindspore.ops.nsa_compress_attention", steps 1-7).
+ *
+ * Conventions shared by every entry point
+ *   - Layout is TND ("mindspore.ops.nsa_compress_attention", note list):
+ *     a tensor (T, N, D) is row-major, D contiguous, then heads, then the
+ *     concatenated tokens of all sequences of the batch.
+ *   - Sequence lengths are HOST int32 arrays of `batch` cumulative ends
+ *     (prefix sums, no leading 0, non-decreasing), as the pages require
+ *     ("cumulative sum mode" on the aclnnNsaCompress page; "prefix-sum mode"
+ *     for actual_seq_qlen / actual_cmp_seq_kvlen / actual_sel_seq_kvlen).
+ *   - Tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
+ *     caller.  The library allocates no memory and keeps no state between
+ *     calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; argument errors are returned
+ *     synchronously before anything is enqueued ("aclnnNsaCompress": the
+ *     first phase validates the parameters and returns a status code).
+ *   - Results are deterministic: two calls with the same inputs produce
+ *     bitwise-identical outputs ("aclnnNsaCompress", deterministic
+ *     computation by default).  No atomics on any result.
+ */
+#ifndef NSA_B200_H
+#define NSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NSA_OK = 0,
+    NSA_ERR_INVALID_ARG = 1,   /* a value, pointer or size breaks a stated constraint */
+    NSA_ERR_UNSUPPORTED = 2,   /* valid per the pages but outside what this build runs */
+    NSA_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small           */
+    NSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed           */
+    NSA_ERR_TIMEOUT = 5        /* a device-side wait gave up (reported after the fact) */
+} nsa_status_t;
+
+typedef enum { NSA_BF16 = 0, NSA_FP16 = 1 } nsa_dtype_t;
+
+/* Human-readable name of a status code.  Never NULL; static storage. */
+const char* nsa_status_string(nsa_status_t status);
+
+/*
+ * Number of compressed blocks per sequence ("aclnnNsaCompress", Formula
+ * section: block i exists for 0 <= i <= floor((S - l)/d); a sequence with
+ * S < l has none).
+ *   cu_seqlens  host, [batch] cumulative raw lengths
+ *   cu_cmp_out  host, [batch] written with the cumulative compressed lengths
+ *   total_out   host, optional (may be NULL): total compressed rows Tc
+ * Errors: NSA_ERR_INVALID_ARG for NULL arrays, batch < 1, l or d < 1, or
+ * decreasing prefix sums.  Pure host function, no CUDA call.
+ */
+nsa_status_t nsa_compress_out_len(const int32_t* cu_seqlens, int batch, int l, int d,
+                                  int32_t* cu_cmp_out, int64_t* total_out);
+
+/*
+ * Sliding-window compression of K and V ("aclnnNsaCompress", Formula
+ * section), with phi read as the weighted sum over the window:
+ *   kcmp[c0+i, n, :] = sum_{j<l} w[j, n] * k[s0 + i*d + j, n, :]
+ *   vcmp[c0+i, n, :] = sum_{j<l} w[j, n] * v[s0 + i*d + j, n, :]
+ * for every sequence (raw rows start at s0, compressed rows at c0) and every
+ * i < n_cmp.  fp32 accumulation in window order, one rounding (RNE) to dtype.
+ *   k     device (T2, N2, D1), dtype        v     device (T2, N2, D2), dtype
+ *   w     device (l, N2), dtype: one weight per window position and head,
+ *         shared by K and V and by every head dimension
+ *   kcmp  device (Tc, N2, D1), written      vcmp  device (Tc, N2, D2), written
+ *   Tc = total of nsa_compress_out_len.  v/vcmp may both be NULL (K only).
+ * Constraints (NSA_ERR_INVALID_ARG): l, d multiples of 16; 16 <= d <= l <= 128
+ * ("select/compress" constraint list of mindspore.ops.nsa_compress_attention);
+ * D1, D2 multiples of 16 and <= 256 (aclnnNsaCompress constraint list);
+ * N2 >= 1; pointers 16-byte aligned.
+ */
+nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, int d,
+                          const int32_t* cu_seqlens, int batch, int n2, int d1, int d2,
+                          nsa_dtype_t dtype, void* kcmp, void* vcmp, void* stream);
+
+/*
+ * Workspace bytes that nsa_compress_attention needs for these arguments.
+ * Same argument meaning as nsa_compress_attention.  Pure host function.
+ */
+nsa_status_t nsa_compress_attention_workspace_size(
+    int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, size_t* bytes);
+
+/*
+ * Compressed attention with importance scores and top-k
+ * ("mindspore.ops.nsa_compress_attention", steps 1-7; returns list).
+ * Per sequence b, query row t_loc sits at position t = t_loc + off_b with
+ * off_b = max(0, (n_cmp_b - 1)*d + l - S_q_b) (0 when n_cmp_b = 0); compressed
+ * block i is visible iff i*d + l - 1 <= t.  For head h of KV group g = h / G
+ * (G = head_num / n2):
+ *   s_i = scale * q[t,h,:] . kcmp[i,g,:]        (step 1)
+ *   P_i = exp(s_i - m) / L,  m = max s, L = sum exp(s - m)   (step 2)
+ *   out[t,h,:] = sum_i P_i vcmp[i,g,:]          (step 3)
+ *   P_slc[j] = sum_{m<l'/d} sum_{n<l/d} P[l'/d*j - m - n]   (step 4)
+ *   P_slc'[t,g,j] = sum over the G heads of group g          (step 5)
+ *   topk_indices[t,g,:] = the min(count, #candidates) largest P_slc' over
+ *     the candidates j < n_sel_b with j*l' <= t, ties to the smaller j,
+ *     listed ascending, then -1 padding (step 7; index convention of
+ *     lite_boost.ops.rain_fusion_attention select_idx).
+ * A row that sees no block gets out = 0, softmax_max = -inf, softmax_sum = 0
+ * and all indices -1.
+ * Arguments
+ *   q         device (T1, N1, D1) dtype      kcmp  device (Tc, N2, D1) dtype
+ *   vcmp      device (Tc, N2, D2) dtype      scale scale_value of step 1
+ *   head_num  N1 (== number of query heads)
+ *   l, d, lp, count  compress_block_size, compress_stride, select_block_size,
+ *             select_block_count
+ *   cu_seqlens_q, cu_cmp_kv, cu_sel_kv  host [batch] prefix sums
+ *   attention_out device (T1, N1, D2) dtype     topk_indices device (T1, N2, count) int32
+ *   softmax_max, softmax_sum  device (T1, N1, 8) fp32, 8 equal copies;
+ *             max of the scaled scores and sum of exp(s - max) (natural exp)
+ *   workspace device, >= nsa_compress_attention_workspace_size bytes,
+ *             256-byte aligned; its first 16 bytes receive a device error
+ *             word read by nsa_workspace_status
+ * Constraints (NSA_ERR_INVALID_ARG, from the note list of
+ * mindspore.ops.nsa_compress_attention): l, d, lp multiples of 16;
+ * 16 <= l <= 128; 16 <= d <= 64; 16 <= lp <= 128; l >= d; lp >= l; lp % d == 0;
+ * 1 <= count <= 32; D1 >= D2; D1, D2 multiples of 16; N1 >= N2, N1 % N2 == 0.
+ * NSA_ERR_UNSUPPORTED: l % d != 0 (the importance sum needs integer l/d),
+ * D1 or D2 > 256, more than 128 query heads per KV group, or shapes whose
+ * on-chip tiles do not fit one SM.
+ */
+nsa_status_t nsa_compress_attention(
+    const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
+    int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+    void* attention_out, int32_t* topk_indices, float* softmax_max, float* softmax_sum,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream` and reads the device error word of `workspace`
+ * (written by the last nsa_compress_attention that used it).  Returns NSA_OK,
+ * NSA_ERR_TIMEOUT when a device-side wait gave up, or NSA_ERR_CUDA.
+ */
+nsa_status_t nsa_workspace_status(const void* workspace, void* stream);
+
+/*
+ * Device-side error word of the compress kernel on the current device
+ * (0 = none).  Synchronises `stream`.  NSA_ERR_TIMEOUT when a wait gave up.
+ */
+nsa_status_t nsa_compress_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_B200_H */

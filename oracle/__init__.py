@@ -74,7 +74,7 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             _i32p, _i32p, _i32p, ctypes.c_int,
-            ctypes.c_void_p, ctypes.c_int64,
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
             _f64p, _f64p, _f64p, _i32p, ctypes.c_void_p, ctypes.c_int,
             ctypes.c_void_p]
         lib.oracle_compress_attention.restype = ctypes.c_int
@@ -161,21 +161,24 @@ def topk(score, n_cand: int, count: int) -> np.ndarray:
 
 def compress_attention(q, kcmp, vcmp, scale: float, l: int, d: int, lp: int,
                        count: int, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
-                       rows=None, sel_cap: int | None = None):
+                       rows=None, sel_cap: int | None = None, q_rows_only: bool = False):
     """Steps 1-7 of mindspore.ops.nsa_compress_attention for query rows.
 
     q (T1, N1, D1), kcmp (Tc, N2, D1), vcmp (Tc, N2, D2): values of the
-    storage-dtype tensors.  ``rows`` selects global query rows (None = all).
+    storage-dtype tensors.  ``rows`` selects global query rows (None = all);
+    with ``q_rows_only`` q holds just those rows, in the order of ``rows``.
     Returns a dict with out (R, N1, D2), softmax_max / softmax_sum (R, N1),
     topk (R, N2, count), score (R, N2, sel_cap) and ncand (R, N2).
     """
     qf, kf, vf = _f64(q), _f64(kcmp), _f64(vcmp)
-    t1, n1, d1 = qf.shape
+    _, n1, d1 = qf.shape
     tc, n2, d1k = kf.shape
     d2 = vf.shape[2]
     assert d1k == d1 and vf.shape[:2] == (tc, n2)
     cq, cc, cs = _i32(cu_seqlens_q), _i32(cu_cmp_kv), _i32(cu_sel_kv)
     batch = cq.size
+    if q_rows_only and rows is None:
+        raise ValueError("q_rows_only needs rows")
     if rows is None:
         rows_arr = np.arange(int(cq[-1]) if batch else 0, dtype=np.int64)
     else:
@@ -198,7 +201,7 @@ def compress_attention(q, kcmp, vcmp, scale: float, l: int, d: int, lp: int,
         rc = _load().oracle_compress_attention(
             qf, kf, vf, float(scale), n1, n2, d1, d2, int(l), int(d), int(lp),
             int(count), cq, cc, cs, batch,
-            rows_arr.ctypes.data_as(ctypes.c_void_p), R,
+            rows_arr.ctypes.data_as(ctypes.c_void_p), R, 1 if q_rows_only else 0,
             out, smax, ssum, tk, score.ctypes.data_as(ctypes.c_void_p), sel_cap,
             ncand.ctypes.data_as(ctypes.c_void_p))
         if rc != 0:

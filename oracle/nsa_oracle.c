@@ -176,6 +176,7 @@ void oracle_topk(const double* score, int n_cand, int count, int32_t* idx)
 /*     storage-dtype tensors (TND layout).                                     */
 /*  cu_q / cu_cmp / cu_sel: cumulative ends per sequence (no leading 0).      */
 /*  rows: global query-row indices to evaluate (nrows of them; NULL = all).   */
+/*  q_compact: when non-zero, q holds only the listed rows, in list order.    */
 /* Outputs, indexed by position r in the row list:                            */
 /*  out   (nrows, N1, D2)  fp64, unrounded                                     */
 /*  smax  (nrows, N1)      max of the scaled scores (-inf for empty rows)      */
@@ -191,7 +192,7 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
                               int l, int d, int lp, int count,
                               const int32_t* cu_q, const int32_t* cu_cmp,
                               const int32_t* cu_sel, int batch,
-                              const int64_t* rows, int64_t nrows,
+                              const int64_t* rows, int64_t nrows, int q_compact,
                               double* out, double* smax, double* ssum,
                               int32_t* topk, double* score, int sel_cap,
                               int32_t* ncand)
@@ -255,7 +256,7 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
                         continue;
                     }
                     /* step 1: QK = scale * query * key^T over the visible blocks */
-                    const double* qr = q + (t * n1 + h) * (int64_t)d1;
+                    const double* qr = q + ((q_compact ? r : t) * n1 + h) * (int64_t)d1;
                     for (int i = 0; i < n_vis; i++) {
                         const double* kr = kc + ((c0 + i) * n2 + g) * (int64_t)d1;
                         double acc = 0.0;

@@ -1,0 +1,254 @@
+"""B200-native NSA compressed-attention path: Python binding of libnsa_b200.so.
+
+This module only marshals arguments: every step of the computation runs in
+the CUDA kernels of the C-ABI library (``include/nsa.h``).  PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: importing
+works without a GPU (for the host-only entry points), and every device entry
+point raises when the library or a CUDA device is missing.
+
+Entry points (same names as the C ABI):
+  nsa_compress_out_len, nsa_compress, nsa_compress_attention_workspace_size,
+  nsa_compress_attention, nsa_workspace_status, nsa_compress_status,
+  nsa_status_string.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnsa_b200.so")
+
+NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED = 0, 1, 2
+NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = 3, 4, 5
+NSA_BF16, NSA_FP16 = 0, 1
+
+EXPORTED = (
+    "nsa_status_string",
+    "nsa_compress_out_len",
+    "nsa_compress",
+    "nsa_compress_attention_workspace_size",
+    "nsa_compress_attention",
+    "nsa_workspace_status",
+    "nsa_compress_status",
+)
+
+_lib = None
+
+
+class NsaError(RuntimeError):
+    """A CUDA failure, a device-side timeout or a workspace problem."""
+
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_status_name(status)}")
+        self.status = status
+
+
+def _status_name(status: int) -> str:
+    try:
+        return load().nsa_status_string(status).decode()
+    except Exception:  # library missing: still report the number
+        return f"status {status}"
+
+
+def load(path: Optional[str] = None):
+    """Load the C-ABI library (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing: build it with sparse_long_context_nsa_b200._build.build()")
+    lib = ctypes.CDLL(p)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    vp, ci, cs = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.nsa_status_string.argtypes = [ci]
+    lib.nsa_status_string.restype = ctypes.c_char_p
+    lib.nsa_compress_out_len.argtypes = [i32p, ci, ci, ci, i32p, ctypes.POINTER(ctypes.c_int64)]
+    lib.nsa_compress_out_len.restype = ci
+    lib.nsa_compress.argtypes = [vp, vp, vp, ci, ci, i32p, ci, ci, ci, ci, ci, vp, vp, vp]
+    lib.nsa_compress.restype = ci
+    lib.nsa_compress_attention_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p, i32p,
+                                                          i32p, ci, ctypes.POINTER(cs)]
+    lib.nsa_compress_attention_workspace_size.restype = ci
+    lib.nsa_compress_attention.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p, i32p,
+                                           i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, cs, vp]
+    lib.nsa_compress_attention.restype = ci
+    lib.nsa_workspace_status.argtypes = [vp, vp]
+    lib.nsa_workspace_status.restype = ci
+    lib.nsa_compress_status.argtypes = [vp]
+    lib.nsa_compress_status.restype = ci
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _raise(status: int, what: str):
+    if status == NSA_OK:
+        return
+    if status in (NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED):
+        raise ValueError(f"{what}: {_status_name(status)}")
+    raise NsaError(status, what)
+
+
+def _cu(x) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(x.cpu() if hasattr(x, "cpu") else x, dtype=np.int32))
+    if a.ndim != 1 or a.size < 1:
+        raise ValueError("sequence lengths must be a non-empty 1-D list of prefix sums")
+    return a
+
+
+def _ip(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return NSA_BF16
+    if t.dtype == torch.float16:
+        return NSA_FP16
+    raise TypeError(f"dtype must be bfloat16 or float16, got {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the library computes on the GPU only)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (TND layout)")
+    return t
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def nsa_status_string(status: int) -> str:
+    return load().nsa_status_string(int(status)).decode()
+
+
+def nsa_compress_out_len(cu_seqlens: Sequence[int], l: int, d: int) -> np.ndarray:
+    """Cumulative compressed lengths of the sequences (host)."""
+    cu = _cu(cu_seqlens)
+    out = np.empty_like(cu)
+    tot = ctypes.c_int64(0)
+    _raise(load().nsa_compress_out_len(_ip(cu), cu.size, int(l), int(d), _ip(out), ctypes.byref(tot)),
+           "nsa_compress_out_len")
+    return out
+
+
+def nsa_compress(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tensor, l: int, d: int,
+                 cu_seqlens: Sequence[int], kcmp: Optional[torch.Tensor] = None,
+                 vcmp: Optional[torch.Tensor] = None, stream=None):
+    """Compress raw K (and V) of shape (T2, N2, D) with weights w (l, N2).
+
+    Returns (kcmp, vcmp) of shape (Tc, N2, D); vcmp is None when v is None.
+    """
+    _dev(k, "k")
+    _dev(w, "w")
+    dt = _dtype_code(k)
+    if w.dtype != k.dtype or (v is not None and v.dtype != k.dtype):
+        raise TypeError("k, v and w must share one dtype")
+    if k.dim() != 3 or w.dim() != 2:
+        raise ValueError("k must be (T2, N2, D1) and w (l, N2)")
+    t2, n2, d1 = k.shape
+    d2 = d1
+    if v is not None:
+        _dev(v, "v")
+        if v.dim() != 3 or v.shape[:2] != k.shape[:2]:
+            raise ValueError("v must be (T2, N2, D2) with the T2, N2 of k")
+        d2 = v.shape[2]
+    if tuple(w.shape) != (l, n2):
+        raise ValueError("w must have shape (l, N2)")
+    cu = _cu(cu_seqlens)
+    if int(cu[-1]) > t2:
+        raise ValueError("cu_seqlens runs past the rows of k")
+    cuc = nsa_compress_out_len(cu, l, d)
+    tc = int(cuc[-1])
+    if kcmp is None:
+        kcmp = torch.empty(tc, n2, d1, dtype=k.dtype, device=k.device)
+    if v is not None and vcmp is None:
+        vcmp = torch.empty(tc, n2, d2, dtype=k.dtype, device=k.device)
+    st = load().nsa_compress(k.data_ptr(), v.data_ptr() if v is not None else None, w.data_ptr(),
+                             int(l), int(d), _ip(cu), cu.size, n2, d1, d2, dt, kcmp.data_ptr(),
+                             vcmp.data_ptr() if v is not None else None, _stream(stream))
+    _raise(st, "nsa_compress")
+    return kcmp, vcmp
+
+
+def nsa_compress_attention_workspace_size(head_num: int, n2: int, d1: int, d2: int, l: int, d: int,
+                                          lp: int, count: int, cu_seqlens_q, cu_cmp_kv,
+                                          cu_sel_kv) -> int:
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size):
+        raise ValueError("the three prefix-sum lists need one entry per sequence")
+    out = ctypes.c_size_t(0)
+    _raise(load().nsa_compress_attention_workspace_size(
+        int(head_num), int(n2), int(d1), int(d2), int(l), int(d), int(lp), int(count), _ip(cq), _ip(cc),
+        _ip(cs), cq.size, ctypes.byref(out)), "nsa_compress_attention_workspace_size")
+    return int(out.value)
+
+
+def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tensor, scale: float,
+                           head_num: int, l: int, d: int, lp: int, count: int, cu_seqlens_q,
+                           cu_cmp_kv, cu_sel_kv, out=None, workspace: Optional[torch.Tensor] = None,
+                           stream=None):
+    """Compressed attention + importance scores + top-k.
+
+    Returns (attention_out (T1,N1,D2), topk_indices (T1,N2,count) int32,
+    softmax_max (T1,N1,8) fp32, softmax_sum (T1,N1,8) fp32).
+    ``out`` may pass these four tensors preallocated.
+    """
+    for t, nm in ((q, "q"), (kcmp, "kcmp"), (vcmp, "vcmp")):
+        _dev(t, nm)
+        if t.dim() != 3:
+            raise ValueError(f"{nm} must be 3-D (TND)")
+    dt = _dtype_code(q)
+    if kcmp.dtype != q.dtype or vcmp.dtype != q.dtype:
+        raise TypeError("q, kcmp and vcmp must share one dtype")
+    t1, n1, d1 = q.shape
+    tc, n2, d1k = kcmp.shape
+    d2 = vcmp.shape[2]
+    if int(head_num) != n1:
+        raise ValueError("head_num must equal the number of query heads")
+    if d1k != d1 or tuple(vcmp.shape[:2]) != (tc, n2):
+        raise ValueError("kcmp must be (Tc, N2, D1) and vcmp (Tc, N2, D2)")
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size):
+        raise ValueError("the three prefix-sum lists need one entry per sequence")
+    if int(cq[-1]) > t1 or int(cc[-1]) > tc:
+        raise ValueError("prefix sums run past the rows of q / kcmp")
+    dev = q.device
+    if out is None:
+        att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
+        tk = torch.empty(t1, n2, count, dtype=torch.int32, device=dev)
+        smax = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
+        ssum = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
+    else:
+        att, tk, smax, ssum = out
+    ws_bytes = nsa_compress_attention_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st = load().nsa_compress_attention(
+        q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
+        int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
+        tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        _stream(stream))
+    _raise(st, "nsa_compress_attention")
+    return att, tk, smax, ssum
+
+
+def nsa_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and read the device error word of an attention workspace."""
+    return int(load().nsa_workspace_status(workspace.data_ptr(), _stream(stream)))
+
+
+def nsa_compress_status(stream=None) -> int:
+    return int(load().nsa_compress_status(_stream(stream)))

@@ -1,0 +1,454 @@
+// nsa_api.cu -- the C ABI: argument validation, work decomposition, tensor
+// maps and launches.  Validation returns a status before anything is enqueued
+// ("aclnnNsaCompress": the first phase checks the parameters and returns a
+// status code); the launches are asynchronous on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/nsa.h"
+#include "nsa_internal.h"
+
+using namespace nsa;
+
+namespace {
+
+constexpr size_t kWsHeader = 256;     // error word + padding
+constexpr int kMaxGrid = 160;         // persistent CTAs sized for one CTA per SM (148 on B200)
+constexpr int kSmemLimit = 232448;    // dynamic shared memory per block on sm_100
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nsa_status_t check_prefix(const int32_t* cu, int batch) {
+    if (cu == nullptr || batch < 1) return NSA_ERR_INVALID_ARG;
+    int32_t prev = 0;
+    for (int b = 0; b < batch; ++b) {
+        if (cu[b] < prev) return NSA_ERR_INVALID_ARG;   // prefix sums never decrease
+        prev = cu[b];
+    }
+    return NSA_OK;
+}
+
+int64_t ncmp_of(int64_t S, int l, int d) {
+    // aclnnNsaCompress Formula: blocks i = 0 .. floor((S-l)/d); none when S < l
+    return S < l ? 0 : (S - l) / d + 1;
+}
+
+inline int nvis_host(int64_t t, int l, int d, int n_cmp) {
+    if (t < l - 1) return 0;
+    return (int)std::min<int64_t>(n_cmp, (t - l + 1) / d + 1);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3D map over a TND tensor (D contiguous, then N, then T), 64-element boxes
+// along D with 128-byte swizzle.
+bool encode_tnd(CUtensorMap* map, const void* base, int dtype, int D, int N, int64_t T, int box_n,
+                int box_t) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)std::max<int64_t>(T, 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * N * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_n, (cuuint32_t)box_t};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------
+// attention plan: everything derived from the host arguments
+// ------------------------------------------------------------------------
+struct AttnPlan {
+    int G = 0, TT = 0, a = 0, b = 0, nkv_cols = 0;
+    std::vector<AttnTile> tiles;
+    int score_cap = 1;
+    int grid = 0;
+    bool score_in_smem = true;
+    int nslot = 0;
+    int off_q = 0, off_ring = 0, slot_bytes = 0, off_p = 0, off_stage = 0, off_score = 0, off_bar = 0,
+        smem_bytes = 0;
+    size_t ws_tiles = 0, ws_score = 0, ws_total = 0;
+};
+
+nsa_status_t validate_attention(int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
+                                const int32_t* cu_q, const int32_t* cu_cmp, const int32_t* cu_sel,
+                                int batch) {
+    // note list of mindspore.ops.nsa_compress_attention
+    if (l % 16 || d % 16 || lp % 16) return NSA_ERR_INVALID_ARG;
+    if (l < 16 || l > 128 || d < 16 || d > 64 || lp < 16 || lp > 128) return NSA_ERR_INVALID_ARG;
+    if (l < d || lp < l || lp % d) return NSA_ERR_INVALID_ARG;
+    if (count < 1 || count > 32) return NSA_ERR_INVALID_ARG;
+    if (d1 < 16 || d2 < 16 || d1 % 16 || d2 % 16 || d1 < d2) return NSA_ERR_INVALID_ARG;
+    if (n2 < 1 || head_num < n2 || head_num % n2) return NSA_ERR_INVALID_ARG;
+    nsa_status_t s;
+    if ((s = check_prefix(cu_q, batch)) != NSA_OK) return s;
+    if ((s = check_prefix(cu_cmp, batch)) != NSA_OK) return s;
+    if ((s = check_prefix(cu_sel, batch)) != NSA_OK) return s;
+    // beyond the pages' constraints: what this build runs
+    if (l % d) return NSA_ERR_UNSUPPORTED;          // l/d must be an integer in step 4
+    if (d1 > 256 || d2 > 256) return NSA_ERR_UNSUPPORTED;
+    if (head_num / n2 > kRows) return NSA_ERR_UNSUPPORTED;
+    return NSA_OK;
+}
+
+nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
+                            const int32_t* cu_q, const int32_t* cu_cmp, const int32_t* cu_sel, int batch,
+                            bool build_tiles, AttnPlan& pl) {
+    nsa_status_t s = validate_attention(head_num, n2, d1, d2, l, d, lp, count, cu_q, cu_cmp, cu_sel, batch);
+    if (s != NSA_OK) return s;
+    pl.G = head_num / n2;
+    pl.TT = kRows / pl.G;
+    pl.a = lp / d;
+    pl.b = l / d;
+    pl.nkv_cols = attention_kv_cols(pl.a);
+    const int NKV = pl.nkv_cols;
+    // tiles: (sequence, group, run of TT tokens)
+    int64_t ntiles = 0;
+    int cap = 1;
+    {
+        int32_t pq = 0, pc = 0, ps = 0;
+        for (int bq = 0; bq < batch; ++bq) {
+            const int64_t Sq = cu_q[bq] - pq;
+            const int n_cmp = cu_cmp[bq] - pc;
+            const int n_sel = cu_sel[bq] - ps;
+            const int64_t off = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
+            if (Sq > 0) {
+                const int64_t tlast = Sq - 1 + off;
+                if (nvis_host(tlast, l, d, n_cmp) > 0)
+                    cap = std::max<int64_t>(cap, std::min<int64_t>(n_sel, tlast / lp + 1));
+                ntiles += ((Sq + pl.TT - 1) / pl.TT) * (int64_t)n2;
+            }
+            pq = cu_q[bq];
+            pc = cu_cmp[bq];
+            ps = cu_sel[bq];
+        }
+    }
+    if (ntiles > (int64_t)1 << 30) return NSA_ERR_UNSUPPORTED;
+    pl.score_cap = (cap + 3) & ~3;
+    pl.grid = (int)std::min<int64_t>(ntiles, kMaxGrid);
+
+    if (build_tiles) {
+        pl.tiles.clear();
+        pl.tiles.reserve((size_t)ntiles);
+        int32_t pq = 0, pc = 0, ps = 0;
+        for (int bq = 0; bq < batch; ++bq) {
+            const int Sq = cu_q[bq] - pq;
+            const int n_cmp = cu_cmp[bq] - pc;
+            const int n_sel = cu_sel[bq] - ps;
+            const int64_t off = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
+            for (int tok0 = 0; tok0 < Sq; tok0 += pl.TT) {
+                AttnTile t;
+                t.q_row0 = pq + tok0;
+                t.ntok = std::min(pl.TT, Sq - tok0);
+                t.cmp_row0 = pc;
+                t.n_cmp = n_cmp;
+                t.n_sel = n_sel;
+                t.t0 = (int)(tok0 + off);
+                const int nv = nvis_host(t.t0 + t.ntok - 1, l, d, n_cmp);
+                t.nkv = (nv + NKV - 1) / NKV;
+                for (int g = 0; g < n2; ++g) {
+                    t.group = g;
+                    pl.tiles.push_back(t);
+                }
+            }
+            pq = cu_q[bq];
+            pc = cu_cmp[bq];
+            ps = cu_sel[bq];
+        }
+        // longest tiles first: with the round-robin hand-out of the persistent
+        // grid this approximates longest-processing-time-first scheduling
+        std::stable_sort(pl.tiles.begin(), pl.tiles.end(),
+                         [](const AttnTile& x, const AttnTile& y) { return x.nkv > y.nkv; });
+    }
+
+    // shared memory layout
+    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
+    const int NJ = NKV / pl.a;
+    const int CHK = std::min(NJ, kBandChunk);
+    pl.off_q = 0;
+    pl.off_ring = nqc * 16384;
+    pl.slot_bytes = std::max(nqc, nvc) * NKV * 128;
+    const int p_bytes = ((NKV + 63) / 64) * 16384;
+    const int stage_bytes = kRows * (CHK + 1) * 4;
+    const int score_bytes = pl.TT * pl.score_cap * 4;
+    const int bar_bytes = 8 * 32 + 64;
+    auto layout = [&](int nslot, bool in_smem) {
+        int off = pl.off_ring + nslot * pl.slot_bytes;
+        pl.off_p = off;
+        off += p_bytes;
+        pl.off_stage = off;
+        off += (stage_bytes + 127) & ~127;
+        pl.off_score = off;
+        if (in_smem) off += (score_bytes + 127) & ~127;
+        pl.off_bar = off;
+        off += bar_bytes;
+        pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
+        pl.nslot = nslot;
+        pl.score_in_smem = in_smem;
+        return pl.smem_bytes <= kSmemLimit;
+    };
+    bool fits = false;
+    for (int ns = 4; ns >= 2 && !fits; --ns) fits = layout(ns, true);
+    for (int ns = 4; ns >= 2 && !fits; --ns) fits = layout(ns, false);
+    if (!fits) return NSA_ERR_UNSUPPORTED;
+
+    pl.ws_tiles = (size_t)ntiles * sizeof(AttnTile);
+    pl.ws_score = pl.score_in_smem ? 0 : (size_t)pl.grid * pl.TT * pl.score_cap * 4;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    pl.ws_total = kWsHeader + up(pl.ws_tiles) + up(pl.ws_score);
+    return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nsa_status_string(nsa_status_t s) {
+    switch (s) {
+        case NSA_OK: return "NSA_OK";
+        case NSA_ERR_INVALID_ARG: return "NSA_ERR_INVALID_ARG";
+        case NSA_ERR_UNSUPPORTED: return "NSA_ERR_UNSUPPORTED";
+        case NSA_ERR_WORKSPACE: return "NSA_ERR_WORKSPACE";
+        case NSA_ERR_CUDA: return "NSA_ERR_CUDA";
+        case NSA_ERR_TIMEOUT: return "NSA_ERR_TIMEOUT";
+    }
+    return "NSA_ERR_UNKNOWN";
+}
+
+nsa_status_t nsa_compress_out_len(const int32_t* cu_seqlens, int batch, int l, int d, int32_t* cu_cmp_out,
+                                  int64_t* total_out) {
+    if (cu_cmp_out == nullptr || l < 1 || d < 1) return NSA_ERR_INVALID_ARG;
+    nsa_status_t s = check_prefix(cu_seqlens, batch);
+    if (s != NSA_OK) return s;
+    int64_t tot = 0;
+    int32_t prev = 0;
+    for (int b = 0; b < batch; ++b) {
+        tot += ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
+        prev = cu_seqlens[b];
+        if (tot > INT32_MAX) return NSA_ERR_INVALID_ARG;
+        cu_cmp_out[b] = (int32_t)tot;
+    }
+    if (total_out) *total_out = tot;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, int d, const int32_t* cu_seqlens,
+                          int batch, int n2, int d1, int d2, nsa_dtype_t dtype, void* kcmp, void* vcmp,
+                          void* stream) {
+    // constraint lists of aclnnNsaCompress and mindspore.ops.nsa_compress_attention
+    if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
+    if (k == nullptr || w == nullptr || kcmp == nullptr) return NSA_ERR_INVALID_ARG;
+    if ((v == nullptr) != (vcmp == nullptr)) return NSA_ERR_INVALID_ARG;
+    if (l % 16 || d % 16 || d < 16 || l < d || l > 128) return NSA_ERR_INVALID_ARG;
+    if (n2 < 1 || d1 < 16 || d1 % 16 || d1 > 256) return NSA_ERR_INVALID_ARG;
+    if (v && (d2 < 16 || d2 % 16 || d2 > 256)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(kcmp) || (v && (!aligned16(v) || !aligned16(vcmp))))
+        return NSA_ERR_INVALID_ARG;
+    nsa_status_t s = check_prefix(cu_seqlens, batch);
+    if (s != NSA_OK) return s;
+    const int dmax = v ? std::max(d1, d2) : d1;
+    const int64_t rowelems = (int64_t)n2 * dmax;
+    if (rowelems / 8 > kCompressMaxThreads) return NSA_ERR_UNSUPPORTED;
+    if ((int64_t)cu_seqlens[batch - 1] * rowelems > ((int64_t)1 << 40)) return NSA_ERR_UNSUPPORTED;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+
+    // sizes of the per-CTA ring and the output run of one CTA
+    const int rowbytes = (int)(rowelems * 2);
+    int rs = std::max(1, 16384 / rowbytes);
+    const int stage_bytes = rs * rowbytes;
+    const int wbytes = ((l * n2 * 4) + 127) & ~127;
+    const size_t smem = (size_t)wbytes + 128 + (size_t)kCompressStages * stage_bytes;
+    if (smem > (size_t)kSmemLimit) return NSA_ERR_UNSUPPORTED;
+    const int occ = std::max(1, std::min(8, (int)(228 * 1024 / (smem + 1024))));
+    int64_t total_out = 0;
+    {
+        int32_t prev = 0;
+        for (int b = 0; b < batch; ++b) {
+            total_out += ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
+            prev = cu_seqlens[b];
+        }
+    }
+    if (total_out == 0) return NSA_OK;
+    const int planes = v ? 2 : 1;
+    const int64_t target = (int64_t)nsm * occ;
+    int chunk = (int)std::min<int64_t>(1024, std::max<int64_t>(4, (total_out * planes + target - 1) / target));
+
+    CompressParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k;
+    p.v = v;
+    p.w = w;
+    p.kcmp = kcmp;
+    p.vcmp = vcmp;
+    p.l = l;
+    p.d = d;
+    p.n2 = n2;
+    p.d1 = d1;
+    p.d2 = v ? d2 : d1;
+    p.dtype = dtype == NSA_BF16 ? 0 : 1;
+    p.chunk = chunk;
+    p.rows_per_stage = rs;
+    const int threads = (int)(((rowelems / 8) + 31) / 32 * 32);
+
+    int32_t prev_raw = 0;
+    int64_t cmp_prev = 0;
+    int b = 0;
+    while (b < batch) {
+        p.nseq = 0;
+        int chunks = 0;
+        for (; b < batch && p.nseq < kCompressMaxSeq; ++b) {
+            const int64_t S = (int64_t)cu_seqlens[b] - prev_raw;
+            const int64_t nc = ncmp_of(S, l, d);
+            CompressSeq& q = p.seq[p.nseq];
+            q.raw_start = prev_raw;
+            q.cmp_start = (int)cmp_prev;
+            q.ncmp = (int)nc;
+            q.nchunks = (int)((nc + chunk - 1) / chunk);
+            chunks += q.nchunks;
+            q.chunk_end = chunks;
+            prev_raw = cu_seqlens[b];
+            cmp_prev += nc;
+            ++p.nseq;
+        }
+        if (chunks == 0) continue;
+        cudaError_t e = launch_compress(p, dim3(chunks, planes), threads, smem, st);
+        if (e != cudaSuccess) return NSA_ERR_CUDA;
+    }
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_status(void* stream) {
+    int err = 0;
+    if (read_compress_error(&err, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NSA_ERR_CUDA;
+    return err ? NSA_ERR_TIMEOUT : NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention_workspace_size(int head_num, int n2, int d1, int d2, int l, int d, int lp,
+                                                   int count, const int32_t* cu_seqlens_q,
+                                                   const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+                                                   int batch, size_t* bytes) {
+    if (bytes == nullptr) return NSA_ERR_INVALID_ARG;
+    AttnPlan pl;
+    nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                    batch, false, pl);
+    if (s != NSA_OK) return s;
+    *bytes = pl.ws_total;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
+                                    int l, int d, int lp, int count, const int32_t* cu_seqlens_q,
+                                    const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv, int batch, int n2, int d1,
+                                    int d2, nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
+                                    float* softmax_max, float* softmax_sum, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
+    if (!q || !kcmp || !vcmp || !attention_out || !topk_indices || !softmax_max || !softmax_sum)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kcmp) || !aligned16(vcmp) || !aligned16(attention_out) ||
+        !aligned16(topk_indices) || !aligned16(softmax_max) || !aligned16(softmax_sum))
+        return NSA_ERR_INVALID_ARG;
+    AttnPlan pl;
+    nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                    batch, true, pl);
+    if (s != NSA_OK) return s;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < pl.ws_total)
+        return NSA_ERR_WORKSPACE;
+    if (pl.tiles.empty()) return NSA_OK;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t t1 = cu_seqlens_q[batch - 1];
+    const int64_t tc = cu_cmp_kv[batch - 1];
+    CUtensorMap tq, tk, tv;
+    if (!encode_tnd(&tq, q, dtype, d1, head_num, t1, pl.G, pl.TT) ||
+        !encode_tnd(&tk, kcmp, dtype, d1, n2, tc, 1, pl.nkv_cols) ||
+        !encode_tnd(&tv, vcmp, dtype, d2, n2, tc, 1, pl.nkv_cols))
+        return NSA_ERR_UNSUPPORTED;
+
+    // workspace: [header: error word][tile list][score buffers]
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    std::vector<uint8_t> host(kWsHeader + pl.ws_tiles, 0);
+    std::memcpy(host.data() + kWsHeader, pl.tiles.data(), pl.ws_tiles);
+    if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.tiles = reinterpret_cast<const AttnTile*>(ws + kWsHeader);
+    p.num_tiles = (int)pl.tiles.size();
+    p.err = reinterpret_cast<int*>(ws);
+    p.score_gmem = pl.score_in_smem ? nullptr
+                                    : reinterpret_cast<float*>(ws + kWsHeader + ((pl.ws_tiles + 255) & ~(size_t)255));
+    p.score_cap = pl.score_cap;
+    p.score_in_smem = pl.score_in_smem ? 1 : 0;
+    p.out = attention_out;
+    p.topk = topk_indices;
+    p.smax = softmax_max;
+    p.ssum = softmax_sum;
+    p.dtype = dtype == NSA_BF16 ? 0 : 1;
+    p.n1 = head_num;
+    p.n2 = n2;
+    p.d1 = d1;
+    p.d2 = d2;
+    p.G = pl.G;
+    p.tok_per_tile = pl.TT;
+    p.l = l;
+    p.d = d;
+    p.lp = lp;
+    p.count = count;
+    p.a = pl.a;
+    p.b = pl.b;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.nkv_cols = pl.nkv_cols;
+    p.nslot = pl.nslot;
+    p.off_q = pl.off_q;
+    p.off_ring = pl.off_ring;
+    p.slot_bytes = pl.slot_bytes;
+    p.off_p = pl.off_p;
+    p.off_stage = pl.off_stage;
+    p.off_score = pl.off_score;
+    p.off_bar = pl.off_bar;
+    p.smem_bytes = pl.smem_bytes;
+    const int grid = std::min(pl.grid, nsm);
+    if (launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_workspace_status(const void* workspace, void* stream) {
+    if (workspace == nullptr) return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return NSA_ERR_CUDA;
+    int err = 0;
+    if (cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NSA_ERR_CUDA;
+    return err ? NSA_ERR_TIMEOUT : NSA_OK;
+}
+
+}  // extern "C"

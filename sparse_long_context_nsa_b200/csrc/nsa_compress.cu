@@ -1,0 +1,257 @@
+// nsa_compress.cu -- sliding-window compression of raw K/V into block tokens.
+//
+// "aclnnNsaCompress", Formula section: block i of a sequence is
+// phi(k[i*d .. i*d+l-1]) for 0 <= i <= floor((S-l)/d); phi is the weighted sum
+// over the window with one weight per window position and head, the same
+// weights for K and V.
+//
+// HBM-bound.  Each CTA owns a run of consecutive output blocks of one sequence
+// and one tensor (K or V).  The raw rows of the run are contiguous in TND
+// layout, so they are streamed through a shared-memory ring with 1D bulk
+// copies (one copy moves a few rows of every head at once).  Every raw row is
+// read from HBM once per CTA; the windows overlap in shared memory only.
+// Each thread owns one 16-byte column vector (8 elements of one head) and
+// keeps the partial sums of the <= ceil(l/d) windows that cover the current
+// row in registers, shifting them by one slot at each group of d rows.
+// fp32 accumulation in window order; one RNE rounding at the store.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "nsa_internal.h"
+#include "ptx.cuh"
+
+namespace nsa {
+
+__device__ int g_compress_err = 0;
+
+template <typename T>
+__device__ __forceinline__ void cvt8(const uint4& u, float (&f)[8]);
+template <>
+__device__ __forceinline__ void cvt8<__nv_bfloat16>(const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+template <>
+__device__ __forceinline__ void cvt8<__half>(const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+        float2 v = __half22float2(h);
+        f[2 * i] = v.x;
+        f[2 * i + 1] = v.y;
+    }
+}
+template <typename T>
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]);
+template <>
+__device__ __forceinline__ uint4 pack8<__nv_bfloat16>(const float (&f)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <>
+__device__ __forceinline__ uint4 pack8<__half>(const float (&f)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half x) { return __half2float(x); }
+
+// One CTA = one run of output blocks [i0, i1) of one sequence of one tensor.
+// BMAX >= ceil(l/d): number of register slots for overlapping windows.
+template <typename T, int BMAX>
+__global__ void __launch_bounds__(kCompressMaxThreads)
+nsa_compress_kernel(const CompressParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // --- locate the work item: blockIdx.y = tensor (0 = K, 1 = V) ---
+    const int plane = blockIdx.y;
+    const int dim = plane == 0 ? p.d1 : p.d2;
+    const T* __restrict__ src = reinterpret_cast<const T*>(plane == 0 ? p.k : p.v);
+    T* __restrict__ dst = reinterpret_cast<T*>(plane == 0 ? p.kcmp : p.vcmp);
+    if (src == nullptr) return;
+    int lo = 0, hi = p.nseq - 1;   // first sequence whose chunk prefix exceeds blockIdx.x
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (p.seq[mid].chunk_end > (int)blockIdx.x) hi = mid; else lo = mid + 1;
+    }
+    const CompressSeq sq = p.seq[lo];
+    const int chunk = blockIdx.x - (sq.chunk_end - sq.nchunks);
+    const int i0 = chunk * p.chunk;
+    const int i1 = min(i0 + p.chunk, sq.ncmp);
+    if (i0 >= i1) return;
+
+    const int l = p.l, d = p.d;
+    const int nb = (l + d - 1) / d;                  // windows covering one row
+    const int rowelems = p.n2 * dim;
+    const int rowbytes = rowelems * (int)sizeof(T);
+    const int nvec = rowelems / 8;                   // 16-byte vectors per row
+    const int64_t rel0 = (int64_t)i0 * d;            // first raw row of the run (in seq)
+    const int nrows = (i1 - 1 - i0) * d + l;         // raw rows of the run
+    const int rs = p.rows_per_stage;
+    const int nstage = (nrows + rs - 1) / rs;
+    const char* gsrc = reinterpret_cast<const char*>(src) +
+                       ((int64_t)sq.raw_start + rel0) * (int64_t)rowbytes;
+
+    // --- shared memory: [weights fp32 l x n2][barriers][stages] ---
+    float* wsm = reinterpret_cast<float*>(smem_raw);
+    const int wbytes = ((l * p.n2 * 4) + 127) & ~127;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + wbytes);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + wbytes + 8 * kCompressStages);
+    uint8_t* stages = smem_raw + wbytes + 128;
+    const int stage_bytes = rs * rowbytes;
+
+    const T* wsrc = reinterpret_cast<const T*>(p.w);
+    for (int i = threadIdx.x; i < l * p.n2; i += blockDim.x) wsm[i] = to_f32<T>(wsrc[i]);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kCompressStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    auto issue = [&](int s) {
+        const int slot = s % kCompressStages;
+        const int rows = min(rs, nrows - s * rs);
+        const uint32_t bytes = (uint32_t)(rows * rowbytes);
+        const uint32_t bar = smem_u32(&bars[slot]);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(smem_u32(stages + slot * stage_bytes), gsrc + (int64_t)s * stage_bytes, bytes, bar);
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kCompressStages && s < nstage; ++s) issue(s);
+    }
+
+    const int cv = threadIdx.x;                      // column vector of this thread
+    const bool active = cv < nvec;
+    const int head = active ? (cv * 8) / dim : 0;
+    float acc[BMAX][8];
+#pragma unroll
+    for (int k = 0; k < BMAX; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+
+    int64_t rel = rel0;                              // raw row within the sequence
+    int q = i0;                                      // rel / d
+    int rin = 0;                                     // rel % d
+    int next_issue = min(kCompressStages, nstage);   // stages handed to the copy engine
+    int s = 0;
+    bool failed = false;
+    for (; s < nstage; ++s) {
+        const int slot = s % kCompressStages;
+        const uint32_t parity = (uint32_t)((s / kCompressStages) & 1);
+        const bool got = mbar_wait(smem_u32(&bars[slot]), parity, abort_flag, &g_compress_err,
+                                   kErrTimeoutBase + 1);
+        const int rows = min(rs, nrows - s * rs);
+        const uint8_t* base = stages + slot * stage_bytes;
+        if (active && got) {
+            for (int r = 0; r < rows; ++r) {
+                const uint4 u = *reinterpret_cast<const uint4*>(base + r * rowbytes + cv * 16);
+                float x[8];
+                cvt8<T>(u, x);
+#pragma unroll
+                for (int k = 0; k < BMAX; ++k) {
+                    const int j = k * d + rin;                // position inside window q-k
+                    if (k < nb && j < l) {
+                        const float wv = wsm[j * p.n2 + head];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wv, x[e], acc[k][e]);
+                    }
+                }
+                ++rel;
+                ++rin;
+                const bool last_row = (s == nstage - 1) && (r == rows - 1);
+                if (rin == d || last_row) {
+                    // window q-(nb-1) has seen its last row: store it, shift slots
+                    const int i = q - (nb - 1);
+                    if (i >= i0 && i < i1) {
+                        float o[8];
+#pragma unroll
+                        for (int kk = 0; kk < BMAX; ++kk)
+                            if (kk == nb - 1)
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) o[e] = acc[kk][e];
+                        T* out = dst + ((int64_t)sq.cmp_start + i) * rowelems + cv * 8;
+                        *reinterpret_cast<uint4*>(out) = pack8<T>(o);
+                    }
+#pragma unroll
+                    for (int kk = BMAX - 1; kk >= 1; --kk)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[kk][e] = acc[kk - 1][e];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[0][e] = 0.f;
+                    rin = 0;
+                    ++q;
+                }
+            }
+        }
+        // every thread is done with this slot, and all agree whether the wait succeeded
+        if (!__syncthreads_and(got ? 1 : 0)) { failed = true; break; }
+        if (threadIdx.x == 0 && next_issue < nstage) issue(next_issue);
+        if (next_issue < nstage) ++next_issue;
+    }
+    if (failed && threadIdx.x == 0) {
+        // a wait gave up: let the copies still in flight land before the CTA exits
+        for (int u = s; u < next_issue; ++u) {
+            const uint32_t bar = smem_u32(&bars[u % kCompressStages]);
+            const uint32_t parity = (uint32_t)((u / kCompressStages) & 1);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < 100000000ull) {
+            }
+        }
+    }
+}
+
+template <typename T, int BMAX>
+static cudaError_t launch_t(const CompressParams& p, dim3 grid, int threads, size_t smem,
+                            cudaStream_t st) {
+    auto kern = nsa_compress_kernel<T, BMAX>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, threads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compress(const CompressParams& p, dim3 grid, int threads, size_t smem,
+                            cudaStream_t st) {
+    const int nb = (p.l + p.d - 1) / p.d;
+    const bool bf = p.dtype == 0;
+#define NSA_DISPATCH(BM)                                                                     \
+    return bf ? launch_t<__nv_bfloat16, BM>(p, grid, threads, smem, st)                      \
+              : launch_t<__half, BM>(p, grid, threads, smem, st);
+    if (nb <= 1) { NSA_DISPATCH(1) }
+    if (nb <= 2) { NSA_DISPATCH(2) }
+    if (nb <= 4) { NSA_DISPATCH(4) }
+    NSA_DISPATCH(8)
+#undef NSA_DISPATCH
+}
+
+cudaError_t read_compress_error(int* out, cudaStream_t st) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(out, g_compress_err, sizeof(int), 0, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess || *out == 0) return e;
+    const int zero = 0;   // reported once: clear for the next call
+    return cudaMemcpyToSymbol(g_compress_err, &zero, sizeof(int), 0, cudaMemcpyHostToDevice);
+}
+
+}  // namespace nsa

@@ -1,0 +1,84 @@
+// nsa_internal.h -- structures shared by the host launcher (nsa_api.cu) and
+// the kernels.  Not part of the public C ABI.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nsa {
+
+// ------------------------------------------------------------ compress
+constexpr int kCompressStages = 4;        // shared-memory ring depth
+constexpr int kCompressMaxThreads = 512;  // one thread per 16-byte column vector
+constexpr int kCompressMaxSeq = 96;       // sequences per launch (kernel-parameter space)
+
+struct CompressSeq {
+    int raw_start;   // first raw row of the sequence (T2 index)
+    int cmp_start;   // first compressed row (Tc index)
+    int ncmp;        // compressed blocks of the sequence
+    int nchunks;     // CTAs given to the sequence
+    int chunk_end;   // inclusive prefix of nchunks over the launch's sequences
+};
+
+struct CompressParams {
+    const void* k;
+    const void* v;
+    const void* w;
+    void* kcmp;
+    void* vcmp;
+    int l, d, n2, d1, d2;
+    int dtype;            // 0 bf16, 1 fp16
+    int chunk;            // output blocks per CTA
+    int rows_per_stage;   // raw rows per bulk copy
+    int nseq;
+    CompressSeq seq[kCompressMaxSeq];
+};
+
+cudaError_t launch_compress(const CompressParams& p, dim3 grid, int threads, size_t smem,
+                            cudaStream_t st);
+cudaError_t read_compress_error(int* out, cudaStream_t st);
+
+// ----------------------------------------------------------- attention
+constexpr int kAttnThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 softmax/epilogue
+constexpr int kRows = 128;          // M of one tile: (tokens x heads of one KV group)
+constexpr int kBandChunk = 16;      // importance scores staged per named-barrier round
+
+// One M-tile: up to 128/G consecutive query tokens of one sequence x the G
+// heads of one KV group.
+struct AttnTile {
+    int q_row0;     // first query row (T1 index)
+    int ntok;       // tokens in the tile (<= tokens per tile)
+    int group;      // KV head g
+    int cmp_row0;   // first compressed row of the sequence (Tc index)
+    int n_cmp;      // compressed blocks of the sequence
+    int n_sel;      // selection blocks of the sequence
+    int t0;         // position of the first token (query offset applied)
+    int nkv;        // KV tiles to visit (both passes)
+};
+
+struct AttnParams {
+    const AttnTile* tiles;
+    int num_tiles;
+    int* err;               // device error word (workspace)
+    float* score_gmem;      // per-CTA score buffers when they do not fit on chip
+    int score_cap;          // floats per token in a score buffer
+    int score_in_smem;
+    void* out;
+    int32_t* topk;
+    float* smax;
+    float* ssum;
+    int dtype;              // 0 bf16, 1 fp16
+    int n1, n2, d1, d2, G, tok_per_tile;
+    int l, d, lp, count, a, b;
+    float scale_log2;       // scale * log2(e)
+    int nkv_cols;           // compressed blocks per KV tile
+    int nslot;              // K/V ring depth
+    // shared-memory layout (byte offsets from a 1024-aligned base)
+    int off_q, off_ring, slot_bytes, off_p, off_stage, off_score, off_bar, smem_bytes;
+};
+
+cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, int grid, cudaStream_t st);
+int attention_kv_cols(int a);   // compressed blocks per KV tile for band factor a
+
+}  // namespace nsa

@@ -1,0 +1,108 @@
+"""Comparison rules between the CUDA path and the fp64 oracle.
+
+Tolerances (written here once, used by every parity test):
+  compress       |gpu - oracle| <= 1 ulp(oracle, storage dtype)
+                                  + l * 2^-24 * sum_j |w_j x_j|
+                 The oracle rounds the exact fp64 sum once; the kernel rounds
+                 an fp32 running sum once.  Away from cancellation the two
+                 differ by at most one unit in the last place; near a
+                 cancelling sum the fp32 accumulation error bound (l terms,
+                 unit roundoff 2^-24, times the sum of magnitudes) decides.
+  attention_out  max |gpu - oracle| <= 1e-2 (the stated bar for bf16 inputs)
+  softmax stats  relative error <= 1e-3, absolute floor 1e-6 where
+                 |oracle| < 1e-3; empty rows exactly -inf / 0; all 8 copies
+                 equal.
+  topk_indices   same number of -1 entries; valid, ascending, distinct
+                 indices; the two index sets may differ only in indices whose
+                 oracle score is within 1e-4 (relative) of the oracle's k-th
+                 largest score (several answers are correct at near-ties).
+"""
+import numpy as np
+import torch
+
+import oracle
+
+
+def ulp(y: np.ndarray, dtype: int) -> np.ndarray:
+    p, emin = (8, -126) if dtype == oracle.BF16 else (11, -14)
+    _, e = np.frexp(np.abs(y))
+    q = np.maximum(e - p, emin - p + 1)
+    return np.ldexp(1.0, q)
+
+
+def check_compress(got: torch.Tensor, x, w, l, d, cu, dtype):
+    """got: (Tc, N2, D) device tensor; x, w: inputs as given to the GPU."""
+    ref, _ = oracle.compress(x, w, l, d, cu, dtype=dtype)
+    mag, _ = oracle.compress(np.abs(oracle._f64(x)), np.abs(oracle._f64(w)), l, d, cu)
+    g = got.double().cpu().numpy()
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    tol = ulp(ref, dtype) + l * 2.0 ** -24 * mag
+    err = np.abs(g - ref)
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} elements off; worst {err.max()} (tol there {tol.ravel()[err.argmax()]})"
+    return float(err.max())
+
+
+def check_attention(res, ref, count, rows=None, tie_rel=1e-4, out_tol=1e-2, stat_rel=1e-3):
+    """res: GPU outputs (att, topk, smax, ssum); ref: oracle dict for `rows`."""
+    att, tk, smax, ssum = res
+    if rows is None:
+        rows = ref["rows"]
+    rows_t = torch.as_tensor(np.asarray(rows), dtype=torch.long, device=att.device)
+    g_out = att.index_select(0, rows_t).double().cpu().numpy()
+    g_tk = tk.index_select(0, rows_t).cpu().numpy()
+    g_max = smax.index_select(0, rows_t).cpu().numpy()
+    g_sum = ssum.index_select(0, rows_t).cpu().numpy()
+    report = {}
+
+    # attention_out
+    assert np.isfinite(g_out).all(), "non-finite attention_out"
+    err = np.abs(g_out - ref["out"])
+    report["out_max_abs"] = float(err.max()) if err.size else 0.0
+    assert report["out_max_abs"] <= out_tol, f"attention_out max abs err {report['out_max_abs']}"
+
+    # stats: 8 equal copies, empty rows exact
+    assert (g_max == g_max[..., :1]).all() and (g_sum == g_sum[..., :1]).all()
+    gm, gs = g_max[..., 0].astype(np.float64), g_sum[..., 0].astype(np.float64)
+    rm, rs = ref["softmax_max"], ref["softmax_sum"]
+    empty = np.isneginf(rm)
+    assert (np.isneginf(gm) == empty).all(), "empty-row max mismatch"
+    assert (gs[empty] == 0).all(), "empty-row sum must be 0"
+    ne = ~empty
+    for name, g, r in (("max", gm[ne], rm[ne]), ("sum", gs[ne], rs[ne])):
+        if g.size == 0:
+            continue
+        denom = np.where(np.abs(r) < 1e-3, 1.0, np.abs(r))
+        floor = np.where(np.abs(r) < 1e-3, 1e-6, 0.0)
+        e = np.abs(g - r)
+        ok = e <= stat_rel * denom + floor
+        report[f"{name}_max_rel"] = float((e / np.maximum(np.abs(r), 1e-30)).max())
+        assert ok.all(), f"softmax_{name}: {(~ok).sum()} rows off, worst rel {report[f'{name}_max_rel']}"
+
+    # top-k: tie-aware set comparison
+    rtk, score, ncand = ref["topk"], ref["score"], ref["ncand"]
+    R, N2, _ = rtk.shape
+    n_tie_diff = 0
+    for r in range(R):
+        for g in range(N2):
+            a = g_tk[r, g]
+            b = rtk[r, g]
+            na, nb = (a >= 0).sum(), (b >= 0).sum()
+            assert na == nb, f"row {rows[r]} group {g}: {na} vs {nb} indices"
+            va, vb = a[:na], b[:nb]
+            assert (a[na:] == -1).all(), "padding must follow the indices"
+            if na == 0:
+                continue
+            assert (np.diff(va) > 0).all(), f"indices not ascending: {va}"
+            assert va.min() >= 0 and va.max() < ncand[r, g], f"index out of candidate range: {va}"
+            if set(va.tolist()) == set(vb.tolist()):
+                continue
+            sc = score[r, g, :ncand[r, g]]
+            kth = np.sort(sc)[::-1][nb - 1]
+            diff = set(va.tolist()) ^ set(vb.tolist())
+            for j in diff:
+                assert abs(sc[j] - kth) <= tie_rel * abs(kth), (
+                    f"row {rows[r]} group {g}: index {j} score {sc[j]} vs k-th {kth}")
+            n_tie_diff += 1
+    report["topk_tie_rows"] = n_tie_diff
+    return report

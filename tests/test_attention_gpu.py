@@ -1,0 +1,194 @@
+"""Parity of the fused CUDA compressed-attention kernel with the fp64 oracle.
+
+Both sides get the same storage-dtype kcmp / vcmp (made by the oracle's
+compression of seeded raw K/V), so the comparison isolates steps 1-7.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import check_attention
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nsa():
+    from sparse_long_context_nsa_b200 import _build
+    _build.build()
+    import sparse_long_context_nsa_b200 as m
+    return m
+
+
+def _prepare(wl, device="cpu"):
+    x = wl.generate(device=device)
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
+    k, v, w = x["k"].cpu(), x["v"].cpu(), x["w"].cpu()
+    kc, cuc = oracle.compress(k, w, wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    vc, _ = oracle.compress(v, w, wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    tdt = wl.torch_dtype
+    kc_t = torch.from_numpy(kc).to(tdt)
+    vc_t = torch.from_numpy(vc).to(tdt)
+    return x, kc_t, vc_t, cuc
+
+
+def _run_both(nsa, wl, rows=None, device="cpu"):
+    x, kc, vc, cuc = _prepare(wl, device)
+    q = x["q"]
+    qd = q if q.is_cuda else q.cuda()
+    res = nsa.nsa_compress_attention(qd, kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp,
+                                     wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    torch.cuda.synchronize()
+    if rows is None:
+        qo = q.cpu()
+        ref = oracle.compress_attention(qo, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
+                                        x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    else:
+        rows = np.asarray(rows, dtype=np.int64)
+        qs = q.index_select(0, torch.from_numpy(rows).to(q.device)).cpu()
+        ref = oracle.compress_attention(qs, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
+                                        x["cu_seqlens_q"], cuc, x["cu_sel_kv"], rows=rows,
+                                        q_rows_only=True)
+    return res, ref, x, (kc, vc, cuc)
+
+
+def _wl(seqs, n1, n2, d1, d2, l, d, lp, count, dtype="bf16", seed=7, q_last=None, std=1.0):
+    return workloads.Workload("case", tuple(seqs), n1, n2, d1, d2, l, d, lp, count, d1 ** -0.5,
+                              dtype, seed=seed, std=std, q_last=q_last)
+
+
+def test_tiny_workload_full(nsa):
+    res, ref, _, _ = _run_both(nsa, workloads.TINY)
+    rep = check_attention(res, ref, workloads.TINY.count)
+    print(rep)
+
+
+GROUPS = [(4, 1), (8, 8), (12, 4), (16, 2), (32, 2), (64, 2), (64, 1), (128, 1)]
+
+
+@pytest.mark.parametrize("n1,n2", GROUPS, ids=lambda v: str(v))
+def test_group_sizes(nsa, n1, n2):
+    # several KV tiles (n_cmp = 155) with a ragged last tile and a ragged token tail
+    wl = _wl([2500], n1, n2, 64, 64, 32, 16, 64, 8)
+    res, ref, _, _ = _run_both(nsa, wl)
+    check_attention(res, ref, wl.count)
+
+
+BANDS = [(16, 16, 16), (32, 16, 32), (32, 16, 48), (32, 16, 64), (64, 16, 80), (32, 16, 96),
+         (64, 16, 112), (128, 16, 128), (64, 32, 64), (128, 64, 128), (64, 32, 128), (48, 16, 96)]
+
+
+@pytest.mark.parametrize("l,d,lp", BANDS, ids=lambda v: str(v))
+def test_band_parameters(nsa, l, d, lp):
+    wl = _wl([3000, 700], 16, 2, 64, 64, l, d, lp, 6)
+    res, ref, _, _ = _run_both(nsa, wl)
+    check_attention(res, ref, wl.count)
+
+
+@pytest.mark.parametrize("d1,d2,dtype", [(64, 64, "fp16"), (128, 128, "bf16"), (192, 128, "fp16"),
+                                         (96, 48, "bf16"), (128, 64, "bf16"), (32, 16, "fp16")])
+def test_head_dims_and_dtypes(nsa, d1, d2, dtype):
+    wl = _wl([1800, 333], 8, 2, d1, d2, 64, 32, 64, 16, dtype=dtype)
+    res, ref, _, _ = _run_both(nsa, wl)
+    check_attention(res, ref, wl.count)
+
+
+def test_varlen_with_empty_and_short_sequences(nsa):
+    wl = _wl([0, 900, 31, 47, 1, 2049, 16, 600], 16, 4, 64, 64, 32, 16, 64, 8)
+    res, ref, _, _ = _run_both(nsa, wl)
+    check_attention(res, ref, wl.count)
+
+
+@pytest.mark.parametrize("count", [1, 32])
+def test_count_extremes(nsa, count):
+    wl = _wl([1500], 8, 1, 64, 64, 32, 16, 32, count)
+    res, ref, _, _ = _run_both(nsa, wl)
+    check_attention(res, ref, wl.count)
+
+
+def test_short_queries_bottom_right_aligned(nsa):
+    wl = _wl([4096, 3000, 2001], 32, 4, 64, 64, 64, 32, 64, 16, q_last=100)
+    res, ref, _, _ = _run_both(nsa, wl)
+    check_attention(res, ref, wl.count)
+
+
+def test_score_buffer_in_global_memory(nsa):
+    # one head per group (128 tokens per tile) and many selection blocks:
+    # the per-token score buffers do not fit on chip and go to the workspace
+    wl = _wl([20000], 2, 2, 64, 64, 16, 16, 16, 32)
+    res, ref, _, _ = _run_both(nsa, wl, rows=workloads.sample_rows(np.array([20000], np.int32),
+                                                                      first=300, last=300, every=37))
+    check_attention(res, ref, wl.count)
+
+
+def test_deterministic_and_status(nsa):
+    wl = _wl([3000], 32, 2, 128, 128, 32, 16, 64, 16)
+    x, kc, vc, cuc = _prepare(wl)
+    args = (x["q"].cuda(), kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count,
+            x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
+        x["cu_sel_kv"]), dtype=torch.uint8, device="cuda")
+    a = nsa.nsa_compress_attention(*args, workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0
+    b = nsa.nsa_compress_attention(*args, workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1], b[1])
+    assert torch.equal(a[2], b[2]) and torch.equal(a[3], b[3])
+
+
+def test_end_to_end_gpu_compress_then_attention(nsa):
+    """GPU compress feeding GPU attention, against oracle compress + oracle
+    attention.  kcmp may differ by one ulp between the two sides, so the
+    top-k sets are reported and only required to agree on nearly all rows."""
+    wl = _wl([4000, 1234], 32, 4, 128, 128, 32, 16, 64, 16)
+    x = wl.generate()
+    kc, vc = nsa.nsa_compress(x["k"].cuda(), x["v"].cuda(), x["w"].cuda(), wl.l, wl.d, x["cu_seqlens"])
+    cuc = nsa.nsa_compress_out_len(x["cu_seqlens"], wl.l, wl.d)
+    res = nsa.nsa_compress_attention(x["q"].cuda(), kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count,
+                                     x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    okc, _ = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=oracle.BF16)
+    ovc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=oracle.BF16)
+    ref = oracle.compress_attention(x["q"], okc, ovc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
+                                    x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    out = res[0].double().cpu().numpy()
+    assert np.abs(out - ref["out"]).max() <= 1e-2
+    same = (res[1].cpu().numpy() == ref["topk"]).all(-1).mean()
+    print(f"end-to-end top-k rows identical: {same:.5f}")
+    assert same > 0.99
+
+
+# ---------------------------------------------------------------- full size
+def _sample(wl, x, first, last, every):
+    return workloads.sample_rows(x["cu_seqlens_q"], first=first, last=last, every=every)
+
+
+@pytest.mark.parametrize("wl,sample", [
+    (workloads.SINGLE_16K, (256, 512, 61)),
+    (workloads.VARLEN_8, (96, 128, 211)),
+    (workloads.LONG_128K, (64, 160, 1999)),
+    (workloads.SHORTQ_4x64K, None),
+], ids=lambda v: getattr(v, "name", "s"))
+def test_full_size_workloads(nsa, wl, sample):
+    """The benchmark's launch configuration at full size; sampled rows are
+    checked one by one against the oracle (all rows for the short-query case)."""
+    x, kc, vc, cuc = _prepare(wl, device="cuda")
+    rows = None if sample is None else workloads.sample_rows(x["cu_seqlens_q"], *sample)
+    q = x["q"]
+    res = nsa.nsa_compress_attention(q, kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp,
+                                     wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    torch.cuda.synchronize()
+    if rows is None:
+        qo = q.cpu()
+        ref = oracle.compress_attention(qo, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
+                                        x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    else:
+        qs = q.index_select(0, torch.from_numpy(rows).cuda()).cpu()
+        ref = oracle.compress_attention(qs, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
+                                        x["cu_seqlens_q"], cuc, x["cu_sel_kv"], rows=rows,
+                                        q_rows_only=True)
+    rep = check_attention(res, ref, wl.count)
+    print(wl.name, rep)
