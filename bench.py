@@ -1,0 +1,439 @@
+"""Benchmark of the NSA compressed-attention hot path on B200.
+
+One step = nsa_compress (raw K/V -> block tokens) + nsa_compress_attention
+(scores, softmax, PV, importance band, group sum, top-k) over one batch of
+seeded synthetic inputs, launched through the C ABI.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle as reference arm
+
+Prints one JSON line (rank 0).  `value` is algorithmic compressed-attention
+TFLOP/s over the whole step (compress + attention, device time, inputs
+resident in HBM), summed over ranks (weak scaling: every rank runs its own
+independent batch, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = ("compressed-attn TFLOP/s + query tok/s (fwd incl. top-k), % bf16 peak; "
+          "compress GB/s")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc", "nsa_attention.cu")
+CMP_SRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc", "nsa_compress.cu")
+
+
+# ------------------------------------------------------------------ work
+def visible_pairs(wl: workloads.Workload) -> int:
+    """sum over query rows of the number of visible compressed blocks."""
+    tot = 0
+    for S, sq in zip(wl.seqlens, wl.q_lengths()):
+        n_cmp = 0 if S < wl.l else (S - wl.l) // wl.d + 1
+        off = max(0, (n_cmp - 1) * wl.d + wl.l - sq) if n_cmp > 0 else 0
+        t = np.arange(sq, dtype=np.int64) + off
+        nv = np.where(t < wl.l - 1, 0, np.minimum(n_cmp, (t - wl.l + 1) // wl.d + 1))
+        tot += int(nv.sum())
+    return tot
+
+
+def attention_flops(wl) -> float:
+    return 2.0 * (wl.d1 + wl.d2) * wl.n1 * visible_pairs(wl)
+
+
+def compress_bytes(wl) -> float:
+    e = 2
+    tc = sum(0 if S < wl.l else (S - wl.l) // wl.d + 1 for S in wl.seqlens)
+    return float(wl.t2 * wl.n2 * (wl.d1 + wl.d2) * e + tc * wl.n2 * (wl.d1 + wl.d2) * e
+                 + wl.l * wl.n2 * e)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profile_traffic(kind):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source still matches the one the counters were taken on."""
+    p = os.path.join(ROOT, "profiles", f"{kind}_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = ATTN_SRC if kind == "attention" else CMP_SRC
+    if d.get("source_sha256_16") != src_hash(src):
+        return None
+    return d.get("bytes_per_launch_full_workload")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index):
+        self.samples, self.reasons = [], set()
+        self.stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop.set()
+            self.t.join()
+
+    def result(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import sparse_long_context_nsa_b200 as nsa
+    from sparse_long_context_nsa_b200 import _build
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workloads.WORKLOADS[args.workload].replace(seed=workloads.WORKLOADS[args.workload].seed + 1000 * rank)
+    x = wl.generate(device=str(dev))
+    q, k, v, w = x["q"], x["k"], x["v"], x["w"]
+    cu, cuq, cus = x["cu_seqlens"], x["cu_seqlens_q"], x["cu_sel_kv"]
+    cuc = nsa.nsa_compress_out_len(cu, wl.l, wl.d)
+    tc = int(cuc[-1])
+    t1 = q.shape[0]
+    kc = torch.empty(tc, wl.n2, wl.d1, dtype=q.dtype, device=dev)
+    vc = torch.empty(tc, wl.n2, wl.d2, dtype=q.dtype, device=dev)
+    outs = (torch.empty(t1, wl.n1, wl.d2, dtype=q.dtype, device=dev),
+            torch.empty(t1, wl.n2, wl.count, dtype=torch.int32, device=dev),
+            torch.empty(t1, wl.n1, 8, dtype=torch.float32, device=dev),
+            torch.empty(t1, wl.n1, 8, dtype=torch.float32, device=dev))
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, cuq, cuc, cus),
+        dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def step():
+        nsa.nsa_compress(k, v, w, wl.l, wl.d, cu, kcmp=kc, vcmp=vc)
+        nsa.nsa_compress_attention(q, kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count, cuq, cuc,
+                                   cus, out=outs, workspace=ws)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nsa.nsa_workspace_status(ws) != 0 or nsa.nsa_compress_status() != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_wall = time.perf_counter()
+        for i in range(K):
+            flush.zero_()                       # L2 flushed between timed steps
+            ev[i][0].record()
+            nsa.nsa_compress(k, v, w, wl.l, wl.d, cu, kcmp=kc, vcmp=vc)
+            ev[i][1].record()
+            nsa.nsa_compress_attention(q, kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count, cuq,
+                                       cuc, cus, out=outs, workspace=ws)
+            ev[i][2].record()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    st_ws = nsa.nsa_workspace_status(ws)
+    if st_ws != 0 or nsa.nsa_compress_status() != 0:
+        raise RuntimeError("device-side timeout in the timed region")
+    t_cmp = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_att = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms = float(np.sum(t_cmp) + np.sum(t_att))    # device time of the K steps
+    att_ms = float(np.mean(t_att))
+    cmp_ms = float(np.mean(t_cmp))
+
+    # ---------------- end to end: host buffers through the public API ----------------
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hw = (t.cpu().pin_memory() for t in (q, k, v, w))
+        ho = tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs)
+        ke = max(3, min(K, args.e2e_steps))
+
+        def e2e_step():
+            dq = hq.to(dev, non_blocking=True)
+            dk = hk.to(dev, non_blocking=True)
+            dv = hv.to(dev, non_blocking=True)
+            dw = hw.to(dev, non_blocking=True)
+            kc2, vc2 = nsa.nsa_compress(dk, dv, dw, wl.l, wl.d, cu)
+            res = nsa.nsa_compress_attention(dq, kc2, vc2, wl.scale, wl.n1, wl.l, wl.d, wl.lp,
+                                             wl.count, cuq, cuc, cus, workspace=ws)
+            for h_, d_ in zip(ho, res):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(ke):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / ke
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hw))
+        d2h = sum(t.numel() * t.element_size() for t in ho)
+        e2e = {"ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": ke}
+
+    return dict(wl=wl, K=K, step_ms=step_ms, att_ms=att_ms, cmp_ms=cmp_ms, t1=t1, wall=t_wall,
+                clocks=clk.result(), e2e=e2e,
+                launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
+
+
+def cpu_baseline(wl, budget_s=15.0, rows_per_seq=None):
+    """The fp64 oracle as it stands, timed on a bounded sample of the workload."""
+    import oracle
+    x = wl.generate(device="cpu")
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
+    # compress: a slice of the raw rows of the first sequence
+    S0 = min(wl.seqlens[0], 8192)
+    t0 = time.perf_counter()
+    oracle.compress(x["k"][:S0], x["w"], wl.l, wl.d, [S0], dtype=dt)
+    oracle.compress(x["v"][:S0], x["w"], wl.l, wl.d, [S0], dtype=dt)
+    t_cmp = time.perf_counter() - t0
+    kc, cuc = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    vc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    # attention: every `stride`-th query row, stride chosen for ~budget_s of CPU
+    cq = x["cu_seqlens_q"]
+    T1 = int(cq[-1])
+    full_pairs = visible_pairs(wl)
+    probe = np.arange(T1 - 1, max(T1 - 33, -1), -1, dtype=np.int64)
+    tp = time.perf_counter()
+    oracle.compress_attention(x["q"][probe], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+                              x["cu_sel_kv"], rows=probe, q_rows_only=True)
+    per_row = (time.perf_counter() - tp) / probe.size
+    nrows = int(max(16, min(T1, budget_s / max(per_row, 1e-6))))
+    stride = max(1, T1 // nrows)
+    rows = np.arange(0, T1, stride, dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.compress_attention(x["q"][rows], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+                              x["cu_sel_kv"], rows=rows, q_rows_only=True)
+    t_att = time.perf_counter() - t0
+    # visible pairs of the sampled rows (all heads)
+    pairs = 0
+    prev = 0
+    for b, end in enumerate(cq.tolist()):
+        sel = rows[(rows >= prev) & (rows < end)]
+        S = wl.seqlens[b]
+        n_cmp = 0 if S < wl.l else (S - wl.l) // wl.d + 1
+        off = max(0, (n_cmp - 1) * wl.d + wl.l - (end - prev)) if n_cmp else 0
+        t = sel - prev + off
+        pairs += int(np.where(t < wl.l - 1, 0, np.minimum(n_cmp, (t - wl.l + 1) // wl.d + 1)).sum())
+        prev = end
+    flops = 2.0 * (wl.d1 + wl.d2) * wl.n1 * pairs
+    tflops = flops / t_att / 1e12
+    cmp_bytes = S0 * wl.n2 * (wl.d1 + wl.d2) * 2 * 2
+    return {"value": tflops, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"attention: {rows.size} of {T1} query rows (every {stride}th), all heads, "
+                      f"{t_att:.1f} s; compress: first {S0} raw rows of K and V, {t_cmp:.2f} s",
+            "compress_gbs": cmp_bytes / t_cmp / 1e9, "seconds": t_att + t_cmp,
+            "full_attention_pairs": full_pairs}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle (the pages publish no code to run)."""
+    if rank != 0:
+        return
+    import oracle
+    wl = workloads.WORKLOADS[args.workload]
+    x = wl.generate(device="cpu")
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
+    kc, cuc = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    vc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    cq = x["cu_seqlens_q"]
+    T1 = int(cq[-1])
+    rows = np.linspace(0, T1 - 1, num=min(T1, args.ref_rows), dtype=np.int64)
+    qs = x["q"][rows]
+
+    def step():
+        oracle.compress_attention(qs, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+                                  x["cu_sel_kv"], rows=rows, q_rows_only=True)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt_s = (time.perf_counter() - t0) / args.steps
+    # algorithmic FLOPs of the sampled rows
+    S = wl.seqlens
+    pairs, prev = 0, 0
+    for b, end in enumerate(cq.tolist()):
+        sel = rows[(rows >= prev) & (rows < end)]
+        n_cmp = 0 if S[b] < wl.l else (S[b] - wl.l) // wl.d + 1
+        off = max(0, (n_cmp - 1) * wl.d + wl.l - (end - prev)) if n_cmp else 0
+        t = sel - prev + off
+        pairs += int(np.where(t < wl.l - 1, 0, np.minimum(n_cmp, (t - wl.l + 1) // wl.d + 1)).sum())
+        prev = end
+    flops = 2.0 * (wl.d1 + wl.d2) * wl.n1 * pairs
+    val = flops / dt_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "sampled_rows": int(rows.size)},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"{rows.size} evenly spaced query rows of {T1}, all heads, "
+                                       "compressed K/V precomputed"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=workloads.SINGLE_16K.name, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=96)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    r = run_ours(args, rank, world, local_rank)
+    wl = r["wl"]
+    # max over ranks of the device time of the timed steps
+    t = torch.tensor([r["step_ms"], r["att_ms"], r["cmp_ms"]], dtype=torch.float64,
+                     device=torch.device("cuda", local_rank))
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    step_total_ms, att_ms, cmp_ms = t.tolist()
+    K = r["K"]
+    ms_per_step = step_total_ms / K
+    flops = attention_flops(wl)
+    cbytes = compress_bytes(wl)
+    peaks, peak_src = load_peaks()
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    att_tflops = flops / (att_ms * 1e-3) / 1e12
+    cmp_gbs = cbytes / (cmp_ms * 1e-3) / 1e9
+    e2e = None
+    if r["e2e"] is not None:
+        e2e = {"value": world * flops / (r["e2e"]["ms_per_step"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
+               "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
+               "ms_per_step": r["e2e"]["ms_per_step"]}
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_baseline(wl, budget_s=args.cpu_budget)
+        peak_t = peaks["bf16_tflops"]
+        traffic = profile_traffic("attention")
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "fp16", "data": "synthetic",
+            "config": {"workload": wl.name, "seqlens": list(wl.seqlens)[:8], "n1": wl.n1, "n2": wl.n2,
+                       "d1": wl.d1, "d2": wl.d2, "l": wl.l, "d": wl.d, "lp": wl.lp, "count": wl.count,
+                       "l2": "flushed (256 MB write) before every timed step",
+                       "parallelism": f"independent batch per GPU x{world}"},
+            "query_tok_s": world * r["t1"] / (ms_per_step * 1e-3),
+            "attention_kernel": {"ms": att_ms, "tflops": att_tflops,
+                                 "pct_of_bf16_peak": 100.0 * att_tflops / peak_t,
+                                 "query_tok_s": r["t1"] / (att_ms * 1e-3)},
+            "compress_kernel": {"ms": cmp_ms, "gbs": cmp_gbs,
+                                "pct_of_hbm": 100.0 * cmp_gbs / peaks["hbm_gbs"],
+                                "bytes": cbytes},
+            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": att_tflops / peak_t, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "flops_per_launch": flops},
+            "roofline_compress": {"bound": "hbm", "achieved": cmp_gbs, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": cmp_gbs / peaks["hbm_gbs"],
+                                  "traffic": profile_traffic("compress"),
+                                  "peak_source": f"{peak_src} hbm_gbs"},
+            "clocks": r["clocks"],
+            "e2e": e2e,
+            "gpu_launches": r["launches_per_step"] * K,
+            "cpu_baseline": cpu,
+            "wall_s_timed_region": r["wall"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

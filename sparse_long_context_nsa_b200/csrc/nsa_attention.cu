@@ -291,6 +291,12 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ++pcnt;
                 }
                 if (!ok) break;
+                // O_FULL of this tile may only complete after the epilogue of the
+                // previous tile has released O: otherwise a tile without PV work
+                // could advance O_FULL by two phases before its consumer looks
+                if (t.nkv == 0)
+                    ok = mbar_wait(bar(B_O_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 7);
+                if (!ok) break;
                 umma_commit(bar(B_O_FULL));
                 umma_commit(bar(B_Q_EMPTY));
             }

@@ -38,9 +38,7 @@ def _run_both(nsa, wl, rows=None, device="cpu"):
     x, kc, vc, cuc = _prepare(wl, device)
     q = x["q"]
     qd = q if q.is_cuda else q.cuda()
-    res = nsa.nsa_compress_attention(qd, kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp,
-                                     wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
-    torch.cuda.synchronize()
+    res = _attn(nsa, qd, kc.cuda(), vc.cuda(), wl, x, cuc)
     if rows is None:
         qo = q.cpu()
         ref = oracle.compress_attention(qo, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
@@ -52,6 +50,17 @@ def _run_both(nsa, wl, rows=None, device="cpu"):
                                         x["cu_seqlens_q"], cuc, x["cu_sel_kv"], rows=rows,
                                         q_rows_only=True)
     return res, ref, x, (kc, vc, cuc)
+
+
+def _attn(nsa, q, kc, vc, wl, x, cuc):
+    """Runs the CUDA path and asserts that no device-side wait gave up."""
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
+        x["cu_sel_kv"]), dtype=torch.uint8, device=q.device)
+    res = nsa.nsa_compress_attention(q, kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count,
+                                     x["cu_seqlens_q"], cuc, x["cu_sel_kv"], workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0, hex(int(ws[:4].view(torch.int32).item()))
+    return res
 
 
 def _wl(seqs, n1, n2, d1, d2, l, d, lp, count, dtype="bf16", seed=7, q_last=None, std=1.0):
@@ -147,9 +156,9 @@ def test_end_to_end_gpu_compress_then_attention(nsa):
     wl = _wl([4000, 1234], 32, 4, 128, 128, 32, 16, 64, 16)
     x = wl.generate()
     kc, vc = nsa.nsa_compress(x["k"].cuda(), x["v"].cuda(), x["w"].cuda(), wl.l, wl.d, x["cu_seqlens"])
+    assert nsa.nsa_compress_status() == 0
     cuc = nsa.nsa_compress_out_len(x["cu_seqlens"], wl.l, wl.d)
-    res = nsa.nsa_compress_attention(x["q"].cuda(), kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count,
-                                     x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    res = _attn(nsa, x["q"].cuda(), kc, vc, wl, x, cuc)
     okc, _ = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=oracle.BF16)
     ovc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=oracle.BF16)
     ref = oracle.compress_attention(x["q"], okc, ovc, wl.scale, wl.l, wl.d, wl.lp, wl.count,
@@ -178,9 +187,7 @@ def test_full_size_workloads(nsa, wl, sample):
     x, kc, vc, cuc = _prepare(wl, device="cuda")
     rows = None if sample is None else workloads.sample_rows(x["cu_seqlens_q"], *sample)
     q = x["q"]
-    res = nsa.nsa_compress_attention(q, kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp,
-                                     wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
-    torch.cuda.synchronize()
+    res = _attn(nsa, q, kc.cuda(), vc.cuda(), wl, x, cuc)
     if rows is None:
         qo = q.cpu()
         ref = oracle.compress_attention(qo, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count,

@@ -57,6 +57,7 @@ def test_compress_parity(nsa, case, dtype):
 def test_compress_k_only(nsa):
     k, v, w, cu = _case([700, 300], 2, 64, 64, 32, 16)
     kc, vc = nsa.nsa_compress(k.cuda(), None, w.cuda(), 32, 16, cu)
+    assert nsa.nsa_compress_status() == 0
     assert vc is None
     check_compress(kc, k, w, 32, 16, cu, oracle.BF16)
 
@@ -86,7 +87,7 @@ def test_compress_full_size_workloads(nsa, wl):
     """The compress launch of the benchmark at full size, every output checked."""
     x = wl.generate(device="cuda")
     kc, vc = nsa.nsa_compress(x["k"], x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"])
-    torch.cuda.synchronize()
+    assert nsa.nsa_compress_status() == 0
     dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
     k, v, w = x["k"].cpu(), x["v"].cpu(), x["w"].cpu()
     check_compress(kc, k, w, wl.l, wl.d, x["cu_seqlens"], dt)
