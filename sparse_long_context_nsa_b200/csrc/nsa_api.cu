@@ -276,7 +276,8 @@ nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, in
 
     // sizes of the per-CTA ring and the output run of one CTA
     const int rowbytes = (int)(rowelems * 2);
-    int rs = std::max(1, 16384 / rowbytes);
+    // rows per bulk copy: about 16 KB, a multiple of 4 (the kernel steps 4 rows at a time)
+    int rs = std::max(4, (16384 / rowbytes) & ~3);
     const int stage_bytes = rs * rowbytes;
     const int wbytes = ((l * n2 * 4) + 127) & ~127;
     const size_t smem = (size_t)wbytes + 128 + (size_t)kCompressStages * stage_bytes;

@@ -150,7 +150,6 @@ nsa_compress_kernel(const CompressParams p) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
 
-    int64_t rel = rel0;                              // raw row within the sequence
     int q = i0;                                      // rel / d
     int rin = 0;                                     // rel % d
     int next_issue = min(kCompressStages, nstage);   // stages handed to the copy engine
@@ -164,22 +163,29 @@ nsa_compress_kernel(const CompressParams p) {
         const int rows = min(rs, nrows - s * rs);
         const uint8_t* base = stages + slot * stage_bytes;
         if (active && got) {
-            for (int r = 0; r < rows; ++r) {
-                const uint4 u = *reinterpret_cast<const uint4*>(base + r * rowbytes + cv * 16);
-                float x[8];
-                cvt8<T>(u, x);
+            // four rows per step: their loads are independent (rows and d are
+            // multiples of 4, so a window group never ends inside a step)
+            for (int r = 0; r < rows; r += 4) {
+                uint4 u[4];
 #pragma unroll
-                for (int k = 0; k < BMAX; ++k) {
-                    const int j = k * d + rin;                // position inside window q-k
-                    if (k < nb && j < l) {
-                        const float wv = wsm[j * p.n2 + head];
+                for (int rr = 0; rr < 4; ++rr)
+                    u[rr] = *reinterpret_cast<const uint4*>(base + (r + rr) * rowbytes + cv * 16);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wv, x[e], acc[k][e]);
+                for (int rr = 0; rr < 4; ++rr) {
+                    float x[8];
+                    cvt8<T>(u[rr], x);
+#pragma unroll
+                    for (int k = 0; k < BMAX; ++k) {
+                        const int j = k * d + rin + rr;       // position inside window q-k
+                        if (k < nb && j < l) {
+                            const float wv = wsm[j * p.n2 + head];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wv, x[e], acc[k][e]);
+                        }
                     }
                 }
-                ++rel;
-                ++rin;
-                const bool last_row = (s == nstage - 1) && (r == rows - 1);
+                rin += 4;
+                const bool last_row = (s == nstage - 1) && (r + 4 == rows);
                 if (rin == d || last_row) {
                     // window q-(nb-1) has seen its last row: store it, shift slots
                     const int i = q - (nb - 1);
