@@ -82,9 +82,9 @@ struct AttnPlan {
     int score_cap = 1;
     int grid = 0;
     bool score_in_smem = true;
-    int nslot = 0;
-    int off_q = 0, off_ring = 0, slot_bytes = 0, off_p = 0, off_stage = 0, off_score = 0, off_bar = 0,
-        smem_bytes = 0;
+    int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_p = 0;
+    int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_stage = 0, stage_entry_bytes = 0,
+        off_score = 0, off_bar = 0, smem_bytes = 0;
     size_t ws_tiles = 0, ws_score = 0, ws_total = 0;
 };
 
@@ -179,35 +179,48 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
                          [](const AttnTile& x, const AttnTile& y) { return x.nkv > y.nkv; });
     }
 
-    // shared memory layout
+    // tensor memory: S buffers (128 columns each), O (D2 columns), P (NKV/2
+    // columns of packed pairs); two S buffers when they fit next to O and P
+    const int d2c = (d2 + 31) & ~31;
+    pl.nsbuf = (256 + d2c + 64 <= 512) ? 2 : 1;
+    pl.tm_o = pl.nsbuf * 128;
+    pl.tm_p = pl.tm_o + d2c;
+    if (pl.tm_p + NKV / 2 > 512) return NSA_ERR_UNSUPPORTED;
+
+    // shared memory: Q buffers, K/V ring, band staging (2 entries), score buffer
     const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
     const int NJ = NKV / pl.a;
-    const int CHK = std::min(NJ, kBandChunk);
-    pl.off_q = 0;
-    pl.off_ring = nqc * 16384;
+    const int ENT = std::min(NJ, kEntryMax);
+    pl.q_bytes = nqc * 16384;
     pl.slot_bytes = std::max(nqc, nvc) * NKV * 128;
-    const int p_bytes = ((NKV + 63) / 64) * 16384;
-    const int stage_bytes = kRows * (CHK + 1) * 4;
+    pl.stage_entry_bytes = kRows * (ENT + 4) * 4;
     const int score_bytes = pl.TT * pl.score_cap * 4;
-    const int bar_bytes = 8 * 32 + 64;
-    auto layout = [&](int nslot, bool in_smem) {
-        int off = pl.off_ring + nslot * pl.slot_bytes;
-        pl.off_p = off;
-        off += p_bytes;
+    const int bar_bytes = 320;
+    auto layout = [&](int nq, int ns, bool in_smem) {
+        int off = 0;
+        pl.off_q = off;
+        off += nq * pl.q_bytes;
+        pl.off_ring = off;
+        off += ns * pl.slot_bytes;
         pl.off_stage = off;
-        off += (stage_bytes + 127) & ~127;
+        off += 2 * pl.stage_entry_bytes;
         pl.off_score = off;
         if (in_smem) off += (score_bytes + 127) & ~127;
         pl.off_bar = off;
         off += bar_bytes;
         pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
-        pl.nslot = nslot;
+        pl.nqbuf = nq;
+        pl.nslot = ns;
         pl.score_in_smem = in_smem;
         return pl.smem_bytes <= kSmemLimit;
     };
+    // preference: deeper K/V ring, then a second Q buffer, then on-chip scores
+    static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}, {2, 2}, {1, 2}};
     bool fits = false;
-    for (int ns = 4; ns >= 2 && !fits; --ns) fits = layout(ns, true);
-    for (int ns = 4; ns >= 2 && !fits; --ns) fits = layout(ns, false);
+    for (const auto& o : kOrder) {
+        if ((fits = layout(o[0], o[1], true))) break;
+        if ((fits = layout(o[0], o[1], false))) break;
+    }
     if (!fits) return NSA_ERR_UNSUPPORTED;
 
     pl.ws_tiles = (size_t)ntiles * sizeof(AttnTile);
@@ -430,11 +443,16 @@ nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void*
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.nkv_cols = pl.nkv_cols;
     p.nslot = pl.nslot;
+    p.nqbuf = pl.nqbuf;
+    p.nsbuf = pl.nsbuf;
+    p.tm_o = pl.tm_o;
+    p.tm_p = pl.tm_p;
     p.off_q = pl.off_q;
+    p.q_bytes = pl.q_bytes;
     p.off_ring = pl.off_ring;
     p.slot_bytes = pl.slot_bytes;
-    p.off_p = pl.off_p;
     p.off_stage = pl.off_stage;
+    p.stage_entry_bytes = pl.stage_entry_bytes;
     p.off_score = pl.off_score;
     p.off_bar = pl.off_bar;
     p.smem_bytes = pl.smem_bytes;

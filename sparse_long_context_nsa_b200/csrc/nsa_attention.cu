@@ -9,26 +9,31 @@
 //   7  top-k of P_slc' over the causal candidates of the query
 //
 // One M-tile = 128 rows = (128/G consecutive tokens) x (the G query heads of
-// one KV group), so every row of the tile shares one K/V head and the group
-// sum of step 5 is a sum over neighbouring rows.  Per tile, two passes over
-// the compressed keys (the importance scores sum *normalised* probabilities
-// over heads, and a head's normaliser is only known at the end of its row):
-//   pass A  S = Q K^T on the tensor cores (tcgen05.mma, fp32 in TMEM),
-//           online max / sum in registers -> exact m and L per row.
-//   pass B  S = Q K^T again, P = exp(S - m) / L in fp32 registers, bf16/fp16 P
-//           -> shared memory -> O += P V on the tensor cores; from the fp32 P
-//           the banded importance sum (step 4) and the group sum (step 5) go
-//           to a per-token score buffer that never leaves the SM.
-//   epilogue O (TMEM) -> out; stats; radix-select top-k per token (step 7).
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues the MMAs
-// and owns the tensor memory, warps 2-5 (one thread per tile row, matching
-// the four 32-lane quadrants of TMEM) run softmax, band sums and epilogue.
-// Q, K and V are staged by TMA with 128-byte swizzle; K/V share one ring.
-// Every mbarrier wait is bounded; a timeout sets the workspace error word.
+// one KV group): every row of a tile shares one K/V head, and the group sum of
+// step 5 is a sum over neighbouring rows.  Two passes over the compressed
+// keys per tile, because step 5 adds *normalised* probabilities of different
+// heads and a head's normaliser is only known at the end of its row:
+//   pass A  S = Q K^T (tcgen05.mma, operands in shared memory, fp32 in tensor
+//           memory); online max / sum in registers -> exact m and L per row;
+//           softmax_max / softmax_sum are written here.
+//   pass B  S = Q K^T again; P = 2^(s*scale*log2e - m - log2 L) in fp32
+//           registers; P (storage dtype) -> tensor memory -> O += P V with the
+//           A operand read from tensor memory; from the fp32 P the banded sum
+//           of step 4 goes to a shared-memory staging ring.
+// Epilogue warps, concurrently with the next tile's passes: sum the staged
+// band values over the G rows of each token into a per-token score buffer
+// (step 5), read O out of tensor memory, and pick the top-k (step 7).
+// Warp roles (384 threads, three warpgroups): warps 0-3 softmax (warp w owns
+// TMEM lanes 32w..32w+31 = tile rows), warps 4-7 epilogue (same lane
+// quadrants), warp 8 TMA producer, warp 9 MMA issuer (and tensor-memory
+// owner), warps 10-11 idle.  Registers move from the third and second
+// warpgroups to the softmax warpgroup with setmaxnreg.
+// Q (double-buffered), K and V are staged by TMA with 128-byte swizzle; K and
+// V share one ring of slots.  Every mbarrier wait is bounded; a timeout sets
+// the workspace error word and every role drains without hanging.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
-#include <cfloat>
 #include <type_traits>
 
 #include "nsa_internal.h"
@@ -38,7 +43,8 @@ namespace nsa {
 
 __host__ __device__ constexpr int kv_cols_for(int a) {
     // largest multiple of lcm(16, a) not above 128: every KV tile then holds a
-    // whole number of importance anchors (anchor of block j = a*j)
+    // whole number of importance anchors (the anchor of selection block j is
+    // compressed block a*j)
     return (a == 1 || a == 2 || a == 4 || a == 8) ? 128
            : (a == 3 || a == 6)                   ? 96
            : (a == 5)                             ? 80
@@ -48,8 +54,10 @@ __host__ __device__ constexpr int kv_cols_for(int a) {
 int attention_kv_cols(int a) { return kv_cols_for(a); }
 
 enum BarId {
-    B_Q_FULL = 0,
-    B_Q_EMPTY,
+    B_Q_FULL0 = 0,
+    B_Q_FULL1,
+    B_Q_EMPTY0,
+    B_Q_EMPTY1,
     B_S_FULL0,
     B_S_FULL1,
     B_S_EMPTY0,
@@ -58,8 +66,12 @@ enum BarId {
     B_P_EMPTY,
     B_O_FULL,
     B_O_EMPTY,
+    B_STG_FULL0,
+    B_STG_FULL1,
+    B_STG_EMPTY0,
+    B_STG_EMPTY1,
     B_MMA_DONE,
-    B_SLOT_FULL0,            // + slot
+    B_SLOT_FULL0,                     // + slot
     B_SLOT_EMPTY0 = B_SLOT_FULL0 + 8,
     B_COUNT = B_SLOT_EMPTY0 + 8
 };
@@ -87,7 +99,8 @@ __device__ __forceinline__ int nvis_of(int t, int l, int d, int n_cmp) {
 // j < ncand; scores for j >= jcov are 0 (no visible block reaches them).
 // Exact k-th largest key by a bitwise search over the fp32 bit patterns
 // (scores are >= 0, so the bit patterns order like the values), then an
-// ordered ballot scan keeps every key above it plus the earliest ties.
+// ordered ballot scan keeps every key above it plus the earliest ties, which
+// also lists the indices in ascending order.
 __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, int count,
                                           int32_t* dst, int lane) {
     const int k = min(count, ncand);
@@ -95,26 +108,47 @@ __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, 
         for (int j = lane; j < count; j += 32) dst[j] = (j < ncand) ? j : -1;
         return;
     }
-    auto key = [&](int j) -> uint32_t { return j < jcov ? __float_as_uint(sc[j]) : 0u; };
+    const int lim = min(ncand, jcov);          // keys at j >= lim are 0
     uint32_t thr = 0;
+    if (ncand <= 32 * 32) {
+        // keys in registers: key[i] belongs to j = lane + 32 i
+        uint32_t key[32];
+        const int nreg = (ncand + 31) >> 5;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int j = lane + 32 * i;
+            key[i] = (i < nreg && j < lim) ? __float_as_uint(sc[j]) : 0u;
+        }
 #pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t trial = thr | (1u << bit);
-        int c = 0;
-        for (int j = lane; j < ncand; j += 32) c += key(j) >= trial ? 1 : 0;
-        c = __reduce_add_sync(0xffffffffu, c);
-        if (c >= k) thr = trial;
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t trial = thr | (1u << bit);
+            int c = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (i < nreg) c += key[i] >= trial ? 1 : 0;
+            c = __reduce_add_sync(0xffffffffu, c);
+            if (c >= k) thr = trial;
+        }
+    } else {
+#pragma unroll 1
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t trial = thr | (1u << bit);
+            int c = 0;
+            for (int j = lane; j < lim; j += 32) c += __float_as_uint(sc[j]) >= trial ? 1 : 0;
+            c = __reduce_add_sync(0xffffffffu, c);
+            if (c >= k) thr = trial;
+        }
     }
     int ngt = 0;
-    for (int j = lane; j < ncand; j += 32) ngt += key(j) > thr ? 1 : 0;
+    for (int j = lane; j < lim; j += 32) ngt += __float_as_uint(sc[j]) > thr ? 1 : 0;
     ngt = __reduce_add_sync(0xffffffffu, ngt);
     const int need_eq = k - ngt;
     const uint32_t lt_mask = (1u << lane) - 1u;
     int eq_seen = 0, written = 0;
-    for (int base = 0; base < ncand; base += 32) {
+    for (int base = 0; base < ncand && written < k; base += 32) {
         const int j = base + lane;
         const bool in = j < ncand;
-        const uint32_t kv = in ? key(j) : 0u;
+        const uint32_t kv = (j < lim) ? __float_as_uint(sc[j]) : 0u;
         const bool gt = in && kv > thr;
         const bool eq = in && kv == thr;
         const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
@@ -135,10 +169,11 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     constexpr int NJ = NKV / A;                    // importance anchors per KV tile
     constexpr int NTAP = 2 * A - 1;                // band taps u = 0 .. 2A-2 (b <= a)
     constexpr int NCARRY = (2 * A - 2) > 0 ? (2 * A - 2) : 1;
-    constexpr int CHK = NJ < kBandChunk ? NJ : kBandChunk;
-    constexpr int STG = CHK + 1;                   // staging row stride (odd: no bank conflicts)
-    constexpr bool kBF16 = sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value;
-    static_assert(NJ % CHK == 0, "anchor chunking");
+    constexpr int ENT = NJ < kEntryMax ? NJ : kEntryMax;   // anchors per staging entry
+    constexpr int NENT = NJ / ENT;                 // staging entries per KV tile
+    constexpr int STR = ENT + 4;                   // staging row stride in floats
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    static_assert(NJ % ENT == 0 && ENT % 4 == 0, "anchor chunking");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -153,8 +188,10 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int TT = p.tok_per_tile;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(B_Q_FULL), 1);
-        mbar_init(bar(B_Q_EMPTY), 1);
+        mbar_init(bar(B_Q_FULL0), 1);
+        mbar_init(bar(B_Q_FULL1), 1);
+        mbar_init(bar(B_Q_EMPTY0), 1);
+        mbar_init(bar(B_Q_EMPTY1), 1);
         mbar_init(bar(B_S_FULL0), 1);
         mbar_init(bar(B_S_FULL1), 1);
         mbar_init(bar(B_S_EMPTY0), 4);
@@ -163,6 +200,10 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(bar(B_P_EMPTY), 1);
         mbar_init(bar(B_O_FULL), 1);
         mbar_init(bar(B_O_EMPTY), 4);
+        mbar_init(bar(B_STG_FULL0), 4);
+        mbar_init(bar(B_STG_FULL1), 4);
+        mbar_init(bar(B_STG_EMPTY0), 4);
+        mbar_init(bar(B_STG_EMPTY1), 4);
         mbar_init(bar(B_MMA_DONE), 1);
         for (int s = 0; s < 8; ++s) {
             mbar_init(bar(B_SLOT_FULL0 + s), 1);
@@ -175,7 +216,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
-    if (warp == 1) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -183,16 +224,19 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_o = tmem + 256;
+    const uint32_t tmem_o = tmem + p.tm_o;
+    const uint32_t tmem_p = tmem + p.tm_p;
 
-    const uint32_t q_addr = smem_u32(smem + p.off_q);
+    const uint32_t q_addr0 = smem_u32(smem + p.off_q);
     const uint32_t ring_addr = smem_u32(smem + p.off_ring);
-    const uint32_t p_addr = smem_u32(smem + p.off_p);
     const int nslot = p.nslot;
+    const int nqbuf = p.nqbuf;
+    const int nsbuf = p.nsbuf;
     const int nqc = (p.d1 + 63) / 64;    // 64-element chunks of a Q/K row
     const int nvc = (p.d2 + 63) / 64;    // 64-element chunks of a V row
 
-    if (warp == 0) {
+    if (warp >= 8) setmaxnreg_dec<kRegsCtl>();
+    if (warp == 8) {
         // ============================ TMA producer ============================
         if (lane == 0) {
             uint32_t item = 0;
@@ -216,11 +260,14 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             };
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
                 const AttnTile t = p.tiles[tile];
-                ok = mbar_wait(bar(B_Q_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 3);
+                const int qb = tcount % nqbuf;
+                const uint32_t qph = (tcount / nqbuf) & 1;
+                ok = mbar_wait(bar(B_Q_EMPTY0 + qb), qph ^ 1, abort_flag, p.err, kErrTimeoutBase + 3);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar(B_Q_FULL), q_bytes);
+                mbar_arrive_expect_tx(bar(B_Q_FULL0 + qb), q_bytes);
+                const uint32_t qdst = q_addr0 + qb * p.q_bytes;
                 for (int c = 0; c < nqc; ++c)
-                    tma_load_3d(q_addr + c * 16384, &tm_q, c * 64, t.group * G, t.q_row0, bar(B_Q_FULL));
+                    tma_load_3d(qdst + c * 16384, &tm_q, c * 64, t.group * G, t.q_row0, bar(B_Q_FULL0 + qb));
                 for (int i = 0; i < t.nkv && ok; ++i) load_kv(false, t.group, t.cmp_row0 + i * NKV);
                 if (t.nkv > 0 && ok) load_kv(false, t.group, t.cmp_row0);
                 for (int i = 0; i < t.nkv && ok; ++i) {
@@ -229,7 +276,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 9) {
         // ============================ MMA issuer =============================
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, NKV, false, false);
@@ -239,9 +286,10 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             uint32_t item = 0, scnt = 0, pcnt = 0;
             int tcount = 0;
             bool ok = true;
+            uint32_t q_addr = q_addr0;
             auto issue_s = [&]() {
-                const int sb = scnt & 1;
-                ok = ok && mbar_wait(bar(B_S_EMPTY0 + sb), ((scnt >> 1) & 1) ^ 1, abort_flag, p.err,
+                const int sb = scnt % nsbuf;
+                ok = ok && mbar_wait(bar(B_S_EMPTY0 + sb), ((scnt / nsbuf) & 1) ^ 1, abort_flag, p.err,
                                      kErrTimeoutBase + 4);
                 const int slot = item % nslot;
                 ok = ok && mbar_wait(bar(B_SLOT_FULL0 + slot), (item / nslot) & 1, abort_flag, p.err,
@@ -262,9 +310,11 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             };
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
                 const AttnTile t = p.tiles[tile];
-                ok = mbar_wait(bar(B_Q_FULL), tcount & 1, abort_flag, p.err, kErrTimeoutBase + 6);
+                const int qb = tcount % nqbuf;
+                ok = mbar_wait(bar(B_Q_FULL0 + qb), (tcount / nqbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 6);
                 if (!ok) break;
                 tc_fence_after();
+                q_addr = q_addr0 + qb * p.q_bytes;
                 for (int i = 0; i < t.nkv && ok; ++i) issue_s();          // pass A
                 if (t.nkv > 0 && ok) issue_s();                          // pass B, S_0
                 for (int i = 0; i < t.nkv && ok; ++i) {
@@ -281,9 +331,8 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const uint32_t vbase = ring_addr + slot * p.slot_bytes;
 #pragma unroll
                     for (int ks = 0; ks < nks_pv; ++ks) {
-                        const uint64_t ad = sdesc_sw128(p_addr + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                         const uint64_t bd = sdesc_sw128(vbase + ks * 2048, NKV * 128, 1024);
-                        umma_ss(tmem_o, ad, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+                        umma_ts(tmem_o, tmem_p + ks * 8, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(bar(B_P_EMPTY));
                     umma_commit(bar(B_SLOT_EMPTY0 + slot));
@@ -298,62 +347,69 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ok = mbar_wait(bar(B_O_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 7);
                 if (!ok) break;
                 umma_commit(bar(B_O_FULL));
-                umma_commit(bar(B_Q_EMPTY));
+                umma_commit(bar(B_Q_EMPTY0 + qb));
             }
             // every MMA issued so far has retired before the tensor memory is freed
             umma_commit(bar(B_MMA_DONE));
             mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
         }
-    } else {
-        // ==================== softmax / band / epilogue (128 thr) ====================
-        const int wq = warp & 3;                  // TMEM lane quadrant of this warp
-        const int row = wq * 32 + lane;           // tile row = TMEM lane
-        const int st = threadIdx.x - 64;          // 0..127, for row-independent work
-        const int sw = warp - 2;                  // 0..3
-        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    } else if (warp < 4) {
+        // ===================== softmax + band values (128 thr) =====================
+        setmaxnreg_inc<kRegsSoftmax>();
+        const int row = warp * 32 + lane;          // tile row = TMEM lane
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const int a = p.a, bb = p.b;
+        const float c2 = p.scale_log2;
         float wband[NTAP];
 #pragma unroll
         for (int u = 0; u < NTAP; ++u) {
-            // multiplicity of m + n = u with m < a, n < b (step 4 double sum)
+            // multiplicity of m + n = u with m < a, n < b (the double sum of step 4)
             const int c = min(min(u, a - 1), min(bb - 1, a + bb - 2 - u)) + 1;
             wband[u] = (u <= a + bb - 2) ? (float)c : 0.f;
         }
         float* stage = reinterpret_cast<float*>(smem + p.off_stage);
-        float* score = p.score_in_smem ? reinterpret_cast<float*>(smem + p.off_score)
-                                       : p.score_gmem + (size_t)blockIdx.x * TT * p.score_cap;
-        const int cap = p.score_cap;
-        uint32_t scnt = 0, pcnt = 0;
-        int tcount = 0;
+        uint32_t scnt = 0, pcnt = 0, stg = 0;
         const int h = row % G;
         const int tok = row / G;
 
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+        auto load_s = [&](float (&s)[NKV]) {
+            const int sb = scnt % nsbuf;
+            mbar_wait(bar(B_S_FULL0 + sb), (scnt / nsbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
+            tc_fence_after();
+            const uint32_t ta = tmem + lane_off + sb * 128;
+#pragma unroll
+            for (int c = 0; c < NKV / 16; ++c) {
+                uint32_t r[16];
+                tmem_ld16(ta + c * 16, r);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) s[c * 16 + e] = __uint_as_float(r[e]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_S_EMPTY0 + sb));
+            ++scnt;
+        };
+        // one staging entry: ENT anchors of this row -> shared memory
+        auto put_entry = [&](const float* v) {
+            const int slot = stg & 1;
+            mbar_wait(bar(B_STG_EMPTY0 + slot), ((stg >> 1) & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 13);
+            float4* dst = reinterpret_cast<float4*>(stage + (size_t)slot * (p.stage_entry_bytes / 4) + row * STR);
+#pragma unroll
+            for (int q4 = 0; q4 < ENT / 4; ++q4)
+                dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_STG_FULL0 + slot));
+            ++stg;
+        };
+
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             const AttnTile t = p.tiles[tile];
             const bool valid = (row < TT * G) && (tok < t.ntok);
             const int tpos = t.t0 + tok;
             const int nvis = valid ? nvis_of(tpos, p.l, p.d, t.n_cmp) : 0;
 
-            auto load_s = [&](float (&s)[NKV]) {
-                const int sb = scnt & 1;
-                mbar_wait(bar(B_S_FULL0 + sb), (scnt >> 1) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
-                tc_fence_after();
-                const uint32_t ta = tmem + lane_off + sb * 128;
-#pragma unroll
-                for (int c = 0; c < NKV / 16; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(ta + c * 16, r);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) s[c * 16 + e] = __uint_as_float(r[e]);
-                }
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_S_EMPTY0 + sb));
-                ++scnt;
-            };
-
-            // ---------------- pass A: exact row max and sum ----------------
+            // ---------------- pass A: exact row max and sum (log2 domain) ----------------
             float m = -INFINITY, L = 0.f;
             for (int i = 0; i < t.nkv; ++i) {
                 float s[NKV];
@@ -362,7 +418,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 float mx = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < NKV; ++c) {
-                    s[c] = (c < lim) ? s[c] * p.scale_log2 : -INFINITY;
+                    s[c] = (c < lim) ? s[c] * c2 : -INFINITY;
                     mx = fmaxf(mx, s[c]);
                 }
                 const float mn = fmaxf(m, mx);
@@ -373,64 +429,62 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 L = L * ex2(m - mref) + sum;
                 m = mn;
             }
+            if (valid) {
+                const size_t si = ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * 8;
+                const float mo = (m == -INFINITY) ? -INFINITY : m * 0.69314718055994530942f;
+                const float4 mv = make_float4(mo, mo, mo, mo);
+                const float4 lv = make_float4(L, L, L, L);
+                reinterpret_cast<float4*>(p.smax + si)[0] = mv;
+                reinterpret_cast<float4*>(p.smax + si)[1] = mv;
+                reinterpret_cast<float4*>(p.ssum + si)[0] = lv;
+                reinterpret_cast<float4*>(p.ssum + si)[1] = lv;
+            }
 
-            // ------------- pass B: P, PV, importance band, group sum -------------
-            const float invL = (L > 0.f) ? 1.f / L : 0.f;
-            const float mref = (m == -INFINITY) ? 0.f : m;
+            // ------------- pass B: P -> TMEM, band values -> staging -------------
+            // P = 2^(s*c2 - m - log2 L): normalised in the exponent
+            const float mb = (L > 0.f) ? m + lg2(L) : INFINITY;
             float carry[NCARRY];
 #pragma unroll
             for (int k = 0; k < NCARRY; ++k) carry[k] = 0.f;
-
-            // stage CHK anchors per round, reduce over the G rows of each token
-            auto band_round = [&](const float* vals, int jfirst) {
-#pragma unroll
-                for (int qq = 0; qq < CHK; ++qq) stage[row * STG + qq] = vals[qq];
-                named_bar_sync(1, 128);
-                for (int pi = st; pi < t.ntok * CHK; pi += 128) {
-                    const int tau = pi / CHK, qq = pi - tau * CHK;
-                    const float* src = stage + (tau * G) * STG + qq;
-                    float acc = 0.f;
-                    for (int hh = 0; hh < G; ++hh) acc += src[hh * STG];
-                    const int j = jfirst + qq;
-                    if (j < cap) score[tau * cap + j] = acc;
-                }
-                named_bar_sync(1, 128);
-            };
-
             for (int i = 0; i < t.nkv; ++i) {
                 float s[NKV];
                 load_s(s);
                 const int lim = nvis - i * NKV;
 #pragma unroll
-                for (int c = 0; c < NKV; ++c)
-                    s[c] = (c < lim) ? ex2(s[c] * p.scale_log2 - mref) * invL : 0.f;
-                // P (storage dtype) -> shared memory, K-major, 128-byte swizzle
+                for (int c = 0; c < NKV; ++c) s[c] = (c < lim) ? ex2(fmaf(s[c], c2, -mb)) : 0.f;
+                // P in the storage dtype -> tensor memory (A operand of P V)
                 mbar_wait(bar(B_P_EMPTY), (pcnt & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 11);
-                {
-                    uint8_t* prow = smem + p.off_p + row * 128;
+                tc_fence_after();
+                if constexpr ((NKV / 2) % 16 == 0) {
 #pragma unroll
-                    for (int v = 0; v < NKV / 8; ++v) {
-                        const int chunk = v >> 3, unit = v & 7;
-                        uint4 w;
-                        w.x = pack2<T>(s[v * 8 + 0], s[v * 8 + 1]);
-                        w.y = pack2<T>(s[v * 8 + 2], s[v * 8 + 3]);
-                        w.z = pack2<T>(s[v * 8 + 4], s[v * 8 + 5]);
-                        w.w = pack2<T>(s[v * 8 + 6], s[v * 8 + 7]);
-                        *reinterpret_cast<uint4*>(prow + chunk * 16384 + ((unit ^ (row & 7)) << 4)) = w;
+                    for (int c = 0; c < NKV / 32; ++c) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) w[e] = pack2<T>(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
+                        tmem_st16(tmem_p + lane_off + c * 16, w);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NKV / 16; ++c) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w[e] = pack2<T>(s[c * 16 + 2 * e], s[c * 16 + 2 * e + 1]);
+                        tmem_st8(tmem_p + lane_off + c * 8, w);
                     }
                 }
-                fence_proxy_async_smem();
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_P_FULL));
                 ++pcnt;
-                // step 4 on the fp32 P: anchors a*jj of this tile, taps reach back
+                // step 4 on the fp32 P: anchors A*jj of this tile; taps reach back
                 // into the previous tile through `carry` (carry[k] = P[c0 - 1 - k])
 #pragma unroll
-                for (int jc = 0; jc < NJ; jc += CHK) {
-                    float vals[CHK];
+                for (int e = 0; e < NENT; ++e) {
+                    float v[ENT];
 #pragma unroll
-                    for (int qq = 0; qq < CHK; ++qq) {
-                        const int anchor = A * (jc + qq);
+                    for (int qq = 0; qq < ENT; ++qq) {
+                        const int anchor = A * (e * ENT + qq);
                         float acc = 0.f;
 #pragma unroll
                         for (int u = 0; u < NTAP; ++u) {
@@ -438,19 +492,18 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             const float pv = (x >= 0) ? s[x >= 0 ? x : 0] : carry[x < 0 ? (-x - 1) : 0];
                             acc = fmaf(wband[u], pv, acc);
                         }
-                        vals[qq] = acc;
+                        v[qq] = acc;
                     }
-                    band_round(vals, i * NJ + jc);
+                    put_entry(v);
                 }
 #pragma unroll
-                for (int k = 0; k < NCARRY; ++k) carry[k] = (NKV - 1 - k >= 0) ? s[NKV - 1 - k] : 0.f;
+                for (int k = 0; k < NCARRY; ++k) carry[k] = s[NKV - 1 - k];
             }
-            int jcov = 0;
             if (t.nkv > 0) {
                 // the first anchors past the last tile still collect taps from it
-                float vals[CHK];
+                float v[ENT];
 #pragma unroll
-                for (int qq = 0; qq < CHK; ++qq) {
+                for (int qq = 0; qq < ENT; ++qq) {
                     const int anchor = A * qq;
                     float acc = 0.f;
 #pragma unroll
@@ -458,18 +511,65 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const int x = anchor - u;
                         if (x < 0) acc = fmaf(wband[u], carry[-x - 1 >= 0 ? -x - 1 : 0], acc);
                     }
-                    vals[qq] = acc;
+                    v[qq] = acc;
                 }
-                band_round(vals, t.nkv * NJ);
-                jcov = t.nkv * NJ + CHK;
+                put_entry(v);
             }
+        }
+    } else if (warp < 8) {
+        // ============ epilogue: group sum, output, top-k (128 thr) ============
+        setmaxnreg_dec<kRegsEpilogue>();
+        const int ew = warp - 4;                   // TMEM lane quadrant
+        const int erow = ew * 32 + lane;
+        const int et = threadIdx.x - 128;          // 0..127
+        const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
+        const float* stage = reinterpret_cast<const float*>(smem + p.off_stage);
+        float* score = p.score_in_smem ? reinterpret_cast<float*>(smem + p.off_score)
+                                       : p.score_gmem + (size_t)blockIdx.x * TT * p.score_cap;
+        const int cap = p.score_cap;
+        uint32_t stg = 0;
+        int tcount = 0;
+        const int eh = erow % G;
+        const int etok = erow / G;
 
-            // ---------------------------- epilogue ----------------------------
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+            const AttnTile t = p.tiles[tile];
+            // step 5: staged band values summed over the G rows of each token
+            const int nent = t.nkv > 0 ? t.nkv * NENT + 1 : 0;
+            for (int e = 0; e < nent; ++e) {
+                const int slot = stg & 1;
+                mbar_wait(bar(B_STG_FULL0 + slot), (stg >> 1) & 1, abort_flag, p.err, kErrTimeoutBase + 14);
+                const int j0 = (e < t.nkv * NENT) ? (e / NENT) * NJ + (e % NENT) * ENT : t.nkv * NJ;
+                const float* st = stage + (size_t)slot * (p.stage_entry_bytes / 4);
+                for (int pi = et; pi < t.ntok * ENT; pi += 128) {
+                    const int tau = pi / ENT, jj = pi - tau * ENT;
+                    const float* src = st + (tau * G) * STR + jj;
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    int hh = 0;
+                    for (; hh + 4 <= G; hh += 4) {
+                        a0 += src[(hh + 0) * STR];
+                        a1 += src[(hh + 1) * STR];
+                        a2 += src[(hh + 2) * STR];
+                        a3 += src[(hh + 3) * STR];
+                    }
+                    for (; hh < G; ++hh) a0 += src[hh * STR];
+                    const int j = j0 + jj;
+                    if (j < cap) score[tau * cap + j] = (a0 + a1) + (a2 + a3);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_STG_EMPTY0 + slot));
+                ++stg;
+            }
+            const int jcov = t.nkv > 0 ? t.nkv * NJ + ENT : 0;
+
+            // O (tensor memory) -> attention_out
             mbar_wait(bar(B_O_FULL), tcount & 1, abort_flag, p.err, kErrTimeoutBase + 12);
             tc_fence_after();
             {
+                const bool valid = (erow < TT * G) && (etok < t.ntok);
+                const int nvis = valid ? nvis_of(t.t0 + etok, p.l, p.d, t.n_cmp) : 0;
                 T* orow = reinterpret_cast<T*>(p.out) +
-                          ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * p.d2;
+                          ((size_t)(t.q_row0 + etok) * p.n1 + (size_t)t.group * G + eh) * p.d2;
                 for (int c = 0; c < p.d2 / 16; ++c) {
                     uint32_t r[16];
                     tmem_ld16(tmem_o + lane_off + c * 16, r);
@@ -478,7 +578,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         uint4 w0, w1;
                         float f[16];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) f[e] = (nvis > 0) ? __uint_as_float(r[e]) : 0.f;
+                        for (int q = 0; q < 16; ++q) f[q] = (nvis > 0) ? __uint_as_float(r[q]) : 0.f;
                         w0.x = pack2<T>(f[0], f[1]);
                         w0.y = pack2<T>(f[2], f[3]);
                         w0.z = pack2<T>(f[4], f[5]);
@@ -495,18 +595,10 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_O_EMPTY));
-            if (valid) {
-                const size_t si = ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * 8;
-                const float mo = (m == -INFINITY) ? -INFINITY : m * 0.69314718055994530942f;
-                const float4 mv = make_float4(mo, mo, mo, mo);
-                const float4 lv = make_float4(L, L, L, L);
-                reinterpret_cast<float4*>(p.smax + si)[0] = mv;
-                reinterpret_cast<float4*>(p.smax + si)[1] = mv;
-                reinterpret_cast<float4*>(p.ssum + si)[0] = lv;
-                reinterpret_cast<float4*>(p.ssum + si)[1] = lv;
-            }
+
+            named_bar_sync(2, 128);   // every group sum of this tile is in the score buffer
             // step 7, one warp per token
-            for (int tau = sw; tau < t.ntok; tau += 4) {
+            for (int tau = ew; tau < t.ntok; tau += 4) {
                 const int tp = t.t0 + tau;
                 int32_t* dst = p.topk + ((size_t)(t.q_row0 + tau) * p.n2 + t.group) * p.count;
                 if (nvis_of(tp, p.l, p.d, t.n_cmp) == 0) {
@@ -516,7 +608,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     warp_topk(score + tau * cap, ncand, jcov, p.count, dst, lane);
                 }
             }
-            named_bar_sync(1, 128);   // score buffer is free for the next tile
+            named_bar_sync(2, 128);   // the score buffer is free for the next tile
         }
     }
 
@@ -529,7 +621,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     }
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -39,9 +39,19 @@ cudaError_t launch_compress(const CompressParams& p, dim3 grid, int threads, siz
 cudaError_t read_compress_error(int* out, cudaStream_t st);
 
 // ----------------------------------------------------------- attention
-constexpr int kAttnThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 softmax/epilogue
+// Warp roles: warps 0-3 softmax (TMEM lanes 32w..32w+31), warps 4-7 epilogue
+// (group sum, output, top-k), warp 8 TMA producer, warp 9 MMA issuer, warps
+// 10-11 idle.  Launched at 168 registers per thread (384 x 168 = 64512); the
+// warpgroups then rebalance to 232 / 152 / 120, whose sum x 128 threads is
+// the same 64512.
+constexpr int kAttnThreads = 384;
+constexpr int kRegsSoftmax = 232;
+constexpr int kRegsEpilogue = 152;
+constexpr int kRegsCtl = 120;
+static_assert((kRegsSoftmax + kRegsEpilogue + kRegsCtl) * 128 <= kAttnThreads * 168,
+              "register split exceeds the launch allocation");
 constexpr int kRows = 128;          // M of one tile: (tokens x heads of one KV group)
-constexpr int kBandChunk = 16;      // importance scores staged per named-barrier round
+constexpr int kEntryMax = 32;       // importance anchors per staging entry
 
 // One M-tile: up to 128/G consecutive query tokens of one sequence x the G
 // heads of one KV group.
@@ -73,8 +83,12 @@ struct AttnParams {
     float scale_log2;       // scale * log2(e)
     int nkv_cols;           // compressed blocks per KV tile
     int nslot;              // K/V ring depth
+    int nqbuf;              // Q buffers (1 or 2)
+    int nsbuf;              // S buffers in tensor memory (1 or 2)
+    int tm_o, tm_p;         // tensor-memory columns of O and of P
     // shared-memory layout (byte offsets from a 1024-aligned base)
-    int off_q, off_ring, slot_bytes, off_p, off_stage, off_score, off_bar, smem_bytes;
+    int off_q, q_bytes, off_ring, slot_bytes, off_stage, stage_entry_bytes, off_score, off_bar,
+        smem_bytes;
 };
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
