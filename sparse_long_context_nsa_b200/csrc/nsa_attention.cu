@@ -95,6 +95,33 @@ __device__ __forceinline__ int nvis_of(int t, int l, int d, int n_cmp) {
     return min(n_cmp, (t - l + 1) / d + 1);
 }
 
+// k-th largest key (fp32 bit pattern) of sc[0 .. ncand) held in registers,
+// NR keys per lane (key i of a lane belongs to j = lane + 32 i); keys at
+// j >= lim are 0.  Bitwise search from the top bit down.
+template <int NR>
+__device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int lim, int k, int lane) {
+    uint32_t key[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+        const int j = lane + 32 * i;
+        key[i] = (j < lim) ? __float_as_uint(sc[j]) : 0u;
+    }
+    uint32_t thr = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t trial = thr | (1u << bit);
+        int c0 = 0, c1 = 0;
+#pragma unroll
+        for (int i = 0; i < NR; i += 2) {
+            c0 += key[i] >= trial ? 1 : 0;
+            c1 += key[i + 1] >= trial ? 1 : 0;
+        }
+        const int c = __reduce_add_sync(0xffffffffu, c0 + c1);
+        if (c >= k) thr = trial;
+    }
+    return thr;
+}
+
 // Top-k of one token's group scores (step 7), one warp.  Candidates are
 // j < ncand; scores for j >= jcov are 0 (no visible block reaches them).
 // Exact k-th largest key by a bitwise search over the fp32 bit patterns
@@ -110,25 +137,12 @@ __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, 
     }
     const int lim = min(ncand, jcov);          // keys at j >= lim are 0
     uint32_t thr = 0;
-    if (ncand <= 32 * 32) {
-        // keys in registers: key[i] belongs to j = lane + 32 i
-        uint32_t key[32];
-        const int nreg = (ncand + 31) >> 5;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int j = lane + 32 * i;
-            key[i] = (i < nreg && j < lim) ? __float_as_uint(sc[j]) : 0u;
-        }
-#pragma unroll 1
-        for (int bit = 31; bit >= 0; --bit) {
-            const uint32_t trial = thr | (1u << bit);
-            int c = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (i < nreg) c += key[i] >= trial ? 1 : 0;
-            c = __reduce_add_sync(0xffffffffu, c);
-            if (c >= k) thr = trial;
-        }
+    if (ncand <= 8 * 32) {
+        thr = kth_key_regs<8>(sc, ncand, lim, k, lane);
+    } else if (ncand <= 16 * 32) {
+        thr = kth_key_regs<16>(sc, ncand, lim, k, lane);
+    } else if (ncand <= 32 * 32) {
+        thr = kth_key_regs<32>(sc, ncand, lim, k, lane);
     } else {
 #pragma unroll 1
         for (int bit = 31; bit >= 0; --bit) {
@@ -378,17 +392,39 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_after();
             const uint32_t ta = tmem + lane_off + sb * 128;
 #pragma unroll
-            for (int c = 0; c < NKV / 16; ++c) {
-                uint32_t r[16];
-                tmem_ld16(ta + c * 16, r);
+            for (int c = 0; c < NKV / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(ta + c * 32, r);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) s[c * 16 + e] = __uint_as_float(r[e]);
+                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+            }
+            if constexpr (NKV % 32 != 0) {
+                uint32_t r[16];
+                tmem_ld16(ta + (NKV / 32) * 32, r);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) s[(NKV / 32) * 32 + e] = __uint_as_float(r[e]);
             }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_S_EMPTY0 + sb));
             ++scnt;
+        };
+        // scores of one KV tile in "exponent units": x = s * ce - shift.  With a
+        // positive scale the raw scores are used as they are (ce = c2); a zero
+        // or negative scale first multiplies them in (ce = 1).  Columns c >= lim
+        // are not visible and become -inf.
+        const bool pos_scale = c2 > 0.f;
+        const float ce = pos_scale ? c2 : 1.f;
+        auto prep = [&](float (&s)[NKV], int lim) {
+            if (!pos_scale) {
+#pragma unroll
+                for (int c = 0; c < NKV; ++c) s[c] *= c2;
+            }
+            if (lim < NKV) {
+#pragma unroll
+                for (int c = 0; c < NKV; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+            }
         };
         // one staging entry: ENT anchors of this row -> shared memory
         auto put_entry = [&](const float* v) {
@@ -414,18 +450,30 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int i = 0; i < t.nkv; ++i) {
                 float s[NKV];
                 load_s(s);
-                const int lim = nvis - i * NKV;     // columns c < lim are visible
-                float mx = -INFINITY;
+                prep(s, nvis - i * NKV);
+                // row maximum: four independent chains of 3-input max
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < NKV; ++c) {
-                    s[c] = (c < lim) ? s[c] * c2 : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
+                for (int c = 0; c < NKV; c += 8) {
+                    mx4[0] = fmax3(mx4[0], s[c + 0], s[c + 1]);
+                    mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
+                    mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
+                    mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
                 }
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
                 const float mn = fmaxf(m, mx);
                 const float mref = (mn == -INFINITY) ? 0.f : mn;
-                float sum = 0.f;
+                // row sum of 2^(x - mref): packed exponent arguments, 8 partial sums
+                const float2 ce2 = make_float2(ce, ce), nm2 = make_float2(-mref, -mref);
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < NKV; ++c) sum += ex2(s[c] - mref);
+                for (int c = 0; c < NKV; c += 2) {
+                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2, nm2);
+                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(x.x), ex2(x.y)));
+                }
+                const float2 t01 = fadd2(acc[0], acc[1]), t23 = fadd2(acc[2], acc[3]);
+                const float sum = (t01.x + t01.y) + (t23.x + t23.y);
                 L = L * ex2(m - mref) + sum;
                 m = mn;
             }
@@ -449,9 +497,16 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int i = 0; i < t.nkv; ++i) {
                 float s[NKV];
                 load_s(s);
-                const int lim = nvis - i * NKV;
+                prep(s, nvis - i * NKV);
+                {
+                    const float2 ce2 = make_float2(ce, ce), nb2 = make_float2(-mb, -mb);
 #pragma unroll
-                for (int c = 0; c < NKV; ++c) s[c] = (c < lim) ? ex2(fmaf(s[c], c2, -mb)) : 0.f;
+                    for (int c = 0; c < NKV; c += 2) {
+                        const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2, nb2);
+                        s[c] = ex2(x.x);
+                        s[c + 1] = ex2(x.y);
+                    }
+                }
                 // P in the storage dtype -> tensor memory (A operand of P V)
                 mbar_wait(bar(B_P_EMPTY), (pcnt & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 11);
                 tc_fence_after();
