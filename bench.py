@@ -90,6 +90,21 @@ def profile_traffic(kind):
     return d.get("bytes_per_launch_full_workload")
 
 
+# ------------------------------------------------------------ ranks
+def rank_workload(name: str, rank: int) -> workloads.Workload:
+    """Each rank runs its own independent batch: same shapes, seed offset by rank."""
+    wl = workloads.WORKLOADS[name]
+    return wl.replace(seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise max of a list of floats over all ranks (identity for one rank)."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML while running."""
@@ -151,7 +166,7 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = workloads.WORKLOADS[args.workload].replace(seed=workloads.WORKLOADS[args.workload].seed + 1000 * rank)
+    wl = rank_workload(args.workload, rank)
     x = wl.generate(device=str(dev))
     q, k, v, w = x["q"], x["k"], x["v"], x["w"]
     cu, cuq, cus = x["cu_seqlens"], x["cu_seqlens_q"], x["cu_sel_kv"]
@@ -374,11 +389,8 @@ def main():
     r = run_ours(args, rank, world, local_rank)
     wl = r["wl"]
     # max over ranks of the device time of the timed steps
-    t = torch.tensor([r["step_ms"], r["att_ms"], r["cmp_ms"]], dtype=torch.float64,
-                     device=torch.device("cuda", local_rank))
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    step_total_ms, att_ms, cmp_ms = t.tolist()
+    step_total_ms, att_ms, cmp_ms = max_over_ranks([r["step_ms"], r["att_ms"], r["cmp_ms"]],
+                                                   torch.device("cuda", local_rank), world)
     K = r["K"]
     ms_per_step = step_total_ms / K
     flops = attention_flops(wl)
