@@ -19,7 +19,8 @@
  *     for actual_seq_qlen / actual_cmp_seq_kvlen / actual_sel_seq_kvlen).
  *   - Tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
  *     caller.  The library allocates no memory and keeps no state between
- *     calls.
+ *     calls (the one exception is the fixed scratch array behind
+ *     nsa_compress_attention_noalloc, declared at the end of this file).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; argument errors are returned
  *     synchronously before anything is enqueued ("aclnnNsaCompress": the
@@ -154,6 +155,35 @@ nsa_status_t nsa_workspace_status(const void* workspace, void* stream);
  * (0 = none).  Synchronises `stream`.  NSA_ERR_TIMEOUT when a wait gave up.
  */
 nsa_status_t nsa_compress_status(void* stream);
+
+/*
+ * Same computation, outputs and argument rules as nsa_compress_attention,
+ * for callers that cannot allocate device memory: for example an application
+ * that has already claimed almost all of the GPU's memory for its own pools,
+ * a plugin that is handed only the tensors it works on, or a path where an
+ * allocation call is not permitted.  The source pages have no counterpart of
+ * this call.
+ *   - No workspace argument: the library uses its own fixed scratch array of
+ *     16 MiB per device (a static device array that every GPU which loads
+ *     the library keeps until the process exits).  Arguments whose workspace
+ *     requirement (nsa_compress_attention_workspace_size) exceeds 16 MiB are
+ *     rejected with NSA_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the contents of
+ *     the last call; each call rewrites the parts that must start at zero.
+ *     Calls whose work can overlap on the GPU (different streams without
+ *     ordering between them) race on the array and must not be issued.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     routine.
+ */
+nsa_status_t nsa_compress_attention_noalloc(
+    const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
+    int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+    void* attention_out, int32_t* topk_indices, float* softmax_max, float* softmax_sum,
+    void* stream);
 
 #ifdef __cplusplus
 }

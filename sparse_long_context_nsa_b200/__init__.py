@@ -35,6 +35,7 @@ EXPORTED = (
     "nsa_compress_attention",
     "nsa_workspace_status",
     "nsa_compress_status",
+    "nsa_compress_attention_noalloc",
 )
 
 _lib = None
@@ -82,6 +83,9 @@ def load(path: Optional[str] = None):
     lib.nsa_workspace_status.restype = ci
     lib.nsa_compress_status.argtypes = [vp]
     lib.nsa_compress_status.restype = ci
+    lib.nsa_compress_attention_noalloc.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p,
+                                                   i32p, i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
+    lib.nsa_compress_attention_noalloc.restype = ci
     if path is None:
         _lib = lib
     return lib
@@ -242,6 +246,33 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
         tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
         _stream(stream))
     _raise(st, "nsa_compress_attention")
+    return att, tk, smax, ssum
+
+
+def nsa_compress_attention_noalloc(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tensor, scale: float,
+                                   head_num: int, l: int, d: int, lp: int, count: int, cu_seqlens_q,
+                                   cu_cmp_kv, cu_sel_kv, out, stream=None):
+    """nsa_compress_attention for callers that cannot allocate device memory.
+
+    The caller passes the four output tensors in ``out`` (attention_out,
+    topk_indices, softmax_max, softmax_sum); the library's own fixed 16 MiB
+    scratch array replaces the workspace.  Nothing is allocated here.
+    """
+    for t, nm in ((q, "q"), (kcmp, "kcmp"), (vcmp, "vcmp")):
+        _dev(t, nm)
+    att, tk, smax, ssum = out
+    for t, nm in ((att, "attention_out"), (tk, "topk_indices"), (smax, "softmax_max"), (ssum, "softmax_sum")):
+        _dev(t, nm)
+    dt = _dtype_code(q)
+    t1, n1, d1 = q.shape
+    tc, n2, _ = kcmp.shape
+    d2 = vcmp.shape[2]
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    st = load().nsa_compress_attention_noalloc(
+        q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
+        int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
+        tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), _stream(stream))
+    _raise(st, "nsa_compress_attention_noalloc")
     return att, tk, smax, ssum
 
 

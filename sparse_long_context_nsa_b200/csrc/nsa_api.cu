@@ -471,3 +471,55 @@ nsa_status_t nsa_workspace_status(const void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Variant with a fixed, library-owned scratch area (no counterpart on the
+// source pages).  Some callers cannot allocate device memory at all: a host
+// application that has already reserved nearly all of the GPU's memory for
+// its own pools, a plugin whose host environment hands it only the tensors
+// it works on, or a latency-critical path where an allocation call is not
+// allowed.  They pass only inputs and outputs; the workspace lives in this
+// file-scope array, which every GPU that loads the library holds until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[256] = {};   // device address of g_static_scratch, per device ordinal
+
+}  // namespace
+
+extern "C" nsa_status_t nsa_compress_attention_noalloc(
+    const void* q, const void* kcmp, const void* vcmp, float scale, int head_num, int l, int d, int lp,
+    int count, const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv, int batch,
+    int n2, int d1, int d2, nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
+    float* softmax_max, float* softmax_sum, void* stream) {
+    size_t need = 0;
+    nsa_status_t s = nsa_compress_attention_workspace_size(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q,
+                                                           cu_cmp_kv, cu_sel_kv, batch, &need);
+    if (s != NSA_OK) return s;
+    if (need > kStaticScratchBytes) return NSA_ERR_WORKSPACE;   // larger than the fixed scratch
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return NSA_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        // first call on a device: look up the device address of the array with
+        // that device current (host code may not use the symbol itself)
+        std::lock_guard<std::mutex> lk(g_scratch_mu);
+        if (g_scratch_addr[dev] == nullptr) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr)
+                return NSA_ERR_CUDA;
+            g_scratch_addr[dev] = ptr;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    // the regular entry point rewrites the scratch header (error word = 0) and
+    // the tile list on every call before its kernel runs
+    return nsa_compress_attention(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
+                                  cu_sel_kv, batch, n2, d1, d2, dtype, attention_out, topk_indices, softmax_max,
+                                  softmax_sum, scratch, kStaticScratchBytes, stream);
+}
