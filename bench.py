@@ -34,8 +34,11 @@ import workloads  # noqa: E402
 METRIC = ("compressed-attn TFLOP/s + query tok/s (fwd incl. top-k), % bf16 peak; "
           "compress GB/s")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc", "nsa_attention.cu")
-CMP_SRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc", "nsa_compress.cu")
+_CSRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc")
+# sources whose change invalidates a recorded DRAM-traffic figure: the two
+# attention kernels and the planner that chooses between them
+ATTN_SRC = [os.path.join(_CSRC, f) for f in ("nsa_attention.cu", "nsa_attention_wide.cu", "nsa_api.cu")]
+CMP_SRC = [os.path.join(_CSRC, "nsa_compress.cu")]
 
 
 # ------------------------------------------------------------------ work
@@ -71,9 +74,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def src_hash(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def src_hash(paths):
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profile_traffic(kind):

@@ -230,6 +230,30 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+// N consecutive columns (N a multiple of 16) into r[0..N).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
+    static_assert(N % 16 == 0, "columns in steps of 16");
+#pragma unroll
+    for (int k = 0; k < N / 32; ++k) tmem_ld32(taddr + 32 * k, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * k));
+    if constexpr (N % 32 != 0) tmem_ld16(taddr + N - 16, *reinterpret_cast<uint32_t(*)[16]>(r + N - 16));
+}
+// Waits for this thread's tensor-memory loads and marks r[0..N) as written
+// after the wait, so that no use of them is scheduled before it.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+// N consecutive columns (N a multiple of 8) from r[0..N).
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* r) {
+    static_assert(N % 8 == 0, "columns in steps of 8");
+#pragma unroll
+    for (int k = 0; k < N / 16; ++k) tmem_st16(taddr + 16 * k, r + 16 * k);
+    if constexpr (N % 16 != 0) tmem_st8(taddr + N - 8, r + N - 8);
+}
 // Packed fp32 pairs (sm_100): two lanes of arithmetic per instruction.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     uint64_t d;
@@ -259,6 +283,12 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+// Moves this warpgroup from the launch budget LAUNCH to N registers per thread.
+template <int N, int LAUNCH>
+__device__ __forceinline__ void setmaxnreg_to() {
+    if constexpr (N > LAUNCH) setmaxnreg_inc<N>();
+    else if constexpr (N < LAUNCH) setmaxnreg_dec<N>();
 }
 __device__ __forceinline__ float lg2(float x) {
     float y;
