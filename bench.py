@@ -82,16 +82,16 @@ def src_hash(paths):
     return h.hexdigest()[:16]
 
 
-def profile_traffic(kind):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    source still matches the one the counters were taken on."""
+def profile_traffic(kind, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    this workload and the kernel source still matches the one it was taken on."""
     p = os.path.join(ROOT, "profiles", f"{kind}_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     src = ATTN_SRC if kind == "attention" else CMP_SRC
-    if d.get("source_sha256_16") != src_hash(src):
+    if d.get("workload") != workload or d.get("source_sha256_16") != src_hash(src):
         return None
     return d.get("bytes_per_launch_full_workload")
 
@@ -267,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
                 launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
 
 
-def cpu_baseline(wl, budget_s=15.0, rows_per_seq=None):
+def cpu_baseline(wl, budget_s=20.0, rows_per_seq=None):
     """The fp64 oracle as it stands, timed on a bounded sample of the workload."""
     import oracle
     x = wl.generate(device="cpu")
@@ -284,7 +284,9 @@ def cpu_baseline(wl, budget_s=15.0, rows_per_seq=None):
     cq = x["cu_seqlens_q"]
     T1 = int(cq[-1])
     full_pairs = visible_pairs(wl)
-    probe = np.arange(T1 - 1, max(T1 - 33, -1), -1, dtype=np.int64)
+    # the cost of a row grows with its position: probe rows spread over the
+    # whole query range so that the estimate is the mean cost per row
+    probe = np.unique(np.linspace(0, T1 - 1, num=min(T1, 48)).astype(np.int64))
     tp = time.perf_counter()
     oracle.compress_attention(x["q"][probe], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
                               x["cu_sel_kv"], rows=probe, q_rows_only=True)
@@ -376,7 +378,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-rows", type=int, default=96)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -416,7 +418,7 @@ def main():
         if not args.no_cpu_baseline and world == 1:
             cpu = cpu_baseline(wl, budget_s=args.cpu_budget)
         peak_t = peaks["bf16_tflops"]
-        traffic = profile_traffic("attention")
+        traffic = profile_traffic("attention", wl.name)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -439,7 +441,7 @@ def main():
                          "flops_per_launch": flops},
             "roofline_compress": {"bound": "hbm", "achieved": cmp_gbs, "peak": peaks["hbm_gbs"],
                                   "unit": "GB/s", "frac": cmp_gbs / peaks["hbm_gbs"],
-                                  "traffic": profile_traffic("compress"),
+                                  "traffic": profile_traffic("compress", wl.name),
                                   "peak_source": f"{peak_src} hbm_gbs"},
             "clocks": r["clocks"],
             "e2e": e2e,

@@ -137,7 +137,13 @@ SHORTQ_4x64K = Workload("compress_t262144_shortq_4x128_n64_n8_d128",
                         (65536,) * 4, 64, 8, 128, 128, 128, 64, 128, 32,
                         128 ** -0.5, "bf16", seed=4, q_last=128)
 
-WORKLOADS = {w.name: w for w in (TINY, SINGLE_16K, VARLEN_8, LONG_128K, SHORTQ_4x64K)}
+# A profiling case, not one of the benchmark's configurations: the shape of the
+# 16K workload at twice the length, so that the M-tiles visit enough KV tiles
+# for the two-CTA attention kernel while the device footprint stays near 1 GB.
+PROFILE_32K = Workload("single_s32768_n64_n4_d128", (32768,), 64, 4, 128, 128,
+                       32, 16, 64, 16, 128 ** -0.5, "bf16", seed=5)
+
+WORKLOADS = {w.name: w for w in (TINY, SINGLE_16K, VARLEN_8, LONG_128K, SHORTQ_4x64K, PROFILE_32K)}
 BY_INDEX = [TINY, SINGLE_16K, VARLEN_8, LONG_128K, SHORTQ_4x64K]
 
 
