@@ -134,11 +134,6 @@ nsa_status_t nsa_compress_attention_workspace_size(
  * NSA_ERR_UNSUPPORTED: l % d != 0 (the importance sum needs integer l/d),
  * D1 or D2 > 256, more than 128 query heads per KV group, or shapes whose
  * on-chip tiles do not fit one SM.
- * Kernel choice: the plan runs two CTAs per SM when the M-tiles visit six or
- * more KV tiles of compressed keys on average and D2 <= 128, else one CTA per
- * SM.  The environment variable NSA_ATTN_CTAS_PER_SM=1 or 2, read at every
- * call (and by nsa_compress_attention_workspace_size), overrides that choice
- * where the requested layout fits; results agree within rounding.
  */
 nsa_status_t nsa_compress_attention(
     const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,

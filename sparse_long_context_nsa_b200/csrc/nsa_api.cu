@@ -6,7 +6,6 @@
 
 #include <algorithm>
 #include <cmath>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -19,10 +18,8 @@ using namespace nsa;
 namespace {
 
 constexpr size_t kWsHeader = 256;     // error word + padding
-constexpr int kMaxGrid = 320;         // persistent CTAs: up to two per SM (148 SMs on B200)
+constexpr int kMaxGrid = 160;         // persistent CTAs sized for one CTA per SM (148 on B200)
 constexpr int kSmemLimit = 232448;    // dynamic shared memory per block on sm_100
-constexpr int kSmemHalf = 113 * 1024; // per block when two blocks share an SM's 228 KB
-constexpr int kMinKvPerTileForTwo = 6;  // KV tiles per M-tile from which two CTAs per SM win
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -84,14 +81,10 @@ struct AttnPlan {
     std::vector<AttnTile> tiles;
     int score_cap = 1;
     int grid = 0;
-    // kernel choice: two CTAs per SM (nsa_attention.cu) or one (nsa_attention_wide.cu)
-    bool wide = false;
     bool score_in_smem = true;
-    int nslot = 0, ctas_per_sm = 1, tmem_cols = 256, sbufs = 1, qbufs = 1;
-    bool shfl_group = false;
-    int nqbuf = 1, nsbuf = 1, tm_o = 0, tm_p = 0;   // one-CTA kernel
+    int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_p = 0;
     int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_stage = 0, stage_entry_bytes = 0,
-        off_score = 0, off_topk = 0, off_bar = 0, smem_bytes = 0;
+        off_score = 0, off_bar = 0, smem_bytes = 0;
     size_t ws_tiles = 0, ws_score = 0, ws_total = 0;
 };
 
@@ -127,10 +120,9 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
     pl.b = l / d;
     pl.nkv_cols = attention_kv_cols(pl.a);
     const int NKV = pl.nkv_cols;
-    // score buffer length (the longest causal candidate list), the M-tile count
-    // and the KV tiles those M-tiles visit
+    // tiles: (sequence, group, run of TT tokens)
+    int64_t ntiles = 0;
     int cap = 1;
-    int64_t nitems = 0, kv_visits = 0;
     {
         int32_t pq = 0, pc = 0, ps = 0;
         for (int bq = 0; bq < batch; ++bq) {
@@ -142,123 +134,20 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
                 const int64_t tlast = Sq - 1 + off;
                 if (nvis_host(tlast, l, d, n_cmp) > 0)
                     cap = std::max<int64_t>(cap, std::min<int64_t>(n_sel, tlast / lp + 1));
-                const int64_t tiles = (Sq + pl.TT - 1) / pl.TT;
-                nitems += tiles * (int64_t)n2;
-                for (int64_t k = 0; k < tiles; ++k) {
-                    const int64_t last = std::min<int64_t>(Sq - 1, (k + 1) * pl.TT - 1) + off;
-                    kv_visits += ((nvis_host(last, l, d, n_cmp) + NKV - 1) / NKV) * (int64_t)n2;
-                }
+                ntiles += ((Sq + pl.TT - 1) / pl.TT) * (int64_t)n2;
             }
             pq = cu_q[bq];
             pc = cu_cmp[bq];
             ps = cu_sel[bq];
         }
     }
-    if (nitems > (int64_t)1 << 30) return NSA_ERR_UNSUPPORTED;
+    if (ntiles > (int64_t)1 << 30) return NSA_ERR_UNSUPPORTED;
     pl.score_cap = (cap + 3) & ~3;
-
-    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
-    const int NJ = NKV / pl.a;
-    pl.q_bytes = nqc * 16384;
-    pl.slot_bytes = std::max(nqc, nvc) * NKV * 128;
-
-    // --- two CTAs per SM: Q, a K/V ring of two tiles, top-k scratch, barriers
-    // (about 110 KB), one score buffer and O in 256 tensor-memory columns.
-    // G a power of two up to 32: the rows of a token share a warp and the
-    // softmax warps sum them by shuffles; else band values are staged through
-    // shared memory and the epilogue sums them.
-    auto plan_two = [&]() {
-        pl.wide = false;
-        pl.shfl_group = (pl.G & (pl.G - 1)) == 0 && pl.G <= 32;
-        pl.stage_entry_bytes = pl.shfl_group ? 0 : kRows * (std::min(NJ, kEntryMax) + 4) * 4;
-        pl.ctas_per_sm = 2;
-        pl.sbufs = 1;
-        pl.qbufs = 1;
-        pl.tmem_cols = 256;
-        if (d2 > 128) return false;
-        auto layout = [&](int ns, bool in_smem) {
-            int off = 0;
-            pl.off_q = off;
-            off += pl.qbufs * pl.q_bytes;
-            pl.off_ring = off;
-            off += ns * pl.slot_bytes;
-            pl.off_stage = off;
-            off += 2 * pl.stage_entry_bytes;
-            pl.off_score = off;
-            if (in_smem) off += (2 * pl.TT * pl.score_cap * 4 + 127) & ~127;   // two score buffers
-            pl.off_topk = off;
-            off += kEpiWarps * 2 * kTopkCap * 4;
-            pl.off_bar = off;
-            off += 512;
-            pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
-            pl.nslot = ns;
-            pl.score_in_smem = in_smem;
-            return pl.smem_bytes <= kSmemHalf;
-        };
-        for (int ns = 4; ns >= 2; --ns)
-            if (layout(ns, true) || layout(ns, false)) return true;
-        return false;
-    };
-
-    // --- one CTA per SM (the kernel of nsa_attention_wide.cu): S buffers
-    // (128 columns each), O (D2 columns), P (NKV/2 columns of packed pairs) in
-    // tensor memory, two S buffers when they fit next to O and P; Q buffers,
-    // K/V ring, band staging (2 entries), score buffer in shared memory
-    auto plan_one = [&]() {
-        pl.wide = true;
-        pl.ctas_per_sm = 1;
-        const int d2c = (d2 + 31) & ~31;
-        pl.nsbuf = (256 + d2c + 64 <= 512) ? 2 : 1;
-        pl.tm_o = pl.nsbuf * 128;
-        pl.tm_p = pl.tm_o + d2c;
-        if (pl.tm_p + NKV / 2 > 512) return false;
-        pl.stage_entry_bytes = kRows * (std::min(NJ, wide::kEntryMax) + 4) * 4;
-        const int score_bytes = pl.TT * pl.score_cap * 4;
-        auto layout = [&](int nq, int ns, bool in_smem) {
-            int off = 0;
-            pl.off_q = off;
-            off += nq * pl.q_bytes;
-            pl.off_ring = off;
-            off += ns * pl.slot_bytes;
-            pl.off_stage = off;
-            off += 2 * pl.stage_entry_bytes;
-            pl.off_score = off;
-            if (in_smem) off += (score_bytes + 127) & ~127;
-            pl.off_bar = off;
-            off += 320;
-            pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
-            pl.nqbuf = nq;
-            pl.nslot = ns;
-            pl.score_in_smem = in_smem;
-            return pl.smem_bytes <= kSmemLimit;
-        };
-        // preference: deeper K/V ring, then a second Q buffer, then on-chip scores
-        static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}, {2, 2}, {1, 2}};
-        for (const auto& o : kOrder)
-            if (layout(o[0], o[1], true) || layout(o[0], o[1], false)) return true;
-        return false;
-    };
-
-    // Two CTAs per SM pay off when the M-tiles visit many KV tiles: one CTA's
-    // exponentials then overlap the other's tensor work for most of a tile.
-    // With few KV tiles per M-tile the per-tile costs (Q load, output
-    // read-out, top-k) dominate, and one CTA with double-buffered scores and
-    // Q runs faster (measured on B200 with the workloads of the benchmark).
-    // NSA_ATTN_CTAS_PER_SM=1 or 2 overrides the choice (where that layout fits)
-    bool two_first = nitems > 0 && kv_visits >= (int64_t)kMinKvPerTileForTwo * nitems;
-    if (const char* force = std::getenv("NSA_ATTN_CTAS_PER_SM")) {
-        if (force[0] == '1' && force[1] == 0) two_first = false;
-        if (force[0] == '2' && force[1] == 0) two_first = true;
-    }
-    bool fits = false;
-    if (two_first) fits = plan_two() || plan_one();
-    else fits = plan_one() || plan_two();
-    if (!fits) return NSA_ERR_UNSUPPORTED;
-    pl.grid = (int)std::min<int64_t>(nitems, pl.wide ? kMaxGrid / 2 : kMaxGrid);
+    pl.grid = (int)std::min<int64_t>(ntiles, kMaxGrid);
 
     if (build_tiles) {
         pl.tiles.clear();
-        pl.tiles.reserve((size_t)nitems);
+        pl.tiles.reserve((size_t)ntiles);
         int32_t pq = 0, pc = 0, ps = 0;
         for (int bq = 0; bq < batch; ++bq) {
             const int Sq = cu_q[bq] - pq;
@@ -290,8 +179,52 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
                          [](const AttnTile& x, const AttnTile& y) { return x.nkv > y.nkv; });
     }
 
-    pl.ws_tiles = (size_t)nitems * sizeof(AttnTile);
-    pl.ws_score = pl.score_in_smem ? 0 : (size_t)pl.grid * (pl.wide ? 1 : 2) * pl.TT * pl.score_cap * 4;
+    // tensor memory: S buffers (128 columns each), O (D2 columns), P (NKV/2
+    // columns of packed pairs); two S buffers when they fit next to O and P
+    const int d2c = (d2 + 31) & ~31;
+    pl.nsbuf = (256 + d2c + 64 <= 512) ? 2 : 1;
+    pl.tm_o = pl.nsbuf * 128;
+    pl.tm_p = pl.tm_o + d2c;
+    if (pl.tm_p + NKV / 2 > 512) return NSA_ERR_UNSUPPORTED;
+
+    // shared memory: Q buffers, K/V ring, band staging (2 entries), score buffer
+    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
+    const int NJ = NKV / pl.a;
+    const int ENT = std::min(NJ, kEntryMax);
+    pl.q_bytes = nqc * 16384;
+    pl.slot_bytes = std::max(nqc, nvc) * NKV * 128;
+    pl.stage_entry_bytes = kRows * (ENT + 4) * 4;
+    const int score_bytes = pl.TT * pl.score_cap * 4;
+    const int bar_bytes = 320;
+    auto layout = [&](int nq, int ns, bool in_smem) {
+        int off = 0;
+        pl.off_q = off;
+        off += nq * pl.q_bytes;
+        pl.off_ring = off;
+        off += ns * pl.slot_bytes;
+        pl.off_stage = off;
+        off += 2 * pl.stage_entry_bytes;
+        pl.off_score = off;
+        if (in_smem) off += (score_bytes + 127) & ~127;
+        pl.off_bar = off;
+        off += bar_bytes;
+        pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
+        pl.nqbuf = nq;
+        pl.nslot = ns;
+        pl.score_in_smem = in_smem;
+        return pl.smem_bytes <= kSmemLimit;
+    };
+    // preference: deeper K/V ring, then a second Q buffer, then on-chip scores
+    static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}, {2, 2}, {1, 2}};
+    bool fits = false;
+    for (const auto& o : kOrder) {
+        if ((fits = layout(o[0], o[1], true))) break;
+        if ((fits = layout(o[0], o[1], false))) break;
+    }
+    if (!fits) return NSA_ERR_UNSUPPORTED;
+
+    pl.ws_tiles = (size_t)ntiles * sizeof(AttnTile);
+    pl.ws_score = pl.score_in_smem ? 0 : (size_t)pl.grid * pl.TT * pl.score_cap * 4;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     pl.ws_total = kWsHeader + up(pl.ws_tiles) + up(pl.ws_score);
     return NSA_OK;
@@ -481,68 +414,51 @@ nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void*
     if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
 
-    // the fields both kernels take
-    auto fill = [&](auto& p) {
-        std::memset(&p, 0, sizeof(p));
-        p.tiles = reinterpret_cast<const AttnTile*>(ws + kWsHeader);
-        p.num_tiles = (int)pl.tiles.size();
-        p.err = reinterpret_cast<int*>(ws);
-        p.score_gmem = pl.score_in_smem
-                           ? nullptr
-                           : reinterpret_cast<float*>(ws + kWsHeader + ((pl.ws_tiles + 255) & ~(size_t)255));
-        p.score_cap = pl.score_cap;
-        p.score_in_smem = pl.score_in_smem ? 1 : 0;
-        p.out = attention_out;
-        p.topk = topk_indices;
-        p.smax = softmax_max;
-        p.ssum = softmax_sum;
-        p.dtype = dtype == NSA_BF16 ? 0 : 1;
-        p.n1 = head_num;
-        p.n2 = n2;
-        p.d1 = d1;
-        p.d2 = d2;
-        p.G = pl.G;
-        p.tok_per_tile = pl.TT;
-        p.l = l;
-        p.d = d;
-        p.lp = lp;
-        p.count = count;
-        p.a = pl.a;
-        p.b = pl.b;
-        p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-        p.nkv_cols = pl.nkv_cols;
-        p.nslot = pl.nslot;
-        p.off_q = pl.off_q;
-        p.q_bytes = pl.q_bytes;
-        p.off_ring = pl.off_ring;
-        p.slot_bytes = pl.slot_bytes;
-        p.off_stage = pl.off_stage;
-        p.stage_entry_bytes = pl.stage_entry_bytes;
-        p.off_score = pl.off_score;
-        p.off_bar = pl.off_bar;
-        p.smem_bytes = pl.smem_bytes;
-    };
-    const int grid = std::min(pl.grid, pl.ctas_per_sm * nsm);
-    cudaError_t e;
-    if (pl.wide) {
-        wide::AttnParams p;
-        fill(p);
-        p.nqbuf = pl.nqbuf;
-        p.nsbuf = pl.nsbuf;
-        p.tm_o = pl.tm_o;
-        p.tm_p = pl.tm_p;
-        e = wide::launch_attention(p, tq, tk, tv, grid, st);
-    } else {
-        AttnParams p;
-        fill(p);
-        p.shfl_group = pl.shfl_group ? 1 : 0;
-        p.tmem_cols = pl.tmem_cols;
-        p.sbufs = pl.sbufs;
-        p.qbufs = pl.qbufs;
-        p.off_topk = pl.off_topk;
-        e = launch_attention(p, tq, tk, tv, grid, st);
-    }
-    return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA;
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.tiles = reinterpret_cast<const AttnTile*>(ws + kWsHeader);
+    p.num_tiles = (int)pl.tiles.size();
+    p.err = reinterpret_cast<int*>(ws);
+    p.score_gmem = pl.score_in_smem ? nullptr
+                                    : reinterpret_cast<float*>(ws + kWsHeader + ((pl.ws_tiles + 255) & ~(size_t)255));
+    p.score_cap = pl.score_cap;
+    p.score_in_smem = pl.score_in_smem ? 1 : 0;
+    p.out = attention_out;
+    p.topk = topk_indices;
+    p.smax = softmax_max;
+    p.ssum = softmax_sum;
+    p.dtype = dtype == NSA_BF16 ? 0 : 1;
+    p.n1 = head_num;
+    p.n2 = n2;
+    p.d1 = d1;
+    p.d2 = d2;
+    p.G = pl.G;
+    p.tok_per_tile = pl.TT;
+    p.l = l;
+    p.d = d;
+    p.lp = lp;
+    p.count = count;
+    p.a = pl.a;
+    p.b = pl.b;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.nkv_cols = pl.nkv_cols;
+    p.nslot = pl.nslot;
+    p.nqbuf = pl.nqbuf;
+    p.nsbuf = pl.nsbuf;
+    p.tm_o = pl.tm_o;
+    p.tm_p = pl.tm_p;
+    p.off_q = pl.off_q;
+    p.q_bytes = pl.q_bytes;
+    p.off_ring = pl.off_ring;
+    p.slot_bytes = pl.slot_bytes;
+    p.off_stage = pl.off_stage;
+    p.stage_entry_bytes = pl.stage_entry_bytes;
+    p.off_score = pl.off_score;
+    p.off_bar = pl.off_bar;
+    p.smem_bytes = pl.smem_bytes;
+    const int grid = std::min(pl.grid, nsm);
+    if (launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
 }
 
 nsa_status_t nsa_workspace_status(const void* workspace, void* stream) {

@@ -39,71 +39,6 @@ cudaError_t launch_compress(const CompressParams& p, dim3 grid, int threads, siz
 cudaError_t read_compress_error(int* out, cudaStream_t st);
 
 // ----------------------------------------------------------- attention
-// Warp roles: warps 0-3 softmax (one TMEM lane quadrant each), warp 4 TMA
-// producer, warp 5 MMA issuer, warps 6-7 epilogue.  Up to two CTAs share an
-// SM, each launched at 128 registers per thread (2 x 256 x 128 = 65536); the
-// softmax warpgroup then grows to 152 and the other warpgroup shrinks to 104,
-// whose sum x 128 threads is the same 32768 per CTA.
-constexpr int kAttnThreads = 256;
-constexpr int kRegsLaunch = 128;
-constexpr int kRegsSoftmax = 152;
-constexpr int kRegsSide = 104;
-static_assert((kRegsSoftmax + kRegsSide) * 128 <= kAttnThreads * kRegsLaunch,
-              "register split exceeds the launch allocation");
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
-constexpr int kWarpEpi0 = 6;
-constexpr int kEpiWarps = 2;
-constexpr int kRows = 128;          // M of one tile: (tokens x heads of one KV group)
-constexpr int kEntryMax = 8;        // importance anchors per staging entry
-constexpr int kTopkCap = 128;       // top-k survivors per epilogue warp (shared-memory scratch)
-
-// One M-tile: up to 128/G consecutive query tokens of one sequence x the G
-// heads of one KV group.
-struct AttnTile {
-    int q_row0;     // first query row (T1 index)
-    int ntok;       // tokens in the tile (<= tokens per tile)
-    int group;      // KV head g
-    int cmp_row0;   // first compressed row of the sequence (Tc index)
-    int n_cmp;      // compressed blocks of the sequence
-    int n_sel;      // selection blocks of the sequence
-    int t0;         // position of the first token (query offset applied)
-    int nkv;        // KV tiles to visit (each pass)
-};
-
-struct AttnParams {
-    const AttnTile* tiles;
-    int num_tiles;
-    int* err;               // device error word (workspace)
-    float* score_gmem;      // per-CTA score buffers when they do not fit on chip
-    int score_cap;          // floats per token in a score buffer
-    int score_in_smem;
-    int shfl_group;         // 1: G is a power of two <= 32, group sums by warp shuffles
-    void* out;
-    int32_t* topk;
-    float* smax;
-    float* ssum;
-    int dtype;              // 0 bf16, 1 fp16
-    int n1, n2, d1, d2, G, tok_per_tile;
-    int l, d, lp, count, a, b;
-    float scale_log2;       // scale * log2(e)
-    int nkv_cols;           // compressed blocks per KV tile
-    int nslot;              // K/V ring depth
-    int tmem_cols;          // tensor-memory columns per CTA (256 or 512)
-    int sbufs;              // score buffers in tensor memory (1 or 2)
-    int qbufs;              // Q buffers in shared memory (1 or 2)
-    // shared-memory layout (byte offsets from a 1024-aligned base)
-    int off_q, q_bytes, off_ring, slot_bytes, off_stage, stage_entry_bytes, off_score, off_topk,
-        off_bar, smem_bytes;
-};
-
-cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, int grid, cudaStream_t st);
-int attention_kv_cols(int a);   // compressed blocks per KV tile for band factor a
-
-// --------------------------------------------- attention, one CTA per SM
-// The kernel of nsa_attention_wide.cu.  It takes the same tile list.
-namespace wide {
 // Warp roles: warps 0-3 softmax (TMEM lanes 32w..32w+31), warps 4-7 epilogue
 // (group sum, output, top-k), warp 8 TMA producer, warp 9 MMA issuer, warps
 // 10-11 idle.  Launched at 168 registers per thread (384 x 168 = 64512); the
@@ -115,7 +50,21 @@ constexpr int kRegsEpilogue = 152;
 constexpr int kRegsCtl = 120;
 static_assert((kRegsSoftmax + kRegsEpilogue + kRegsCtl) * 128 <= kAttnThreads * 168,
               "register split exceeds the launch allocation");
+constexpr int kRows = 128;          // M of one tile: (tokens x heads of one KV group)
 constexpr int kEntryMax = 32;       // importance anchors per staging entry
+
+// One M-tile: up to 128/G consecutive query tokens of one sequence x the G
+// heads of one KV group.
+struct AttnTile {
+    int q_row0;     // first query row (T1 index)
+    int ntok;       // tokens in the tile (<= tokens per tile)
+    int group;      // KV head g
+    int cmp_row0;   // first compressed row of the sequence (Tc index)
+    int n_cmp;      // compressed blocks of the sequence
+    int n_sel;      // selection blocks of the sequence
+    int t0;         // position of the first token (query offset applied)
+    int nkv;        // KV tiles to visit (both passes)
+};
 
 struct AttnParams {
     const AttnTile* tiles;
@@ -144,6 +93,6 @@ struct AttnParams {
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, int grid, cudaStream_t st);
-}  // namespace wide
+int attention_kv_cols(int a);   // compressed blocks per KV tile for band factor a
 
 }  // namespace nsa

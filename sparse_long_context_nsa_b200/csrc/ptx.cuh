@@ -246,14 +246,6 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
 #pragma unroll
     for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
-// N consecutive columns (N a multiple of 8) from r[0..N).
-template <int N>
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* r) {
-    static_assert(N % 8 == 0, "columns in steps of 8");
-#pragma unroll
-    for (int k = 0; k < N / 16; ++k) tmem_st16(taddr + 16 * k, r + 16 * k);
-    if constexpr (N % 16 != 0) tmem_st8(taddr + N - 8, r + N - 8);
-}
 // Packed fp32 pairs (sm_100): two lanes of arithmetic per instruction.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     uint64_t d;
@@ -283,12 +275,6 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-// Moves this warpgroup from the launch budget LAUNCH to N registers per thread.
-template <int N, int LAUNCH>
-__device__ __forceinline__ void setmaxnreg_to() {
-    if constexpr (N > LAUNCH) setmaxnreg_inc<N>();
-    else if constexpr (N < LAUNCH) setmaxnreg_dec<N>();
 }
 __device__ __forceinline__ float lg2(float x) {
     float y;

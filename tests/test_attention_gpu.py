@@ -14,17 +14,6 @@ from parity import check_attention
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["auto", "1", "2"], autouse=True, ids=lambda v: f"ctas{v}")
-def ctas_per_sm(request, monkeypatch):
-    """Every case runs with the plan's own kernel choice and with each layout
-    forced (one or two CTAs per SM; a layout that does not fit falls back)."""
-    if request.param == "auto":
-        monkeypatch.delenv("NSA_ATTN_CTAS_PER_SM", raising=False)
-    else:
-        monkeypatch.setenv("NSA_ATTN_CTAS_PER_SM", request.param)
-    return request.param
-
-
 @pytest.fixture(scope="module")
 def nsa():
     from sparse_long_context_nsa_b200 import _build

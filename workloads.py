@@ -138,8 +138,8 @@ SHORTQ_4x64K = Workload("compress_t262144_shortq_4x128_n64_n8_d128",
                         128 ** -0.5, "bf16", seed=4, q_last=128)
 
 # A profiling case, not one of the benchmark's configurations: the shape of the
-# 16K workload at twice the length, so that the M-tiles visit enough KV tiles
-# for the two-CTA attention kernel while the device footprint stays near 1 GB.
+# 16K workload at twice the length (M-tiles visit twice as many KV tiles), with
+# a device footprint near 1 GB, small enough for a full ncu capture.
 PROFILE_32K = Workload("single_s32768_n64_n4_d128", (32768,), 64, 4, 128, 128,
                        32, 16, 64, 16, 128 ** -0.5, "bf16", seed=5)
 
