@@ -79,6 +79,13 @@ def _load():
             ctypes.c_void_p]
         lib.oracle_compress_attention.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_select_attention.argtypes = [
+            _f64p, _f64p, _f64p, _i32p, ctypes.c_double,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _i32p, _i32p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+            _f64p, _f64p]
+        lib.oracle_select_attention.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
         return lib
@@ -208,3 +215,47 @@ def compress_attention(q, kcmp, vcmp, scale: float, l: int, d: int, lp: int,
             raise ValueError("oracle: l % d and l' % d must be 0")
     return {"out": out, "softmax_max": smax, "softmax_sum": ssum, "topk": tk,
             "score": score, "ncand": ncand, "rows": rows_arr}
+
+
+def select_attention(q, k, v, sel, scale: float, lp: int, count: int, cu_seqlens_q,
+                     cu_seqlens_kv, rows=None, q_rows_only: bool = False):
+    """Selection attention over the l'-token KV blocks listed per (query row,
+    KV group) in ``sel`` ("lite_boost.ops.rain_fusion_attention": index lists,
+    causal mask, GQA; fed with the top-k of the compressed branch).
+
+    q (T1, N1, D1), k (T2, N2, D1), v (T2, N2, D2): values of the storage-dtype
+    tensors; sel (T1, N2, count) int32 over all query rows.  ``rows`` /
+    ``q_rows_only`` as in compress_attention.  Returns a dict with out
+    (R, N1, D2) and lse (R, N1).
+    """
+    qf, kf, vf = _f64(q), _f64(k), _f64(v)
+    _, n1, d1 = qf.shape
+    t2, n2, d1k = kf.shape
+    d2 = vf.shape[2]
+    assert d1k == d1 and vf.shape[:2] == (t2, n2)
+    sl = np.ascontiguousarray(np.asarray(sel, dtype=np.int32))
+    assert sl.shape[1:] == (n2, count)
+    cq, ck = _i32(cu_seqlens_q), _i32(cu_seqlens_kv)
+    batch = cq.size
+    if q_rows_only and rows is None:
+        raise ValueError("q_rows_only needs rows")
+    if rows is None:
+        rows_arr = np.arange(int(cq[-1]) if batch else 0, dtype=np.int64)
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    R = rows_arr.size
+    out = np.zeros((R, n1, d2))
+    lse = np.zeros((R, n1))
+    if kf.size == 0:
+        kf = np.zeros(1)
+    if vf.size == 0:
+        vf = np.zeros(1)
+    if sl.size == 0:
+        sl = np.zeros(1, dtype=np.int32)
+    if R > 0:
+        rc = _load().oracle_select_attention(
+            qf, kf, vf, sl, float(scale), n1, n2, d1, d2, int(lp), int(count), cq, ck, batch,
+            rows_arr.ctypes.data_as(ctypes.c_void_p), R, 1 if q_rows_only else 0, out, lse)
+        if rc != 0:
+            raise ValueError("oracle: bad selection-attention arguments")
+    return {"out": out, "lse": lse, "rows": rows_arr}

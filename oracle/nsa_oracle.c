@@ -11,7 +11,9 @@
  *          description, the note list (TND layout, prefix-sum lengths,
  *          constraints) and the Returns list (output shapes).
  *   [RFA]  "lite_boost.ops.rain_fusion_attention" -- select_idx parameter:
- *          valid indices listed in ascending order first, then -1 padding.
+ *          valid indices listed in ascending order first, then -1 padding;
+ *          block-sparse attention over the listed KV blocks, causal mask
+ *          (mask_type 0), GQA, attention_out and softmax_lse returns.
  *
  * Readings taken where the pages are silent or garbled (each one is listed in
  * the design notes of this repository):
@@ -297,6 +299,103 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
             }
         }
         free(sc); free(P); free(pslc); free(grp);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Selection attention ([RFA], block-sparse attention driven by index lists), */
+/* in the reading that feeds it with the top-k of the compressed branch:       */
+/* query row t_loc of sequence b sits at key position                          */
+/* t = t_loc + (S_kv - S_q) (bottom-right alignment); for head h of group      */
+/* g = h / G it attends to the raw keys p of the selection blocks listed for   */
+/* (t, g) in sel (block j holds positions j*l' .. j*l'+l'-1), restricted to    */
+/* p <= t (causal, mask_type 0) and p < S_kv.  The list is read as a set:      */
+/* -1 entries, blocks past the end of the sequence and repeats are skipped.    */
+/*   out[t,h,:] = sum_p softmax_p(scale * q . k_p) v_p                         */
+/*   lse[t,h]   = m + log(sum_p exp(s_p - m))   (natural log)                  */
+/* An empty key set gives out = 0 and lse = -inf.                              */
+/*  q (T1,N1,D1) or (nrows,N1,D1) when q_compact; k (T2,N2,D1); v (T2,N2,D2);  */
+/*  sel (T1,N2,count) int32 over all query rows; cu_q / cu_kv prefix sums;     */
+/*  rows: global query rows to evaluate (NULL = all); out (nrows,N1,D2);       */
+/*  lse (nrows,N1).                                                            */
+/* ------------------------------------------------------------------------- */
+int oracle_select_attention(const double* q, const double* k, const double* v,
+                            const int32_t* sel, double scale, int n1, int n2,
+                            int d1, int d2, int lp, int count,
+                            const int32_t* cu_q, const int32_t* cu_kv, int batch,
+                            const int64_t* rows, int64_t nrows, int q_compact,
+                            double* out, double* lse)
+{
+    if (lp <= 0 || n2 <= 0 || n1 % n2 != 0) return -1;
+    const int G = n1 / n2;
+    if (rows == NULL) nrows = cu_q[batch - 1];
+
+    #pragma omp parallel
+    {
+        int64_t max_kv = 0;
+        for (int s = 0; s < batch; s++) {
+            int64_t n = cu_kv[s] - (s ? cu_kv[s - 1] : 0);
+            if (n > max_kv) max_kv = n;
+        }
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)(max_kv + 1));
+        double* sc = (double*)malloc(sizeof(double) * (size_t)(max_kv + 1));
+
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < nrows; r++) {
+            int64_t t = rows ? rows[r] : r;
+            int s = 0;
+            while (cu_q[s] <= t) s++;
+            int64_t q0 = s ? cu_q[s - 1] : 0;
+            int64_t k0 = s ? cu_kv[s - 1] : 0;
+            int64_t Sq = cu_q[s] - q0;
+            int64_t Skv = cu_kv[s] - k0;
+            int64_t tpos = (t - q0) + (Skv - Sq);
+            int64_t n_blk = (Skv + lp - 1) / lp;
+
+            for (int g = 0; g < n2; g++) {
+                /* the key set of (t, g): listed blocks, each once, causal */
+                const int32_t* list = sel + (t * n2 + g) * (int64_t)count;
+                int64_t nk = 0;
+                for (int c = 0; c < count; c++) {
+                    int64_t j = list[c];
+                    if (j < 0 || j >= n_blk) continue;
+                    int seen = 0;
+                    for (int c2 = 0; c2 < c; c2++)
+                        if (list[c2] == list[c]) seen = 1;
+                    if (seen) continue;
+                    for (int64_t p = j * lp; p < (j + 1) * lp && p < Skv; p++)
+                        if (p <= tpos) keys[nk++] = p;
+                }
+                for (int hh = 0; hh < G; hh++) {
+                    int h = g * G + hh;
+                    double* o = out + (r * n1 + h) * (int64_t)d2;
+                    for (int e = 0; e < d2; e++) o[e] = 0.0;
+                    if (nk == 0) {
+                        lse[r * n1 + h] = -INFINITY;
+                        continue;
+                    }
+                    const double* qr = q + ((q_compact ? r : t) * n1 + h) * (int64_t)d1;
+                    for (int64_t i = 0; i < nk; i++) {
+                        const double* kr = k + ((k0 + keys[i]) * n2 + g) * (int64_t)d1;
+                        double acc = 0.0;
+                        for (int e = 0; e < d1; e++) acc += qr[e] * kr[e];
+                        sc[i] = scale * acc;
+                    }
+                    double m = sc[0];
+                    for (int64_t i = 1; i < nk; i++) if (sc[i] > m) m = sc[i];
+                    double L = 0.0;
+                    for (int64_t i = 0; i < nk; i++) L += exp(sc[i] - m);
+                    for (int64_t i = 0; i < nk; i++) {
+                        const double pw = exp(sc[i] - m) / L;
+                        const double* vr = v + ((k0 + keys[i]) * n2 + g) * (int64_t)d2;
+                        for (int e = 0; e < d2; e++) o[e] += pw * vr[e];
+                    }
+                    lse[r * n1 + h] = m + log(L);
+                }
+            }
+        }
+        free(keys); free(sc);
     }
     return 0;
 }
