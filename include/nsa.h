@@ -7,7 +7,9 @@
  *   nsa_compress_attention  causal GQA attention over the compressed blocks,
  *                           importance scores, head-group sum and per-query
  *                           top-k of selection blocks
- *                           ("mindspore.ops.nsa_compress_attention", steps 1-7).
+ *                           ("mindspore.ops.nsa_compress_attention", steps 1-7);
+ *   nsa_select_attention    attention over the raw K/V blocks that top-k lists
+ *                           ("lite_boost.ops.rain_fusion_attention").
  *
  * Conventions shared by every entry point
  *   - Layout is TND ("mindspore.ops.nsa_compress_attention", note list):
@@ -144,8 +146,54 @@ nsa_status_t nsa_compress_attention(
     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of device workspace nsa_select_attention needs for these shapes
+ * (same arguments; a pure host computation).
+ */
+nsa_status_t nsa_select_attention_workspace_size(
+    int head_num, int n2, int d1, int d2, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv, int batch, size_t* bytes);
+
+/*
+ * Selection attention: attention over the raw K/V blocks of l' tokens listed
+ * per (query row, KV group) -- the consumer of nsa_compress_attention's
+ * topk_indices ("lite_boost.ops.rain_fusion_attention": block-sparse
+ * attention over index lists that hold ascending valid block indices, then
+ * -1 padding; causal mask, mask_type 0; GQA; returns attention_out and
+ * softmax_lse).  Query row t_loc of sequence b sits at key position
+ * t = t_loc + (S_kv_b - S_q_b); for head h of group g = h / G it attends to
+ * the keys p of the blocks listed in topk_indices[t, g, :] (block j holds
+ * p = j*lp .. j*lp + lp - 1) with p <= t and p < S_kv_b:
+ *   attention_out[t,h,:] = sum_p softmax_p(scale * q[t,h,:] . k[p,g,:]) v[p,g,:]
+ *   softmax_lse[t,h]     = log sum_p exp(scale * q . k_p)  (natural log)
+ * The list is read as a set: -1 entries, blocks past the end of the
+ * sequence and repeats are skipped.  A row that attends to nothing gets
+ * attention_out = 0 and softmax_lse = -inf.
+ * Arguments
+ *   q             device (T1, N1, D1) dtype      k device (T2, N2, D1) dtype
+ *   v             device (T2, N2, D2) dtype
+ *   topk_indices  device (T1, N2, count) int32 (as written by nsa_compress_attention)
+ *   scale, head_num (N1), lp (block size l'), count (entries per list)
+ *   cu_seqlens_q, cu_seqlens_kv  host [batch] prefix sums (no leading 0)
+ *   attention_out device (T1, N1, D2) dtype      softmax_lse device (T1, N1) fp32
+ *   workspace     device, >= nsa_select_attention_workspace_size bytes,
+ *                 256-byte aligned; its first 16 bytes receive the device error
+ *                 word read by nsa_workspace_status
+ * Constraints: lp a multiple of 16 in [16, 128]; 1 <= count <= 32; D1, D2
+ * multiples of 16 (NSA_ERR_INVALID_ARG); D1 or D2 > 256, more than 128 query
+ * heads per KV group, or sequences of more than about 6.5e6 blocks
+ * (NSA_ERR_UNSUPPORTED).  Two launches on `stream`: a planning kernel that
+ * gathers each tile's union of listed blocks, then the attention kernel.
+ */
+nsa_status_t nsa_select_attention(
+    const void* q, const void* k, const void* v, const int32_t* topk_indices, float scale,
+    int head_num, int lp, int count, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+    int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+    void* attention_out, float* softmax_lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream` and reads the device error word of `workspace`
- * (written by the last nsa_compress_attention that used it).  Returns NSA_OK,
+ * (written by the last nsa_compress_attention or nsa_select_attention that
+ * used it).  Returns NSA_OK,
  * NSA_ERR_TIMEOUT when a device-side wait gave up, or NSA_ERR_CUDA.
  */
 nsa_status_t nsa_workspace_status(const void* workspace, void* stream);

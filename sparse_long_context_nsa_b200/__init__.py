@@ -36,6 +36,8 @@ EXPORTED = (
     "nsa_workspace_status",
     "nsa_compress_status",
     "nsa_compress_attention_noalloc",
+    "nsa_select_attention_workspace_size",
+    "nsa_select_attention",
 )
 
 _lib = None
@@ -86,6 +88,12 @@ def load(path: Optional[str] = None):
     lib.nsa_compress_attention_noalloc.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p,
                                                    i32p, i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
     lib.nsa_compress_attention_noalloc.restype = ci
+    lib.nsa_select_attention_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, i32p, i32p, ci,
+                                                        ctypes.POINTER(cs)]
+    lib.nsa_select_attention_workspace_size.restype = ci
+    lib.nsa_select_attention.argtypes = [vp, vp, vp, vp, ctypes.c_float, ci, ci, ci, i32p, i32p, ci, ci, ci,
+                                         ci, ci, vp, vp, vp, cs, vp]
+    lib.nsa_select_attention.restype = ci
     if path is None:
         _lib = lib
     return lib
@@ -283,3 +291,65 @@ def nsa_workspace_status(workspace: torch.Tensor, stream=None) -> int:
 
 def nsa_compress_status(stream=None) -> int:
     return int(load().nsa_compress_status(_stream(stream)))
+
+
+def nsa_select_attention_workspace_size(head_num: int, n2: int, d1: int, d2: int, lp: int, count: int,
+                                        cu_seqlens_q, cu_seqlens_kv) -> int:
+    cq, ck = _cu(cu_seqlens_q), _cu(cu_seqlens_kv)
+    if cq.size != ck.size:
+        raise ValueError("the two prefix-sum lists need one entry per sequence")
+    out = ctypes.c_size_t(0)
+    _raise(load().nsa_select_attention_workspace_size(
+        int(head_num), int(n2), int(d1), int(d2), int(lp), int(count), _ip(cq), _ip(ck), cq.size,
+        ctypes.byref(out)), "nsa_select_attention_workspace_size")
+    return int(out.value)
+
+
+def nsa_select_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_indices: torch.Tensor,
+                         scale: float, head_num: int, lp: int, cu_seqlens_q, cu_seqlens_kv, out=None,
+                         workspace: Optional[torch.Tensor] = None, stream=None):
+    """Attention over the l'-token K/V blocks listed in ``topk_indices``
+    (T1, N2, count) int32, as written by nsa_compress_attention.
+
+    Returns (attention_out (T1,N1,D2), softmax_lse (T1,N1) fp32); ``out`` may
+    pass both preallocated.
+    """
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (topk_indices, "topk_indices")):
+        _dev(t, nm)
+        if t.dim() != 3:
+            raise ValueError(f"{nm} must be 3-D")
+    dt = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if topk_indices.dtype != torch.int32 or not topk_indices.is_contiguous():
+        raise TypeError("topk_indices must be a contiguous int32 tensor")
+    t1, n1, d1 = q.shape
+    t2, n2, d1k = k.shape
+    d2 = v.shape[2]
+    count = topk_indices.shape[2]
+    if int(head_num) != n1:
+        raise ValueError("head_num must equal the number of query heads")
+    if d1k != d1 or tuple(v.shape[:2]) != (t2, n2):
+        raise ValueError("k must be (T2, N2, D1) and v (T2, N2, D2)")
+    if tuple(topk_indices.shape[:2]) != (t1, n2):
+        raise ValueError("topk_indices must be (T1, N2, count)")
+    cq, ck = _cu(cu_seqlens_q), _cu(cu_seqlens_kv)
+    if cq.size != ck.size:
+        raise ValueError("the two prefix-sum lists need one entry per sequence")
+    if int(cq[-1]) > t1 or int(ck[-1]) > t2:
+        raise ValueError("prefix sums run past the rows of q / k")
+    dev = q.device
+    if out is None:
+        att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
+        lse = torch.empty(t1, n1, dtype=torch.float32, device=dev)
+    else:
+        att, lse = out
+    ws_bytes = nsa_select_attention_workspace_size(n1, n2, d1, d2, lp, count, cq, ck)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st = load().nsa_select_attention(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), topk_indices.data_ptr(), float(scale), int(head_num),
+        int(lp), int(count), _ip(cq), _ip(ck), cq.size, n2, d1, d2, dt, att.data_ptr(), lse.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _raise(st, "nsa_select_attention")
+    return att, lse

@@ -230,6 +230,114 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
     return NSA_OK;
 }
 
+// ------------------------------------------------------------------------
+// selection-attention plan
+// ------------------------------------------------------------------------
+struct SelPlan {
+    int G = 0, TT = 0, cap = 1, max_words = 1, grid = 0;
+    std::vector<sel::Tile> tiles;
+    int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_p = 0;
+    int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_bar = 0, smem_bytes = 0;
+    size_t ws_tiles = 0, ws_n = 0, ws_blk = 0, ws_mask = 0, ws_total = 0;
+};
+
+nsa_status_t plan_select(int head_num, int n2, int d1, int d2, int lp, int count, const int32_t* cu_q,
+                         const int32_t* cu_kv, int batch, bool build_tiles, SelPlan& pl) {
+    // block shape of the index lists: l' (select_block_size of the compressed
+    // branch) keys per block; tiles of 16-column multiples for the MMA
+    if (lp % 16 || lp < 16 || lp > 128) return NSA_ERR_INVALID_ARG;
+    if (count < 1 || count > 32) return NSA_ERR_INVALID_ARG;
+    if (d1 < 16 || d2 < 16 || d1 % 16 || d2 % 16) return NSA_ERR_INVALID_ARG;
+    if (n2 < 1 || head_num < n2 || head_num % n2) return NSA_ERR_INVALID_ARG;
+    nsa_status_t s;
+    if ((s = check_prefix(cu_q, batch)) != NSA_OK) return s;
+    if ((s = check_prefix(cu_kv, batch)) != NSA_OK) return s;
+    if (d1 > 256 || d2 > 256) return NSA_ERR_UNSUPPORTED;
+    if (head_num / n2 > kRows) return NSA_ERR_UNSUPPORTED;
+    pl.G = head_num / n2;
+    pl.TT = kRows / pl.G;
+    int64_t ntiles = 0, max_blk = 1;
+    {
+        int32_t pq = 0, pk = 0;
+        for (int bq = 0; bq < batch; ++bq) {
+            const int64_t Sq = cu_q[bq] - pq, Skv = cu_kv[bq] - pk;
+            ntiles += ((Sq + pl.TT - 1) / pl.TT) * (int64_t)n2;
+            max_blk = std::max<int64_t>(max_blk, (Skv + lp - 1) / lp);
+            pq = cu_q[bq];
+            pk = cu_kv[bq];
+        }
+    }
+    if (ntiles > (int64_t)1 << 30) return NSA_ERR_UNSUPPORTED;
+    // the planning kernel keeps a bit map and a prefix word per 32 blocks on chip
+    pl.max_words = (int)((max_blk + 31) / 32);
+    if ((int64_t)pl.max_words * 8 > 200 * 1024) return NSA_ERR_UNSUPPORTED;
+    pl.cap = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)pl.TT * count, max_blk));
+
+    // tensor memory: S buffers (128 columns each), O, P (l'/2 columns)
+    const int d2c = (d2 + 31) & ~31;
+    pl.nsbuf = (256 + d2c + 64 <= 512) ? 2 : 1;
+    pl.tm_o = pl.nsbuf * 128;
+    pl.tm_p = pl.tm_o + d2c;
+    if (pl.tm_p + lp / 2 > 512) return NSA_ERR_UNSUPPORTED;
+    // shared memory: Q buffers and the K/V ring
+    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
+    pl.q_bytes = nqc * 16384;
+    pl.slot_bytes = std::max(nqc, nvc) * lp * 128;
+    auto layout = [&](int nq, int ns) {
+        int off = 0;
+        pl.off_q = off;
+        off += nq * pl.q_bytes;
+        pl.off_ring = off;
+        off += ns * pl.slot_bytes;
+        pl.off_bar = off;
+        off += 320;
+        pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
+        pl.nqbuf = nq;
+        pl.nslot = ns;
+        return pl.smem_bytes <= kSmemLimit;
+    };
+    static const int kOrder[][2] = {{2, 8}, {2, 6}, {2, 4}, {1, 4}, {2, 2}, {1, 2}};
+    bool fits = false;
+    for (const auto& o : kOrder)
+        if ((fits = layout(o[0], o[1]))) break;
+    if (!fits) return NSA_ERR_UNSUPPORTED;
+    // the kernel takes all 512 tensor-memory columns: keep a second CTA off the SM
+    pl.smem_bytes = std::max(pl.smem_bytes, 120 * 1024);
+    pl.grid = (int)std::min<int64_t>(ntiles, kMaxGrid);
+
+    if (build_tiles) {
+        pl.tiles.clear();
+        pl.tiles.reserve((size_t)ntiles);
+        int32_t pq = 0, pk = 0;
+        for (int bq = 0; bq < batch; ++bq) {
+            const int Sq = cu_q[bq] - pq, Skv = cu_kv[bq] - pk;
+            for (int tok0 = 0; tok0 < Sq; tok0 += pl.TT) {
+                sel::Tile t;
+                t.q_row0 = pq + tok0;
+                t.ntok = std::min(pl.TT, Sq - tok0);
+                t.kv_row0 = pk;
+                t.s_kv = Skv;
+                t.t0 = tok0 + (Skv - Sq);
+                t.n_blk = (Skv + lp - 1) / lp;
+                t.pad = 0;
+                for (int g = 0; g < n2; ++g) {
+                    t.group = g;
+                    pl.tiles.push_back(t);
+                }
+            }
+            pq = cu_q[bq];
+            pk = cu_kv[bq];
+        }
+    }
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    pl.ws_tiles = up((size_t)ntiles * sizeof(sel::Tile));
+    pl.ws_n = up((size_t)ntiles * 4);
+    pl.ws_blk = up((size_t)ntiles * pl.cap * 4);
+    pl.ws_mask = up((size_t)ntiles * pl.cap * 16);
+    pl.ws_total = kWsHeader + pl.ws_tiles + pl.ws_n + pl.ws_blk + pl.ws_mask;
+    return NSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -458,6 +566,92 @@ nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void*
     p.smem_bytes = pl.smem_bytes;
     const int grid = std::min(pl.grid, nsm);
     if (launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_select_attention_workspace_size(int head_num, int n2, int d1, int d2, int lp, int count,
+                                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+                                                 int batch, size_t* bytes) {
+    if (bytes == nullptr) return NSA_ERR_INVALID_ARG;
+    SelPlan pl;
+    nsa_status_t s = plan_select(head_num, n2, d1, d2, lp, count, cu_seqlens_q, cu_seqlens_kv, batch, false, pl);
+    if (s != NSA_OK) return s;
+    *bytes = pl.ws_total;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_select_attention(const void* q, const void* k, const void* v, const int32_t* topk_indices,
+                                  float scale, int head_num, int lp, int count, const int32_t* cu_seqlens_q,
+                                  const int32_t* cu_seqlens_kv, int batch, int n2, int d1, int d2,
+                                  nsa_dtype_t dtype, void* attention_out, float* softmax_lse, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !topk_indices || !attention_out || !softmax_lse) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(attention_out) ||
+        (reinterpret_cast<uintptr_t>(topk_indices) & 3u) || (reinterpret_cast<uintptr_t>(softmax_lse) & 3u))
+        return NSA_ERR_INVALID_ARG;
+    SelPlan pl;
+    nsa_status_t s = plan_select(head_num, n2, d1, d2, lp, count, cu_seqlens_q, cu_seqlens_kv, batch, true, pl);
+    if (s != NSA_OK) return s;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < pl.ws_total)
+        return NSA_ERR_WORKSPACE;
+    if (pl.tiles.empty()) return NSA_OK;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t t1 = cu_seqlens_q[batch - 1];
+    const int64_t t2 = cu_seqlens_kv[batch - 1];
+    CUtensorMap tq, tk, tv;
+    if (!encode_tnd(&tq, q, dtype, d1, head_num, t1, pl.G, pl.TT) ||
+        !encode_tnd(&tk, k, dtype, d1, n2, t2, 1, lp) || !encode_tnd(&tv, v, dtype, d2, n2, t2, 1, lp))
+        return NSA_ERR_UNSUPPORTED;
+
+    // workspace: [header: error word][tiles][list counts][list blocks][list masks]
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    std::vector<uint8_t> host(kWsHeader + pl.tiles.size() * sizeof(sel::Tile), 0);
+    std::memcpy(host.data() + kWsHeader, pl.tiles.data(), pl.tiles.size() * sizeof(sel::Tile));
+    if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+
+    sel::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.tiles = reinterpret_cast<const sel::Tile*>(ws + kWsHeader);
+    p.num_tiles = (int)pl.tiles.size();
+    p.err = reinterpret_cast<int*>(ws);
+    p.topk = topk_indices;
+    p.count = count;
+    p.list_n = reinterpret_cast<int*>(ws + kWsHeader + pl.ws_tiles);
+    p.list_blk = reinterpret_cast<int32_t*>(ws + kWsHeader + pl.ws_tiles + pl.ws_n);
+    p.list_mask = reinterpret_cast<uint32_t*>(ws + kWsHeader + pl.ws_tiles + pl.ws_n + pl.ws_blk);
+    p.cap = pl.cap;
+    p.out = attention_out;
+    p.lse = softmax_lse;
+    p.dtype = dtype == NSA_BF16 ? 0 : 1;
+    p.n1 = head_num;
+    p.n2 = n2;
+    p.d1 = d1;
+    p.d2 = d2;
+    p.G = pl.G;
+    p.tok_per_tile = pl.TT;
+    p.lp = lp;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.nslot = pl.nslot;
+    p.nqbuf = pl.nqbuf;
+    p.nsbuf = pl.nsbuf;
+    p.tm_o = pl.tm_o;
+    p.tm_p = pl.tm_p;
+    p.off_q = pl.off_q;
+    p.q_bytes = pl.q_bytes;
+    p.off_ring = pl.off_ring;
+    p.slot_bytes = pl.slot_bytes;
+    p.off_bar = pl.off_bar;
+    p.smem_bytes = pl.smem_bytes;
+    if (sel::launch_plan(p, pl.max_words, st) != cudaSuccess) return NSA_ERR_CUDA;
+    const int grid = std::min(pl.grid, nsm);
+    if (sel::launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
     return NSA_OK;
 }
 

@@ -95,4 +95,54 @@ cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const C
                              const CUtensorMap& tv, int grid, cudaStream_t st);
 int attention_kv_cols(int a);   // compressed blocks per KV tile for band factor a
 
+// ------------------------------------------------ selection attention
+// Attention over the raw K/V blocks of l' tokens that the compressed branch's
+// top-k lists per (query row, KV group).  Same warp roles and register split
+// as the compressed-attention kernel.
+namespace sel {
+constexpr int kThreads = 384;
+constexpr int kRegsSoftmax = 232;
+constexpr int kRegsEpilogue = 152;
+constexpr int kRegsCtl = 120;
+constexpr int kPlanThreads = 256;
+
+// One M-tile: up to 128/G consecutive query tokens of one sequence x the G
+// heads of one KV group.
+struct Tile {
+    int q_row0;     // first query row (T1 index)
+    int ntok;       // tokens in the tile
+    int group;      // KV head g
+    int kv_row0;    // first raw K/V row of the sequence (T2 index)
+    int s_kv;       // K/V length of the sequence
+    int t0;         // key position of the first token (bottom-right alignment)
+    int n_blk;      // selection blocks of the sequence: ceil(s_kv / l')
+    int pad;
+};
+
+struct Params {
+    const Tile* tiles;
+    int num_tiles;
+    int* err;                   // device error word (workspace)
+    const int32_t* topk;        // (T1, N2, count) block lists
+    int count;
+    int* list_n;                // per tile: blocks in the union of its tokens' lists
+    int32_t* list_blk;          // per tile: cap block indices, ascending
+    uint32_t* list_mask;        // per tile: cap x 4 words, bit tau = token tau listed the block
+    int cap;                    // list capacity per tile
+    void* out;
+    float* lse;
+    int dtype;                  // 0 bf16, 1 fp16
+    int n1, n2, d1, d2, G, tok_per_tile, lp;
+    float scale_log2;           // scale * log2(e)
+    int nslot, nqbuf, nsbuf;    // K/V ring depth, Q buffers, S buffers
+    int tm_o, tm_p;             // tensor-memory columns of O and of P
+    // shared-memory layout (byte offsets from a 1024-aligned base)
+    int off_q, q_bytes, off_ring, slot_bytes, off_bar, smem_bytes;
+};
+
+cudaError_t launch_plan(const Params& p, int max_words, cudaStream_t st);
+cudaError_t launch_attention(const Params& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, int grid, cudaStream_t st);
+}  // namespace sel
+
 }  // namespace nsa
