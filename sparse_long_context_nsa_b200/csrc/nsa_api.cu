@@ -236,7 +236,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
 struct SelPlan {
     int G = 0, TT = 0, cap = 1, max_words = 1, grid = 0;
     std::vector<sel::Tile> tiles;
-    int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_p = 0;
+    int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_s = 0, s_stride = 0;
     int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_bar = 0, smem_bytes = 0;
     size_t ws_tiles = 0, ws_n = 0, ws_blk = 0, ws_mask = 0, ws_total = 0;
 };
@@ -273,16 +273,19 @@ nsa_status_t plan_select(int head_num, int n2, int d1, int d2, int lp, int count
     if ((int64_t)pl.max_words * 8 > 200 * 1024) return NSA_ERR_UNSUPPORTED;
     pl.cap = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)pl.TT * count, max_blk));
 
-    // tensor memory: S buffers (128 columns each), O, P (l'/2 columns)
-    const int d2c = (d2 + 31) & ~31;
-    pl.nsbuf = (256 + d2c + 64 <= 512) ? 2 : 1;
-    pl.tm_o = pl.nsbuf * 128;
-    pl.tm_p = pl.tm_o + d2c;
-    if (pl.tm_p + lp / 2 > 512) return NSA_ERR_UNSUPPORTED;
+    // tensor memory: O (d2 columns), then up to kMaxSBuf score buffers of one
+    // KV tile each (P is written over the first half of its buffer), all at
+    // 32-column boundaries
+    pl.tm_o = 0;
+    pl.tm_s = (d2 + 31) & ~31;
+    const int nkv_keys = sel::blocks_per_tile(lp) * lp;     // keys per KV tile
+    pl.s_stride = (nkv_keys + 31) & ~31;
+    pl.nsbuf = std::min(sel::kMaxSBuf, (512 - pl.tm_s) / pl.s_stride);
+    if (pl.nsbuf < 2) return NSA_ERR_UNSUPPORTED;
     // shared memory: Q buffers and the K/V ring
     const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
     pl.q_bytes = nqc * 16384;
-    pl.slot_bytes = std::max(nqc, nvc) * lp * 128;
+    pl.slot_bytes = std::max(nqc, nvc) * nkv_keys * 128;
     auto layout = [&](int nq, int ns) {
         int off = 0;
         pl.off_q = off;
@@ -290,7 +293,7 @@ nsa_status_t plan_select(int head_num, int n2, int d1, int d2, int lp, int count
         pl.off_ring = off;
         off += ns * pl.slot_bytes;
         pl.off_bar = off;
-        off += 320;
+        off += sel::kBarBytes;
         pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
         pl.nqbuf = nq;
         pl.nslot = ns;
@@ -308,25 +311,28 @@ nsa_status_t plan_select(int head_num, int n2, int d1, int d2, int lp, int count
     if (build_tiles) {
         pl.tiles.clear();
         pl.tiles.reserve((size_t)ntiles);
-        int32_t pq = 0, pk = 0;
-        for (int bq = 0; bq < batch; ++bq) {
-            const int Sq = cu_q[bq] - pq, Skv = cu_kv[bq] - pk;
-            for (int tok0 = 0; tok0 < Sq; tok0 += pl.TT) {
-                sel::Tile t;
-                t.q_row0 = pq + tok0;
-                t.ntok = std::min(pl.TT, Sq - tok0);
-                t.kv_row0 = pk;
-                t.s_kv = Skv;
-                t.t0 = tok0 + (Skv - Sq);
-                t.n_blk = (Skv + lp - 1) / lp;
-                t.pad = 0;
-                for (int g = 0; g < n2; ++g) {
+        // KV group outermost: the CTAs run neighbouring tiles at the same
+        // time, and these then read the blocks of one group's K/V, which
+        // stays in L2 while they do
+        for (int g = 0; g < n2; ++g) {
+            int32_t pq = 0, pk = 0;
+            for (int bq = 0; bq < batch; ++bq) {
+                const int Sq = cu_q[bq] - pq, Skv = cu_kv[bq] - pk;
+                for (int tok0 = 0; tok0 < Sq; tok0 += pl.TT) {
+                    sel::Tile t;
+                    t.q_row0 = pq + tok0;
+                    t.ntok = std::min(pl.TT, Sq - tok0);
                     t.group = g;
+                    t.kv_row0 = pk;
+                    t.s_kv = Skv;
+                    t.t0 = tok0 + (Skv - Sq);
+                    t.n_blk = (Skv + lp - 1) / lp;
+                    t.pad = 0;
                     pl.tiles.push_back(t);
                 }
+                pq = cu_q[bq];
+                pk = cu_kv[bq];
             }
-            pq = cu_q[bq];
-            pk = cu_kv[bq];
         }
     }
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -642,7 +648,8 @@ nsa_status_t nsa_select_attention(const void* q, const void* k, const void* v, c
     p.nqbuf = pl.nqbuf;
     p.nsbuf = pl.nsbuf;
     p.tm_o = pl.tm_o;
-    p.tm_p = pl.tm_p;
+    p.tm_s = pl.tm_s;
+    p.s_stride = pl.s_stride;
     p.off_q = pl.off_q;
     p.q_bytes = pl.q_bytes;
     p.off_ring = pl.off_ring;

@@ -100,11 +100,13 @@ int attention_kv_cols(int a);   // compressed blocks per KV tile for band factor
 // top-k lists per (query row, KV group).  Same warp roles and register split
 // as the compressed-attention kernel.
 namespace sel {
-constexpr int kThreads = 384;
-constexpr int kRegsSoftmax = 232;
-constexpr int kRegsEpilogue = 152;
-constexpr int kRegsCtl = 120;
+constexpr int kThreads = 192;      // warps 0-3 softmax + output, 4 TMA, 5 MMA
+constexpr int kMaxSBuf = 8;        // score buffers in tensor memory
+constexpr int kBarBytes = 512;     // mbarriers, tensor-memory address, abort flag
 constexpr int kPlanThreads = 256;
+// listed blocks of lp keys placed side by side in one KV tile: 128 keys when
+// lp divides 128, else one block per tile
+constexpr int blocks_per_tile(int lp) { return (128 % lp == 0) ? 128 / lp : 1; }
 
 // One M-tile: up to 128/G consecutive query tokens of one sequence x the G
 // heads of one KV group.
@@ -135,7 +137,8 @@ struct Params {
     int n1, n2, d1, d2, G, tok_per_tile, lp;
     float scale_log2;           // scale * log2(e)
     int nslot, nqbuf, nsbuf;    // K/V ring depth, Q buffers, S buffers
-    int tm_o, tm_p;             // tensor-memory columns of O and of P
+    int tm_o;                   // tensor-memory column of O (d2 columns)
+    int tm_s, s_stride;         // column of score buffer 0, columns between buffers
     // shared-memory layout (byte offsets from a 1024-aligned base)
     int off_q, q_bytes, off_ring, slot_bytes, off_bar, smem_bytes;
 };

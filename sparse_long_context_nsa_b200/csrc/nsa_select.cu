@@ -15,16 +15,16 @@
 //   sel_plan_kernel  one CTA per M-tile (128/G tokens x the G heads of one KV
 //                    group): the union of the tiles' listed blocks, ascending,
 //                    and per block a bit mask of the tokens that listed it.
-//   sel_attn_kernel  the two-pass tcgen05 attention of nsa_attention.cu over
-//                    those blocks (one KV tile of l' keys per listed block):
-//                    pass A exact max / sum per row and softmax_lse, pass B
-//                    P = 2^(s*scale*log2e - m - log2 L) into tensor memory and
-//                    O += P V; a row masks the columns of a block it did not
-//                    list, and the causal / sequence-end columns.
-// Warp roles as in nsa_attention.cu (384 threads): warps 0-3 softmax, warps
-// 4-7 epilogue (O read-out), warp 8 TMA producer, warp 9 MMA issuer (and
-// tensor-memory owner), warps 10-11 idle.  Every mbarrier wait is bounded; a
-// timeout sets the workspace error word and every role drains.
+//   sel_attn_kernel  tcgen05 attention over those blocks, one KV tile of l'
+//                    keys per listed block, with a one-pass online softmax:
+//                    S = Q K^T into tensor memory, P = 2^(s*scale*log2e - m)
+//                    written back over S, O += P V; a row masks the columns
+//                    of a block it did not list and the causal / sequence-end
+//                    columns; O / L and softmax_lse at the end of the tile.
+// Warp roles (192 threads): warps 0-3 softmax and output (one tile row per
+// thread), warp 4 TMA producer, warp 5 MMA issuer and tensor-memory owner.
+// Every mbarrier wait is bounded; a timeout sets the workspace error word and
+// every role drains.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -37,19 +37,19 @@ namespace nsa {
 namespace sel {
 
 enum BarId {
-    B_Q_FULL0 = 0,                    // + Q buffer (2)
-    B_Q_EMPTY0 = B_Q_FULL0 + 2,       // + Q buffer (2)
-    B_S_FULL0 = B_Q_EMPTY0 + 2,       // + score buffer (2)
-    B_S_EMPTY0 = B_S_FULL0 + 2,       // + score buffer (2)
-    B_P_FULL = B_S_EMPTY0 + 2,
-    B_P_EMPTY,
-    B_O_FULL,
+    B_Q_FULL0 = 0,                        // + Q buffer (2)
+    B_Q_EMPTY0 = B_Q_FULL0 + 2,           // + Q buffer (2)
+    B_S_FULL0 = B_Q_EMPTY0 + 2,           // + score buffer: S = Q K^T landed
+    B_S_EMPTY0 = B_S_FULL0 + kMaxSBuf,    // + score buffer: the P V reading it retired
+    B_P_FULL0 = B_S_EMPTY0 + kMaxSBuf,    // + score buffer: P written (4 warps)
+    B_O_FULL = B_P_FULL0 + kMaxSBuf,
     B_O_EMPTY,
     B_MMA_DONE,
-    B_SLOT_FULL0,                     // + slot (8)
+    B_SLOT_FULL0,                         // + slot (8)
     B_SLOT_EMPTY0 = B_SLOT_FULL0 + 8,
     B_COUNT = B_SLOT_EMPTY0 + 8
 };
+static_assert(8 * B_COUNT + 8 <= kBarBytes, "barrier area");
 
 template <typename T>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi);
@@ -146,13 +146,25 @@ cudaError_t launch_plan(const Params& p, int max_words, cudaStream_t st) {
 
 // ---------------------------------------------------------------------------
 // Attention over the listed blocks.  LP = l' keys per KV tile.
+//
+// One pass with an online softmax per row.  The row's reference maximum m
+// moves up only when a block's maximum exceeds it by more than 8 (exponent
+// units, base 2): P = 2^(x - m) then stays at most 2^8, and O and L are
+// rescaled by 2^(m_old - m_new) only at those moves.  O / L and the
+// log-sum-exp are formed once per tile.  P is written, in the storage dtype,
+// over the first l'/2 columns of the score buffer it came from; the buffer is
+// reused once the P V that reads it has retired.  A warp none of whose rows
+// attend to a block skips the exponentials and writes zero P.
 // ---------------------------------------------------------------------------
 template <typename T, int LP>
 __global__ void __launch_bounds__(kThreads, 1)
 sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    constexpr int NKV = LP;
+    // BPT listed blocks side by side in one KV tile of NKV keys
+    constexpr int BPT = blocks_per_tile(LP);
+    constexpr int NKV = BPT * LP;
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr int kWarpTma = 4, kWarpMma = 5;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,11 +182,12 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(B_Q_FULL0 + i), 1);
             mbar_init(bar(B_Q_EMPTY0 + i), 1);
-            mbar_init(bar(B_S_FULL0 + i), 1);
-            mbar_init(bar(B_S_EMPTY0 + i), 4);
         }
-        mbar_init(bar(B_P_FULL), 4);
-        mbar_init(bar(B_P_EMPTY), 1);
+        for (int i = 0; i < kMaxSBuf; ++i) {
+            mbar_init(bar(B_S_FULL0 + i), 1);
+            mbar_init(bar(B_S_EMPTY0 + i), 1);
+            mbar_init(bar(B_P_FULL0 + i), 4);
+        }
         mbar_init(bar(B_O_FULL), 1);
         mbar_init(bar(B_O_EMPTY), 4);
         mbar_init(bar(B_MMA_DONE), 1);
@@ -189,7 +202,7 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
-    if (warp == 9) {
+    if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -198,7 +211,6 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tmem_o = tmem + p.tm_o;
-    const uint32_t tmem_p = tmem + p.tm_p;
 
     const uint32_t q_addr0 = smem_u32(smem + p.off_q);
     const uint32_t ring_addr = smem_u32(smem + p.off_ring);
@@ -207,23 +219,32 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int nsbuf = p.nsbuf;
     const int nqc = (p.d1 + 63) / 64;    // 64-element chunks of a Q/K row
     const int nvc = (p.d2 + 63) / 64;    // 64-element chunks of a V row
+    // tensor-memory column of score buffer sb
+    auto s_col = [&](uint32_t sb) { return (uint32_t)p.tm_s + sb * (uint32_t)p.s_stride; };
     // the block list of tile `tile` (written by sel_plan_kernel)
     auto list_n = [&](int tile) { return min(p.list_n[tile], p.cap); };
     auto list_blk = [&](int tile, int i) { return p.list_blk[(size_t)tile * p.cap + i]; };
+    // KV tile i of a tile holds its listed blocks i*BPT .. i*BPT+BPT-1 (a
+    // slot past the list repeats the tile's first block and is masked).
+    // Every role walks the same tiles and counts them alike: a tile with an
+    // empty list takes no Q, no K/V and no MMA, and is not counted in qc / oc.
+    // A tile's KV tiles are consumed in the order S_0 .. S_{min(nkv,nsbuf)-1},
+    // then for i = 0 .. nkv-1: P V_i, and S_{i-lag+nsbuf} once i >= lag.  S_j
+    // thus lands nsbuf - lag steps before its P V is due, and a buffer is
+    // refilled lag steps after the P V that frees it was issued.
+    const int lag = max(1, nsbuf / 2);
 
-    if (warp >= 8) setmaxnreg_dec<kRegsCtl>();
-    if (warp == 8) {
+    if (warp == kWarpTma) {
         // ============================ TMA producer ============================
-        // per tile: Q; pass A: K of the listed blocks; pass B: K_0, then
-        // K_{i+1}, V_i for each i
         if (lane == 0) {
-            uint32_t item = 0;
-            int tcount = 0;
+            uint32_t item = 0, qc = 0;
             const uint32_t q_bytes = (uint32_t)(nqc * 64 * G * TT * 2);
             const uint32_t k_bytes = (uint32_t)(nqc * 64 * NKV * 2);
             const uint32_t v_bytes = (uint32_t)(nvc * 64 * NKV * 2);
             bool ok = true;
-            auto load_kv = [&](bool is_v, int g, int row) {
+            // K or V of KV tile i: block q of the tile to rows q*LP.. of each
+            // 64-column chunk
+            auto load_kv = [&](bool is_v, int tile, const Tile& t, int n, int i) {
                 const int slot = item % nslot;
                 const uint32_t ph = (item / nslot) & 1;
                 ok = ok && mbar_wait(bar(B_SLOT_EMPTY0 + slot), ph ^ 1, abort_flag, p.err, kErrTimeoutBase + 2);
@@ -232,43 +253,51 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t dst = ring_addr + slot * p.slot_bytes;
                 mbar_arrive_expect_tx(fb, is_v ? v_bytes : k_bytes);
                 const int nc = is_v ? nvc : nqc;
-                for (int c = 0; c < nc; ++c)
-                    tma_load_3d(dst + c * NKV * 128, is_v ? &tm_v : &tm_k, c * 64, g, row, fb);
+                for (int q = 0; q < BPT; ++q) {
+                    const int e = (i * BPT + q < n) ? i * BPT + q : i * BPT;
+                    const int row = t.kv_row0 + list_blk(tile, e) * LP;
+                    for (int c = 0; c < nc; ++c)
+                        tma_load_3d(dst + c * NKV * 128 + q * LP * 128, is_v ? &tm_v : &tm_k, c * 64, t.group, row,
+                                    fb);
+                }
                 ++item;
             };
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
-                const Tile t = p.tiles[tile];
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
                 const int n = list_n(tile);
-                const int qb = tcount % nqbuf;
-                const uint32_t qph = (tcount / nqbuf) & 1;
-                ok = mbar_wait(bar(B_Q_EMPTY0 + qb), qph ^ 1, abort_flag, p.err, kErrTimeoutBase + 3);
+                if (n == 0) continue;
+                const Tile t = p.tiles[tile];
+                const int qb = qc % nqbuf;
+                ok = mbar_wait(bar(B_Q_EMPTY0 + qb), ((qc / nqbuf) & 1) ^ 1, abort_flag, p.err,
+                               kErrTimeoutBase + 3);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(B_Q_FULL0 + qb), q_bytes);
                 const uint32_t qdst = q_addr0 + qb * p.q_bytes;
                 for (int c = 0; c < nqc; ++c)
                     tma_load_3d(qdst + c * 16384, &tm_q, c * 64, t.group * G, t.q_row0, bar(B_Q_FULL0 + qb));
-                auto row_of = [&](int i) { return t.kv_row0 + list_blk(tile, i) * NKV; };
-                for (int i = 0; i < n && ok; ++i) load_kv(false, t.group, row_of(i));
-                if (n > 0 && ok) load_kv(false, t.group, row_of(0));
-                for (int i = 0; i < n && ok; ++i) {
-                    if (i + 1 < n) load_kv(false, t.group, row_of(i + 1));
-                    load_kv(true, t.group, row_of(i));
+                const int nkv = (n + BPT - 1) / BPT;
+                const int npro = min(nkv, nsbuf);
+                for (int i = 0; i < npro && ok; ++i) load_kv(false, tile, t, n, i);
+                for (int i = 0; i < nkv && ok; ++i) {
+                    load_kv(true, tile, t, n, i);
+                    if (i >= lag && i - lag + nsbuf < nkv) load_kv(false, tile, t, n, i - lag + nsbuf);
                 }
+                ++qc;
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == kWarpMma) {
         // ============================ MMA issuer =============================
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, NKV, false, false);
             const uint32_t idesc_pv = idesc_f16(kBF16, 128, p.d2, false, true);
             const int nks_qk = p.d1 / 16;
             constexpr int nks_pv = NKV / 16;
-            uint32_t item = 0, scnt = 0, pcnt = 0;
-            int tcount = 0;
+            uint32_t item = 0, scnt = 0, qc = 0, oc = 0;
             bool ok = true;
             uint32_t q_addr = q_addr0;
+            // S = Q K^T of the next block into its score buffer, once the P V
+            // that last read the buffer has retired
             auto issue_s = [&]() {
-                const int sb = scnt % nsbuf;
+                const uint32_t sb = scnt % nsbuf;
                 ok = ok && mbar_wait(bar(B_S_EMPTY0 + sb), ((scnt / nsbuf) & 1) ^ 1, abort_flag, p.err,
                                      kErrTimeoutBase + 4);
                 const int slot = item % nslot;
@@ -279,30 +308,36 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t kbase = ring_addr + slot * p.slot_bytes;
                 for (int ks = 0; ks < nks_qk; ++ks) {
                     const uint32_t off = (ks & 3) * 32;   // 16 elements inside a 128-byte row
-                    const uint64_t ad = sdesc_sw128(q_addr + (ks >> 2) * 16384 + off, 16, 1024);
                     const uint64_t bd = sdesc_sw128(kbase + (ks >> 2) * (NKV * 128) + off, 16, 1024);
-                    umma_ss(tmem + sb * 128, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
+                    const uint64_t ad = sdesc_sw128(q_addr + (ks >> 2) * 16384 + off, 16, 1024);
+                    umma_ss(tmem + s_col(sb), ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(bar(B_S_FULL0 + sb));
                 umma_commit(bar(B_SLOT_EMPTY0 + slot));
                 ++item;
                 ++scnt;
             };
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
                 const int n = list_n(tile);
-                const int qb = tcount % nqbuf;
-                ok = mbar_wait(bar(B_Q_FULL0 + qb), (tcount / nqbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 6);
+                if (n == 0) continue;
+                const int qb = qc % nqbuf;
+                ok = mbar_wait(bar(B_Q_FULL0 + qb), (qc / nqbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 6);
                 if (!ok) break;
                 tc_fence_after();
                 q_addr = q_addr0 + qb * p.q_bytes;
-                for (int i = 0; i < n && ok; ++i) issue_s();          // pass A
-                if (n > 0 && ok) issue_s();                          // pass B, S_0
-                for (int i = 0; i < n && ok; ++i) {
-                    if (i + 1 < n) issue_s();
+                const uint32_t s0 = scnt;               // running index of the tile's KV tile 0
+                const int nkv = (n + BPT - 1) / BPT;
+                const int npro = min(nkv, nsbuf);
+                for (int i = 0; i < npro && ok; ++i) issue_s();
+                for (int i = 0; i < nkv && ok; ++i) {
+                    const uint32_t gi = s0 + i;
+                    const uint32_t sb = gi % nsbuf;
+                    // O of the previous tile has been read out before P V_0 overwrites it
                     if (i == 0)
-                        ok = ok && mbar_wait(bar(B_O_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err,
+                        ok = ok && mbar_wait(bar(B_O_EMPTY), (oc & 1) ^ 1, abort_flag, p.err,
                                              kErrTimeoutBase + 7);
-                    ok = ok && mbar_wait(bar(B_P_FULL), pcnt & 1, abort_flag, p.err, kErrTimeoutBase + 8);
+                    ok = ok && mbar_wait(bar(B_P_FULL0 + sb), (gi / nsbuf) & 1, abort_flag, p.err,
+                                         kErrTimeoutBase + 8);
                     const int slot = item % nslot;
                     ok = ok && mbar_wait(bar(B_SLOT_FULL0 + slot), (item / nslot) & 1, abort_flag, p.err,
                                          kErrTimeoutBase + 9);
@@ -312,217 +347,204 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int ks = 0; ks < nks_pv; ++ks) {
                         const uint64_t bd = sdesc_sw128(vbase + ks * 2048, NKV * 128, 1024);
-                        umma_ts(tmem_o, tmem_p + ks * 8, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+                        umma_ts(tmem_o, tmem + s_col(sb) + ks * 8, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
                     }
-                    umma_commit(bar(B_P_EMPTY));
+                    umma_commit(bar(B_S_EMPTY0 + sb));     // the buffer is free, O holds P V_0..i
                     umma_commit(bar(B_SLOT_EMPTY0 + slot));
                     ++item;
-                    ++pcnt;
+                    // refill the buffer of block i - lag: its P V was issued lag
+                    // steps ago and has had that long to retire
+                    if (i >= lag && i - lag + nsbuf < nkv) issue_s();
                 }
-                if (!ok) break;
-                // a tile without P V work waits for the previous read-out, so that
-                // O_FULL never runs two phases ahead of its consumer
-                if (n == 0)
-                    ok = mbar_wait(bar(B_O_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 7);
                 if (!ok) break;
                 umma_commit(bar(B_O_FULL));
                 umma_commit(bar(B_Q_EMPTY0 + qb));
+                ++qc;
+                ++oc;
             }
             // every MMA issued so far has retired before the tensor memory is freed
             umma_commit(bar(B_MMA_DONE));
             mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
         }
     } else if (warp < 4) {
-        // ===================== softmax (128 thr) =====================
-        setmaxnreg_inc<kRegsSoftmax>();
+        // ============ softmax and output (128 thr, one row each) ============
         const int row = warp * 32 + lane;          // tile row = TMEM lane
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const float c2 = p.scale_log2;
         const int h = row % G;
         const int tok = row / G;
-        uint32_t scnt = 0, pcnt = 0;
-
-        auto load_s = [&](float (&s)[NKV]) {
-            const int sb = scnt % nsbuf;
-            mbar_wait(bar(B_S_FULL0 + sb), (scnt / nsbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
-            tc_fence_after();
-            const uint32_t ta = tmem + lane_off + sb * 128;
-#pragma unroll
-            for (int c = 0; c < NKV / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(ta + c * 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
-            }
-            if constexpr (NKV % 32 != 0) {
-                uint32_t r[16];
-                tmem_ld16(ta + (NKV / 32) * 32, r);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) s[(NKV / 32) * 32 + e] = __uint_as_float(r[e]);
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_S_EMPTY0 + sb));
-            ++scnt;
-        };
-        // scores in "exponent units": x = s * ce - shift.  With a positive scale
-        // the raw scores are used as they are (ce = c2); a zero or negative
-        // scale first multiplies them in (ce = 1).  Columns c >= lim are not
-        // attended to and become -inf.
+        // scores in "exponent units": x = s * ce.  With a positive scale the
+        // raw scores are used as they are (ce = c2); a zero or negative scale
+        // first multiplies them in (ce = 1).  Key k of block q of the KV tile
+        // is attended to iff k < lim[q]; the others become -inf.
         const bool pos_scale = c2 > 0.f;
         const float ce = pos_scale ? c2 : 1.f;
-        auto prep = [&](float (&s)[NKV], int lim) {
+        auto prep = [&](float (&s)[NKV], const int (&lim)[BPT]) {
             if (!pos_scale) {
 #pragma unroll
                 for (int c = 0; c < NKV; ++c) s[c] *= c2;
             }
-            if (lim < NKV) {
+            bool full = true;
 #pragma unroll
-                for (int c = 0; c < NKV; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+            for (int q = 0; q < BPT; ++q) full = full && lim[q] == LP;
+            if (!full) {
+#pragma unroll
+                for (int c = 0; c < NKV; ++c) s[c] = (c % LP < lim[c / LP]) ? s[c] : -INFINITY;
             }
         };
+        uint32_t scnt = 0, oc = 0;
 
-        int tcount = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             const Tile t = p.tiles[tile];
             const int n = list_n(tile);
             const bool valid = (row < TT * G) && (tok < t.ntok);
+            const size_t ridx = (size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h;
+            T* orow = reinterpret_cast<T*>(p.out) + ridx * p.d2;
+            if (n == 0) {
+                // no listed block: nothing is attended to
+                if (valid) {
+                    p.lse[ridx] = -INFINITY;
+                    for (int c = 0; c < p.d2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                continue;
+            }
             const int tpos = t.t0 + tok;
-            // columns of listed block i this row attends to: a prefix, cut by the
+            // keys of listed block e this row attends to: a prefix, cut by the
             // causal rule and the end of the sequence; none when its token did
-            // not list the block
-            auto lim_of = [&](int i) {
-                if (!valid) return 0;
-                const int b = list_blk(tile, i);
-                const uint32_t w = p.list_mask[((size_t)tile * p.cap + i) * 4 + (tok >> 5)];
+            // not list the block (or e is past the list)
+            auto lim_of = [&](int e) {
+                if (!valid || e >= n) return 0;
+                const int b = list_blk(tile, e);
+                const uint32_t w = p.list_mask[((size_t)tile * p.cap + e) * 4 + (tok >> 5)];
                 if (!((w >> (tok & 31)) & 1u)) return 0;
-                const int lim = min(NKV, min(tpos - b * NKV + 1, t.s_kv - b * NKV));
+                const int lim = min(LP, min(tpos - b * LP + 1, t.s_kv - b * LP));
                 return lim > 0 ? lim : 0;
             };
 
-            // ---------------- pass A: exact row max and sum (log2 domain) ----------------
-            float m = -INFINITY, L = 0.f;
-            for (int i = 0; i < n; ++i) {
-                float s[NKV];
-                const int lim = lim_of(i);
-                load_s(s);
-                prep(s, lim);
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float m = -INFINITY, L = 0.f;   // reference max (exponent units), sum of 2^(x - m)
+            const int nkv = (n + BPT - 1) / BPT;
+            int lim[BPT];
 #pragma unroll
-                for (int c = 0; c < NKV; c += 8) {
-                    mx4[0] = fmax3(mx4[0], s[c + 0], s[c + 1]);
-                    mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
-                    mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
-                    mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
-                }
-                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
-                const float mn = fmaxf(m, mx);
-                const float mref = (mn == -INFINITY) ? 0.f : mn;
-                const float2 ce2 = make_float2(ce, ce), nm2 = make_float2(-mref, -mref);
-                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                 make_float2(0.f, 0.f)};
+            for (int q = 0; q < BPT; ++q) lim[q] = lim_of(q);
+            for (int i = 0; i < nkv; ++i) {
+                const uint32_t sb = scnt % nsbuf;
+                const uint32_t ts = tmem + lane_off + s_col(sb);
+                int lim_next[BPT];
+                bool any = false;
 #pragma unroll
-                for (int c = 0; c < NKV; c += 2) {
-                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2, nm2);
-                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(x.x), ex2(x.y)));
+                for (int q = 0; q < BPT; ++q) {
+                    lim_next[q] = (i + 1 < nkv) ? lim_of((i + 1) * BPT + q) : 0;
+                    any = any || lim[q] > 0;
                 }
-                const float2 t01 = fadd2(acc[0], acc[1]), t23 = fadd2(acc[2], acc[3]);
-                const float sum = (t01.x + t01.y) + (t23.x + t23.y);
-                L = L * ex2(m - mref) + sum;
-                m = mn;
-            }
-            if (valid) {
-                // natural log-sum-exp: (m + log2 L) * ln 2
-                p.lse[(size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h] =
-                    (L > 0.f) ? (m + lg2(L)) * 0.69314718055994530942f : -INFINITY;
-            }
-
-            // ------------- pass B: P -> TMEM -------------
-            // P = 2^(s*c2 - m - log2 L): normalised in the exponent
-            const float mb = (L > 0.f) ? m + lg2(L) : INFINITY;
-            const float2 ce2b = make_float2(ce, ce), nb2 = make_float2(-mb, -mb);
-            for (int i = 0; i < n; ++i) {
-                float s[NKV];
-                const int lim = lim_of(i);
-                load_s(s);
-                prep(s, lim);
-#pragma unroll
-                for (int c = 0; c < NKV; c += 2) {
-                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2b, nb2);
-                    s[c] = ex2(x.x);
-                    s[c + 1] = ex2(x.y);
-                }
-                // P in the storage dtype -> tensor memory (A operand of P V)
-                mbar_wait(bar(B_P_EMPTY), (pcnt & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 11);
+                const bool work = __any_sync(0xffffffffu, any);
+                mbar_wait(bar(B_S_FULL0 + sb), (scnt / nsbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
                 tc_fence_after();
-                if constexpr ((NKV / 2) % 16 == 0) {
+                uint32_t pw[NKV / 2];
+                if (work) {
+                    float s[NKV];
+                    {
+                        uint32_t r[NKV];
+                        tmem_ld_cols<NKV>(ts, r);
+                        tmem_wait_ld_regs<NKV>(r);
 #pragma unroll
-                    for (int c = 0; c < NKV / 32; ++c) {
-                        uint32_t w[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) w[e] = pack2<T>(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
-                        tmem_st16(tmem_p + lane_off + c * 16, w);
+                        for (int c = 0; c < NKV; ++c) s[c] = __uint_as_float(r[c]);
                     }
+                    prep(s, lim);
+                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int c = 0; c < NKV; c += 8) {
+                        mx4[0] = fmax3(mx4[0], s[c + 0], s[c + 1]);
+                        mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
+                        mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
+                        mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
+                    }
+                    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
+                    // move the reference up only by more than 8: P <= 2^8 in between
+                    const bool raise = mx > m + 8.f;            // from -inf: any finite maximum
+                    const bool resc = raise && (m != -INFINITY); // O holds earlier blocks' P V
+                    float corr = 1.f;
+                    if (raise) {
+                        corr = ex2(m - mx);                     // 0 from -inf
+                        L *= corr;
+                        m = mx;
+                    }
+                    if (__any_sync(0xffffffffu, resc)) {
+                        // O rows of this warp times corr, after P V of the previous block
+                        const uint32_t pg = scnt - 1;
+                        mbar_wait(bar(B_S_EMPTY0 + pg % nsbuf), (pg / nsbuf) & 1, abort_flag, p.err,
+                                  kErrTimeoutBase + 11);
+                        tc_fence_after();
+                        const float f = resc ? corr : 1.f;
+                        for (int c = 0; c < p.d2; c += 16) {
+                            uint32_t r[16];
+                            tmem_ld16(tmem_o + lane_off + c, r);
+                            tmem_wait_ld_regs<16>(r);
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+                            tmem_st16(tmem_o + lane_off + c, r);
+                        }
+                    }
+                    const float mref = (m == -INFINITY) ? 0.f : m;
+                    const float2 ce2 = make_float2(ce, ce), nm2 = make_float2(-mref, -mref);
+                    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                     make_float2(0.f, 0.f)};
+#pragma unroll
+                    for (int c = 0; c < NKV; c += 2) {
+                        const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2, nm2);
+                        const float2 e2 = make_float2(ex2(x.x), ex2(x.y));
+                        acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e2);
+                        pw[c >> 1] = pack2<T>(e2.x, e2.y);
+                    }
+                    const float2 t01 = fadd2(acc[0], acc[1]), t23 = fadd2(acc[2], acc[3]);
+                    L += (t01.x + t01.y) + (t23.x + t23.y);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < NKV / 16; ++c) {
-                        uint32_t w[8];
+                    for (int c = 0; c < NKV / 2; ++c) pw[c] = 0u;
+                }
+                // P in the storage dtype over the first NKV/2 columns of the buffer
+                if constexpr ((NKV / 2) % 16 == 0) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) w[e] = pack2<T>(s[c * 16 + 2 * e], s[c * 16 + 2 * e + 1]);
-                        tmem_st8(tmem_p + lane_off + c * 8, w);
-                    }
+                    for (int c = 0; c < NKV / 32; ++c) tmem_st16(ts + c * 16, pw + c * 16);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NKV / 16; ++c) tmem_st8(ts + c * 8, pw + c * 8);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_P_FULL));
-                ++pcnt;
+                if (lane == 0) mbar_arrive(bar(B_P_FULL0 + sb));
+                ++scnt;
+#pragma unroll
+                for (int q = 0; q < BPT; ++q) lim[q] = lim_next[q];
             }
-        }
-    } else if (warp < 8) {
-        // ============ epilogue: O read-out (128 thr) ============
-        setmaxnreg_dec<kRegsEpilogue>();
-        const int ew = warp - 4;                   // TMEM lane quadrant
-        const int erow = ew * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
-        const int eh = erow % G;
-        const int etok = erow / G;
-        int tcount = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-            const Tile t = p.tiles[tile];
-            const int n = list_n(tile);
-            mbar_wait(bar(B_O_FULL), tcount & 1, abort_flag, p.err, kErrTimeoutBase + 12);
+
+            // ------------- O / L -> attention_out, log-sum-exp -------------
+            mbar_wait(bar(B_O_FULL), oc & 1, abort_flag, p.err, kErrTimeoutBase + 12);
             tc_fence_after();
-            const bool valid = (erow < TT * G) && (etok < t.ntok);
-            T* orow = reinterpret_cast<T*>(p.out) +
-                      ((size_t)(t.q_row0 + etok) * p.n1 + (size_t)t.group * G + eh) * p.d2;
-            // a row whose token attends to nothing has P = 0 everywhere, so O = 0
-            // from the P V products; a tile with no listed block has no P V
-            for (int c = 0; c < p.d2 / 16; ++c) {
+            if (valid) p.lse[ridx] = (L > 0.f) ? (m + lg2(L)) * 0.69314718055994530942f : -INFINITY;
+            const float inv = (L > 0.f) ? 1.f / L : 0.f;
+            for (int c = 0; c < p.d2; c += 16) {
                 uint32_t r[16];
-                tmem_ld16(tmem_o + lane_off + c * 16, r);
-                tmem_wait_ld();
+                tmem_ld16(tmem_o + lane_off + c, r);
+                tmem_wait_ld_regs<16>(r);
                 if (valid) {
                     uint4 w0, w1;
-                    float f[16];
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) f[q] = (n > 0) ? __uint_as_float(r[q]) : 0.f;
-                    w0.x = pack2<T>(f[0], f[1]);
-                    w0.y = pack2<T>(f[2], f[3]);
-                    w0.z = pack2<T>(f[4], f[5]);
-                    w0.w = pack2<T>(f[6], f[7]);
-                    w1.x = pack2<T>(f[8], f[9]);
-                    w1.y = pack2<T>(f[10], f[11]);
-                    w1.z = pack2<T>(f[12], f[13]);
-                    w1.w = pack2<T>(f[14], f[15]);
-                    *reinterpret_cast<uint4*>(orow + c * 16) = w0;
-                    *reinterpret_cast<uint4*>(orow + c * 16 + 8) = w1;
+                    w0.x = pack2<T>(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
+                    w0.y = pack2<T>(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
+                    w0.z = pack2<T>(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
+                    w0.w = pack2<T>(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
+                    w1.x = pack2<T>(__uint_as_float(r[8]) * inv, __uint_as_float(r[9]) * inv);
+                    w1.y = pack2<T>(__uint_as_float(r[10]) * inv, __uint_as_float(r[11]) * inv);
+                    w1.z = pack2<T>(__uint_as_float(r[12]) * inv, __uint_as_float(r[13]) * inv);
+                    w1.w = pack2<T>(__uint_as_float(r[14]) * inv, __uint_as_float(r[15]) * inv);
+                    *reinterpret_cast<uint4*>(orow + c) = w0;
+                    *reinterpret_cast<uint4*>(orow + c + 8) = w1;
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_O_EMPTY));
+            ++oc;
         }
     }
 
@@ -535,7 +557,7 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     }
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
