@@ -38,6 +38,7 @@ _CSRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc")
 # sources whose change invalidates a recorded DRAM-traffic figure
 ATTN_SRC = [os.path.join(_CSRC, "nsa_attention.cu")]
 CMP_SRC = [os.path.join(_CSRC, "nsa_compress.cu")]
+SEL_SRC = [os.path.join(_CSRC, "nsa_select.cu")]
 
 
 # ------------------------------------------------------------------ work
@@ -62,6 +63,30 @@ def compress_bytes(wl) -> float:
     tc = sum(0 if S < wl.l else (S - wl.l) // wl.d + 1 for S in wl.seqlens)
     return float(wl.t2 * wl.n2 * (wl.d1 + wl.d2) * e + tc * wl.n2 * (wl.d1 + wl.d2) * e
                  + wl.l * wl.n2 * e)
+
+
+def row_keys(topk, cu_q, cu_kv, lp):
+    """(T1, N2): keys each (query row, KV group) attends to through its listed
+    blocks: block j gives keys j*lp .. j*lp+lp-1 up to the row's key position
+    t and the end of the sequence (repeats and -1 give none)."""
+    out = np.zeros(topk.shape[:2], np.int64)
+    q0 = k0 = 0
+    for b in range(len(cu_q)):
+        sq, skv = int(cu_q[b]) - q0, int(cu_kv[b]) - k0
+        if sq > 0:
+            t = (np.arange(sq, dtype=np.int64) + skv - sq)[:, None, None]
+            srt = np.sort(topk[q0:q0 + sq].astype(np.int64), axis=-1)
+            first = np.ones_like(srt, dtype=bool)
+            first[..., 1:] = srt[..., 1:] != srt[..., :-1]
+            kk = np.minimum(np.minimum(lp, t - srt * lp + 1), skv - srt * lp)
+            out[q0:q0 + sq] = np.where((srt >= 0) & first & (kk > 0), kk, 0).sum(-1)
+        q0, k0 = int(cu_q[b]), int(cu_kv[b])
+    return out
+
+
+def select_flops(wl, keys) -> float:
+    """algorithmic FLOPs of selection attention: QK^T and PV over the attended keys, all heads."""
+    return 2.0 * (wl.d1 + wl.d2) * (wl.n1 // wl.n2) * float(np.sum(keys))
 
 
 def load_peaks():
@@ -89,7 +114,7 @@ def profile_traffic(kind, workload):
         return None
     with open(p) as f:
         d = json.load(f)
-    src = ATTN_SRC if kind == "attention" else CMP_SRC
+    src = {"attention": ATTN_SRC, "compress": CMP_SRC, "select": SEL_SRC}[kind]
     if d.get("workload") != workload or d.get("source_sha256_16") != src_hash(src):
         return None
     return d.get("bytes_per_launch_full_workload")
@@ -261,8 +286,38 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": ke}
 
+    # ---------- selection attention over the step's own top-k lists ----------
+    sel = None
+    if not args.no_select:
+        topk = outs[1]
+        sws = torch.empty(nsa.nsa_select_attention_workspace_size(wl.n1, wl.n2, wl.d1, wl.d2, wl.lp, wl.count,
+                                                                  cuq, cu), dtype=torch.uint8, device=dev)
+        sout = (torch.empty(t1, wl.n1, wl.d2, dtype=q.dtype, device=dev),
+                torch.empty(t1, wl.n1, dtype=torch.float32, device=dev))
+
+        def sel_call():
+            nsa.nsa_select_attention(q, k, v, topk, wl.scale, wl.n1, wl.lp, cuq, cu, out=sout, workspace=sws)
+
+        for _ in range(max(args.warmup, 0)):
+            flush.zero_()
+            sel_call()
+        torch.cuda.synchronize()
+        ks = max(3, min(K, args.select_steps))
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(ks)]
+        for i in range(ks):
+            flush.zero_()
+            sev[i][0].record()
+            sel_call()
+            sev[i][1].record()
+        torch.cuda.synchronize()
+        if nsa.nsa_workspace_status(sws) != 0:
+            raise RuntimeError("device-side timeout in selection attention")
+        tk_host = topk.cpu().numpy()
+        sel = dict(ms=float(np.mean([e[0].elapsed_time(e[1]) for e in sev])), steps=ks,
+                   keys=row_keys(tk_host, cuq, cu, wl.lp), topk=tk_host)
+
     return dict(wl=wl, K=K, step_ms=step_ms, att_ms=att_ms, cmp_ms=cmp_ms, t1=t1, wall=t_wall,
-                clocks=clk.result(), e2e=e2e,
+                clocks=clk.result(), e2e=e2e, sel=sel,
                 launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
 
 
@@ -316,6 +371,27 @@ def cpu_baseline(wl, budget_s=20.0, rows_per_seq=None):
                       f"{t_att:.1f} s; compress: first {S0} raw rows of K and V, {t_cmp:.2f} s",
             "compress_gbs": cmp_bytes / t_cmp / 1e9, "seconds": t_att + t_cmp,
             "full_attention_pairs": full_pairs}
+
+
+def select_cpu_baseline(wl, topk, keys, budget_s=8.0):
+    """The selection-attention oracle as it stands, on evenly spaced query rows
+    (all heads) of the same workload and the same top-k lists."""
+    import oracle
+    x = wl.generate(device="cpu")
+    q, k, v = x["q"].float(), x["k"].float(), x["v"].float()
+    cq, ck = x["cu_seqlens_q"], x["cu_seqlens"]
+    T1 = int(cq[-1])
+    probe = np.unique(np.linspace(0, T1 - 1, num=min(T1, 32)).astype(np.int64))
+    tp = time.perf_counter()
+    oracle.select_attention(q[probe], k, v, topk, wl.scale, wl.lp, wl.count, cq, ck, rows=probe, q_rows_only=True)
+    per_row = (time.perf_counter() - tp) / probe.size
+    nrows = int(max(16, min(T1, budget_s / max(per_row, 1e-6))))
+    rows = np.unique(np.linspace(0, T1 - 1, num=nrows).astype(np.int64))
+    t0 = time.perf_counter()
+    oracle.select_attention(q[rows], k, v, topk, wl.scale, wl.lp, wl.count, cq, ck, rows=rows, q_rows_only=True)
+    dt = time.perf_counter() - t0
+    return {"value": select_flops(wl, keys[rows]) / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{rows.size} of {T1} evenly spaced query rows, all heads, {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
@@ -379,6 +455,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-rows", type=int, default=96)
+    ap.add_argument("--no-select", action="store_true", help="skip the selection-attention measurement")
+    ap.add_argument("--select-steps", type=int, default=20)
+    ap.add_argument("--select-cpu-budget", type=float, default=8.0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -448,6 +527,23 @@ def main():
             "cpu_baseline": cpu,
             "wall_s_timed_region": r["wall"],
         }
+        if r["sel"] is not None:
+            sf = select_flops(wl, r["sel"]["keys"])
+            st = sf / (r["sel"]["ms"] * 1e-3) / 1e12
+            line["select_attention"] = {
+                "what": "nsa_select_attention over the step's own top-k lists (plan + attention kernels)",
+                "ms": r["sel"]["ms"], "steps": r["sel"]["steps"], "tflops": st,
+                "flops_per_launch": sf,
+                "keys_per_row_group": float(np.mean(r["sel"]["keys"])),
+                "l2": "flushed (256 MB write) before every timed call",
+                "roofline": {"bound": "tensor", "achieved": st, "peak": peak_t, "unit": "TFLOP/s",
+                             "frac": st / peak_t, "traffic": profile_traffic("select", wl.name),
+                             "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                "cpu_baseline": (select_cpu_baseline(wl, r["sel"]["topk"], r["sel"]["keys"],
+                                                     budget_s=args.select_cpu_budget)
+                                 if (not args.no_cpu_baseline and world == 1) else None),
+                "gpu_launches": 2 * r["sel"]["steps"],
+            }
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

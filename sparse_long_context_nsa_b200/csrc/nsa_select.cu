@@ -409,23 +409,34 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 continue;
             }
             const int tpos = t.t0 + tok;
-            // keys of listed block e this row attends to: a prefix, cut by the
-            // causal rule and the end of the sequence; none when its token did
-            // not list the block (or e is past the list)
-            auto lim_of = [&](int e) {
-                if (!valid || e >= n) return 0;
-                const int b = list_blk(tile, e);
-                const uint32_t w = p.list_mask[((size_t)tile * p.cap + e) * 4 + (tok >> 5)];
-                if (!((w >> (tok & 31)) & 1u)) return 0;
+            // list entry e: its block and the mask word of this row's token (a
+            // zero word past the list).  The entries of KV tile i + 2 are read
+            // while tile i is processed, so that their latency is hidden.
+            auto fetch = [&](int e, int& b, uint32_t& w) {
+                b = (e < n) ? list_blk(tile, e) : 0;
+                w = (e < n) ? p.list_mask[((size_t)tile * p.cap + e) * 4 + (tok >> 5)] : 0u;
+            };
+            // keys of the block this row attends to: a prefix, cut by the causal
+            // rule and the end of the sequence; none when its token did not
+            // list the block
+            auto lim_of = [&](int b, uint32_t w) {
+                if (!valid || !((w >> (tok & 31)) & 1u)) return 0;
                 const int lim = min(LP, min(tpos - b * LP + 1, t.s_kv - b * LP));
                 return lim > 0 ? lim : 0;
             };
 
             float m = -INFINITY, L = 0.f;   // reference max (exponent units), sum of 2^(x - m)
             const int nkv = (n + BPT - 1) / BPT;
-            int lim[BPT];
+            int lim[BPT], nb[BPT];
+            uint32_t nw[BPT];
 #pragma unroll
-            for (int q = 0; q < BPT; ++q) lim[q] = lim_of(q);
+            for (int q = 0; q < BPT; ++q) {
+                int b0;
+                uint32_t w0;
+                fetch(q, b0, w0);
+                lim[q] = lim_of(b0, w0);
+                fetch(BPT + q, nb[q], nw[q]);
+            }
             for (int i = 0; i < nkv; ++i) {
                 const uint32_t sb = scnt % nsbuf;
                 const uint32_t ts = tmem + lane_off + s_col(sb);
@@ -433,7 +444,8 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 bool any = false;
 #pragma unroll
                 for (int q = 0; q < BPT; ++q) {
-                    lim_next[q] = (i + 1 < nkv) ? lim_of((i + 1) * BPT + q) : 0;
+                    lim_next[q] = lim_of(nb[q], nw[q]);
+                    fetch((i + 2) * BPT + q, nb[q], nw[q]);
                     any = any || lim[q] > 0;
                 }
                 const bool work = __any_sync(0xffffffffu, any);
