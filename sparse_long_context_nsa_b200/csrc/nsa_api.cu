@@ -403,8 +403,10 @@ nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, in
 
     // sizes of the per-CTA ring and the output run of one CTA
     const int rowbytes = (int)(rowelems * 2);
-    // rows per bulk copy: about 16 KB, a multiple of 4 (the kernel steps 4 rows at a time)
-    int rs = std::max(4, (16384 / rowbytes) & ~3);
+    // rows per bulk copy: about 8 KB, a multiple of 4 (the kernel steps 4 rows at a time).
+    // Measured on B200 against 16 KB and 32 KB stages and 3-8 deep rings: 8 KB x 4 gives
+    // the smallest CTAs (about 6 per SM) and the highest read rate.
+    int rs = std::max(4, (8192 / rowbytes) & ~3);
     const int stage_bytes = rs * rowbytes;
     const int wbytes = ((l * n2 * 4) + 127) & ~127;
     const size_t smem = (size_t)wbytes + 128 + (size_t)kCompressStages * stage_bytes;
