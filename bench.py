@@ -135,6 +135,14 @@ def max_over_ranks(values, device, world: int):
     return t.tolist()
 
 
+def sum_over_ranks(values, device, world: int):
+    """Element-wise sum of a list of floats over all ranks (identity for one rank)."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return t.tolist()
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML while running."""
@@ -491,6 +499,13 @@ def main():
                "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
                "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
                "ms_per_step": r["e2e"]["ms_per_step"]}
+    # selection attention: every rank times its own batch; max of the times,
+    # sum of the algorithmic work (the lists differ from rank to rank)
+    sel_ms = sel_flops_all = None
+    if r["sel"] is not None:
+        dev0 = torch.device("cuda", local_rank)
+        sel_ms = max_over_ranks([r["sel"]["ms"]], dev0, world)[0]
+        sel_flops_all = sum_over_ranks([select_flops(wl, r["sel"]["keys"])], dev0, world)[0]
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
@@ -529,10 +544,11 @@ def main():
         }
         if r["sel"] is not None:
             sf = select_flops(wl, r["sel"]["keys"])
-            st = sf / (r["sel"]["ms"] * 1e-3) / 1e12
+            st = sf / (r["sel"]["ms"] * 1e-3) / 1e12                  # this GPU (rank 0)
             line["select_attention"] = {
                 "what": "nsa_select_attention over the step's own top-k lists (plan + attention kernels)",
-                "ms": r["sel"]["ms"], "steps": r["sel"]["steps"], "tflops": st,
+                "ms": sel_ms, "steps": r["sel"]["steps"], "tflops": st,
+                "tflops_all_ranks": sel_flops_all / (sel_ms * 1e-3) / 1e12,
                 "flops_per_launch": sf,
                 "keys_per_row_group": float(np.mean(r["sel"]["keys"])),
                 "l2": "flushed (256 MB write) before every timed call",

@@ -160,3 +160,71 @@ def test_python_binding_rejects_host_tensors(lib):
     w = torch.zeros(32, 1, dtype=torch.bfloat16)
     with pytest.raises(TypeError, match="CUDA tensor"):
         nsa.nsa_compress(k, None, w, 32, 16, [64])
+
+
+# ------------------------------------------------------------ selection attention
+def _sws(**kw):
+    a = dict(head_num=64, n2=4, d1=128, d2=128, lp=64, count=16, cu_seqlens_q=[16384], cu_seqlens_kv=[16384])
+    a.update(kw)
+    return nsa.nsa_select_attention_workspace_size(**a)
+
+
+def test_select_workspace_size_is_positive_and_grows_with_tiles(lib):
+    small = _sws(cu_seqlens_q=[1024], cu_seqlens_kv=[1024])
+    big = _sws()
+    assert 256 < small < big
+    # short queries against long keys: the lists are sized by the keys' blocks
+    assert _sws(cu_seqlens_q=[128], cu_seqlens_kv=[65536]) > _sws(cu_seqlens_q=[128], cu_seqlens_kv=[1024])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(lp=40), dict(lp=8), dict(lp=144), dict(count=0), dict(count=33), dict(d1=120), dict(d2=40),
+    dict(head_num=6, n2=4), dict(head_num=2, n2=4), dict(cu_seqlens_q=[10, 5], cu_seqlens_kv=[10, 20]),
+    dict(cu_seqlens_q=[10, 20], cu_seqlens_kv=[10, 5]),
+])
+def test_select_constraints_invalid(lib, kw):
+    with pytest.raises(ValueError, match="INVALID_ARG"):
+        _sws(**kw)
+
+
+@pytest.mark.parametrize("kw", [dict(d1=272), dict(d2=272), dict(head_num=256, n2=1)])
+def test_select_constraints_unsupported(lib, kw):
+    with pytest.raises(ValueError, match="UNSUPPORTED"):
+        _sws(**kw)
+
+
+def test_select_prefix_lists_must_pair_up(lib):
+    with pytest.raises(ValueError):
+        _sws(cu_seqlens_q=[100, 200], cu_seqlens_kv=[200])
+
+
+def _call_select(lib, **kw):
+    a = dict(q=4096, k=4096, v=4096, tk=4096, scale=0.1, head_num=64, lp=64, count=16, cq=[16384], ck=[16384],
+             n2=4, d1=128, d2=128, dtype=0, out=4096, lse=4096, ws=4096, wsb=1 << 30)
+    a.update(kw)
+    arr = lambda x: np.ascontiguousarray(np.asarray(x, np.int32))
+    cq, ck = arr(a["cq"]), arr(a["ck"])
+    ip = lambda x: x.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    return lib.nsa_select_attention(a["q"], a["k"], a["v"], a["tk"], a["scale"], a["head_num"], a["lp"],
+                                    a["count"], ip(cq), ip(ck), cq.size, a["n2"], a["d1"], a["d2"], a["dtype"],
+                                    a["out"], a["lse"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), nsa.NSA_ERR_INVALID_ARG),
+    (dict(tk=None), nsa.NSA_ERR_INVALID_ARG),
+    (dict(lse=None), nsa.NSA_ERR_INVALID_ARG),
+    (dict(k=4100), nsa.NSA_ERR_INVALID_ARG),            # misaligned
+    (dict(tk=4098), nsa.NSA_ERR_INVALID_ARG),           # int32 list not 4-byte aligned
+    (dict(lse=4097), nsa.NSA_ERR_INVALID_ARG),
+    (dict(dtype=5), nsa.NSA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), nsa.NSA_ERR_INVALID_ARG),
+    (dict(lp=24), nsa.NSA_ERR_INVALID_ARG),
+    (dict(count=64), nsa.NSA_ERR_INVALID_ARG),
+    (dict(ws=None), nsa.NSA_ERR_WORKSPACE),
+    (dict(ws=4096 + 64), nsa.NSA_ERR_WORKSPACE),        # workspace must be 256-byte aligned
+    (dict(wsb=256), nsa.NSA_ERR_WORKSPACE),             # undersized
+    (dict(cq=[0], ck=[16384]), nsa.NSA_OK),             # no query rows: nothing to launch
+])
+def test_select_rejects_before_launch(lib, kw, status):
+    assert _call_select(lib, **kw) == status

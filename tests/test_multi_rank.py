@@ -32,12 +32,13 @@ def _worker(rank, world, port, q):
         gathered = [None] * world
         dist.all_gather_object(gathered, (wl.seed, tuple(x["q"].shape), checksum))
         mx = bench.max_over_ranks([1.0 + rank, 10.0 - rank], torch.device("cpu"), world)
+        sm = bench.sum_over_ranks([1.0 + rank, 0.5], torch.device("cpu"), world)
 
         class A:
             workload = workloads.TINY.name
             steps, warmup, ref_rows = 1, 0, 4
         ref_printed = bench.run_reference(A, rank, world) if rank != 0 else "rank0"
-        q.put((rank, gathered, mx, ref_printed))
+        q.put((rank, gathered, mx + sm, ref_printed))
     finally:
         dist.destroy_process_group()
 
@@ -61,5 +62,5 @@ def test_two_ranks_independent_batches_and_max_reduction():
     assert seeds[0] != seeds[1]
     assert g0[0][1] == g0[1][1]                 # same shapes
     assert g0[0][2] != g0[1][2]                 # different data
-    assert mx0 == mx1 == [2.0, 10.0]            # max over ranks, identical everywhere
+    assert mx0 == mx1 == [2.0, 10.0, 3.0, 1.0]  # max (then sum) over ranks, identical everywhere
     assert ref1 is None                         # reference arm: rank 0 only
