@@ -179,10 +179,11 @@ nsa_status_t nsa_select_attention_workspace_size(
  *                 256-byte aligned; its first 16 bytes receive the device error
  *                 word read by nsa_workspace_status
  * Constraints: lp a multiple of 16 in [16, 128]; 1 <= count <= 32; D1, D2
- * multiples of 16 (NSA_ERR_INVALID_ARG); D1 or D2 > 256, more than 128 query
- * heads per KV group, or sequences of more than about 6.5e6 blocks
- * (NSA_ERR_UNSUPPORTED).  Two launches on `stream`: a planning kernel that
- * gathers each tile's union of listed blocks, then the attention kernel.
+ * multiples of 16; topk_indices and softmax_lse 4-byte aligned, the other
+ * tensors 16-byte aligned (NSA_ERR_INVALID_ARG); D1 or D2 > 256, more than
+ * 128 query heads per KV group, or a sequence of more than 819200 blocks of
+ * lp keys (NSA_ERR_UNSUPPORTED).  Two launches on `stream`: a planning kernel
+ * that gathers each tile's union of listed blocks, then the attention kernel.
  */
 nsa_status_t nsa_select_attention(
     const void* q, const void* k, const void* v, const int32_t* topk_indices, float scale,
