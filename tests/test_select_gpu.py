@@ -126,11 +126,19 @@ def test_count_extremes(nsa):
         _check(out, lse, ref)
 
 
-def test_pipeline_on_the_16k_workload(nsa):
-    """Compress -> compressed attention -> selection attention on the 16K
-    workload at full size, sampled rows against the oracle fed with the GPU's
-    own top-k lists."""
-    wl = workloads.SINGLE_16K
+@pytest.mark.parametrize("name,first,last,every", [
+    ("single_s16384_n64_n4_d128", 64, 64, 257),
+    ("varlen8_t158963_n32_n2_d192x128_fp16", 32, 32, 997),
+    ("long_s131072_n128_n8_d128", 48, 48, 2039),
+    ("compress_t262144_shortq_4x128_n64_n8_d128", 128, 128, 1),
+], ids=["16k", "varlen", "long", "shortq"])
+def test_pipeline_on_full_workloads(nsa, name, first, last, every):
+    """Compress -> compressed attention -> selection attention on a workload at
+    full size (the 16K one is the bench's; varlen runs fp16 with D1=192, the long
+    one l'=128 and 32-entry lists, the short-query one bottom-right aligned
+    queries).  Sampled rows against the oracle fed with the GPU's own top-k
+    lists; every row of the short-query case."""
+    wl = workloads.WORKLOADS[name]
     x = wl.generate(device="cuda")
     cuc = nsa.nsa_compress_out_len(x["cu_seqlens"], wl.l, wl.d)
     kc, vc = nsa.nsa_compress(x["k"], x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"])
@@ -139,7 +147,7 @@ def test_pipeline_on_the_16k_workload(nsa):
     out, lse = nsa.nsa_select_attention(x["q"], x["k"], x["v"], tk, wl.scale, wl.n1, wl.lp,
                                         x["cu_seqlens_q"], x["cu_seqlens"])
     torch.cuda.synchronize()
-    rows = workloads.sample_rows(x["cu_seqlens_q"], first=64, last=64, every=257)
+    rows = workloads.sample_rows(x["cu_seqlens_q"], first=first, last=last, every=every)
     sel = tk.cpu().numpy()
     rows_t = torch.from_numpy(rows).cuda()
     ref = oracle.select_attention(x["q"].index_select(0, rows_t).float().cpu(), x["k"].float().cpu(),
