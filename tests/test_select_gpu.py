@@ -90,13 +90,14 @@ def test_small_case(nsa):
     _check(out, lse, ref)
 
 
-@pytest.mark.parametrize("n1,n2", [(4, 4), (8, 1), (32, 2), (16, 1), (64, 2)], ids=lambda v: str(v))
+@pytest.mark.parametrize("n1,n2", [(4, 4), (8, 1), (32, 2), (16, 1), (64, 2), (128, 1), (6, 2)],
+                         ids=lambda v: str(v))
 def test_group_sizes(nsa, n1, n2):
     out, lse, ref = _run(nsa, [700, 333], [700, 333], n1, n2, 64, 64, 32, 6, seed=1)
     _check(out, lse, ref)
 
 
-@pytest.mark.parametrize("lp", [16, 48, 64, 112, 128])
+@pytest.mark.parametrize("lp", [16, 32, 48, 64, 80, 96, 112, 128])
 def test_block_sizes(nsa, lp):
     out, lse, ref = _run(nsa, [1500], [1500], 16, 2, 64, 64, lp, 5, seed=2)
     _check(out, lse, ref)
