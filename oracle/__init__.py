@@ -76,7 +76,7 @@ def _load():
             _i32p, _i32p, _i32p, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
             _f64p, _f64p, _f64p, _i32p, ctypes.c_void_p, ctypes.c_int,
-            ctypes.c_void_p]
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64]
         lib.oracle_compress_attention.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_select_attention.argtypes = [
@@ -168,12 +168,17 @@ def topk(score, n_cand: int, count: int) -> np.ndarray:
 
 def compress_attention(q, kcmp, vcmp, scale: float, l: int, d: int, lp: int,
                        count: int, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
-                       rows=None, sel_cap: int | None = None, q_rows_only: bool = False):
+                       rows=None, sel_cap: int | None = None, q_rows_only: bool = False,
+                       atten_mask=None, topk_mask=None):
     """Steps 1-7 of mindspore.ops.nsa_compress_attention for query rows.
 
     q (T1, N1, D1), kcmp (Tc, N2, D1), vcmp (Tc, N2, D2): values of the
     storage-dtype tensors.  ``rows`` selects global query rows (None = all);
     with ``q_rows_only`` q holds just those rows, in the order of ``rows``.
+    ``atten_mask`` (S1, S2cmp) and ``topk_mask`` (S1, S2sel), bool, optional:
+    one matrix for every sequence and head, indexed by (query index inside the
+    sequence, block); True removes the block from the visible set (step 1) or
+    from the top-k candidates (step 6).
     Returns a dict with out (R, N1, D2), softmax_max / softmax_sum (R, N1),
     topk (R, N2, count), score (R, N2, sel_cap) and ncand (R, N2).
     """
@@ -204,13 +209,27 @@ def compress_attention(q, kcmp, vcmp, scale: float, l: int, d: int, lp: int,
         kf = np.zeros(1)
     if vf.size == 0:
         vf = np.zeros(1)
+    def _mask(mk, need_cols, what):
+        if mk is None:
+            return None, 0
+        mk = np.ascontiguousarray(np.asarray(mk).astype(np.uint8))
+        seq_q = np.diff(np.concatenate([[0], cq])) if batch else np.zeros(1, np.int64)
+        if mk.ndim != 2 or mk.shape[0] < int(np.max(seq_q, initial=0)) or mk.shape[1] < need_cols:
+            raise ValueError(f"{what} must be (S1, S2) covering every sequence's queries and blocks")
+        return mk, mk.shape[1]
+    max_cmp = int(np.max(np.diff(np.concatenate([[0], cc])), initial=0)) if batch else 0
+    max_sel = int(np.max(np.diff(np.concatenate([[0], cs])), initial=0)) if batch else 0
+    am, am_s2 = _mask(atten_mask, max_cmp, "atten_mask")
+    tm, tm_s2 = _mask(topk_mask, max_sel, "topk_mask")
     if R > 0:
         rc = _load().oracle_compress_attention(
             qf, kf, vf, float(scale), n1, n2, d1, d2, int(l), int(d), int(lp),
             int(count), cq, cc, cs, batch,
             rows_arr.ctypes.data_as(ctypes.c_void_p), R, 1 if q_rows_only else 0,
             out, smax, ssum, tk, score.ctypes.data_as(ctypes.c_void_p), sel_cap,
-            ncand.ctypes.data_as(ctypes.c_void_p))
+            ncand.ctypes.data_as(ctypes.c_void_p),
+            am.ctypes.data_as(ctypes.c_void_p) if am is not None else None, am_s2,
+            tm.ctypes.data_as(ctypes.c_void_p) if tm is not None else None, tm_s2)
         if rc != 0:
             raise ValueError("oracle: l % d and l' % d must be 0")
     return {"out": out, "softmax_max": smax, "softmax_sum": ssum, "topk": tk,

@@ -153,14 +153,26 @@ void oracle_importance(const double* P, int n_vis, int a, int b, int n_sel,
 /* descending score, ties to the smaller j, then lists them ascending ([RFA]  */
 /* select_idx convention) and pads with -1 up to count.                       */
 /* ------------------------------------------------------------------------- */
+void oracle_topk_excl(const double* score, int n_cand, const uint8_t* excl, int count, int32_t* idx);
 void oracle_topk(const double* score, int n_cand, int count, int32_t* idx)
 {
-    int kstar = (count < n_cand) ? count : n_cand;
+    oracle_topk_excl(score, n_cand, NULL, count, idx);
+}
+
+/* As above over the candidates j < n_cand with excl[j] == 0 (excl may be     */
+/* NULL): [ATT] step 6, P'_slc = topk_mask(P'_slc), read as removing the      */
+/* masked blocks from the candidate set.                                     */
+void oracle_topk_excl(const double* score, int n_cand, const uint8_t* excl, int count, int32_t* idx)
+{
+    int n_in = 0;
+    for (int j = 0; j < n_cand; j++)
+        if (!(excl && excl[j])) n_in++;
+    int kstar = (count < n_in) ? count : n_in;
     char* taken = (char*)calloc((size_t)(n_cand > 0 ? n_cand : 1), 1);
     for (int r = 0; r < kstar; r++) {
         int best = -1;
         for (int j = 0; j < n_cand; j++) {
-            if (taken[j]) continue;
+            if (taken[j] || (excl && excl[j])) continue;
             if (best < 0 || score[j] > score[best]) best = j;   /* strict: earlier j wins ties */
         }
         taken[best] = 1;
@@ -184,6 +196,11 @@ void oracle_topk(const double* score, int n_cand, int count, int32_t* idx)
 /*  smax  (nrows, N1)      max of the scaled scores (-inf for empty rows)      */
 /*  ssum  (nrows, N1)      sum of exp(s - max) (0 for empty rows)              */
 /*  topk  (nrows, N2, count)                                                   */
+/* Optional masks of [ATT] steps 1 and 6 (NULL = none), bool bytes, one (S1,  */
+/* S2) matrix shared by every sequence and head, indexed by the row's query   */
+/* index inside its sequence and the block index; a true entry removes the    */
+/* pair: amask (S1, >= n_cmp) row stride am_s2, tmask (S1, >= n_sel) row      */
+/* stride tm_s2.                                                              */
 /*  score (nrows, N2, sel_cap) or NULL: P_slc' for j < min(n_sel, sel_cap)     */
 /*  ncand (nrows, N2) or NULL: number of top-k candidates of the row (0 when   */
 /*        the row sees no block)                                               */
@@ -197,7 +214,9 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
                               const int64_t* rows, int64_t nrows, int q_compact,
                               double* out, double* smax, double* ssum,
                               int32_t* topk, double* score, int sel_cap,
-                              int32_t* ncand)
+                              int32_t* ncand,
+                              const uint8_t* amask, int64_t am_s2,
+                              const uint8_t* tmask, int64_t tm_s2)
 {
     if (l % d != 0 || lp % d != 0) return -1;
     const int a = lp / d, bb = l / d;
@@ -240,11 +259,23 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
             int n_vis = 0;
             for (int i = 0; i < n_cmp; i++)
                 if ((int64_t)i * d + l - 1 <= tpos) n_vis++;
+            /* step 1's optional atten_mask (S1, S2cmp): a true entry at (query  */
+            /* row of the sequence, block) removes the block from the visible    */
+            /* set; a row left without a block is an empty row                   */
+            const int64_t tloc = t - q0;
+            const uint8_t* arow = amask ? amask + tloc * am_s2 : NULL;
+            const uint8_t* trow = tmask ? tmask + tloc * tm_s2 : NULL;
+            int n_att = 0;
+            for (int i = 0; i < n_vis; i++)
+                if (!(arow && arow[i])) n_att++;
 
             /* candidates: j < n_sel with j*l' <= tpos */
             int n_cand = 0;
             for (int j = 0; j < n_sel; j++)
                 if ((int64_t)j * lp <= tpos) n_cand++;
+            int n_cand_in = 0;
+            for (int j = 0; j < n_cand; j++)
+                if (!(trow && trow[j])) n_cand_in++;
 
             for (int g = 0; g < n2; g++) {
                 for (int j = 0; j < n_sel; j++) grp[j] = 0.0;
@@ -252,7 +283,7 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
                     int h = g * G + hh;
                     double* o = out + (r * n1 + h) * (int64_t)d2;
                     for (int e = 0; e < d2; e++) o[e] = 0.0;
-                    if (n_vis == 0) {
+                    if (n_att == 0) {
                         smax[r * n1 + h] = -INFINITY;
                         ssum[r * n1 + h] = 0.0;
                         continue;
@@ -265,12 +296,15 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
                         for (int k = 0; k < d1; k++) acc += qr[k] * kr[k];
                         sc[i] = scale * acc;
                     }
-                    /* step 2: P_cmp = softmax(QK) */
-                    double m = sc[0];
-                    for (int i = 1; i < n_vis; i++) if (sc[i] > m) m = sc[i];
+                    /* step 2: P_cmp = softmax(QK) over the attended blocks */
+                    double m = -INFINITY;
+                    for (int i = 0; i < n_vis; i++)
+                        if (!(arow && arow[i]) && sc[i] > m) m = sc[i];
                     double L = 0.0;
-                    for (int i = 0; i < n_vis; i++) L += exp(sc[i] - m);
-                    for (int i = 0; i < n_vis; i++) P[i] = exp(sc[i] - m) / L;
+                    for (int i = 0; i < n_vis; i++)
+                        if (!(arow && arow[i])) L += exp(sc[i] - m);
+                    for (int i = 0; i < n_vis; i++)
+                        P[i] = (arow && arow[i]) ? 0.0 : exp(sc[i] - m) / L;
                     smax[r * n1 + h] = m;
                     ssum[r * n1 + h] = L;
                     /* step 3: attentionOut = P_cmp * value */
@@ -288,13 +322,13 @@ int oracle_compress_attention(const double* q, const double* kc, const double* v
                     double* dst = score + (r * n2 + g) * (int64_t)sel_cap;
                     for (int j = 0; j < sel_cap; j++) dst[j] = (j < lim) ? grp[j] : 0.0;
                 }
-                if (ncand) ncand[r * n2 + g] = (n_vis == 0) ? 0 : n_cand;
-                /* steps 6-7: causal candidate set, then top-k */
+                if (ncand) ncand[r * n2 + g] = (n_att == 0) ? 0 : n_cand_in;
+                /* steps 6-7: causal candidate set less the topk_mask, then top-k */
                 int32_t* ti = topk + (r * n2 + g) * (int64_t)count;
-                if (n_vis == 0) {
+                if (n_att == 0) {
                     for (int k = 0; k < count; k++) ti[k] = -1;
                 } else {
-                    oracle_topk(grp, n_cand, count, ti);
+                    oracle_topk_excl(grp, n_cand, trow, count, ti);
                 }
             }
         }
