@@ -325,6 +325,48 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": ke, "overlap": "copy-in, compute and copy-out of consecutive steps on three streams"}
 
+    # ---------- the optional masks of steps 1 and 6 (seeded, 30 % set) ----------
+    msk = None
+    if not args.no_masks:
+        rng = np.random.default_rng(wl.seed + 77)
+        sq = np.diff(np.concatenate([[0], cuq]))
+        ncs = np.diff(np.concatenate([[0], cuc]))
+        nss = np.diff(np.concatenate([[0], cus]))
+        am = rng.random((int(sq.max()), max(1, int(ncs.max())))) < 0.3
+        tm = rng.random((int(sq.max()), max(1, int(nss.max())))) < 0.3
+        am_d, tm_d = torch.from_numpy(am).to(dev), torch.from_numpy(tm).to(dev)
+        mouts = tuple(torch.empty_like(t) for t in outs)
+
+        def masked_call():
+            nsa.nsa_compress_attention(q, kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count, cuq, cuc, cus,
+                                       out=mouts, workspace=ws, atten_mask=am_d, topk_mask=tm_d)
+
+        for _ in range(max(args.warmup, 0)):
+            flush.zero_()
+            masked_call()
+        km = max(3, min(K, args.select_steps))
+        mev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(km)]
+        for i in range(km):
+            flush.zero_()
+            mev[i][0].record()
+            masked_call()
+            mev[i][1].record()
+        torch.cuda.synchronize()
+        if nsa.nsa_workspace_status(ws) != 0:
+            raise RuntimeError("device-side timeout in masked attention")
+        # attended (row, block) pairs: visible by the causal rule and not masked
+        pairs = 0
+        for b in range(len(cuq)):
+            n_q, n_c = int(sq[b]), int(ncs[b])
+            if n_q == 0 or n_c == 0:
+                continue
+            off = max(0, (n_c - 1) * wl.d + wl.l - n_q)
+            tpos = np.arange(n_q)[:, None] + off
+            vis = np.arange(n_c)[None, :] * wl.d + wl.l - 1 <= tpos
+            pairs += int((vis & ~am[:n_q, :n_c]).sum())
+        msk = dict(ms=float(np.mean([e[0].elapsed_time(e[1]) for e in mev])), steps=km,
+                   flops=2.0 * (wl.d1 + wl.d2) * wl.n1 * pairs)
+
     # ---------- selection attention over the step's own top-k lists ----------
     sel = None
     if not args.no_select:
@@ -356,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
                    keys=row_keys(tk_host, cuq, cu, wl.lp), topk=tk_host)
 
     return dict(wl=wl, K=K, step_ms=step_ms, att_ms=att_ms, cmp_ms=cmp_ms, t1=t1, wall=t_wall,
-                clocks=clk.result(), e2e=e2e, sel=sel,
+                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk,
                 launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
 
 
@@ -495,6 +537,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-rows", type=int, default=96)
     ap.add_argument("--no-select", action="store_true", help="skip the selection-attention measurement")
+    ap.add_argument("--no-masks", action="store_true", help="skip the masked-attention measurement")
     ap.add_argument("--select-steps", type=int, default=20)
     ap.add_argument("--select-cpu-budget", type=float, default=8.0)
     args = ap.parse_args()
@@ -574,6 +617,14 @@ def main():
             "cpu_baseline": cpu,
             "wall_s_timed_region": r["wall"],
         }
+        if r["msk"] is not None:
+            mt = r["msk"]["flops"] / (r["msk"]["ms"] * 1e-3) / 1e12
+            line["masked_attention"] = {
+                "what": "nsa_compress_attention with atten_mask and topk_mask (seeded, 30 % of entries set); "
+                        "FLOPs over the attended (visible, unmasked) pairs",
+                "ms": r["msk"]["ms"], "steps": r["msk"]["steps"], "tflops": mt,
+                "pct_of_bf16_peak": 100.0 * mt / peak_t, "flops_per_launch": r["msk"]["flops"],
+                "unmasked_ms": att_ms, "gpu_launches": r["msk"]["steps"]}
         if r["sel"] is not None:
             sf = select_flops(wl, r["sel"]["keys"])
             st = sf / (r["sel"]["ms"] * 1e-3) / 1e12                  # this GPU (rank 0)

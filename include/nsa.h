@@ -8,6 +8,8 @@
  *                           importance scores, head-group sum and per-query
  *                           top-k of selection blocks
  *                           ("mindspore.ops.nsa_compress_attention", steps 1-7);
+ *   nsa_compress_attention_masked  the same with the optional atten_mask /
+ *                           topk_mask of the page's keyword arguments
  *   nsa_select_attention    attention over the raw K/V blocks that top-k lists
  *                           ("lite_boost.ops.rain_fusion_attention").
  *
@@ -142,6 +144,38 @@ nsa_status_t nsa_compress_attention(
     int l, int d, int lp, int count,
     const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
     int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+    void* attention_out, int32_t* topk_indices, float* softmax_max, float* softmax_sum,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nsa_compress_attention with the page's optional keyword arguments
+ * ("mindspore.ops.nsa_compress_attention": atten_mask, shape (S1, S2) with S2
+ * the compressed KV length, applied to QK in step 1; topk_mask, shape
+ * (S1, S2) with S2 the select KV length, applied to P'_slc in step 6; dtype
+ * bool).  Reading of the page, which leaves both open: a non-zero byte at
+ * (row, block) removes that pair -- the block from the visible set of the
+ * row, or the selection block from its top-k candidates; one matrix serves
+ * every sequence of the batch and every head, and its row is the query's
+ * index inside its sequence (0 .. S_q-1).  The masks act on top of the
+ * built-in causal rules; a row left without an attended block is an empty
+ * row (zeros, max -inf, sum 0, indices -1).
+ *   atten_mask  device bytes, row-major, am_rows x am_cols (row stride
+ *               am_cols); NULL = no mask.  Needs am_rows >= every S_q and
+ *               am_cols >= every sequence's compressed block count.
+ *   topk_mask   device bytes, tm_rows x tm_cols, NULL = no mask.  Needs
+ *               tm_rows >= every S_q and tm_cols >= every n_sel.
+ * Other arguments, outputs, workspace (nsa_compress_attention_workspace_size)
+ * and errors as nsa_compress_attention; a mask too small for the batch is
+ * NSA_ERR_INVALID_ARG.  With both masks NULL the call is
+ * nsa_compress_attention.
+ */
+nsa_status_t nsa_compress_attention_masked(
+    const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
+    int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+    const uint8_t* atten_mask, int am_rows, int am_cols,
+    const uint8_t* topk_mask, int tm_rows, int tm_cols,
     void* attention_out, int32_t* topk_indices, float* softmax_max, float* softmax_sum,
     void* workspace, size_t workspace_bytes, void* stream);
 

@@ -33,6 +33,7 @@ EXPORTED = (
     "nsa_compress",
     "nsa_compress_attention_workspace_size",
     "nsa_compress_attention",
+    "nsa_compress_attention_masked",
     "nsa_workspace_status",
     "nsa_compress_status",
     "nsa_compress_attention_noalloc",
@@ -81,6 +82,10 @@ def load(path: Optional[str] = None):
     lib.nsa_compress_attention.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p, i32p,
                                            i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, cs, vp]
     lib.nsa_compress_attention.restype = ci
+    lib.nsa_compress_attention_masked.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p, i32p,
+                                                  i32p, ci, ci, ci, ci, ci, vp, ci, ci, vp, ci, ci, vp, vp, vp,
+                                                  vp, vp, cs, vp]
+    lib.nsa_compress_attention_masked.restype = ci
     lib.nsa_workspace_status.argtypes = [vp, vp]
     lib.nsa_workspace_status.restype = ci
     lib.nsa_compress_status.argtypes = [vp]
@@ -211,12 +216,16 @@ def nsa_compress_attention_workspace_size(head_num: int, n2: int, d1: int, d2: i
 def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tensor, scale: float,
                            head_num: int, l: int, d: int, lp: int, count: int, cu_seqlens_q,
                            cu_cmp_kv, cu_sel_kv, out=None, workspace: Optional[torch.Tensor] = None,
-                           stream=None):
+                           stream=None, atten_mask: Optional[torch.Tensor] = None,
+                           topk_mask: Optional[torch.Tensor] = None):
     """Compressed attention + importance scores + top-k.
 
     Returns (attention_out (T1,N1,D2), topk_indices (T1,N2,count) int32,
     softmax_max (T1,N1,8) fp32, softmax_sum (T1,N1,8) fp32).
-    ``out`` may pass these four tensors preallocated.
+    ``out`` may pass these four tensors preallocated.  ``atten_mask``
+    (S1, S2cmp) and ``topk_mask`` (S1, S2sel), bool or uint8 device tensors,
+    are the page's optional masks: True removes the (query, block) pair, one
+    matrix for every sequence and head, row = query index inside the sequence.
     """
     for t, nm in ((q, "q"), (kcmp, "kcmp"), (vcmp, "vcmp")):
         _dev(t, nm)
@@ -248,12 +257,31 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
     ws_bytes = nsa_compress_attention_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs)
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    st = load().nsa_compress_attention(
+    if atten_mask is None and topk_mask is None:
+        st = load().nsa_compress_attention(
+            q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
+            int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
+            tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
+            _stream(stream))
+        _raise(st, "nsa_compress_attention")
+        return att, tk, smax, ssum
+    masks = []
+    for mk, nm in ((atten_mask, "atten_mask"), (topk_mask, "topk_mask")):
+        if mk is None:
+            masks.append((None, 0, 0))
+            continue
+        _dev(mk, nm)
+        if mk.dim() != 2 or mk.dtype not in (torch.bool, torch.uint8) or not mk.is_contiguous():
+            raise TypeError(f"{nm} must be a contiguous 2-D bool or uint8 tensor (S1, S2)")
+        masks.append((mk, int(mk.shape[0]), int(mk.shape[1])))
+    (am, ar, ac), (tm, tr, tc_) = masks
+    st = load().nsa_compress_attention_masked(
         q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
-        int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
-        tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt,
+        am.data_ptr() if am is not None else None, ar, ac, tm.data_ptr() if tm is not None else None, tr, tc_,
+        att.data_ptr(), tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
         _stream(stream))
-    _raise(st, "nsa_compress_attention")
+    _raise(st, "nsa_compress_attention_masked")
     return att, tk, smax, ssum
 
 

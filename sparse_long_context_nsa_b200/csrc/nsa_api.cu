@@ -162,6 +162,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
                 t.n_cmp = n_cmp;
                 t.n_sel = n_sel;
                 t.t0 = (int)(tok0 + off);
+                t.tloc0 = (int)tok0;
                 const int nv = nvis_host(t.t0 + t.ntok - 1, l, d, n_cmp);
                 t.nkv = (nv + NKV - 1) / NKV;
                 for (int g = 0; g < n2; ++g) {
@@ -488,12 +489,16 @@ nsa_status_t nsa_compress_attention_workspace_size(int head_num, int n2, int d1,
     return NSA_OK;
 }
 
-nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
-                                    int l, int d, int lp, int count, const int32_t* cu_seqlens_q,
-                                    const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv, int batch, int n2, int d1,
-                                    int d2, nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
-                                    float* softmax_max, float* softmax_sum, void* workspace,
-                                    size_t workspace_bytes, void* stream) {
+// Steps 1-7 with the optional masks of steps 1 and 6 (null = none), already
+// validated against the shapes.
+static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, const void* vcmp, float scale,
+                                            int head_num, int l, int d, int lp, int count,
+                                            const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv,
+                                            const int32_t* cu_sel_kv, int batch, int n2, int d1, int d2,
+                                            nsa_dtype_t dtype, const uint8_t* atten_mask, int am_s2,
+                                            const uint8_t* topk_mask, int tm_s2, void* attention_out,
+                                            int32_t* topk_indices, float* softmax_max, float* softmax_sum,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
     if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
     if (!q || !kcmp || !vcmp || !attention_out || !topk_indices || !softmax_max || !softmax_sum)
@@ -572,9 +577,52 @@ nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void*
     p.off_score = pl.off_score;
     p.off_bar = pl.off_bar;
     p.smem_bytes = pl.smem_bytes;
+    p.amask = atten_mask;
+    p.am_s2 = am_s2;
+    p.tmask = topk_mask;
+    p.tm_s2 = tm_s2;
     const int grid = std::min(pl.grid, nsm);
     if (launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
     return NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
+                                    int l, int d, int lp, int count, const int32_t* cu_seqlens_q,
+                                    const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv, int batch, int n2, int d1,
+                                    int d2, nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
+                                    float* softmax_max, float* softmax_sum, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    return compress_attention_impl(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
+                                   cu_sel_kv, batch, n2, d1, d2, dtype, nullptr, 0, nullptr, 0, attention_out,
+                                   topk_indices, softmax_max, softmax_sum, workspace, workspace_bytes, stream);
+}
+
+nsa_status_t nsa_compress_attention_masked(const void* q, const void* kcmp, const void* vcmp, float scale,
+                                           int head_num, int l, int d, int lp, int count,
+                                           const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv,
+                                           const int32_t* cu_sel_kv, int batch, int n2, int d1, int d2,
+                                           nsa_dtype_t dtype, const uint8_t* atten_mask, int am_rows,
+                                           int am_cols, const uint8_t* topk_mask, int tm_rows, int tm_cols,
+                                           void* attention_out, int32_t* topk_indices, float* softmax_max,
+                                           float* softmax_sum, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+    // every sequence's query rows and blocks must lie inside each given mask
+    nsa_status_t s;
+    if ((s = check_prefix(cu_seqlens_q, batch)) != NSA_OK) return s;
+    if ((s = check_prefix(cu_cmp_kv, batch)) != NSA_OK) return s;
+    if ((s = check_prefix(cu_sel_kv, batch)) != NSA_OK) return s;
+    int64_t max_q = 0, max_c = 0, max_s = 0;
+    for (int b = 0; b < batch; ++b) {
+        max_q = std::max<int64_t>(max_q, cu_seqlens_q[b] - (b ? cu_seqlens_q[b - 1] : 0));
+        max_c = std::max<int64_t>(max_c, cu_cmp_kv[b] - (b ? cu_cmp_kv[b - 1] : 0));
+        max_s = std::max<int64_t>(max_s, cu_sel_kv[b] - (b ? cu_sel_kv[b - 1] : 0));
+    }
+    if (atten_mask && (am_rows < max_q || am_cols < max_c || am_cols < 1)) return NSA_ERR_INVALID_ARG;
+    if (topk_mask && (tm_rows < max_q || tm_cols < max_s || tm_cols < 1)) return NSA_ERR_INVALID_ARG;
+    return compress_attention_impl(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
+                                   cu_sel_kv, batch, n2, d1, d2, dtype, atten_mask, am_cols, topk_mask, tm_cols,
+                                   attention_out, topk_indices, softmax_max, softmax_sum, workspace,
+                                   workspace_bytes, stream);
 }
 
 nsa_status_t nsa_select_attention_workspace_size(int head_num, int n2, int d1, int d2, int lp, int count,

@@ -102,13 +102,16 @@ __device__ __forceinline__ int nvis_of(int t, int l, int d, int n_cmp) {
 // k-th largest key (fp32 bit pattern) of sc[0 .. ncand) held in registers,
 // NR keys per lane (key i of a lane belongs to j = lane + 32 i); keys at
 // j >= lim are 0.  Bitwise search from the top bit down.
-template <int NR>
-__device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int lim, int k, int lane) {
+template <int NR, bool kMask>
+__device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int lim, int k, int lane,
+                                                 const uint8_t* trow) {
     uint32_t key[NR];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
         const int j = lane + 32 * i;
-        key[i] = (j < lim) ? __float_as_uint(sc[j]) : 0u;
+        bool in = j < lim;
+        if constexpr (kMask) in = in && !(trow && trow[j]);
+        key[i] = in ? __float_as_uint(sc[j]) : 0u;
     }
     uint32_t thr = 0;
 #pragma unroll 1
@@ -131,41 +134,57 @@ __device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int
 // Exact k-th largest key by a bitwise search over the fp32 bit patterns
 // (scores are >= 0, so the bit patterns order like the values), then an
 // ordered ballot scan keeps every key above it plus the earliest ties, which
-// also lists the indices in ascending order.
+// also lists the indices in ascending order.  With a topk_mask row (kMask),
+// candidates whose mask byte is set are out of the set (step 6).
+template <bool kMask>
 __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, int count,
-                                          int32_t* dst, int lane) {
-    const int k = min(count, ncand);
-    if (k == ncand) {
+                                          int32_t* dst, int lane, const uint8_t* trow) {
+    auto masked = [&](int j) {
+        if constexpr (kMask) return trow != nullptr && trow[j] != 0;
+        return false;
+    };
+    int n_in = ncand;
+    if constexpr (kMask) {
+        if (trow) {
+            int nm = 0;
+            for (int j = lane; j < ncand; j += 32) nm += trow[j] ? 1 : 0;
+            n_in = ncand - __reduce_add_sync(0xffffffffu, nm);
+        }
+    }
+    const int k = min(count, n_in);
+    if (k == n_in && (!kMask || n_in == ncand)) {
         for (int j = lane; j < count; j += 32) dst[j] = (j < ncand) ? j : -1;
         return;
     }
     const int lim = min(ncand, jcov);          // keys at j >= lim are 0
     uint32_t thr = 0;
-    if (ncand <= 8 * 32) {
-        thr = kth_key_regs<8>(sc, ncand, lim, k, lane);
+    if (k == n_in) {
+        thr = 0;                               // every remaining candidate is taken
+    } else if (ncand <= 8 * 32) {
+        thr = kth_key_regs<8, kMask>(sc, ncand, lim, k, lane, trow);
     } else if (ncand <= 16 * 32) {
-        thr = kth_key_regs<16>(sc, ncand, lim, k, lane);
+        thr = kth_key_regs<16, kMask>(sc, ncand, lim, k, lane, trow);
     } else if (ncand <= 32 * 32) {
-        thr = kth_key_regs<32>(sc, ncand, lim, k, lane);
+        thr = kth_key_regs<32, kMask>(sc, ncand, lim, k, lane, trow);
     } else {
 #pragma unroll 1
         for (int bit = 31; bit >= 0; --bit) {
             const uint32_t trial = thr | (1u << bit);
             int c = 0;
-            for (int j = lane; j < lim; j += 32) c += __float_as_uint(sc[j]) >= trial ? 1 : 0;
+            for (int j = lane; j < lim; j += 32) c += (!masked(j) && __float_as_uint(sc[j]) >= trial) ? 1 : 0;
             c = __reduce_add_sync(0xffffffffu, c);
             if (c >= k) thr = trial;
         }
     }
     int ngt = 0;
-    for (int j = lane; j < lim; j += 32) ngt += __float_as_uint(sc[j]) > thr ? 1 : 0;
+    for (int j = lane; j < lim; j += 32) ngt += (!masked(j) && __float_as_uint(sc[j]) > thr) ? 1 : 0;
     ngt = __reduce_add_sync(0xffffffffu, ngt);
     const int need_eq = k - ngt;
     const uint32_t lt_mask = (1u << lane) - 1u;
     int eq_seen = 0, written = 0;
     for (int base = 0; base < ncand && written < k; base += 32) {
         const int j = base + lane;
-        const bool in = j < ncand;
+        const bool in = j < ncand && !masked(j < ncand ? j : 0);
         const uint32_t kv = (j < lim) ? __float_as_uint(sc[j]) : 0u;
         const bool gt = in && kv > thr;
         const bool eq = in && kv == thr;
@@ -226,7 +245,7 @@ __device__ __forceinline__ void p_half(float (&s)[N], float2 ce2, float2 nb2, ui
     }
 }
 
-template <typename T, int A>
+template <typename T, int A, bool kMask>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -494,6 +513,20 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int c = 0; c < NH; ++c) s[c0 + c] = (c0 + c < lim) ? s[c0 + c] : -INFINITY;
             }
         };
+        // atten_mask (step 1), masked kernel only: a set byte at (the row's
+        // query index, block) removes a visible block.  arow is the row's mask
+        // row, null for rows outside the tile or without a mask.
+        const uint8_t* arow = nullptr;
+        auto amask_cols = [&](float (&s)[NKV], int c0, int w, int i, int lim) {
+            if constexpr (kMask) {
+                if (arow != nullptr) {
+                    const uint8_t* mr = arow + (long long)i * NKV;
+#pragma unroll
+                    for (int c = 0; c < NKV; ++c)
+                        if (c >= c0 && c < c0 + w && c < lim && mr[c]) s[c] = -INFINITY;
+                }
+            }
+        };
         uint32_t split_sb = 0;
         auto open_half0 = [&](float (&s)[NKV], uint32_t (&r1)[NH]) {
             split_sb = scnt % nsbuf;
@@ -534,6 +567,8 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const bool valid = (row < TT * G) && (tok < t.ntok);
             const int tpos = t.t0 + tok;
             const int nvis = valid ? nvis_of(tpos, p.l, p.d, t.n_cmp) : 0;
+            if constexpr (kMask)
+                arow = (valid && p.amask != nullptr) ? p.amask + (long long)(t.tloc0 + tok) * p.am_s2 : nullptr;
 
             // ---------------- pass A: exact row max and sum (log2 domain) ----------------
             float m = -INFINITY, L = 0.f;
@@ -542,15 +577,18 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 uint32_t r1[NH];
                 open_half0(s, r1);
                 mask_half(s, 0, nvis - i * NKV);
+                amask_cols(s, 0, NH, i, nvis - i * NKV);
                 online_update<0, NH>(s, ce, m, L);
                 close_half1(s, r1);
                 mask_half(s, NH, nvis - i * NKV);
+                amask_cols(s, NH, NH, i, nvis - i * NKV);
                 online_update<NH, NH>(s, ce, m, L);
             }
             for (int i = 0; i < t.nkv && !kSplit; ++i) {
                 float s[NKV];
                 load_s(s);
                 prep(s, nvis - i * NKV);
+                amask_cols(s, 0, NKV, i, nvis - i * NKV);
                 // row maximum: four independent chains of 3-input max
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -601,16 +639,19 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     uint32_t r1[NH];
                     open_half0(s, r1);
                     mask_half(s, 0, nvis - i * NKV);
+                    amask_cols(s, 0, NH, i, nvis - i * NKV);
                     // P of the previous tile has been read by its P V
                     mbar_wait(bar(B_P_EMPTY), (pcnt & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 11);
                     tc_fence_after();
                     p_half<T, 0, NH>(s, ce2b, nb2, tmem_p + lane_off);
                     close_half1(s, r1);
                     mask_half(s, NH, nvis - i * NKV);
+                    amask_cols(s, NH, NH, i, nvis - i * NKV);
                     p_half<T, NH, NH>(s, ce2b, nb2, tmem_p + lane_off);
                 } else {
                 load_s(s);
                 prep(s, nvis - i * NKV);
+                amask_cols(s, 0, NKV, i, nvis - i * NKV);
                 {
 #pragma unroll
                     for (int c = 0; c < NKV; c += 2) {
@@ -769,11 +810,24 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int tau = ew; tau < t.ntok; tau += 4) {
                 const int tp = t.t0 + tau;
                 int32_t* dst = p.topk + ((size_t)(t.q_row0 + tau) * p.n2 + t.group) * p.count;
-                if (nvis_of(tp, p.l, p.d, t.n_cmp) == 0) {
+                const int nv = nvis_of(tp, p.l, p.d, t.n_cmp);
+                bool empty = nv == 0;
+                const uint8_t* trow = nullptr;
+                if constexpr (kMask) {
+                    // a token whose visible blocks are all masked attends to nothing
+                    if (!empty && p.amask != nullptr) {
+                        const uint8_t* ar = p.amask + (long long)(t.tloc0 + tau) * p.am_s2;
+                        int keep = 0;
+                        for (int c = lane; c < nv; c += 32) keep |= (ar[c] == 0) ? 1 : 0;
+                        empty = !__any_sync(0xffffffffu, keep);
+                    }
+                    if (p.tmask != nullptr) trow = p.tmask + (long long)(t.tloc0 + tau) * p.tm_s2;
+                }
+                if (empty) {
                     for (int j = lane; j < p.count; j += 32) dst[j] = -1;
                 } else {
                     const int ncand = min(t.n_sel, tp / p.lp + 1);
-                    warp_topk(score + tau * cap, ncand, jcov, p.count, dst, lane);
+                    warp_topk<kMask>(score + tau * cap, ncand, jcov, p.count, dst, lane, trow);
                 }
             }
             named_bar_sync(2, 128);   // the score buffer is free for the next tile
@@ -795,36 +849,40 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 }
 
-template <typename T, int A>
+template <typename T, int A, bool kMask>
 static cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, int grid, cudaStream_t st) {
-    auto kern = nsa_cmp_attn_kernel<T, A>;
+    auto kern = nsa_cmp_attn_kernel<T, A, kMask>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
     kern<<<grid, kAttnThreads, p.smem_bytes, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, bool kMask>
 static cudaError_t launch_a(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, int grid, cudaStream_t st) {
     switch (p.a) {
-        case 1: return launch_t<T, 1>(p, tq, tk, tv, grid, st);
-        case 2: return launch_t<T, 2>(p, tq, tk, tv, grid, st);
-        case 3: return launch_t<T, 3>(p, tq, tk, tv, grid, st);
-        case 4: return launch_t<T, 4>(p, tq, tk, tv, grid, st);
-        case 5: return launch_t<T, 5>(p, tq, tk, tv, grid, st);
-        case 6: return launch_t<T, 6>(p, tq, tk, tv, grid, st);
-        case 7: return launch_t<T, 7>(p, tq, tk, tv, grid, st);
-        case 8: return launch_t<T, 8>(p, tq, tk, tv, grid, st);
+        case 1: return launch_t<T, 1, kMask>(p, tq, tk, tv, grid, st);
+        case 2: return launch_t<T, 2, kMask>(p, tq, tk, tv, grid, st);
+        case 3: return launch_t<T, 3, kMask>(p, tq, tk, tv, grid, st);
+        case 4: return launch_t<T, 4, kMask>(p, tq, tk, tv, grid, st);
+        case 5: return launch_t<T, 5, kMask>(p, tq, tk, tv, grid, st);
+        case 6: return launch_t<T, 6, kMask>(p, tq, tk, tv, grid, st);
+        case 7: return launch_t<T, 7, kMask>(p, tq, tk, tv, grid, st);
+        case 8: return launch_t<T, 8, kMask>(p, tq, tk, tv, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, int grid, cudaStream_t st) {
-    return p.dtype == 0 ? launch_a<__nv_bfloat16>(p, tq, tk, tv, grid, st)
-                        : launch_a<__half>(p, tq, tk, tv, grid, st);
+    // the masked kernel only where a mask is given: the unmasked one is unchanged
+    if (p.amask != nullptr || p.tmask != nullptr)
+        return p.dtype == 0 ? launch_a<__nv_bfloat16, true>(p, tq, tk, tv, grid, st)
+                            : launch_a<__half, true>(p, tq, tk, tv, grid, st);
+    return p.dtype == 0 ? launch_a<__nv_bfloat16, false>(p, tq, tk, tv, grid, st)
+                        : launch_a<__half, false>(p, tq, tk, tv, grid, st);
 }
 
 }  // namespace nsa

@@ -64,6 +64,7 @@ struct AttnTile {
     int n_sel;      // selection blocks of the sequence
     int t0;         // position of the first token (query offset applied)
     int nkv;        // KV tiles to visit (both passes)
+    int tloc0;      // query index of the first token inside its sequence (mask rows)
 };
 
 struct AttnParams {
@@ -89,6 +90,12 @@ struct AttnParams {
     // shared-memory layout (byte offsets from a 1024-aligned base)
     int off_q, q_bytes, off_ring, slot_bytes, off_stage, stage_entry_bytes, off_score, off_bar,
         smem_bytes;
+    // optional masks (null = none): bool bytes (S1, row stride), one matrix for
+    // every sequence and head, row = query index inside the sequence
+    const uint8_t* amask;   // (S1, >= n_cmp): true removes the compressed block (step 1)
+    long long am_s2;
+    const uint8_t* tmask;   // (S1, >= n_sel): true removes the top-k candidate (step 6)
+    long long tm_s2;
 };
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,

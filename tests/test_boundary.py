@@ -228,3 +228,31 @@ def _call_select(lib, **kw):
 ])
 def test_select_rejects_before_launch(lib, kw, status):
     assert _call_select(lib, **kw) == status
+
+
+def _call_masked(lib, **kw):
+    a = dict(q=4096, kcmp=4096, vcmp=4096, scale=0.1, head_num=64, l=32, d=16, lp=64, count=16,
+             cq=[16384], cc=[1023], cs=[256], n2=4, d1=128, d2=128, dtype=0, am=4096, ar=16384, ac=1023,
+             tm=4096, tr=16384, tc=256, out=4096, tk=4096, smax=4096, ssum=4096, ws=4096, wsb=1 << 30)
+    a.update(kw)
+    arr = lambda x: np.ascontiguousarray(np.asarray(x, np.int32))
+    cq, cc, cs = arr(a["cq"]), arr(a["cc"]), arr(a["cs"])
+    ip = lambda x: x.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    return lib.nsa_compress_attention_masked(
+        a["q"], a["kcmp"], a["vcmp"], a["scale"], a["head_num"], a["l"], a["d"], a["lp"], a["count"], ip(cq),
+        ip(cc), ip(cs), cq.size, a["n2"], a["d1"], a["d2"], a["dtype"], a["am"], a["ar"], a["ac"], a["tm"],
+        a["tr"], a["tc"], a["out"], a["tk"], a["smax"], a["ssum"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ar=16383), nsa.NSA_ERR_INVALID_ARG),          # fewer mask rows than queries
+    (dict(ac=1022), nsa.NSA_ERR_INVALID_ARG),           # fewer columns than compressed blocks
+    (dict(tr=100), nsa.NSA_ERR_INVALID_ARG),
+    (dict(tc=255), nsa.NSA_ERR_INVALID_ARG),            # fewer columns than selection blocks
+    (dict(cq=[10, 5], cc=[0, 0], cs=[1, 1]), nsa.NSA_ERR_INVALID_ARG),
+    (dict(q=None), nsa.NSA_ERR_INVALID_ARG),
+    (dict(ws=None), nsa.NSA_ERR_WORKSPACE),
+    (dict(am=None, ar=0, ac=0, ws=4096 + 8), nsa.NSA_ERR_WORKSPACE),   # a mask may be absent
+])
+def test_masked_attention_rejects_before_launch(lib, kw, status):
+    assert _call_masked(lib, **kw) == status
