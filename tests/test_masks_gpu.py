@@ -102,6 +102,22 @@ def test_random_masks(nsa, l, d, lp):
     _check(res, ref, wl, x, tm)
 
 
+@pytest.mark.parametrize("l,d,lp", [(32, 16, 64), (32, 16, 32)], ids=["a4", "a2"])
+def test_masks_wider_than_the_blocks(nsa, l, d, lp):
+    # mask rows longer than the blocks of any sequence (padded to a multiple
+    # of 16 bytes); the extra columns are set and must be ignored
+    wl = _wl([1300, 200], 16, 2, 64, l, d, lp, 6, seed=25)
+    x, kc, vc, cuc = _inputs(wl)
+    am, tm = _masks(wl, x, cuc, 0.3, 0.3, seed=6)
+    pad = lambda m_: np.concatenate([m_, np.ones((m_.shape[0], -m_.shape[1] % 16 or 16), bool)], axis=1)
+    am, tm = pad(am), pad(tm)
+    assert am.shape[1] % 16 == 0 and tm.shape[1] % 16 == 0
+    res = _gpu(nsa, wl, x, kc, vc, cuc, am, tm)
+    ref = oracle.compress_attention(x["q"], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
+                                    x["cu_sel_kv"], atten_mask=am, topk_mask=tm)
+    _check(res, ref, wl, x, tm)
+
+
 def test_one_mask_at_a_time_and_fully_masked_rows(nsa):
     wl = _wl([900], 8, 2, 64, 32, 16, 64, 5, seed=22)
     x, kc, vc, cuc = _inputs(wl)
