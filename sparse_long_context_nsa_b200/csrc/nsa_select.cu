@@ -147,14 +147,15 @@ cudaError_t launch_plan(const Params& p, int max_words, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 // Attention over the listed blocks.  LP = l' keys per KV tile.
 //
-// One pass with an online softmax per row.  The row's reference maximum m
-// moves up only when a block's maximum exceeds it by more than 8 (exponent
-// units, base 2): P = 2^(x - m) then stays at most 2^8, and O and L are
-// rescaled by 2^(m_old - m_new) only at those moves.  O / L and the
-// log-sum-exp are formed once per tile.  P is written, in the storage dtype,
-// over the first l'/2 columns of the score buffer it came from; the buffer is
-// reused once the P V that reads it has retired.  A warp none of whose rows
-// attend to a block skips the exponentials and writes zero P.
+// A KV tile holds BPT listed blocks side by side (NKV = BPT * l' keys).  One
+// pass with an online softmax per row: the row's reference maximum m moves
+// up only when a KV tile's maximum exceeds it by more than 8 (exponent units,
+// base 2): P = 2^(x - m) then stays at most 2^8, and O and L are rescaled by
+// 2^(m_old - m_new) only at those moves.  O / L and the log-sum-exp are
+// formed once per M-tile.  P is written, in the storage dtype, over the first
+// NKV/2 columns of the score buffer it came from; the buffer is reused once
+// the P V that reads it has retired.  A warp none of whose rows attend to a
+// KV tile skips the exponentials and writes zero P.
 // ---------------------------------------------------------------------------
 template <typename T, int LP>
 __global__ void __launch_bounds__(kThreads, 1)
