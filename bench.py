@@ -365,7 +365,7 @@ def run_ours(args, rank, world, local_rank):
             vis = np.arange(n_c)[None, :] * wl.d + wl.l - 1 <= tpos
             pairs += int((vis & ~am[:n_q, :n_c]).sum())
         msk = dict(ms=float(np.mean([e[0].elapsed_time(e[1]) for e in mev])), steps=km,
-                   flops=2.0 * (wl.d1 + wl.d2) * wl.n1 * pairs)
+                   flops=2.0 * (wl.d1 + wl.d2) * wl.n1 * pairs, am=am, tm=tm)
 
     # ---------- selection attention over the step's own top-k lists ----------
     sel = None
@@ -473,6 +473,45 @@ def select_cpu_baseline(wl, topk, keys, budget_s=8.0):
     dt = time.perf_counter() - t0
     return {"value": select_flops(wl, keys[rows]) / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "sample": f"{rows.size} of {T1} evenly spaced query rows, all heads, {dt:.1f} s"}
+
+
+def masked_cpu_baseline(wl, am, tm, budget_s=8.0):
+    """The oracle with the same masks, as it stands, on evenly spaced query rows
+    (all heads); FLOPs over the attended (visible, unmasked) pairs of those rows."""
+    import oracle
+    x = wl.generate(device="cpu")
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
+    kc, cuc = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    vc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    cq = x["cu_seqlens_q"]
+    T1 = int(cq[-1])
+
+    def run(rows):
+        oracle.compress_attention(x["q"][rows], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+                                  x["cu_sel_kv"], rows=rows, q_rows_only=True, atten_mask=am, topk_mask=tm)
+
+    probe = np.unique(np.linspace(0, T1 - 1, num=min(T1, 32)).astype(np.int64))
+    tp = time.perf_counter()
+    run(probe)
+    per_row = (time.perf_counter() - tp) / probe.size
+    rows = np.unique(np.linspace(0, T1 - 1, num=int(max(16, min(T1, budget_s / max(per_row, 1e-6))))).astype(np.int64))
+    t0 = time.perf_counter()
+    run(rows)
+    dt_s = time.perf_counter() - t0
+    pairs, prev = 0, 0
+    for b, end in enumerate(cq.tolist()):
+        sel = rows[(rows >= prev) & (rows < end)]
+        S = wl.seqlens[b]
+        n_cmp = 0 if S < wl.l else (S - wl.l) // wl.d + 1
+        if n_cmp and sel.size:
+            off = max(0, (n_cmp - 1) * wl.d + wl.l - (end - prev))
+            tloc = sel - prev
+            vis = np.arange(n_cmp)[None, :] * wl.d + wl.l - 1 <= (tloc + off)[:, None]
+            pairs += int((vis & ~am[tloc, :n_cmp]).sum())
+        prev = end
+    return {"value": 2.0 * (wl.d1 + wl.d2) * wl.n1 * pairs / dt_s / 1e12, "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows.size} of {T1} evenly spaced query rows, all heads, same masks, {dt_s:.1f} s"}
 
 
 def run_reference(args, rank, world):
@@ -624,7 +663,13 @@ def main():
                         "FLOPs over the attended (visible, unmasked) pairs",
                 "ms": r["msk"]["ms"], "steps": r["msk"]["steps"], "tflops": mt,
                 "pct_of_bf16_peak": 100.0 * mt / peak_t, "flops_per_launch": r["msk"]["flops"],
-                "unmasked_ms": att_ms, "gpu_launches": r["msk"]["steps"]}
+                "unmasked_ms": att_ms, "gpu_launches": r["msk"]["steps"],
+                "roofline": {"bound": "tensor", "achieved": mt, "peak": peak_t, "unit": "TFLOP/s",
+                             "frac": mt / peak_t, "traffic": None,
+                             "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                "cpu_baseline": (masked_cpu_baseline(wl, r["msk"]["am"], r["msk"]["tm"],
+                                                     budget_s=args.select_cpu_budget)
+                                 if (not args.no_cpu_baseline and world == 1) else None)}
         if r["sel"] is not None:
             sf = select_flops(wl, r["sel"]["keys"])
             st = sf / (r["sel"]["ms"] * 1e-3) / 1e12                  # this GPU (rank 0)
