@@ -131,6 +131,32 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"dtype must be bfloat16 or float16, got {t.dtype}")
 
 
+def _same_device(ref: torch.Tensor, *named) -> None:
+    for t, name in named:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} must be on {ref.device}")
+
+
+def _out(t: torch.Tensor, shape, dtype, device, name: str) -> torch.Tensor:
+    """A caller-provided output: the kernels write exactly this shape, so
+    anything else is refused before the launch."""
+    _dev(t, name)
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+    return t
+
+
+def _workspace(ws: torch.Tensor, nbytes: int, device) -> torch.Tensor:
+    if ws is None or ws.numel() < nbytes:
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    _dev(ws, "workspace")
+    if ws.device != device or ws.dtype != torch.uint8:
+        raise ValueError(f"workspace must be a uint8 tensor on {device}")
+    return ws
+
+
 def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -177,6 +203,7 @@ def nsa_compress(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tensor, l:
         raise ValueError("k must be (T2, N2, D1) and w (l, N2)")
     t2, n2, d1 = k.shape
     d2 = d1
+    _same_device(k, (w, "w"), (v, "v"))
     if v is not None:
         _dev(v, "v")
         if v.dim() != 3 or v.shape[:2] != k.shape[:2]:
@@ -191,8 +218,12 @@ def nsa_compress(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tensor, l:
     tc = int(cuc[-1])
     if kcmp is None:
         kcmp = torch.empty(tc, n2, d1, dtype=k.dtype, device=k.device)
+    else:
+        _out(kcmp, (tc, n2, d1), k.dtype, k.device, "kcmp")
     if v is not None and vcmp is None:
         vcmp = torch.empty(tc, n2, d2, dtype=k.dtype, device=k.device)
+    elif v is not None:
+        _out(vcmp, (tc, n2, d2), k.dtype, k.device, "vcmp")
     st = load().nsa_compress(k.data_ptr(), v.data_ptr() if v is not None else None, w.data_ptr(),
                              int(l), int(d), _ip(cu), cu.size, n2, d1, d2, dt, kcmp.data_ptr(),
                              vcmp.data_ptr() if v is not None else None, _stream(stream))
@@ -247,6 +278,7 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
     if int(cq[-1]) > t1 or int(cc[-1]) > tc:
         raise ValueError("prefix sums run past the rows of q / kcmp")
     dev = q.device
+    _same_device(q, (kcmp, "kcmp"), (vcmp, "vcmp"))
     if out is None:
         att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
         tk = torch.empty(t1, n2, count, dtype=torch.int32, device=dev)
@@ -254,9 +286,12 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
         ssum = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
     else:
         att, tk, smax, ssum = out
+        _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
+        _out(tk, (t1, n2, count), torch.int32, dev, "topk_indices")
+        _out(smax, (t1, n1, 8), torch.float32, dev, "softmax_max")
+        _out(ssum, (t1, n1, 8), torch.float32, dev, "softmax_sum")
     ws_bytes = nsa_compress_attention_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs)
-    if workspace is None or workspace.numel() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    workspace = _workspace(workspace, ws_bytes, dev)
     if atten_mask is None and topk_mask is None:
         st = load().nsa_compress_attention(
             q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
@@ -271,6 +306,8 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
             masks.append((None, 0, 0))
             continue
         _dev(mk, nm)
+        if mk.device != q.device:
+            raise ValueError(f"{nm} must be on the device of q")
         if mk.dim() != 2 or mk.dtype not in (torch.bool, torch.uint8) or not mk.is_contiguous():
             raise TypeError(f"{nm} must be a contiguous 2-D bool or uint8 tensor (S1, S2)")
         masks.append((mk, int(mk.shape[0]), int(mk.shape[1])))
@@ -296,14 +333,29 @@ def nsa_compress_attention_noalloc(q: torch.Tensor, kcmp: torch.Tensor, vcmp: to
     """
     for t, nm in ((q, "q"), (kcmp, "kcmp"), (vcmp, "vcmp")):
         _dev(t, nm)
-    att, tk, smax, ssum = out
-    for t, nm in ((att, "attention_out"), (tk, "topk_indices"), (smax, "softmax_max"), (ssum, "softmax_sum")):
-        _dev(t, nm)
+        if t.dim() != 3:
+            raise ValueError(f"{nm} must be 3-D (TND)")
+    _same_device(q, (kcmp, "kcmp"), (vcmp, "vcmp"))
     dt = _dtype_code(q)
+    if kcmp.dtype != q.dtype or vcmp.dtype != q.dtype:
+        raise TypeError("q, kcmp and vcmp must share one dtype")
     t1, n1, d1 = q.shape
-    tc, n2, _ = kcmp.shape
+    tc, n2, d1k = kcmp.shape
     d2 = vcmp.shape[2]
+    if int(head_num) != n1:
+        raise ValueError("head_num must equal the number of query heads")
+    if d1k != d1 or tuple(vcmp.shape[:2]) != (tc, n2):
+        raise ValueError("kcmp must be (Tc, N2, D1) and vcmp (Tc, N2, D2)")
     cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size):
+        raise ValueError("the three prefix-sum lists need one entry per sequence")
+    if int(cq[-1]) > t1 or int(cc[-1]) > tc:
+        raise ValueError("prefix sums run past the rows of q / kcmp")
+    att, tk, smax, ssum = out
+    _out(att, (t1, n1, d2), q.dtype, q.device, "attention_out")
+    _out(tk, (t1, n2, count), torch.int32, q.device, "topk_indices")
+    _out(smax, (t1, n1, 8), torch.float32, q.device, "softmax_max")
+    _out(ssum, (t1, n1, 8), torch.float32, q.device, "softmax_sum")
     st = load().nsa_compress_attention_noalloc(
         q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
         int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
@@ -367,14 +419,16 @@ def nsa_select_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk
     if int(cq[-1]) > t1 or int(ck[-1]) > t2:
         raise ValueError("prefix sums run past the rows of q / k")
     dev = q.device
+    _same_device(q, (k, "k"), (v, "v"), (topk_indices, "topk_indices"))
     if out is None:
         att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
         lse = torch.empty(t1, n1, dtype=torch.float32, device=dev)
     else:
         att, lse = out
+        _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
+        _out(lse, (t1, n1), torch.float32, dev, "softmax_lse")
     ws_bytes = nsa_select_attention_workspace_size(n1, n2, d1, d2, lp, count, cq, ck)
-    if workspace is None or workspace.numel() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    workspace = _workspace(workspace, ws_bytes, dev)
     st = load().nsa_select_attention(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), topk_indices.data_ptr(), float(scale), int(head_num),
         int(lp), int(count), _ip(cq), _ip(ck), cq.size, n2, d1, d2, dt, att.data_ptr(), lse.data_ptr(),
