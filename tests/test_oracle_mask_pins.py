@@ -142,3 +142,24 @@ def test_masks_are_indexed_by_the_query_inside_its_sequence():
         for key in ("out", "topk", "softmax_sum"):
             assert np.array_equal(one[key], both[key][q0:cq[b]]), key
         q0, c0 = cq[b], cc[b]
+
+
+def test_closed_form_equal_scores_under_a_mask():
+    # q = 0: every visible score is 0, so a row's output is the mean of its
+    # visible, unmasked value blocks, softmax_max = 0 and softmax_sum = their count
+    S, n1, n2, dd = 200, 2, 1, 4
+    n_cmp = (S - L_) // D_ + 1
+    n_sel = -(-S // LP_)
+    q = np.zeros((S, n1, dd))
+    kc = np.random.default_rng(0).standard_normal((n_cmp, n2, dd))
+    vc = np.arange(n_cmp, dtype=np.float64)[:, None, None] * np.ones((1, n2, dd))
+    am = np.zeros((S, n_cmp), bool)
+    am[:, 1::3] = True                     # every third block from 1 on
+    r = oracle.compress_attention(q, kc, vc, 0.5, L_, D_, LP_, 2, [S], [n_cmp], [n_sel], atten_mask=am)
+    for t in range(S):
+        kept = [i for i in range(n_cmp) if i * D_ + L_ - 1 <= t and not am[t, i]]
+        if not kept:
+            assert np.isneginf(r["softmax_max"][t]).all() and (r["out"][t] == 0).all()
+            continue
+        assert np.allclose(r["out"][t], np.mean(kept), rtol=0, atol=1e-12)
+        assert (r["softmax_max"][t] == 0).all() and np.allclose(r["softmax_sum"][t], len(kept), atol=1e-12)

@@ -142,3 +142,32 @@ def test_varlen_sequences_are_independent_and_rows_sample():
     rows = np.array([0, 29, 30, 31, 75], dtype=np.int64)
     samp = oracle.select_attention(q[rows], k, v, sel, 0.4, lp, 3, cq, ck, rows=rows, q_rows_only=True)
     assert np.array_equal(samp["out"], allr["out"][rows])
+
+
+def test_closed_form_two_keys():
+    # q = (1, 0); k_0 = (1, 0), k_1 = (0, 1); v_0 = (1, 0), v_1 = (0, 2); scale 1;
+    # blocks of one key, row 1 lists both: weights e/(e+1), 1/(e+1)
+    q = np.array([[[0.0, 0.0]], [[1.0, 0.0]]])
+    k = np.array([[[1.0, 0.0]], [[0.0, 1.0]]])
+    v = np.array([[[1.0, 0.0]], [[0.0, 2.0]]])
+    sel = np.array([[[0, -1]], [[0, 1]]], np.int32)
+    r = oracle.select_attention(q, k, v, sel, 1.0, 1, 2, [2], [2])
+    e = np.e
+    assert np.allclose(r["out"][1, 0], [e / (e + 1), 2 / (e + 1)], rtol=0, atol=1e-15)
+    assert abs(r["lse"][1, 0] - np.log(e + 1)) < 1e-15
+    # row 0 sees only key 0: the output is v_0, the lse its scaled score (0)
+    assert np.array_equal(r["out"][0, 0], [1.0, 0.0]) and r["lse"][0, 0] == 0.0
+
+
+def test_closed_form_causal_cut_inside_a_block():
+    # one block of 4 keys; row t sees keys 0..t: with equal scores the output
+    # is the mean of the first t+1 value rows and the lse is log(t+1)
+    S = 4
+    q = np.zeros((S, 1, 2))
+    k = np.zeros((S, 1, 2))
+    v = np.arange(S, dtype=np.float64).reshape(S, 1, 1) * np.ones((1, 1, 2))
+    sel = np.zeros((S, 1, 1), np.int32)
+    r = oracle.select_attention(q, k, v, sel, 0.7, 4, 1, [S], [S])
+    for t in range(S):
+        assert np.allclose(r["out"][t, 0], np.full(2, t / 2.0), rtol=0, atol=1e-15)
+        assert abs(r["lse"][t, 0] - np.log(t + 1)) < 1e-15
