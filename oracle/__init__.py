@@ -86,6 +86,15 @@ def _load():
             ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
             _f64p, _f64p]
         lib.oracle_select_attention.restype = ctypes.c_int
+        lib.oracle_compress_attention_backward.argtypes = [
+            _f64p, _f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_int64, _f64p, _f64p, _f64p]
+        lib.oracle_compress_attention_backward.restype = ctypes.c_int
+        lib.oracle_compress_backward.argtypes = [
+            _f64p, _f64p, _f64p, ctypes.c_int, ctypes.c_int, _i32p, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, _f64p, _f64p]
+        lib.oracle_compress_backward.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
         return lib
@@ -278,3 +287,44 @@ def select_attention(q, k, v, sel, scale: float, lp: int, count: int, cu_seqlens
         if rc != 0:
             raise ValueError("oracle: bad selection-attention arguments")
     return {"out": out, "lse": lse, "rows": rows_arr}
+
+
+def compress_attention_backward(q, kcmp, vcmp, dout, scale: float, l: int, d: int, cu_seqlens_q,
+                                cu_cmp_kv, atten_mask=None):
+    """Gradient of attention_out (steps 1-3) with respect to q, kcmp and vcmp
+    for the incoming dout (T1, N1, D2); the importance scores and the top-k
+    carry none.  ``atten_mask`` as in compress_attention.  Returns a dict
+    with dq (T1, N1, D1), dkcmp (Tc, N2, D1), dvcmp (Tc, N2, D2), fp64."""
+    qf, kf, vf, gf = _f64(q), _f64(kcmp), _f64(vcmp), _f64(dout)
+    t1, n1, d1 = qf.shape
+    tc, n2, _ = kf.shape
+    d2 = vf.shape[2]
+    assert gf.shape == (t1, n1, d2)
+    cq, cc = _i32(cu_seqlens_q), _i32(cu_cmp_kv)
+    am, am_s2 = None, 0
+    if atten_mask is not None:
+        am = np.ascontiguousarray(np.asarray(atten_mask).astype(np.uint8))
+        am_s2 = am.shape[1]
+    dq = np.zeros((t1, n1, d1))
+    dk = np.zeros((max(tc, 1), n2, d1))
+    dv = np.zeros((max(tc, 1), n2, d2))
+    rc = _load().oracle_compress_attention_backward(
+        qf, kf if kf.size else np.zeros(1), vf if vf.size else np.zeros(1), gf, float(scale), n1, n2, d1, d2,
+        int(l), int(d), cq, cc, cq.size, am.ctypes.data_as(ctypes.c_void_p) if am is not None else None,
+        am_s2, dq, dk, dv)
+    if rc != 0:
+        raise ValueError("oracle: N1 must be a multiple of N2")
+    return {"dq": dq, "dkcmp": dk[:tc], "dvcmp": dv[:tc]}
+
+
+def compress_backward(x, w, dcmp, l: int, d: int, cu_seqlens):
+    """Gradient of the compression of x (T, N2, D) with weights w (l, N2) for
+    the incoming dcmp (Tc, N2, D).  Returns (dx (T, N2, D), dw (l, N2)), fp64."""
+    xf, wf, gf = _f64(x), _f64(w), _f64(dcmp)
+    T, n2, dim = xf.shape
+    cu = _i32(cu_seqlens)
+    dx = np.zeros((T, n2, dim))
+    dw = np.zeros((l, n2))
+    _load().oracle_compress_backward(xf, wf, gf if gf.size else np.zeros(1), int(l), int(d), cu, cu.size, n2,
+                                     dim, dx, dw)
+    return dx, dw

@@ -442,3 +442,138 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------- */
+/* Backward of [ATT] steps 1-3: the gradient of attention_out with respect   */
+/* to q, kcmp and vcmp (the importance scores and the top-k are indices and  */
+/* carry none).  Derived from the forward definition: for query row t, head  */
+/* h of group g and its attended blocks i (visible by the causal rule and    */
+/* not removed by amask), with s_i = scale q.k_i, P = softmax(s), O = sum    */
+/* P_i v_i and the incoming dO:                                              */
+/*   dv_i += P_i dO                                                          */
+/*   dP_i  = dO . v_i,   dS_i = P_i (dP_i - sum_j P_j dP_j)                  */
+/*   dq    = scale sum_i dS_i k_i,   dk_i += scale dS_i q                    */
+/* A row that attends to nothing contributes nothing.  dq (T1, N1, D1);      */
+/* dkc (Tc, N2, D1) and dvc (Tc, N2, D2) sum over the rows and the G heads  */
+/* of each group.  Single-threaded (the sums are shared between rows).       */
+/* ------------------------------------------------------------------------- */
+int oracle_compress_attention_backward(const double* q, const double* kc, const double* vc,
+                                       const double* dout, double scale, int n1, int n2,
+                                       int d1, int d2, int l, int d,
+                                       const int32_t* cu_q, const int32_t* cu_cmp, int batch,
+                                       const uint8_t* amask, int64_t am_s2,
+                                       double* dq, double* dkc, double* dvc)
+{
+    if (n2 <= 0 || n1 % n2 != 0) return -1;
+    const int G = n1 / n2;
+    const int64_t T1 = batch ? cu_q[batch - 1] : 0;
+    const int64_t Tc = batch ? cu_cmp[batch - 1] : 0;
+    for (int64_t x = 0; x < T1 * n1 * d1; x++) dq[x] = 0.0;
+    for (int64_t x = 0; x < Tc * n2 * d1; x++) dkc[x] = 0.0;
+    for (int64_t x = 0; x < Tc * n2 * d2; x++) dvc[x] = 0.0;
+    int max_cmp = 1;
+    for (int s = 0; s < batch; s++) {
+        int nc = cu_cmp[s] - (s ? cu_cmp[s - 1] : 0);
+        if (nc > max_cmp) max_cmp = nc;
+    }
+    double* sc = (double*)malloc(sizeof(double) * (size_t)max_cmp);
+    double* P = (double*)malloc(sizeof(double) * (size_t)max_cmp);
+    double* dP = (double*)malloc(sizeof(double) * (size_t)max_cmp);
+    char* att = (char*)malloc((size_t)max_cmp);
+    for (int s = 0; s < batch; s++) {
+        const int64_t q0 = s ? cu_q[s - 1] : 0, c0 = s ? cu_cmp[s - 1] : 0;
+        const int64_t Sq = cu_q[s] - q0;
+        const int n_cmp = (int)(cu_cmp[s] - c0);
+        int64_t off = 0;
+        if (n_cmp > 0) {
+            off = (int64_t)(n_cmp - 1) * d + l - Sq;
+            if (off < 0) off = 0;
+        }
+        for (int64_t tl = 0; tl < Sq; tl++) {
+            const int64_t t = q0 + tl, tpos = tl + off;
+            int n_att = 0;
+            for (int i = 0; i < n_cmp; i++) {
+                att[i] = ((int64_t)i * d + l - 1 <= tpos) && !(amask && amask[tl * am_s2 + i]);
+                n_att += att[i];
+            }
+            if (n_att == 0) continue;
+            for (int h = 0; h < n1; h++) {
+                const int g = h / G;
+                const double* qr = q + (t * n1 + h) * (int64_t)d1;
+                const double* dor = dout + (t * n1 + h) * (int64_t)d2;
+                double m = -INFINITY;
+                for (int i = 0; i < n_cmp; i++) {
+                    if (!att[i]) continue;
+                    const double* kr = kc + ((c0 + i) * n2 + g) * (int64_t)d1;
+                    double acc = 0.0;
+                    for (int e = 0; e < d1; e++) acc += qr[e] * kr[e];
+                    sc[i] = scale * acc;
+                    if (sc[i] > m) m = sc[i];
+                }
+                double L = 0.0;
+                for (int i = 0; i < n_cmp; i++) if (att[i]) L += exp(sc[i] - m);
+                double delta = 0.0;
+                for (int i = 0; i < n_cmp; i++) {
+                    if (!att[i]) continue;
+                    P[i] = exp(sc[i] - m) / L;
+                    const double* vr = vc + ((c0 + i) * n2 + g) * (int64_t)d2;
+                    double acc = 0.0;
+                    for (int e = 0; e < d2; e++) acc += dor[e] * vr[e];
+                    dP[i] = acc;
+                    delta += P[i] * acc;
+                }
+                double* dqr = dq + (t * n1 + h) * (int64_t)d1;
+                for (int i = 0; i < n_cmp; i++) {
+                    if (!att[i]) continue;
+                    const double dS = P[i] * (dP[i] - delta);
+                    const double* kr = kc + ((c0 + i) * n2 + g) * (int64_t)d1;
+                    double* dkr = dkc + ((c0 + i) * n2 + g) * (int64_t)d1;
+                    double* dvr = dvc + ((c0 + i) * n2 + g) * (int64_t)d2;
+                    for (int e = 0; e < d1; e++) {
+                        dqr[e] += scale * dS * kr[e];
+                        dkr[e] += scale * dS * qr[e];
+                    }
+                    for (int e = 0; e < d2; e++) dvr[e] += P[i] * dor[e];
+                }
+            }
+        }
+    }
+    free(sc); free(P); free(dP); free(att);
+    return 0;
+}
+
+/* Backward of the compression ([NSA-C] Formula, phi = weighted window sum): */
+/* out[c0+i, n, :] = sum_{j<l} w[j, n] x[s0 + i d + j, n, :] is linear in x  */
+/* and w, so dx[s0 + i d + j, n, :] += w[j, n] dout[c0+i, n, :] and          */
+/* dw[j, n] += x[s0 + i d + j, n, :] . dout[c0+i, n, :].  dx (T, N2, D) and  */
+/* dw (l, N2) are zeroed here; for K and V sharing w, dw is their sum.       */
+int oracle_compress_backward(const double* x, const double* w, const double* dout, int l, int d,
+                             const int32_t* cu, int batch, int n2, int dim, double* dx, double* dw)
+{
+    const int64_t T = batch ? cu[batch - 1] : 0;
+    for (int64_t e = 0; e < T * n2 * dim; e++) dx[e] = 0.0;
+    for (int e = 0; e < l * n2; e++) dw[e] = 0.0;
+    int64_t c0 = 0;
+    for (int s = 0; s < batch; s++) {
+        const int64_t s0 = s ? cu[s - 1] : 0, S = cu[s] - s0;
+        const int64_t n_cmp = (S < l) ? 0 : (S - l) / d + 1;
+        for (int64_t i = 0; i < n_cmp; i++) {
+            for (int j = 0; j < l; j++) {
+                const int64_t row = s0 + i * d + j;
+                for (int n = 0; n < n2; n++) {
+                    const double* gr = dout + ((c0 + i) * n2 + n) * (int64_t)dim;
+                    const double* xr = x + (row * n2 + n) * (int64_t)dim;
+                    double* dxr = dx + (row * n2 + n) * (int64_t)dim;
+                    double acc = 0.0;
+                    for (int e = 0; e < dim; e++) {
+                        dxr[e] += w[j * n2 + n] * gr[e];
+                        acc += xr[e] * gr[e];
+                    }
+                    dw[j * n2 + n] += acc;
+                }
+            }
+        }
+        c0 += n_cmp;
+    }
+    return 0;
+}
