@@ -2,7 +2,12 @@
 
 One step = nsa_compress (raw K/V -> block tokens) + nsa_compress_attention
 (scores, softmax, PV, importance band, group sum, top-k) over one batch of
-seeded synthetic inputs, launched through the C ABI.
+seeded synthetic inputs, launched through the C ABI.  The default workload is
+the largest single-GPU one: one sequence of 131072 tokens, 128 query heads in
+8 KV groups.  The same JSON line also carries the bandwidth-bound compress of
+262144 raw tokens (4 sequences of 65536, N2 = 8, D = 128, l = 128, d = 64) and
+the short-query attention of its last 128 tokens per sequence, each timed in
+the same run with its own roofline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the fp64 CPU oracle as reference arm
@@ -397,15 +402,104 @@ def run_ours(args, rank, world, local_rank):
         sel = dict(ms=float(np.mean([e[0].elapsed_time(e[1]) for e in sev])), steps=ks,
                    keys=row_keys(tk_host, cuq, cu, wl.lp), topk=tk_host)
 
+    side = None
+    if not args.no_side:
+        del flush
+        side = time_side_case(args, nsa, dev, rank)
+
     return dict(wl=wl, K=K, step_ms=step_ms, att_ms=att_ms, cmp_ms=cmp_ms, t1=t1, wall=t_wall,
-                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk,
+                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk, side=side, x=x,
                 launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
 
 
-def cpu_baseline(wl, budget_s=20.0, rows_per_seq=None):
-    """The fp64 oracle as it stands, timed on a bounded sample of the workload."""
+def time_side_case(args, nsa, dev, rank):
+    """The bandwidth-bound compress of 262144 raw tokens (4 x 65536, N2 = 8,
+    D = 128, l = 128, d = 64) and the compressed attention of the last 128
+    queries of each sequence against all of its blocks (N1 = 64, l' = 128,
+    count = 32): each timed on its own, L2 flushed before every launch."""
+    wl = rank_workload(args.side_workload, rank)
+    x = wl.generate(device=str(dev))
+    q, k, v, w = x["q"], x["k"], x["v"], x["w"]
+    cu, cuq, cus = x["cu_seqlens"], x["cu_seqlens_q"], x["cu_sel_kv"]
+    cuc = nsa.nsa_compress_out_len(cu, wl.l, wl.d)
+    tc, t1 = int(cuc[-1]), q.shape[0]
+    kc = torch.empty(tc, wl.n2, wl.d1, dtype=q.dtype, device=dev)
+    vc = torch.empty(tc, wl.n2, wl.d2, dtype=q.dtype, device=dev)
+    outs = (torch.empty(t1, wl.n1, wl.d2, dtype=q.dtype, device=dev),
+            torch.empty(t1, wl.n2, wl.count, dtype=torch.int32, device=dev),
+            torch.empty(t1, wl.n1, 8, dtype=torch.float32, device=dev),
+            torch.empty(t1, wl.n1, 8, dtype=torch.float32, device=dev))
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, cuq, cuc, cus), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def timed(fn, n):
+        for _ in range(max(args.warmup, 0)):
+            flush.zero_()
+            fn()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            evs[i][0].record()
+            fn()
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        return float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+
+    n = max(3, min(args.steps, args.side_steps))
+    cmp_ms = timed(lambda: nsa.nsa_compress(k, v, w, wl.l, wl.d, cu, kcmp=kc, vcmp=vc), n)
+    if nsa.nsa_compress_status() != 0:
+        raise RuntimeError("device-side timeout in the 262144-token compress")
+    att_ms = timed(lambda: nsa.nsa_compress_attention(q, kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count,
+                                                      cuq, cuc, cus, out=outs, workspace=ws), n)
+    if nsa.nsa_workspace_status(ws) != 0:
+        raise RuntimeError("device-side timeout in the short-query attention")
+    return dict(wl=wl, cmp_ms=cmp_ms, att_ms=att_ms, steps=n, x={kk: x[kk] for kk in ("k", "v", "w")},
+                cu=cu)
+
+
+def compress_cpu_baseline(wl, x, budget_rows=8192):
+    """The oracle's compression as it stands, on the first raw rows of the
+    first sequence of a workload (x: generated inputs on any device)."""
     import oracle
-    x = wl.generate(device="cpu")
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
+    S0 = min(wl.seqlens[0], budget_rows)
+    k, v, w = x["k"][:S0].cpu(), x["v"][:S0].cpu(), x["w"].cpu()
+    t0 = time.perf_counter()
+    oracle.compress(k, w, wl.l, wl.d, [S0], dtype=dt)
+    oracle.compress(v, w, wl.l, wl.d, [S0], dtype=dt)
+    dt_s = time.perf_counter() - t0
+    nc = 0 if S0 < wl.l else (S0 - wl.l) // wl.d + 1
+    nbytes = (S0 + nc) * wl.n2 * (wl.d1 + wl.d2) * 2 + wl.l * wl.n2 * 2
+    return {"value": nbytes / dt_s / 1e9, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {S0} raw rows of K and V of the first sequence, {dt_s:.2f} s"}
+
+
+def gen_device():
+    """Where seeded inputs are drawn: the CUDA generator when a GPU is present
+    (the large workloads hold several GB of float32 draws), else the CPU."""
+    return "cuda" if torch.cuda.is_available() else "cpu"
+
+
+def host_inputs(x, rows=None):
+    """CPU copies of the generated inputs the oracle needs: k, v, w whole and
+    q whole or only the query rows in ``rows``."""
+    out = {kk: x[kk] for kk in ("cu_seqlens", "cu_seqlens_q", "cu_sel_kv")}
+    for kk in ("k", "v", "w"):
+        out[kk] = x[kk].cpu()
+    if rows is None:
+        out["q"] = x["q"].cpu()
+    else:
+        idx = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=x["q"].device)
+        out["q"] = x["q"].index_select(0, idx).cpu()
+    return out
+
+
+def cpu_baseline(wl, x, budget_s=20.0):
+    """The fp64 oracle as it stands, timed on a bounded sample of the workload
+    (x: the generated inputs, on any device; the oracle gets CPU copies)."""
+    import oracle
+    x = {kk: (vv.cpu() if torch.is_tensor(vv) and kk != "q" else vv) for kk, vv in x.items()}
     dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
     # compress: a slice of the raw rows of the first sequence
     S0 = min(wl.seqlens[0], 8192)
@@ -422,15 +516,17 @@ def cpu_baseline(wl, budget_s=20.0, rows_per_seq=None):
     # the cost of a row grows with its position: probe rows spread over the
     # whole query range so that the estimate is the mean cost per row
     probe = np.unique(np.linspace(0, T1 - 1, num=min(T1, 48)).astype(np.int64))
+    qp = x["q"].index_select(0, torch.as_tensor(probe, device=x["q"].device)).cpu()
     tp = time.perf_counter()
-    oracle.compress_attention(x["q"][probe], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+    oracle.compress_attention(qp, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
                               x["cu_sel_kv"], rows=probe, q_rows_only=True)
     per_row = (time.perf_counter() - tp) / probe.size
     nrows = int(max(16, min(T1, budget_s / max(per_row, 1e-6))))
     stride = max(1, T1 // nrows)
     rows = np.arange(0, T1, stride, dtype=np.int64)
+    qr = x["q"].index_select(0, torch.as_tensor(rows, device=x["q"].device)).cpu()
     t0 = time.perf_counter()
-    oracle.compress_attention(x["q"][rows], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+    oracle.compress_attention(qr, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
                               x["cu_sel_kv"], rows=rows, q_rows_only=True)
     t_att = time.perf_counter() - t0
     # visible pairs of the sampled rows (all heads)
@@ -454,49 +550,58 @@ def cpu_baseline(wl, budget_s=20.0, rows_per_seq=None):
             "full_attention_pairs": full_pairs}
 
 
-def select_cpu_baseline(wl, topk, keys, budget_s=8.0):
+def select_cpu_baseline(wl, x, topk, keys, budget_s=8.0):
     """The selection-attention oracle as it stands, on evenly spaced query rows
     (all heads) of the same workload and the same top-k lists."""
     import oracle
-    x = wl.generate(device="cpu")
-    q, k, v = x["q"].float(), x["k"].float(), x["v"].float()
+    k, v = x["k"].cpu().float(), x["v"].cpu().float()
     cq, ck = x["cu_seqlens_q"], x["cu_seqlens"]
     T1 = int(cq[-1])
+
+    def qrows(r):
+        return x["q"].index_select(0, torch.as_tensor(r, device=x["q"].device)).cpu().float()
+
     probe = np.unique(np.linspace(0, T1 - 1, num=min(T1, 32)).astype(np.int64))
+    qp = qrows(probe)
     tp = time.perf_counter()
-    oracle.select_attention(q[probe], k, v, topk, wl.scale, wl.lp, wl.count, cq, ck, rows=probe, q_rows_only=True)
+    oracle.select_attention(qp, k, v, topk, wl.scale, wl.lp, wl.count, cq, ck, rows=probe, q_rows_only=True)
     per_row = (time.perf_counter() - tp) / probe.size
     nrows = int(max(16, min(T1, budget_s / max(per_row, 1e-6))))
     rows = np.unique(np.linspace(0, T1 - 1, num=nrows).astype(np.int64))
+    qr = qrows(rows)
     t0 = time.perf_counter()
-    oracle.select_attention(q[rows], k, v, topk, wl.scale, wl.lp, wl.count, cq, ck, rows=rows, q_rows_only=True)
+    oracle.select_attention(qr, k, v, topk, wl.scale, wl.lp, wl.count, cq, ck, rows=rows, q_rows_only=True)
     dt = time.perf_counter() - t0
     return {"value": select_flops(wl, keys[rows]) / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "sample": f"{rows.size} of {T1} evenly spaced query rows, all heads, {dt:.1f} s"}
 
 
-def masked_cpu_baseline(wl, am, tm, budget_s=8.0):
+def masked_cpu_baseline(wl, x, am, tm, budget_s=8.0):
     """The oracle with the same masks, as it stands, on evenly spaced query rows
     (all heads); FLOPs over the attended (visible, unmasked) pairs of those rows."""
     import oracle
-    x = wl.generate(device="cpu")
     dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
-    kc, cuc = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
-    vc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    kc, cuc = oracle.compress(x["k"].cpu(), x["w"].cpu(), wl.l, wl.d, x["cu_seqlens"], dtype=dt)
+    vc, _ = oracle.compress(x["v"].cpu(), x["w"].cpu(), wl.l, wl.d, x["cu_seqlens"], dtype=dt)
     cq = x["cu_seqlens_q"]
     T1 = int(cq[-1])
 
-    def run(rows):
-        oracle.compress_attention(x["q"][rows], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
+    def run(rows, qr):
+        oracle.compress_attention(qr, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
                                   x["cu_sel_kv"], rows=rows, q_rows_only=True, atten_mask=am, topk_mask=tm)
 
+    def qrows(r):
+        return x["q"].index_select(0, torch.as_tensor(r, device=x["q"].device)).cpu()
+
     probe = np.unique(np.linspace(0, T1 - 1, num=min(T1, 32)).astype(np.int64))
+    qp = qrows(probe)
     tp = time.perf_counter()
-    run(probe)
+    run(probe, qp)
     per_row = (time.perf_counter() - tp) / probe.size
     rows = np.unique(np.linspace(0, T1 - 1, num=int(max(16, min(T1, budget_s / max(per_row, 1e-6))))).astype(np.int64))
+    qr = qrows(rows)
     t0 = time.perf_counter()
-    run(rows)
+    run(rows, qr)
     dt_s = time.perf_counter() - t0
     pairs, prev = 0, 0
     for b, end in enumerate(cq.tolist()):
@@ -520,14 +625,16 @@ def run_reference(args, rank, world):
         return
     import oracle
     wl = workloads.WORKLOADS[args.workload]
-    x = wl.generate(device="cpu")
+    cq = wl.cu_seqlens_q()
+    T1 = int(cq[-1])
+    rows = np.linspace(0, T1 - 1, num=min(T1, args.ref_rows), dtype=np.int64)
+    # inputs drawn where they are cheapest; the oracle gets CPU copies of k, v,
+    # w and of the sampled query rows
+    x = host_inputs(wl.generate(device=gen_device()), rows)
     dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
     kc, cuc = oracle.compress(x["k"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
     vc, _ = oracle.compress(x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"], dtype=dt)
-    cq = x["cu_seqlens_q"]
-    T1 = int(cq[-1])
-    rows = np.linspace(0, T1 - 1, num=min(T1, args.ref_rows), dtype=np.int64)
-    qs = x["q"][rows]
+    qs = x["q"]
 
     def step():
         oracle.compress_attention(qs, kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, cq, cuc,
@@ -569,7 +676,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=workloads.SINGLE_16K.name, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=workloads.LONG_128K.name, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--side-workload", default=workloads.SHORTQ_4x64K.name, choices=list(workloads.WORKLOADS),
+                    help="workload of the separately timed compress and short-query attention")
+    ap.add_argument("--no-side", action="store_true", help="skip the separately timed compress case")
+    ap.add_argument("--side-steps", type=int, default=50)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -613,6 +724,11 @@ def main():
                "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
                "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
                "ms_per_step": e2e_ms, "overlap": r["e2e"]["overlap"]}
+    # the separately timed compress / short-query case: max over ranks too
+    side_cmp_ms = side_att_ms = None
+    if r["side"] is not None:
+        side_cmp_ms, side_att_ms = max_over_ranks([r["side"]["cmp_ms"], r["side"]["att_ms"]],
+                                                  torch.device("cuda", local_rank), world)
     # selection attention: every rank times its own batch; max of the times,
     # sum of the algorithmic work (the lists differ from rank to rank)
     sel_ms = sel_flops_all = None
@@ -623,7 +739,7 @@ def main():
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            cpu = cpu_baseline(wl, budget_s=args.cpu_budget)
+            cpu = cpu_baseline(wl, r["x"], budget_s=args.cpu_budget)
         peak_t = peaks["bf16_tflops"]
         traffic = profile_traffic("attention", wl.name)
         line = {
@@ -639,23 +755,46 @@ def main():
             "attention_kernel": {"ms": att_ms, "tflops": att_tflops,
                                  "pct_of_bf16_peak": 100.0 * att_tflops / peak_t,
                                  "query_tok_s": r["t1"] / (att_ms * 1e-3)},
-            "compress_kernel": {"ms": cmp_ms, "gbs": cmp_gbs,
-                                "pct_of_hbm": 100.0 * cmp_gbs / peaks["hbm_gbs"],
-                                "bytes": cbytes},
+            "compress_in_step": {"ms": cmp_ms, "gbs": cmp_gbs,
+                                 "pct_of_hbm": 100.0 * cmp_gbs / peaks["hbm_gbs"],
+                                 "bytes": cbytes, "workload": wl.name},
             "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": att_tflops / peak_t, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "frac_of_sustained": att_tflops / peaks.get("bf16_tflops_sustained", peak_t),
                          "flops_per_launch": flops},
-            "roofline_compress": {"bound": "hbm", "achieved": cmp_gbs, "peak": peaks["hbm_gbs"],
-                                  "unit": "GB/s", "frac": cmp_gbs / peaks["hbm_gbs"],
-                                  "traffic": profile_traffic("compress", wl.name),
-                                  "peak_source": f"{peak_src} hbm_gbs"},
             "clocks": r["clocks"],
             "e2e": e2e,
             "gpu_launches": r["launches_per_step"] * K,
             "cpu_baseline": cpu,
             "wall_s_timed_region": r["wall"],
         }
+        if r["side"] is not None:
+            swl = r["side"]["wl"]
+            sb = compress_bytes(swl)
+            sg = sb / (side_cmp_ms * 1e-3) / 1e9
+            line["compress_kernel"] = {
+                "what": f"nsa_compress alone on {swl.t2} raw tokens ({len(swl.seqlens)} x {swl.seqlens[0]}), "
+                        f"N2={swl.n2}, D={swl.d1}, l={swl.l}, d={swl.d}; L2 flushed before every launch",
+                "workload": swl.name, "ms": side_cmp_ms, "gbs": sg, "pct_of_hbm": 100.0 * sg / peaks["hbm_gbs"],
+                "bytes": sb, "steps": r["side"]["steps"], "gpu_launches": r["side"]["steps"]}
+            line["roofline_compress"] = {
+                "bound": "hbm", "achieved": sg, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": sg / peaks["hbm_gbs"], "traffic": profile_traffic("compress", swl.name),
+                "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": sb}
+            sf4 = attention_flops(swl)
+            st4 = sf4 / (side_att_ms * 1e-3) / 1e12
+            line["shortq_attention"] = {
+                "what": f"nsa_compress_attention for the last {swl.q_last} queries of each sequence of the "
+                        f"same workload (N1={swl.n1}, l'={swl.lp}, count={swl.count}); L2 flushed before every launch",
+                "ms": side_att_ms, "tflops": st4, "pct_of_bf16_peak": 100.0 * st4 / peak_t,
+                "query_tok_s": sum(swl.q_lengths()) / (side_att_ms * 1e-3), "flops_per_launch": sf4,
+                "steps": r["side"]["steps"], "gpu_launches": r["side"]["steps"],
+                "roofline": {"bound": "tensor", "achieved": st4, "peak": peak_t, "unit": "TFLOP/s",
+                             "frac": st4 / peak_t, "traffic": None,
+                             "peak_source": f"{peak_src} bf16_tflops (burst)"}}
+            if not args.no_cpu_baseline and world == 1:
+                line["compress_kernel"]["cpu_baseline"] = compress_cpu_baseline(swl, r["side"]["x"])
         if r["msk"] is not None:
             mt = r["msk"]["flops"] / (r["msk"]["ms"] * 1e-3) / 1e12
             line["masked_attention"] = {
@@ -667,7 +806,7 @@ def main():
                 "roofline": {"bound": "tensor", "achieved": mt, "peak": peak_t, "unit": "TFLOP/s",
                              "frac": mt / peak_t, "traffic": None,
                              "peak_source": f"{peak_src} bf16_tflops (burst)"},
-                "cpu_baseline": (masked_cpu_baseline(wl, r["msk"]["am"], r["msk"]["tm"],
+                "cpu_baseline": (masked_cpu_baseline(wl, r["x"], r["msk"]["am"], r["msk"]["tm"],
                                                      budget_s=args.select_cpu_budget)
                                  if (not args.no_cpu_baseline and world == 1) else None)}
         if r["sel"] is not None:
@@ -683,7 +822,7 @@ def main():
                 "roofline": {"bound": "tensor", "achieved": st, "peak": peak_t, "unit": "TFLOP/s",
                              "frac": st / peak_t, "traffic": profile_traffic("select", wl.name),
                              "peak_source": f"{peak_src} bf16_tflops (burst)"},
-                "cpu_baseline": (select_cpu_baseline(wl, r["sel"]["topk"], r["sel"]["keys"],
+                "cpu_baseline": (select_cpu_baseline(wl, r["x"], r["sel"]["topk"], r["sel"]["keys"],
                                                      budget_s=args.select_cpu_budget)
                                  if (not args.no_cpu_baseline and world == 1) else None),
                 "gpu_launches": 2 * r["sel"]["steps"],

@@ -253,6 +253,12 @@ nsa_status_t nsa_compress_status(void* stream);
  *     rejected with NSA_ERR_WORKSPACE before anything is enqueued.
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
+ *     Under CUDA's lazy module loading (the default since CUDA 12.2) the
+ *     array's 16 MiB are committed on a device when the library's module is
+ *     first loaded there, which is this first call: make it before the
+ *     application claims the rest of the device's memory for its own pools.
+ *     The looked-up address is kept per device ordinal; a cudaDeviceReset
+ *     invalidates it, so do not call this entry point after one.
  *   - All calls on a device share the one array, which keeps the contents of
  *     the last call; each call rewrites the parts that must start at zero.
  *     Calls whose work can overlap on the GPU (different streams without
@@ -267,6 +273,15 @@ nsa_status_t nsa_compress_attention_noalloc(
     int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
     void* attention_out, int32_t* topk_indices, float* softmax_max, float* softmax_sum,
     void* stream);
+
+/*
+ * Device error word of the last nsa_compress_attention_noalloc on the
+ * current device (the counterpart of nsa_workspace_status for the fixed
+ * scratch array, which the caller has no pointer to).  Synchronises `stream`
+ * first.  Returns NSA_OK, NSA_ERR_TIMEOUT when a device-side wait of that
+ * call gave up (its outputs are then not valid), or NSA_ERR_CUDA.
+ */
+nsa_status_t nsa_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

@@ -8,7 +8,8 @@ point raises when the library or a CUDA device is missing.
 
 Entry points (same names as the C ABI):
   nsa_compress_out_len, nsa_compress, nsa_compress_attention_workspace_size,
-  nsa_compress_attention, nsa_workspace_status, nsa_compress_status,
+  nsa_compress_attention, nsa_compress_attention_noalloc, nsa_select_attention,
+  nsa_workspace_status, nsa_compress_status, nsa_noalloc_status,
   nsa_status_string.
 """
 from __future__ import annotations
@@ -37,6 +38,7 @@ EXPORTED = (
     "nsa_workspace_status",
     "nsa_compress_status",
     "nsa_compress_attention_noalloc",
+    "nsa_noalloc_status",
     "nsa_select_attention_workspace_size",
     "nsa_select_attention",
 )
@@ -93,6 +95,8 @@ def load(path: Optional[str] = None):
     lib.nsa_compress_attention_noalloc.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p,
                                                    i32p, i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
     lib.nsa_compress_attention_noalloc.restype = ci
+    lib.nsa_noalloc_status.argtypes = [vp]
+    lib.nsa_noalloc_status.restype = ci
     lib.nsa_select_attention_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, i32p, i32p, ci,
                                                         ctypes.POINTER(cs)]
     lib.nsa_select_attention_workspace_size.restype = ci
@@ -149,11 +153,18 @@ def _out(t: torch.Tensor, shape, dtype, device, name: str) -> torch.Tensor:
 
 
 def _workspace(ws: torch.Tensor, nbytes: int, device) -> torch.Tensor:
-    if ws is None or ws.numel() < nbytes:
+    """The caller's workspace, checked; a fresh one only when none is given.
+
+    A caller-provided workspace that is too small is refused rather than
+    replaced: the kernel writes its error word into the workspace it runs
+    on, and the caller reads that word back from its own tensor."""
+    if ws is None:
         return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
     _dev(ws, "workspace")
     if ws.device != device or ws.dtype != torch.uint8:
         raise ValueError(f"workspace must be a uint8 tensor on {device}")
+    if ws.numel() < nbytes:
+        raise ValueError(f"workspace holds {ws.numel()} bytes; this call needs {nbytes}")
     return ws
 
 
@@ -371,6 +382,12 @@ def nsa_workspace_status(workspace: torch.Tensor, stream=None) -> int:
 
 def nsa_compress_status(stream=None) -> int:
     return int(load().nsa_compress_status(_stream(stream)))
+
+
+def nsa_noalloc_status(stream=None) -> int:
+    """Synchronise and read the device error word of the last
+    nsa_compress_attention_noalloc on the current device."""
+    return int(load().nsa_noalloc_status(_stream(stream)))
 
 
 def nsa_select_attention_workspace_size(head_num: int, n2: int, d1: int, d2: int, lp: int, count: int,

@@ -774,3 +774,13 @@ extern "C" nsa_status_t nsa_compress_attention_noalloc(
                                   cu_sel_kv, batch, n2, d1, d2, dtype, attention_out, topk_indices, softmax_max,
                                   softmax_sum, scratch, kStaticScratchBytes, stream);
 }
+
+// Error word of the last nsa_compress_attention_noalloc on the current device:
+// the first int of the fixed scratch array, read after `stream` has drained.
+extern "C" nsa_status_t nsa_noalloc_status(void* stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NSA_ERR_CUDA;
+    int err = 0;
+    if (cudaMemcpyFromSymbol(&err, g_static_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    return err ? NSA_ERR_TIMEOUT : NSA_OK;
+}

@@ -54,6 +54,17 @@ def test_attention_checks_outputs_workspace_and_masks(nsa):
         nsa.nsa_compress_attention(*args, out=(att, tk, st.half(), st.clone()))
     with pytest.raises(ValueError, match="workspace"):
         nsa.nsa_compress_attention(*args, workspace=torch.empty(1 << 20, dtype=torch.float32, device="cuda"))
+    # an undersized workspace is refused, never silently replaced: the kernel's
+    # error word must land in the tensor the caller reads it back from
+    need = nsa.nsa_compress_attention_workspace_size(8, 2, 64, 64, 32, 16, 64, 4, [512], cuc, [8])
+    small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError, match="workspace"):
+        nsa.nsa_compress_attention(*args, workspace=small)
+    sneed = nsa.nsa_select_attention_workspace_size(8, 2, 64, 64, 64, 4, [512], [512])
+    tk0 = torch.zeros(512, 2, 4, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError, match="workspace"):
+        nsa.nsa_select_attention(q, k, v, tk0, 0.125, 8, 64, [512], [512],
+                                 workspace=torch.zeros(sneed - 1, dtype=torch.uint8, device="cuda"))
     with pytest.raises(TypeError, match="atten_mask"):
         nsa.nsa_compress_attention(*args, atten_mask=torch.zeros(512, 64, dtype=torch.float32, device="cuda"))
     res = nsa.nsa_compress_attention(*args, out=(att, tk, st, st.clone()))

@@ -69,10 +69,19 @@ def _check(res, ref, wl, x, tm, rows=None, tie_rel=1e-4):
         denom = np.where(np.abs(r) < 1e-3, 1.0, np.abs(r))
         assert (np.abs(g - r) <= 1e-3 * denom + np.where(np.abs(r) < 1e-3, 1e-6, 0)).all()
     cq = x["cu_seqlens_q"]
+    cs = x["cu_sel_kv"]
     g_tk = tk.numpy()[rows]
     for ri, row in enumerate(rows):
         b = int(np.searchsorted(cq, row, side="right"))
         tloc = row - (int(cq[b - 1]) if b else 0)
+        # the row's position t (query offset of the sequence, as in step 1's
+        # causal rule) and its selection-block count: a causal candidate j has
+        # j < n_sel and j * l' <= t
+        s_raw = wl.seqlens[b]
+        n_cmp = 0 if s_raw < wl.l else (s_raw - wl.l) // wl.d + 1
+        s_q = int(cq[b]) - (int(cq[b - 1]) if b else 0)
+        t_pos = tloc + (max(0, (n_cmp - 1) * wl.d + wl.l - s_q) if n_cmp else 0)
+        n_sel = int(cs[b]) - (int(cs[b - 1]) if b else 0)
         for g in range(wl.n2):
             a, r = g_tk[ri, g], ref["topk"][ri, g]
             na, nr = int((a >= 0).sum()), int((r >= 0).sum())
@@ -81,6 +90,9 @@ def _check(res, ref, wl, x, tm, rows=None, tie_rel=1e-4):
             if na == 0:
                 continue
             assert (np.diff(va) > 0).all()
+            assert va.min() >= 0 and va.max() < n_sel, f"row {row} group {g}: index past the sequence {va}"
+            assert (va.astype(np.int64) * wl.lp <= t_pos).all(), f"row {row} group {g}: future block in {va}"
+            assert va.max() < ref["ncand"][ri, g], f"row {row} group {g}: index outside the candidates {va}"
             if tm is not None:
                 assert not tm[tloc, va].any(), "a masked candidate was selected"
             if set(va.tolist()) != set(vr.tolist()):

@@ -5,7 +5,8 @@ memory (for instance an application that has reserved nearly all GPU memory
 for its own pools, or a plugin handed only its tensors).  It takes inputs and
 outputs only and runs in the library's fixed scratch array.  This file checks,
 through the C ABI, that two calls in a row reproduce the regular entry point
-within the parity tolerances, and that oversized problems are refused.  It is
+within the parity tolerances with a clean device error word after each
+(nsa_noalloc_status), and that oversized problems are refused.  It is
 named so that pytest collects it last.
 """
 import numpy as np
@@ -63,12 +64,17 @@ def test_noalloc_matches_regular_entry_point_twice(nsa, wl):
     x, kc, vc, cuc = _inputs(wl)
     args = (x["q"], kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
             x["cu_sel_kv"])
-    ref = nsa.nsa_compress_attention(*args)
-    torch.cuda.synchronize()
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"]),
+        dtype=torch.uint8, device="cuda")
+    ref = nsa.nsa_compress_attention(*args, workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0
     t1 = x["q"].shape[0]
     for _ in range(2):                       # the scratch keeps the previous call's contents
         got = nsa.nsa_compress_attention_noalloc(*args, out=_empty_outputs(wl, t1))
-        torch.cuda.synchronize()
+        # the error word lives in the fixed scratch array: read it through the
+        # status call made for it (it also synchronises the stream)
+        assert nsa.nsa_noalloc_status() == 0
         _close(got, ref)
 
 
