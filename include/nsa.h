@@ -248,9 +248,13 @@ nsa_status_t nsa_compress_status(void* stream);
  * this call.
  *   - No workspace argument: the library uses its own fixed scratch array of
  *     16 MiB per device (a static device array that every GPU which loads
- *     the library keeps until the process exits).  Arguments whose workspace
- *     requirement (nsa_compress_attention_workspace_size) exceeds 16 MiB are
- *     rejected with NSA_ERR_WORKSPACE before anything is enqueued.
+ *     the library keeps until the process exits).  When the workspace that
+ *     nsa_compress_attention_workspace_size reports exceeds 16 MiB, the call
+ *     runs on fewer persistent CTAs (each CTA needs its own importance
+ *     scratch), then with one M-tile per work item, until it fits: same
+ *     results, lower throughput.  Arguments for which even one CTA's scratch
+ *     exceeds 16 MiB are rejected with NSA_ERR_WORKSPACE before anything is
+ *     enqueued.
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *     Under CUDA's lazy module loading (the default since CUDA 12.2) the

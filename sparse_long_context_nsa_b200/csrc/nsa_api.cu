@@ -77,15 +77,16 @@ bool encode_tnd(CUtensorMap* map, const void* base, int dtype, int D, int N, int
 // attention plan: everything derived from the host arguments
 // ------------------------------------------------------------------------
 struct AttnPlan {
-    int G = 0, TT = 0, a = 0, b = 0, nkv_cols = 0;
+    int G = 0, TT = 0, a = 0, b = 0, nkv_cols = 0, chunk = 0, npipe = 1, nsb = 2;
     std::vector<AttnTile> tiles;
-    int score_cap = 1;
-    int grid = 0;
+    int score_cap = 4;
+    int grid = 0, max_nkv = 0, capj = 4, capc = 4, region = 64;
     bool score_in_smem = true;
-    int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_p = 0;
-    int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_stage = 0, stage_entry_bytes = 0,
-        off_score = 0, off_bar = 0, smem_bytes = 0;
-    size_t ws_tiles = 0, ws_score = 0, ws_total = 0;
+    int nslot = 0, nqbuf = 1, tm_s[2] = {0, 0}, tm_o[2] = {0, 0};
+    int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_rowstat = 0, off_score = 0, off_bar = 0,
+        smem_bytes = 0;
+    size_t ws_tiles = 0, ws_score = 0, ws_band = 0, ws_total = 0;
+    size_t ws_fixed = 0, ws_per_cta = 0;   // ws_total = ws_fixed + grid * ws_per_cta
 };
 
 nsa_status_t validate_attention(int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
@@ -109,9 +110,12 @@ nsa_status_t validate_attention(int head_num, int n2, int d1, int d2, int l, int
     return NSA_OK;
 }
 
+// Work items of npipe x TT tokens; grid_cap bounds the persistent grid (and
+// with it the per-CTA scratch of the workspace); npipe_max = 1 forces one
+// M-tile per item.
 nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
                             const int32_t* cu_q, const int32_t* cu_cmp, const int32_t* cu_sel, int batch,
-                            bool build_tiles, AttnPlan& pl) {
+                            bool build_tiles, AttnPlan& pl, int grid_cap = kMaxGrid, int npipe_max = 2) {
     nsa_status_t s = validate_attention(head_num, n2, d1, d2, l, d, lp, count, cu_q, cu_cmp, cu_sel, batch);
     if (s != NSA_OK) return s;
     pl.G = head_num / n2;
@@ -119,10 +123,14 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
     pl.a = lp / d;
     pl.b = l / d;
     pl.nkv_cols = attention_kv_cols(pl.a);
+    pl.chunk = attention_chunk_cols(pl.a);
     const int NKV = pl.nkv_cols;
-    // tiles: (sequence, group, run of TT tokens)
-    int64_t ntiles = 0;
-    int cap = 1;
+    const int NCH = NKV / pl.chunk;
+    const int NJ = NKV / pl.a;
+    const int NJC = pl.chunk / pl.a;
+
+    // score-row capacity (largest candidate count) and the longest KV walk
+    int cap = 1, max_nkv = 0;
     {
         int32_t pq = 0, pc = 0, ps = 0;
         for (int bq = 0; bq < batch; ++bq) {
@@ -132,18 +140,89 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
             const int64_t off = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
             if (Sq > 0) {
                 const int64_t tlast = Sq - 1 + off;
-                if (nvis_host(tlast, l, d, n_cmp) > 0)
-                    cap = std::max<int64_t>(cap, std::min<int64_t>(n_sel, tlast / lp + 1));
-                ntiles += ((Sq + pl.TT - 1) / pl.TT) * (int64_t)n2;
+                const int nv = nvis_host(tlast, l, d, n_cmp);
+                if (nv > 0) cap = std::max<int64_t>(cap, std::min<int64_t>(n_sel, tlast / lp + 1));
+                max_nkv = std::max(max_nkv, (nv + NKV - 1) / NKV);
             }
             pq = cu_q[bq];
             pc = cu_cmp[bq];
             ps = cu_sel[bq];
         }
     }
-    if (ntiles > (int64_t)1 << 30) return NSA_ERR_UNSUPPORTED;
     pl.score_cap = (cap + 3) & ~3;
-    pl.grid = (int)std::min<int64_t>(ntiles, kMaxGrid);
+    pl.max_nkv = max_nkv;
+    // importance scratch of one slot: chunks of every KV tile plus the one past
+    // the last (its first anchors still collect taps), 128 rows each
+    const int nchk = max_nkv * NCH + 1;
+    pl.capj = nchk * kRows * NJC;
+    pl.capc = (nchk + 3) & ~3;
+    pl.region = (pl.capj + kRows * pl.capc + 63) & ~63;
+
+    // shared memory: Q buffers (npipe M-tiles each), K/V ring, row statistics,
+    // per-warp score rows, mbarriers.  Tensor memory: with two pipelines one
+    // score buffer and O each (O within 128 columns); with one, two score
+    // buffers and O.
+    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
+    const int score_bytes = 4 * pl.score_cap * 4;
+    const int rowstat_bytes = (2 * 2 * 2 * kRows + 4 * kRows) * 4;   // row statistics + per-warp normalisers
+    const int bar_bytes = 512;
+    pl.slot_bytes = std::max(nqc, nvc) * NKV * 128;
+    auto layout = [&](int np, int nq, int ns, bool in_smem) {
+        int off = 0;
+        pl.q_bytes = np * nqc * 16384;
+        pl.off_q = off;
+        off += nq * pl.q_bytes;
+        pl.off_ring = off;
+        off += ns * pl.slot_bytes;
+        pl.off_rowstat = off;
+        off += rowstat_bytes;
+        pl.off_score = off;
+        if (in_smem) off += (score_bytes + 127) & ~127;
+        pl.off_bar = off;
+        off += bar_bytes;
+        pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
+        pl.npipe = np;
+        pl.nqbuf = nq;
+        pl.nslot = ns;
+        pl.score_in_smem = in_smem;
+        return pl.smem_bytes <= kSmemLimit;
+    };
+    // preference: two pipelines, then a deeper K/V ring, a second Q buffer,
+    // on-chip score rows
+    static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}, {2, 2}, {1, 2}};
+    bool fits = false;
+    for (int np = std::min(npipe_max, d2 <= 128 ? 2 : 1); np >= 1 && !fits; --np)
+        for (const auto& o : kOrder) {
+            if ((fits = layout(np, o[0], o[1], true))) break;
+            if ((fits = layout(np, o[0], o[1], false))) break;
+        }
+    if (!fits) return NSA_ERR_UNSUPPORTED;
+    if (pl.npipe == 2) {
+        pl.nsb = 1;
+        pl.tm_s[0] = 0;
+        pl.tm_s[1] = 128;
+        pl.tm_o[0] = 256;
+        pl.tm_o[1] = 384;
+    } else {
+        pl.nsb = 2;
+        pl.tm_s[0] = pl.tm_s[1] = 0;
+        pl.tm_o[0] = pl.tm_o[1] = 256;
+        if (256 + d2 > 512) return NSA_ERR_UNSUPPORTED;
+    }
+
+    // items: (sequence, group, run of npipe * TT tokens)
+    const int run = pl.npipe * pl.TT;
+    int64_t ntiles = 0;
+    {
+        int32_t pq = 0;
+        for (int bq = 0; bq < batch; ++bq) {
+            const int64_t Sq = cu_q[bq] - pq;
+            ntiles += ((Sq + run - 1) / run) * (int64_t)n2;
+            pq = cu_q[bq];
+        }
+    }
+    if (ntiles > (int64_t)1 << 30) return NSA_ERR_UNSUPPORTED;
+    pl.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, std::max(1, grid_cap)));
 
     if (build_tiles) {
         pl.tiles.clear();
@@ -154,10 +233,10 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
             const int n_cmp = cu_cmp[bq] - pc;
             const int n_sel = cu_sel[bq] - ps;
             const int64_t off = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
-            for (int tok0 = 0; tok0 < Sq; tok0 += pl.TT) {
+            for (int tok0 = 0; tok0 < Sq; tok0 += run) {
                 AttnTile t;
                 t.q_row0 = pq + tok0;
-                t.ntok = std::min(pl.TT, Sq - tok0);
+                t.ntok = std::min(run, Sq - tok0);
                 t.cmp_row0 = pc;
                 t.n_cmp = n_cmp;
                 t.n_sel = n_sel;
@@ -174,60 +253,21 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
             pc = cu_cmp[bq];
             ps = cu_sel[bq];
         }
-        // longest tiles first: with the round-robin hand-out of the persistent
+        // longest items first: with the round-robin hand-out of the persistent
         // grid this approximates longest-processing-time-first scheduling
         std::stable_sort(pl.tiles.begin(), pl.tiles.end(),
                          [](const AttnTile& x, const AttnTile& y) { return x.nkv > y.nkv; });
     }
 
-    // tensor memory: S buffers (128 columns each), O (D2 columns), P (NKV/2
-    // columns of packed pairs); two S buffers when they fit next to O and P
-    const int d2c = (d2 + 31) & ~31;
-    pl.nsbuf = (256 + d2c + 64 <= 512) ? 2 : 1;
-    pl.tm_o = pl.nsbuf * 128;
-    pl.tm_p = pl.tm_o + d2c;
-    if (pl.tm_p + NKV / 2 > 512) return NSA_ERR_UNSUPPORTED;
-
-    // shared memory: Q buffers, K/V ring, band staging (2 entries), score buffer
-    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
-    const int NJ = NKV / pl.a;
-    const int ENT = std::min(NJ, kEntryMax);
-    pl.q_bytes = nqc * 16384;
-    pl.slot_bytes = std::max(nqc, nvc) * NKV * 128;
-    pl.stage_entry_bytes = kRows * (ENT + 4) * 4;
-    const int score_bytes = pl.TT * pl.score_cap * 4;
-    const int bar_bytes = 320;
-    auto layout = [&](int nq, int ns, bool in_smem) {
-        int off = 0;
-        pl.off_q = off;
-        off += nq * pl.q_bytes;
-        pl.off_ring = off;
-        off += ns * pl.slot_bytes;
-        pl.off_stage = off;
-        off += 2 * pl.stage_entry_bytes;
-        pl.off_score = off;
-        if (in_smem) off += (score_bytes + 127) & ~127;
-        pl.off_bar = off;
-        off += bar_bytes;
-        pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
-        pl.nqbuf = nq;
-        pl.nslot = ns;
-        pl.score_in_smem = in_smem;
-        return pl.smem_bytes <= kSmemLimit;
-    };
-    // preference: deeper K/V ring, then a second Q buffer, then on-chip scores
-    static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}, {2, 2}, {1, 2}};
-    bool fits = false;
-    for (const auto& o : kOrder) {
-        if ((fits = layout(o[0], o[1], true))) break;
-        if ((fits = layout(o[0], o[1], false))) break;
-    }
-    if (!fits) return NSA_ERR_UNSUPPORTED;
-
-    pl.ws_tiles = (size_t)ntiles * sizeof(AttnTile);
-    pl.ws_score = pl.score_in_smem ? 0 : (size_t)pl.grid * pl.TT * pl.score_cap * 4;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    pl.ws_total = kWsHeader + up(pl.ws_tiles) + up(pl.ws_score);
+    pl.ws_tiles = (size_t)ntiles * sizeof(AttnTile);
+    const size_t score_per_cta = pl.score_in_smem ? 0 : (size_t)4 * pl.score_cap * 4;
+    const size_t band_per_cta = (size_t)pl.npipe * 2 * (size_t)pl.region * 4;
+    pl.ws_score = up((size_t)pl.grid * score_per_cta);
+    pl.ws_band = up((size_t)pl.grid * band_per_cta);
+    pl.ws_fixed = kWsHeader + up(pl.ws_tiles) + 512;
+    pl.ws_per_cta = score_per_cta + band_per_cta;
+    pl.ws_total = kWsHeader + up(pl.ws_tiles) + pl.ws_score + pl.ws_band;
     return NSA_OK;
 }
 
@@ -498,7 +538,8 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
                                             nsa_dtype_t dtype, const uint8_t* atten_mask, int am_s2,
                                             const uint8_t* topk_mask, int tm_s2, void* attention_out,
                                             int32_t* topk_indices, float* softmax_max, float* softmax_sum,
-                                            void* workspace, size_t workspace_bytes, void* stream) {
+                                            void* workspace, size_t workspace_bytes, void* stream,
+                                            int grid_cap = kMaxGrid, int npipe_max = 2) {
     if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
     if (!q || !kcmp || !vcmp || !attention_out || !topk_indices || !softmax_max || !softmax_sum)
@@ -508,7 +549,7 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
         return NSA_ERR_INVALID_ARG;
     AttnPlan pl;
     nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
-                                    batch, true, pl);
+                                    batch, true, pl, grid_cap, npipe_max);
     if (s != NSA_OK) return s;
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         workspace_bytes < pl.ws_total)
@@ -524,7 +565,7 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
         !encode_tnd(&tv, vcmp, dtype, d2, n2, tc, 1, pl.nkv_cols))
         return NSA_ERR_UNSUPPORTED;
 
-    // workspace: [header: error word][tile list][score buffers]
+    // workspace: [header: error word][item list][score rows][importance scratch]
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     std::vector<uint8_t> host(kWsHeader + pl.ws_tiles, 0);
     std::memcpy(host.data() + kWsHeader, pl.tiles.data(), pl.ws_tiles);
@@ -537,11 +578,15 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
 
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
+    const size_t off_score = kWsHeader + ((pl.ws_tiles + 255) & ~(size_t)255);
     p.tiles = reinterpret_cast<const AttnTile*>(ws + kWsHeader);
     p.num_tiles = (int)pl.tiles.size();
     p.err = reinterpret_cast<int*>(ws);
-    p.score_gmem = pl.score_in_smem ? nullptr
-                                    : reinterpret_cast<float*>(ws + kWsHeader + ((pl.ws_tiles + 255) & ~(size_t)255));
+    p.score_gmem = pl.score_in_smem ? nullptr : reinterpret_cast<float*>(ws + off_score);
+    p.band = reinterpret_cast<float*>(ws + off_score + pl.ws_score);
+    p.capj = pl.capj;
+    p.capc = pl.capc;
+    p.region = pl.region;
     p.score_cap = pl.score_cap;
     p.score_in_smem = pl.score_in_smem ? 1 : 0;
     p.out = attention_out;
@@ -565,15 +610,17 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     p.nkv_cols = pl.nkv_cols;
     p.nslot = pl.nslot;
     p.nqbuf = pl.nqbuf;
-    p.nsbuf = pl.nsbuf;
-    p.tm_o = pl.tm_o;
-    p.tm_p = pl.tm_p;
+    p.npipe = pl.npipe;
+    p.nsb = pl.nsb;
+    for (int i = 0; i < 2; ++i) {
+        p.tm_s[i] = pl.tm_s[i];
+        p.tm_o[i] = pl.tm_o[i];
+    }
     p.off_q = pl.off_q;
     p.q_bytes = pl.q_bytes;
     p.off_ring = pl.off_ring;
     p.slot_bytes = pl.slot_bytes;
-    p.off_stage = pl.off_stage;
-    p.stage_entry_bytes = pl.stage_entry_bytes;
+    p.off_rowstat = pl.off_rowstat;
     p.off_score = pl.off_score;
     p.off_bar = pl.off_bar;
     p.smem_bytes = pl.smem_bytes;
@@ -581,7 +628,7 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     p.am_s2 = am_s2;
     p.tmask = topk_mask;
     p.tm_s2 = tm_s2;
-    const int grid = std::min(pl.grid, nsm);
+    const int grid = std::min(pl.grid, nsm);   // the workspace holds pl.grid CTAs' scratch
     if (launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
     return NSA_OK;
 }
@@ -748,11 +795,30 @@ extern "C" nsa_status_t nsa_compress_attention_noalloc(
     int count, const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv, int batch,
     int n2, int d1, int d2, nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
     float* softmax_max, float* softmax_sum, void* stream) {
-    size_t need = 0;
-    nsa_status_t s = nsa_compress_attention_workspace_size(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q,
-                                                           cu_cmp_kv, cu_sel_kv, batch, &need);
+    AttnPlan pl;
+    nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                    batch, false, pl);
     if (s != NSA_OK) return s;
-    if (need > kStaticScratchBytes) return NSA_ERR_WORKSPACE;   // larger than the fixed scratch
+    int grid_cap = kMaxGrid, npipe_max = 2;
+    if (pl.ws_total > kStaticScratchBytes) {
+        // the per-CTA scratch of the full grid does not fit the fixed array: run
+        // fewer persistent CTAs, then one M-tile per item, before refusing
+        bool fit = false;
+        for (int np = pl.npipe; np >= 1 && !fit; --np) {
+            AttnPlan q;
+            if (plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv, batch,
+                               false, q, kMaxGrid, np) != NSA_OK ||
+                q.ws_fixed >= kStaticScratchBytes || q.ws_per_cta == 0)
+                continue;
+            const size_t n = (kStaticScratchBytes - q.ws_fixed) / q.ws_per_cta;
+            if (n >= 1) {
+                grid_cap = (int)std::min<size_t>(n, kMaxGrid);
+                npipe_max = np;
+                fit = true;
+            }
+        }
+        if (!fit) return NSA_ERR_WORKSPACE;   // one CTA's scratch exceeds the fixed array
+    }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return NSA_ERR_CUDA;
     void* scratch = nullptr;
@@ -770,9 +836,10 @@ extern "C" nsa_status_t nsa_compress_attention_noalloc(
     }
     // the regular entry point rewrites the scratch header (error word = 0) and
     // the tile list on every call before its kernel runs
-    return nsa_compress_attention(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
-                                  cu_sel_kv, batch, n2, d1, d2, dtype, attention_out, topk_indices, softmax_max,
-                                  softmax_sum, scratch, kStaticScratchBytes, stream);
+    return compress_attention_impl(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
+                                   cu_sel_kv, batch, n2, d1, d2, dtype, nullptr, 0, nullptr, 0, attention_out,
+                                   topk_indices, softmax_max, softmax_sum, scratch, kStaticScratchBytes, stream,
+                                   grid_cap, npipe_max);
 }
 
 // Error word of the last nsa_compress_attention_noalloc on the current device:

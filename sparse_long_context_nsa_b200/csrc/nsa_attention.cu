@@ -10,30 +10,35 @@
 //
 // One M-tile = 128 rows = (128/G consecutive tokens) x (the G query heads of
 // one KV group): every row of a tile shares one K/V head, and the group sum of
-// step 5 is a sum over neighbouring rows.  Two passes over the compressed
-// keys per tile, because step 5 adds *normalised* probabilities of different
-// heads and a head's normaliser is only known at the end of its row:
-//   pass A  S = Q K^T (tcgen05.mma, operands in shared memory, fp32 in tensor
-//           memory); online max / sum in registers -> exact m and L per row;
-//           softmax_max / softmax_sum are written here.
-//   pass B  S = Q K^T again; P = 2^(s*scale*log2e - m - log2 L) in fp32
-//           registers; P (storage dtype) -> tensor memory -> O += P V with the
-//           A operand read from tensor memory; from the fp32 P the banded sum
-//           of step 4 goes to a shared-memory staging ring.
-// A 128-column score tile (a >= 4) is read from tensor memory in two halves:
-// the second half's load is in flight while the first half's exponentials
-// run.
-// Epilogue warps, concurrently with the next tile's passes: sum the staged
-// band values over the G rows of each token into a per-token score buffer
-// (step 5), read O out of tensor memory, and pick the top-k (step 7).
-// Warp roles (384 threads, three warpgroups): warps 0-3 softmax (warp w owns
-// TMEM lanes 32w..32w+31 = tile rows), warps 4-7 epilogue (same lane
-// quadrants), warp 8 TMA producer, warp 9 MMA issuer (and tensor-memory
-// owner), warps 10-11 idle.  Registers move from the third and second
-// warpgroups to the softmax warpgroup with setmaxnreg.  One persistent CTA
-// per SM.
-// Q (double-buffered), K and V are staged by TMA with 128-byte swizzle; K and
-// V share one ring of slots.  Every mbarrier wait is bounded; a timeout sets
+// step 5 runs over neighbouring rows.  A work item holds one M-tile, or two
+// adjacent M-tiles of the same sequence and group that read the same K/V
+// tiles (two "pipelines", one softmax warpgroup each).
+//
+// One pass over the compressed keys per M-tile, online softmax:
+//   S = Q K^T (tcgen05.mma, operands in shared memory, fp32 in tensor memory).
+//   The softmax warps read S in chunks of CH columns.  Each row keeps a
+//   reference maximum m_ref (log2 units) that moves only when a chunk's
+//   maximum exceeds it by more than kRescaleLog2; then the row's sum L, the
+//   P values already written for the tile and O are rescaled.  P =
+//   2^(s*scale*log2e - m_ref) goes, in the storage dtype, over the score
+//   columns it came from and O += P V reads it from there (A operand in
+//   tensor memory).  The exact maximum is tracked as well for softmax_max.
+//   Step 4 needs the *normalised* P of each head, known only at the end of
+//   the row, while step 5 adds heads with different normalisers: so the
+//   banded sums of the unnormalised fp32 P (step 4 up to a factor) go, per
+//   chunk, to a per-CTA scratch row in global memory (sized to stay in L2),
+//   with the chunk's m_ref; the row's final m_ref and L go to shared memory.
+// Epilogue warps, concurrently with the next item: O / L -> attention_out;
+// for each token, P_slc' = sum over the G heads of 2^(m_ref_chunk - m_ref -
+// log2 L) x banded value (steps 4-5) into a per-warp score row, then the
+// top-k (step 7).
+// Warp roles (512 threads, four warpgroups): warps 0-3 softmax of pipeline
+// 0, warps 4-7 softmax of pipeline 1 (warp w owns TMEM lanes 32(w%4).. =
+// tile rows), warps 8-11 epilogue (same lane quadrants), warp 12 TMA
+// producer, warp 13 MMA issuer (and tensor-memory owner), warps 14-15 idle.
+// Registers move to the softmax warpgroups with setmaxnreg.  One persistent
+// CTA per SM.  Q, K and V are staged by TMA with 128-byte swizzle; K and V
+// share one ring of slots.  Every mbarrier wait is bounded; a timeout sets
 // the workspace error word and every role drains without hanging.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -55,30 +60,36 @@ __host__ __device__ constexpr int kv_cols_for(int a) {
                                                   : 112;
 }
 
+__host__ __device__ constexpr int chunk_cols_for(int a) {
+    // score columns per softmax step: a whole number of anchors, a divisor of
+    // the KV tile, loadable from tensor memory in pieces of 32/16/8 columns.
+    // Measured on B200: 64-column chunks beat 32-column chunks with the next
+    // chunk's load in flight (16K workload 1.17 vs 1.26 ms, 128K 49.1 vs 54.1 ms)
+    return (a == 1 || a == 2 || a == 4 || a == 8) ? 64 : 8 * a;
+}
+
 int attention_kv_cols(int a) { return kv_cols_for(a); }
+int attention_chunk_cols(int a) { return chunk_cols_for(a); }
 
 enum BarId {
     B_Q_FULL0 = 0,
     B_Q_FULL1,
     B_Q_EMPTY0,
     B_Q_EMPTY1,
-    B_S_FULL0,
-    B_S_FULL1,
-    B_S_EMPTY0,
-    B_S_EMPTY1,
-    B_P_FULL,
-    B_P_EMPTY,
-    B_O_FULL,
-    B_O_EMPTY,
-    B_STG_FULL0,
-    B_STG_FULL1,
-    B_STG_EMPTY0,
-    B_STG_EMPTY1,
-    B_MMA_DONE,
-    B_SLOT_FULL0,                     // + slot
+    B_S_FULL = 4,        // + 2 * pipeline + buffer
+    B_P_FULL = 8,        // + pipeline: P of the tile written (4 softmax warps)
+    B_P_EMPTY = 10,      // + pipeline: the P V of that pipeline completed
+    B_O_FULL = 12,       // + pipeline: last P V of the item completed
+    B_O_EMPTY = 14,      // + pipeline: O read out (4 epilogue warps)
+    B_ROW_DONE = 16,     // + 2 * pipeline + slot: scratch rows and row statistics written (4 softmax
+                         // warps); one per slot, so that it never runs two phases ahead of its waiter
+    B_SCR_EMPTY = 20,    // + 2 * pipeline + slot: scratch slot read (4 epilogue warps)
+    B_MMA_DONE = 24,
+    B_SLOT_FULL0 = 25,   // + ring slot
     B_SLOT_EMPTY0 = B_SLOT_FULL0 + 8,
     B_COUNT = B_SLOT_EMPTY0 + 8
 };
+static_assert(B_COUNT * 8 + 8 <= 512, "barrier area");
 
 template <typename T>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi);
@@ -91,6 +102,16 @@ template <>
 __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t w);
+template <>
+__device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w));
+}
+template <>
+__device__ __forceinline__ float2 unpack2<__half>(uint32_t w) {
+    return __half22float2(*reinterpret_cast<__half2*>(&w));
 }
 
 __device__ __forceinline__ int nvis_of(int t, int l, int d, int n_cmp) {
@@ -198,51 +219,32 @@ __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, 
     for (int j = written + lane; j < count; j += 32) dst[j] = -1;
 }
 
-// Online max / sum update (log2 domain) with score columns [C0, C0 + W).
-template <int C0, int W, int N>
-__device__ __forceinline__ void online_update(const float (&s)[N], float ce, float& m, float& L) {
-    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+
+// Multiplies n_cols fp32 columns of this warp's 32 tensor-memory lanes by the
+// per-lane factor f, in 16-column pieces.
+__device__ __noinline__ void tmem_scale_f32(uint32_t taddr, int n_cols, float f) {
+    for (int c = 0; c < n_cols; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c, r);
+        tmem_wait_ld_regs<16>(r);
 #pragma unroll
-    for (int c = 0; c < W; c += 8) {
-        mx4[0] = fmax3(mx4[0], s[C0 + c + 0], s[C0 + c + 1]);
-        mx4[1] = fmax3(mx4[1], s[C0 + c + 2], s[C0 + c + 3]);
-        mx4[2] = fmax3(mx4[2], s[C0 + c + 4], s[C0 + c + 5]);
-        mx4[3] = fmax3(mx4[3], s[C0 + c + 6], s[C0 + c + 7]);
+        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+        tmem_st16(taddr + c, r);
     }
-    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
-    const float mn = fmaxf(m, mx);
-    const float mref = (mn == -INFINITY) ? 0.f : mn;
-    // sum of 2^(x - mref): packed exponent arguments, 8 partial sums
-    const float2 ce2 = make_float2(ce, ce), nm2 = make_float2(-mref, -mref);
-    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int c = 0; c < W; c += 2) {
-        const float2 x = ffma2(make_float2(s[C0 + c], s[C0 + c + 1]), ce2, nm2);
-        acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(x.x), ex2(x.y)));
-    }
-    const float2 t01 = fadd2(acc[0], acc[1]), t23 = fadd2(acc[2], acc[3]);
-    const float sum = (t01.x + t01.y) + (t23.x + t23.y);
-    L = L * ex2(m - mref) + sum;
-    m = mn;
 }
 
-// P = 2^(x * ce - mb) over score columns [C0, C0 + W), then those P in the
-// storage dtype -> tensor memory, W/2 packed columns from tp + C0/2.
-template <typename T, int C0, int W, int N>
-__device__ __forceinline__ void p_half(float (&s)[N], float2 ce2, float2 nb2, uint32_t tp) {
+// Multiplies NP columns of packed 16-bit pairs (P in the storage dtype) by f.
+template <typename T, int NP>
+__device__ __noinline__ void tmem_scale_packed(uint32_t taddr, float f) {
+    uint32_t r[NP];
+    tmem_ld_n<NP>(taddr, r);
+    tmem_wait_ld_regs<NP>(r);
 #pragma unroll
-    for (int c = 0; c < W; c += 2) {
-        const float2 x = ffma2(make_float2(s[C0 + c], s[C0 + c + 1]), ce2, nb2);
-        s[C0 + c] = ex2(x.x);
-        s[C0 + c + 1] = ex2(x.y);
+    for (int e = 0; e < NP; ++e) {
+        const float2 v = unpack2<T>(r[e]);
+        r[e] = pack2<T>(v.x * f, v.y * f);
     }
-#pragma unroll
-    for (int c = 0; c < W / 32; ++c) {
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = pack2<T>(s[C0 + c * 32 + 2 * e], s[C0 + c * 32 + 2 * e + 1]);
-        tmem_st16(tp + C0 / 2 + c * 16, w);
-    }
+    tmem_st_n<NP>(taddr, r);
 }
 
 template <typename T, int A, bool kMask>
@@ -250,44 +252,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
     constexpr int NKV = kv_cols_for(A);            // compressed blocks per KV tile
+    constexpr int CH = chunk_cols_for(A);          // score columns per softmax chunk
+    constexpr int NCH = NKV / CH;                  // chunks per KV tile
     constexpr int NJ = NKV / A;                    // importance anchors per KV tile
+    constexpr int NJC = CH / A;                    // importance anchors per chunk
     constexpr int NTAP = 2 * A - 1;                // band taps u = 0 .. 2A-2 (b <= a)
     constexpr int NCARRY = (2 * A - 2) > 0 ? (2 * A - 2) : 1;
-    constexpr int ENT = NJ < kEntryMax ? NJ : kEntryMax;   // anchors per staging entry
-    constexpr int NENT = NJ / ENT;                 // staging entries per KV tile
-    constexpr int STR = ENT + 4;                   // staging row stride in floats
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
-    static_assert(NJ % ENT == 0 && ENT % 4 == 0, "anchor chunking");
+    constexpr bool kPrefetch = CH <= 32;           // next chunk's load in flight while this one runs
+                                                   // (32-column chunks only: registers)
+    static_assert(NKV % CH == 0 && CH % A == 0 && NJC % 4 == 0 && CH >= NCARRY, "chunking");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.off_bar + 8 * B_COUNT);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.off_bar + 8 * B_COUNT + 4);
+    float* rowstat = reinterpret_cast<float*>(smem + p.off_rowstat);   // [pipe][slot][m_ref, L][128]
     auto bar = [&](int id) { return smem_u32(&bars[id]); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.G;
     const int TT = p.tok_per_tile;
+    const int npipe = p.npipe;
+    const int nsb = p.nsb;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(B_Q_FULL0), 1);
-        mbar_init(bar(B_Q_FULL1), 1);
-        mbar_init(bar(B_Q_EMPTY0), 1);
-        mbar_init(bar(B_Q_EMPTY1), 1);
-        mbar_init(bar(B_S_FULL0), 1);
-        mbar_init(bar(B_S_FULL1), 1);
-        mbar_init(bar(B_S_EMPTY0), 4);
-        mbar_init(bar(B_S_EMPTY1), 4);
-        mbar_init(bar(B_P_FULL), 4);
-        mbar_init(bar(B_P_EMPTY), 1);
-        mbar_init(bar(B_O_FULL), 1);
-        mbar_init(bar(B_O_EMPTY), 4);
-        mbar_init(bar(B_STG_FULL0), 4);
-        mbar_init(bar(B_STG_FULL1), 4);
-        mbar_init(bar(B_STG_EMPTY0), 4);
-        mbar_init(bar(B_STG_EMPTY1), 4);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(B_Q_FULL0 + i), 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(B_S_FULL + i), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(B_P_FULL + i), 4);
+            mbar_init(bar(B_P_EMPTY + i), 1);
+            mbar_init(bar(B_O_FULL + i), 1);
+            mbar_init(bar(B_O_EMPTY + i), 4);
+        }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar(B_ROW_DONE + i), 4);
+            mbar_init(bar(B_SCR_EMPTY + i), 4);
+        }
         mbar_init(bar(B_MMA_DONE), 1);
         for (int s = 0; s < 8; ++s) {
             mbar_init(bar(B_SLOT_FULL0 + s), 1);
@@ -300,7 +303,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
-    if (warp == 9) {
+    if (warp == 13) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -308,24 +311,23 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_o = tmem + p.tm_o;
-    const uint32_t tmem_p = tmem + p.tm_p;
 
     const uint32_t q_addr0 = smem_u32(smem + p.off_q);
     const uint32_t ring_addr = smem_u32(smem + p.off_ring);
     const int nslot = p.nslot;
     const int nqbuf = p.nqbuf;
-    const int nsbuf = p.nsbuf;
     const int nqc = (p.d1 + 63) / 64;    // 64-element chunks of a Q/K row
     const int nvc = (p.d2 + 63) / 64;    // 64-element chunks of a V row
+    const uint32_t q_tile_stride = (uint32_t)nqc * 16384u;   // one M-tile of Q in shared memory
 
-    if (warp >= 8) setmaxnreg_dec<kRegsCtl>();
-    if (warp == 8) {
-        // ============================ TMA producer ============================
-        if (lane == 0) {
+    if (warp >= 12) {
+        setmaxnreg_dec<kRegsCtl>();
+        if (warp == 12 && lane == 0) {
+            // ============================ TMA producer ============================
             uint32_t item = 0;
             int tcount = 0;
-            const uint32_t q_bytes = (uint32_t)(nqc * 64 * G * TT * 2);
+            const uint64_t q_policy = l2_policy_evict_first();
+            const uint32_t q_bytes = (uint32_t)(nqc * 64 * G * TT * 2);   // one M-tile box
             const uint32_t k_bytes = (uint32_t)(nqc * 64 * NKV * 2);
             const uint32_t v_bytes = (uint32_t)(nvc * 64 * NKV * 2);
             bool ok = true;
@@ -348,49 +350,72 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t qph = (tcount / nqbuf) & 1;
                 ok = mbar_wait(bar(B_Q_EMPTY0 + qb), qph ^ 1, abort_flag, p.err, kErrTimeoutBase + 3);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar(B_Q_FULL0 + qb), q_bytes);
+                mbar_arrive_expect_tx(bar(B_Q_FULL0 + qb), q_bytes * npipe);
                 const uint32_t qdst = q_addr0 + qb * p.q_bytes;
-                for (int c = 0; c < nqc; ++c)
-                    tma_load_3d(qdst + c * 16384, &tm_q, c * 64, t.group * G, t.q_row0, bar(B_Q_FULL0 + qb));
-                for (int i = 0; i < t.nkv && ok; ++i) load_kv(false, t.group, t.cmp_row0 + i * NKV);
+                // Q is read once: evict it first and keep L2 for K/V and the scratch
+                for (int pp = 0; pp < npipe; ++pp)
+                    for (int c = 0; c < nqc; ++c)
+                        tma_load_3d_hint(qdst + pp * q_tile_stride + c * 16384, &tm_q, c * 64, t.group * G,
+                                         t.q_row0 + pp * TT, bar(B_Q_FULL0 + qb), q_policy);
+                // K_0, then K_{i+1} ahead of V_i: the order the MMA issuer consumes them
                 if (t.nkv > 0 && ok) load_kv(false, t.group, t.cmp_row0);
                 for (int i = 0; i < t.nkv && ok; ++i) {
                     if (i + 1 < t.nkv) load_kv(false, t.group, t.cmp_row0 + (i + 1) * NKV);
                     load_kv(true, t.group, t.cmp_row0 + i * NKV);
                 }
             }
-        }
-    } else if (warp == 9) {
-        // ============================ MMA issuer =============================
-        if (lane == 0) {
+        } else if (warp == 13 && lane == 0) {
+            // ============================ MMA issuer =============================
             constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, NKV, false, false);
             const uint32_t idesc_pv = idesc_f16(kBF16, 128, p.d2, false, true);
             const int nks_qk = p.d1 / 16;
             constexpr int nks_pv = NKV / 16;
-            uint32_t item = 0, scnt = 0, pcnt = 0;
+            uint32_t item = 0;
+            int scnt0 = 0, scnt1 = 0, pvc0 = 0, pvc1 = 0;   // per pipeline: Q K^T and P V issued
+            const uint32_t tm_s0 = tmem + p.tm_s[0], tm_s1 = tmem + p.tm_s[1];
+            const uint32_t tm_o0 = tmem + p.tm_o[0], tm_o1 = tmem + p.tm_o[1];
             int tcount = 0;
             bool ok = true;
-            uint32_t q_addr = q_addr0;
-            auto issue_s = [&]() {
-                const int sb = scnt % nsbuf;
-                ok = ok && mbar_wait(bar(B_S_EMPTY0 + sb), ((scnt / nsbuf) & 1) ^ 1, abort_flag, p.err,
-                                     kErrTimeoutBase + 4);
+            auto wait_slot = [&]() {
                 const int slot = item % nslot;
                 ok = ok && mbar_wait(bar(B_SLOT_FULL0 + slot), (item / nslot) & 1, abort_flag, p.err,
                                      kErrTimeoutBase + 5);
-                if (!ok) return;
-                tc_fence_after();
-                const uint32_t kbase = ring_addr + slot * p.slot_bytes;
+                ++item;
+                return slot;
+            };
+            // S_pp = Q_pp K^T into the next score buffer of pipeline pp
+            auto qk = [&](int pp, uint32_t qaddr, int kslot) {
+                int& sc = pp ? scnt1 : scnt0;
+                const int sb = sc % nsb;
+                const uint32_t kbase = ring_addr + kslot * p.slot_bytes;
+                const uint32_t qa = qaddr + pp * q_tile_stride;
+                const uint32_t dst = (pp ? tm_s1 : tm_s0) + sb * 128;
                 for (int ks = 0; ks < nks_qk; ++ks) {
                     const uint32_t off = (ks & 3) * 32;   // 16 elements inside a 128-byte row
-                    const uint64_t ad = sdesc_sw128(q_addr + (ks >> 2) * 16384 + off, 16, 1024);
+                    const uint64_t ad = sdesc_sw128(qa + (ks >> 2) * 16384 + off, 16, 1024);
                     const uint64_t bd = sdesc_sw128(kbase + (ks >> 2) * (NKV * 128) + off, 16, 1024);
-                    umma_ss(tmem + sb * 128, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
+                    umma_ss(dst, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(bar(B_S_FULL0 + sb));
-                umma_commit(bar(B_SLOT_EMPTY0 + slot));
-                ++item;
-                ++scnt;
+                umma_commit(bar(B_S_FULL + 2 * pp + sb));
+                ++sc;
+            };
+            // O_pp (+)= P_pp V, P read from the score buffer it was written over
+            auto pv = [&](int pp, int vslot, bool acc) {
+                int& pc = pp ? pvc1 : pvc0;
+                ok = ok && mbar_wait(bar(B_P_FULL + pp), pc & 1, abort_flag, p.err, kErrTimeoutBase + 8);
+                if (!ok) return;
+                tc_fence_after();
+                const int sb = pc % nsb;
+                const uint32_t vbase = ring_addr + vslot * p.slot_bytes;
+                const uint32_t pa = (pp ? tm_s1 : tm_s0) + sb * 128;
+                const uint32_t od = pp ? tm_o1 : tm_o0;
+#pragma unroll
+                for (int ks = 0; ks < nks_pv; ++ks) {
+                    const uint64_t bd = sdesc_sw128(vbase + ks * 2048, NKV * 128, 1024);
+                    umma_ts(od, pa + ks * 8, bd, idesc_pv, (acc || ks > 0) ? 1u : 0u);
+                }
+                umma_commit(bar(B_P_EMPTY + pp));
+                ++pc;
             };
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
                 const AttnTile t = p.tiles[tile];
@@ -398,396 +423,100 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok = mbar_wait(bar(B_Q_FULL0 + qb), (tcount / nqbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 6);
                 if (!ok) break;
                 tc_fence_after();
-                q_addr = q_addr0 + qb * p.q_bytes;
-                for (int i = 0; i < t.nkv && ok; ++i) issue_s();          // pass A
-                if (t.nkv > 0 && ok) issue_s();                          // pass B, S_0
-                for (int i = 0; i < t.nkv && ok; ++i) {
-                    if (i + 1 < t.nkv) issue_s();
-                    if (i == 0)
-                        ok = ok && mbar_wait(bar(B_O_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err,
-                                             kErrTimeoutBase + 7);
-                    ok = ok && mbar_wait(bar(B_P_FULL), pcnt & 1, abort_flag, p.err, kErrTimeoutBase + 8);
-                    const int slot = item % nslot;
-                    ok = ok && mbar_wait(bar(B_SLOT_FULL0 + slot), (item / nslot) & 1, abort_flag, p.err,
-                                         kErrTimeoutBase + 9);
+                const uint32_t qaddr = q_addr0 + qb * p.q_bytes;
+                if (t.nkv > 0) {
+                    const int k0 = wait_slot();
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t vbase = ring_addr + slot * p.slot_bytes;
-#pragma unroll
-                    for (int ks = 0; ks < nks_pv; ++ks) {
-                        const uint64_t bd = sdesc_sw128(vbase + ks * 2048, NKV * 128, 1024);
-                        umma_ts(tmem_o, tmem_p + ks * 8, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+                    for (int pp = 0; pp < npipe; ++pp) qk(pp, qaddr, k0);
+                    if (t.nkv == 1) umma_commit(bar(B_Q_EMPTY0 + qb));
+                    umma_commit(bar(B_SLOT_EMPTY0 + k0));
+                    for (int i = 0; i < t.nkv && ok; ++i) {
+                        const int kslot = (i + 1 < t.nkv) ? wait_slot() : -1;
+                        const int vslot = wait_slot();
+                        if (!ok) break;
+                        tc_fence_after();
+                        // the epilogue has read the previous item's O out.  Waited for
+                        // before S_{i+1} is issued: between that issue and the wait for
+                        // P_i nothing may block, or the softmax could finish tiles i and
+                        // i+1 first and P_FULL would run two phases ahead of this wait
+                        if (i == 0)
+                            for (int pp = 0; pp < npipe; ++pp)
+                                ok = ok && mbar_wait(bar(B_O_EMPTY + pp), (tcount & 1) ^ 1, abort_flag, p.err,
+                                                     kErrTimeoutBase + 7);
+                        if (!ok) break;
+                        // two score buffers (one pipeline): S_{i+1} goes into the
+                        // buffer whose P was consumed by the previous P V
+                        if (nsb == 2 && kslot >= 0) qk(0, qaddr, kslot);
+                        for (int pp = 0; pp < npipe; ++pp) {
+                            pv(pp, vslot, i > 0);
+                            // one score buffer: S_{i+1} overwrites P_i after its P V
+                            // (tcgen05.mma of one thread execute in issue order)
+                            if (nsb == 1 && kslot >= 0 && ok) qk(pp, qaddr, kslot);
+                        }
+                        if (!ok) break;
+                        if (i + 2 == t.nkv) umma_commit(bar(B_Q_EMPTY0 + qb));   // last Q K^T issued
+                        umma_commit(bar(B_SLOT_EMPTY0 + vslot));
+                        if (kslot >= 0) umma_commit(bar(B_SLOT_EMPTY0 + kslot));
                     }
-                    umma_commit(bar(B_P_EMPTY));
-                    umma_commit(bar(B_SLOT_EMPTY0 + slot));
-                    ++item;
-                    ++pcnt;
+                } else {
+                    // no visible block in the item: keep the O hand-off in step
+                    for (int pp = 0; pp < npipe; ++pp)
+                        ok = ok && mbar_wait(bar(B_O_EMPTY + pp), (tcount & 1) ^ 1, abort_flag, p.err,
+                                             kErrTimeoutBase + 7);
+                    umma_commit(bar(B_Q_EMPTY0 + qb));
                 }
                 if (!ok) break;
-                // O_FULL of this tile may only complete after the epilogue of the
-                // previous tile has released O: otherwise a tile without PV work
-                // could advance O_FULL by two phases before its consumer looks
-                if (t.nkv == 0)
-                    ok = mbar_wait(bar(B_O_EMPTY), (tcount & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 7);
-                if (!ok) break;
-                umma_commit(bar(B_O_FULL));
-                umma_commit(bar(B_Q_EMPTY0 + qb));
+                for (int pp = 0; pp < npipe; ++pp) umma_commit(bar(B_O_FULL + pp));
             }
             // every MMA issued so far has retired before the tensor memory is freed
             umma_commit(bar(B_MMA_DONE));
             mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
         }
-    } else if (warp < 4) {
-        // ===================== softmax + band values (128 thr) =====================
-        setmaxnreg_inc<kRegsSoftmax>();
-        const int row = warp * 32 + lane;          // tile row = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const int a = p.a, bb = p.b;
-        const float c2 = p.scale_log2;
-        float wband[NTAP];
-#pragma unroll
-        for (int u = 0; u < NTAP; ++u) {
-            // multiplicity of m + n = u with m < a, n < b (the double sum of step 4)
-            const int c = min(min(u, a - 1), min(bb - 1, a + bb - 2 - u)) + 1;
-            wband[u] = (u <= a + bb - 2) ? (float)c : 0.f;
-        }
-        float* stage = reinterpret_cast<float*>(smem + p.off_stage);
-        uint32_t scnt = 0, pcnt = 0, stg = 0;
-        const int h = row % G;
-        const int tok = row / G;
-
-        auto load_s = [&](float (&s)[NKV]) {
-            const int sb = scnt % nsbuf;
-            mbar_wait(bar(B_S_FULL0 + sb), (scnt / nsbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
-            tc_fence_after();
-            const uint32_t ta = tmem + lane_off + sb * 128;
-#pragma unroll
-            for (int c = 0; c < NKV / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(ta + c * 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
-            }
-            if constexpr (NKV % 32 != 0) {
-                uint32_t r[16];
-                tmem_ld16(ta + (NKV / 32) * 32, r);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) s[(NKV / 32) * 32 + e] = __uint_as_float(r[e]);
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_S_EMPTY0 + sb));
-            ++scnt;
-        };
-        // scores of one KV tile in "exponent units": x = s * ce - shift.  With a
-        // positive scale the raw scores are used as they are (ce = c2); a zero
-        // or negative scale first multiplies them in (ce = 1).  Columns c >= lim
-        // are not visible and become -inf.
-        const bool pos_scale = c2 > 0.f;
-        const float ce = pos_scale ? c2 : 1.f;
-        auto prep = [&](float (&s)[NKV], int lim) {
-            if (!pos_scale) {
-#pragma unroll
-                for (int c = 0; c < NKV; ++c) s[c] *= c2;
-            }
-            if (lim < NKV) {
-#pragma unroll
-                for (int c = 0; c < NKV; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
-            }
-        };
-        // A 128-column score tile is taken in two halves: the second half's
-        // tensor-memory load is in flight while the first half is processed.
-        // open_half0 waits for the tile, loads columns [0, 64) and starts the
-        // load of [64, 128) into r1; close_half1 waits for it and releases the
-        // score buffer.  Columns c >= lim are masked as in prep.
-        constexpr bool kSplit = (NKV == 128 && A >= 4);   // measured: no gain for a <= 2
-        constexpr int NH = kSplit ? NKV / 2 : 16;   // (16: the split helpers are unused then)
-        auto mask_half = [&](float (&s)[NKV], int c0, int lim) {
-            if (!pos_scale) {
-#pragma unroll
-                for (int c = 0; c < NH; ++c) s[c0 + c] *= c2;
-            }
-            if (lim < c0 + NH) {
-#pragma unroll
-                for (int c = 0; c < NH; ++c) s[c0 + c] = (c0 + c < lim) ? s[c0 + c] : -INFINITY;
-            }
-        };
-        // atten_mask (step 1), masked kernel only: a set byte at (the row's
-        // query index, block) removes a visible block.  arow is the row's mask
-        // row, null for rows outside the tile or without a mask.
-        const uint8_t* arow = nullptr;
-        auto amask_cols = [&](float (&s)[NKV], int c0, int w, int i, int lim) {
-            if constexpr (kMask) {
-                if (arow != nullptr) {
-                    const uint8_t* mr = arow + (long long)i * NKV;
-#pragma unroll
-                    for (int c = 0; c < NKV; ++c)
-                        if (c >= c0 && c < c0 + w && c < lim && mr[c]) s[c] = -INFINITY;
-                }
-            }
-        };
-        uint32_t split_sb = 0;
-        auto open_half0 = [&](float (&s)[NKV], uint32_t (&r1)[NH]) {
-            split_sb = scnt % nsbuf;
-            mbar_wait(bar(B_S_FULL0 + split_sb), (scnt / nsbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
-            tc_fence_after();
-            const uint32_t ta = tmem + lane_off + split_sb * 128;
-            uint32_t r0[NH];
-            tmem_ld_cols<NH>(ta, r0);
-            tmem_wait_ld_regs<NH>(r0);
-#pragma unroll
-            for (int e = 0; e < NH; ++e) s[e] = __uint_as_float(r0[e]);
-            tmem_ld_cols<NH>(ta + NH, r1);
-        };
-        auto close_half1 = [&](float (&s)[NKV], uint32_t (&r1)[NH]) {
-            tmem_wait_ld_regs<NH>(r1);
-#pragma unroll
-            for (int e = 0; e < NH; ++e) s[NH + e] = __uint_as_float(r1[e]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_S_EMPTY0 + split_sb));
-            ++scnt;
-        };
-        // one staging entry: ENT anchors of this row -> shared memory
-        auto put_entry = [&](const float* v) {
-            const int slot = stg & 1;
-            mbar_wait(bar(B_STG_EMPTY0 + slot), ((stg >> 1) & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 13);
-            float4* dst = reinterpret_cast<float4*>(stage + (size_t)slot * (p.stage_entry_bytes / 4) + row * STR);
-#pragma unroll
-            for (int q4 = 0; q4 < ENT / 4; ++q4)
-                dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_STG_FULL0 + slot));
-            ++stg;
-        };
-
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-            const AttnTile t = p.tiles[tile];
-            const bool valid = (row < TT * G) && (tok < t.ntok);
-            const int tpos = t.t0 + tok;
-            const int nvis = valid ? nvis_of(tpos, p.l, p.d, t.n_cmp) : 0;
-            if constexpr (kMask)
-                arow = (valid && p.amask != nullptr) ? p.amask + (long long)(t.tloc0 + tok) * p.am_s2 : nullptr;
-
-            // ---------------- pass A: exact row max and sum (log2 domain) ----------------
-            float m = -INFINITY, L = 0.f;
-            for (int i = 0; i < t.nkv && kSplit; ++i) {
-                float s[NKV];
-                uint32_t r1[NH];
-                open_half0(s, r1);
-                mask_half(s, 0, nvis - i * NKV);
-                amask_cols(s, 0, NH, i, nvis - i * NKV);
-                online_update<0, NH>(s, ce, m, L);
-                close_half1(s, r1);
-                mask_half(s, NH, nvis - i * NKV);
-                amask_cols(s, NH, NH, i, nvis - i * NKV);
-                online_update<NH, NH>(s, ce, m, L);
-            }
-            for (int i = 0; i < t.nkv && !kSplit; ++i) {
-                float s[NKV];
-                load_s(s);
-                prep(s, nvis - i * NKV);
-                amask_cols(s, 0, NKV, i, nvis - i * NKV);
-                // row maximum: four independent chains of 3-input max
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int c = 0; c < NKV; c += 8) {
-                    mx4[0] = fmax3(mx4[0], s[c + 0], s[c + 1]);
-                    mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
-                    mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
-                    mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
-                }
-                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
-                const float mn = fmaxf(m, mx);
-                const float mref = (mn == -INFINITY) ? 0.f : mn;
-                // row sum of 2^(x - mref): packed exponent arguments, 8 partial sums
-                const float2 ce2 = make_float2(ce, ce), nm2 = make_float2(-mref, -mref);
-                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                 make_float2(0.f, 0.f)};
-#pragma unroll
-                for (int c = 0; c < NKV; c += 2) {
-                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2, nm2);
-                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(x.x), ex2(x.y)));
-                }
-                const float2 t01 = fadd2(acc[0], acc[1]), t23 = fadd2(acc[2], acc[3]);
-                const float sum = (t01.x + t01.y) + (t23.x + t23.y);
-                L = L * ex2(m - mref) + sum;
-                m = mn;
-            }
-            if (valid) {
-                const size_t si = ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * 8;
-                const float mo = (m == -INFINITY) ? -INFINITY : m * 0.69314718055994530942f;
-                const float4 mv = make_float4(mo, mo, mo, mo);
-                const float4 lv = make_float4(L, L, L, L);
-                reinterpret_cast<float4*>(p.smax + si)[0] = mv;
-                reinterpret_cast<float4*>(p.smax + si)[1] = mv;
-                reinterpret_cast<float4*>(p.ssum + si)[0] = lv;
-                reinterpret_cast<float4*>(p.ssum + si)[1] = lv;
-            }
-
-            // ------------- pass B: P -> TMEM, band values -> staging -------------
-            // P = 2^(s*c2 - m - log2 L): normalised in the exponent
-            const float mb = (L > 0.f) ? m + lg2(L) : INFINITY;
-            float carry[NCARRY];
-#pragma unroll
-            for (int k = 0; k < NCARRY; ++k) carry[k] = 0.f;
-            const float2 ce2b = make_float2(ce, ce), nb2 = make_float2(-mb, -mb);
-            for (int i = 0; i < t.nkv; ++i) {
-                float s[NKV];
-                if constexpr (kSplit) {
-                    uint32_t r1[NH];
-                    open_half0(s, r1);
-                    mask_half(s, 0, nvis - i * NKV);
-                    amask_cols(s, 0, NH, i, nvis - i * NKV);
-                    // P of the previous tile has been read by its P V
-                    mbar_wait(bar(B_P_EMPTY), (pcnt & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 11);
-                    tc_fence_after();
-                    p_half<T, 0, NH>(s, ce2b, nb2, tmem_p + lane_off);
-                    close_half1(s, r1);
-                    mask_half(s, NH, nvis - i * NKV);
-                    amask_cols(s, NH, NH, i, nvis - i * NKV);
-                    p_half<T, NH, NH>(s, ce2b, nb2, tmem_p + lane_off);
-                } else {
-                load_s(s);
-                prep(s, nvis - i * NKV);
-                amask_cols(s, 0, NKV, i, nvis - i * NKV);
-                {
-#pragma unroll
-                    for (int c = 0; c < NKV; c += 2) {
-                        const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2b, nb2);
-                        s[c] = ex2(x.x);
-                        s[c + 1] = ex2(x.y);
-                    }
-                }
-                // P in the storage dtype -> tensor memory (A operand of P V)
-                mbar_wait(bar(B_P_EMPTY), (pcnt & 1) ^ 1, abort_flag, p.err, kErrTimeoutBase + 11);
-                tc_fence_after();
-                if constexpr ((NKV / 2) % 16 == 0) {
-#pragma unroll
-                    for (int c = 0; c < NKV / 32; ++c) {
-                        uint32_t w[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) w[e] = pack2<T>(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
-                        tmem_st16(tmem_p + lane_off + c * 16, w);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < NKV / 16; ++c) {
-                        uint32_t w[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) w[e] = pack2<T>(s[c * 16 + 2 * e], s[c * 16 + 2 * e + 1]);
-                        tmem_st8(tmem_p + lane_off + c * 8, w);
-                    }
-                }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_P_FULL));
-                ++pcnt;
-                // step 4 on the fp32 P: anchors A*jj of this tile; taps reach back
-                // into the previous tile through `carry` (carry[k] = P[c0 - 1 - k])
-#pragma unroll
-                for (int e = 0; e < NENT; ++e) {
-                    float v[ENT];
-#pragma unroll
-                    for (int qq = 0; qq < ENT; ++qq) {
-                        const int anchor = A * (e * ENT + qq);
-                        float acc = 0.f;
-#pragma unroll
-                        for (int u = 0; u < NTAP; ++u) {
-                            const int x = anchor - u;
-                            const float pv = (x >= 0) ? s[x >= 0 ? x : 0] : carry[x < 0 ? (-x - 1) : 0];
-                            acc = fmaf(wband[u], pv, acc);
-                        }
-                        v[qq] = acc;
-                    }
-                    put_entry(v);
-                }
-#pragma unroll
-                for (int k = 0; k < NCARRY; ++k) carry[k] = s[NKV - 1 - k];
-            }
-            if (t.nkv > 0) {
-                // the first anchors past the last tile still collect taps from it
-                float v[ENT];
-#pragma unroll
-                for (int qq = 0; qq < ENT; ++qq) {
-                    const int anchor = A * qq;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int u = 0; u < NTAP; ++u) {
-                        const int x = anchor - u;
-                        if (x < 0) acc = fmaf(wband[u], carry[-x - 1 >= 0 ? -x - 1 : 0], acc);
-                    }
-                    v[qq] = acc;
-                }
-                put_entry(v);
-            }
-        }
-    } else if (warp < 8) {
-        // ============ epilogue: group sum, output, top-k (128 thr) ============
+    } else if (warp >= 8) {
+        // ============ epilogue: output, group sum, top-k (128 thr) ============
         setmaxnreg_dec<kRegsEpilogue>();
-        const int ew = warp - 4;                   // TMEM lane quadrant
+        const int ew = warp - 8;                   // TMEM lane quadrant
         const int erow = ew * 32 + lane;
-        const int et = threadIdx.x - 128;          // 0..127
         const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
-        const float* stage = reinterpret_cast<const float*>(smem + p.off_stage);
-        float* score = p.score_in_smem ? reinterpret_cast<float*>(smem + p.off_score)
-                                       : p.score_gmem + (size_t)blockIdx.x * TT * p.score_cap;
         const int cap = p.score_cap;
-        uint32_t stg = 0;
+        float* score = p.score_in_smem ? reinterpret_cast<float*>(smem + p.off_score) + ew * cap
+                                       : p.score_gmem + ((size_t)blockIdx.x * 4 + ew) * cap;
+        float* mbw = reinterpret_cast<float*>(smem + p.off_rowstat) + 2 * 2 * 2 * 128 + ew * 128;
+        const uint64_t out_policy = l2_policy_evict_first();   // attention_out is written once
         int tcount = 0;
         const int eh = erow % G;
         const int etok = erow / G;
 
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
             const AttnTile t = p.tiles[tile];
-            // step 5: staged band values summed over the G rows of each token
-            const int nent = t.nkv > 0 ? t.nkv * NENT + 1 : 0;
-            for (int e = 0; e < nent; ++e) {
-                const int slot = stg & 1;
-                mbar_wait(bar(B_STG_FULL0 + slot), (stg >> 1) & 1, abort_flag, p.err, kErrTimeoutBase + 14);
-                const int j0 = (e < t.nkv * NENT) ? (e / NENT) * NJ + (e % NENT) * ENT : t.nkv * NJ;
-                const float* st = stage + (size_t)slot * (p.stage_entry_bytes / 4);
-                for (int pi = et; pi < t.ntok * ENT; pi += 128) {
-                    const int tau = pi / ENT, jj = pi - tau * ENT;
-                    const float* src = st + (tau * G) * STR + jj;
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    int hh = 0;
-                    for (; hh + 4 <= G; hh += 4) {
-                        a0 += src[(hh + 0) * STR];
-                        a1 += src[(hh + 1) * STR];
-                        a2 += src[(hh + 2) * STR];
-                        a3 += src[(hh + 3) * STR];
-                    }
-                    for (; hh < G; ++hh) a0 += src[hh * STR];
-                    const int j = j0 + jj;
-                    if (j < cap) score[tau * cap + j] = (a0 + a1) + (a2 + a3);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_STG_EMPTY0 + slot));
-                ++stg;
-            }
-            const int jcov = t.nkv > 0 ? t.nkv * NJ + ENT : 0;
-
-            // O (tensor memory) -> attention_out
-            mbar_wait(bar(B_O_FULL), tcount & 1, abort_flag, p.err, kErrTimeoutBase + 12);
-            tc_fence_after();
-            {
-                const bool valid = (erow < TT * G) && (etok < t.ntok);
-                const int nvis = valid ? nvis_of(t.t0 + etok, p.l, p.d, t.n_cmp) : 0;
+            const int slot = tcount & 1;
+            for (int pp = 0; pp < npipe; ++pp) {
+                mbar_wait(bar(B_ROW_DONE + 2 * pp + slot), (tcount >> 1) & 1, abort_flag, p.err,
+                          kErrTimeoutBase + 14);
+                mbar_wait(bar(B_O_FULL + pp), tcount & 1, abort_flag, p.err, kErrTimeoutBase + 12);
+                tc_fence_after();
+                // O (tensor memory) / L -> attention_out
+                const int tok = pp * TT + etok;
+                const bool valid = (erow < TT * G) && (tok < t.ntok);
+                const int nvis = valid ? nvis_of(t.t0 + tok, p.l, p.d, t.n_cmp) : 0;
+                const float Lr = rowstat[((pp * 2 + slot) * 2 + 1) * 128 + erow];
+                // rows that attend to nothing write zeros (their O may never have been
+                // written: select, do not multiply)
+                const bool live = nvis > 0 && Lr > 0.f;
+                const float inv = live ? 1.f / Lr : 0.f;
                 T* orow = reinterpret_cast<T*>(p.out) +
-                          ((size_t)(t.q_row0 + etok) * p.n1 + (size_t)t.group * G + eh) * p.d2;
+                          ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + eh) * p.d2;
+                const uint32_t obase = tmem + lane_off + (pp ? p.tm_o[1] : p.tm_o[0]);
                 for (int c = 0; c < p.d2 / 16; ++c) {
                     uint32_t r[16];
-                    tmem_ld16(tmem_o + lane_off + c * 16, r);
-                    tmem_wait_ld();
+                    tmem_ld16(obase + c * 16, r);
+                    tmem_wait_ld_regs<16>(r);
                     if (valid) {
                         uint4 w0, w1;
                         float f[16];
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) f[q] = (nvis > 0) ? __uint_as_float(r[q]) : 0.f;
+                        for (int q = 0; q < 16; ++q) f[q] = live ? __uint_as_float(r[q]) * inv : 0.f;
                         w0.x = pack2<T>(f[0], f[1]);
                         w0.y = pack2<T>(f[2], f[3]);
                         w0.z = pack2<T>(f[4], f[5]);
@@ -796,18 +525,19 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         w1.y = pack2<T>(f[10], f[11]);
                         w1.z = pack2<T>(f[12], f[13]);
                         w1.w = pack2<T>(f[14], f[15]);
-                        *reinterpret_cast<uint4*>(orow + c * 16) = w0;
-                        *reinterpret_cast<uint4*>(orow + c * 16 + 8) = w1;
+                        st_global_v4_hint(orow + c * 16, w0, out_policy);
+                        st_global_v4_hint(orow + c * 16 + 8, w1, out_policy);
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_O_EMPTY + pp));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_O_EMPTY));
 
-            named_bar_sync(2, 128);   // every group sum of this tile is in the score buffer
-            // step 7, one warp per token
+            // steps 4-5 from the scratch rows, then step 7; one warp per token
             for (int tau = ew; tau < t.ntok; tau += 4) {
+                const int pp = tau / TT;
+                const int tl = tau - pp * TT;
                 const int tp = t.t0 + tau;
                 int32_t* dst = p.topk + ((size_t)(t.q_row0 + tau) * p.n2 + t.group) * p.count;
                 const int nv = nvis_of(tp, p.l, p.d, t.n_cmp);
@@ -825,12 +555,317 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (empty) {
                     for (int j = lane; j < p.count; j += 32) dst[j] = -1;
-                } else {
-                    const int ncand = min(t.n_sel, tp / p.lp + 1);
-                    warp_topk<kMask>(score + tau * cap, ncand, jcov, p.count, dst, lane, trow);
+                    continue;
+                }
+                const int ncand = min(t.n_sel, tp / p.lp + 1);
+                // anchors past nkv*NJ + NJC collect no tap from a visible block
+                const int jn = min(ncand, t.nkv * NJ + NJC);
+                const float* base = p.band + (((size_t)blockIdx.x * npipe + pp) * 2 + slot) * (size_t)p.region;
+                const float* rs = rowstat + (pp * 2 + slot) * 2 * 128 + tl * G;
+                // the token's heads' normalisers m_ref + log2 L, once
+                for (int hh = lane; hh < G; hh += 32) {
+                    const float Lh = rs[128 + hh];
+                    mbw[hh] = (Lh > 0.f) ? rs[hh] + lg2(Lh) : INFINITY;
+                }
+                __syncwarp();
+                // P_slc'[j] = sum_h 2^(m_c - m_ref - log2 L) x banded value, where m_c
+                // is the reference the value's chunk was written against (steps 4-5).
+                // Lane l takes anchors 4l..4l+3 of every 128 (in one chunk, NJC % 4 == 0)
+                // and loops over the heads, eight at a time for loads in flight.
+                const float* wbase = base + p.capj + (size_t)(tl * G) * p.capc;
+                for (int j0 = 0; j0 < jn; j0 += 128) {
+                    const int j4 = j0 + 4 * lane;
+                    const bool live = j4 < jn;
+                    const int c = j4 / NJC;                     // chunk of the four anchors
+                    const float* bp = base + ((size_t)c * 128 + tl * G) * NJC + (j4 - c * NJC);
+                    const float* wp = wbase + c;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    int hh = 0;
+                    for (; hh + 8 <= G; hh += 8) {
+                        float4 bv[8];
+                        float mv[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            bv[u] = live ? __ldcg(reinterpret_cast<const float4*>(bp + (size_t)(hh + u) * NJC))
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                            mv[u] = live ? __ldcg(wp + (size_t)(hh + u) * p.capc) : 0.f;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float w = live ? ex2(mv[u] - mbw[hh + u]) : 0.f;
+                            acc.x = fmaf(w, bv[u].x, acc.x);
+                            acc.y = fmaf(w, bv[u].y, acc.y);
+                            acc.z = fmaf(w, bv[u].z, acc.z);
+                            acc.w = fmaf(w, bv[u].w, acc.w);
+                        }
+                    }
+                    for (; hh < G; ++hh) {
+                        if (live) {
+                            const float4 b1 = __ldcg(reinterpret_cast<const float4*>(bp + (size_t)hh * NJC));
+                            const float w = ex2(__ldcg(wp + (size_t)hh * p.capc) - mbw[hh]);
+                            acc.x = fmaf(w, b1.x, acc.x);
+                            acc.y = fmaf(w, b1.y, acc.y);
+                            acc.z = fmaf(w, b1.z, acc.z);
+                            acc.w = fmaf(w, b1.w, acc.w);
+                        }
+                    }
+                    if (live) *reinterpret_cast<float4*>(score + j4) = acc;
+                }
+                __syncwarp();
+                warp_topk<kMask>(score, ncand, jn, p.count, dst, lane, trow);
+                __syncwarp();   // the score row is free for the next token
+            }
+            // every token of the item is done: the slot's scratch is dead, so its
+            // lines leave L2 without a write-back; then slot and row statistics
+            // are free
+            named_bar_sync(2, 128);
+            if (t.nkv > 0) {
+                const size_t band_bytes = (size_t)(t.nkv * NCH + 1) * 128 * NJC * 4;
+                for (int pp = 0; pp < npipe; ++pp) {
+                    const char* sb0 = reinterpret_cast<const char*>(
+                        p.band + (((size_t)blockIdx.x * npipe + pp) * 2 + slot) * (size_t)p.region);
+                    for (size_t o = (size_t)(warp - 8) * 32 + lane; o * 128 < band_bytes; o += 128)
+                        discard_l2_line(sb0 + o * 128);
+                    const size_t mref_bytes = (size_t)128 * p.capc * 4;
+                    const char* mb0 = sb0 + (size_t)p.capj * 4;
+                    for (size_t o = (size_t)(warp - 8) * 32 + lane; o * 128 < mref_bytes; o += 128)
+                        discard_l2_line(mb0 + o * 128);
                 }
             }
-            named_bar_sync(2, 128);   // the score buffer is free for the next tile
+            __syncwarp();
+            if (lane == 0)
+                for (int pp = 0; pp < npipe; ++pp) mbar_arrive(bar(B_SCR_EMPTY + 2 * pp + slot));
+        }
+    } else {
+        // ========== softmax, P, banded values (128 threads per pipeline) ==========
+        setmaxnreg_inc<kRegsSoftmax>();
+        const int pp = warp >> 2;                  // pipeline
+        if (pp < npipe) {
+            const int wq = warp & 3;               // TMEM lane quadrant
+            const int row = wq * 32 + lane;        // tile row = TMEM lane
+            const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+            const int a = p.a, bb = p.b;
+            const float c2 = p.scale_log2;
+            float wband[NTAP];
+#pragma unroll
+            for (int u = 0; u < NTAP; ++u) {
+                // multiplicity of m + n = u with m < a, n < b (the double sum of step 4)
+                const int c = min(min(u, a - 1), min(bb - 1, a + bb - 2 - u)) + 1;
+                wband[u] = (u <= a + bb - 2) ? (float)c : 0.f;
+            }
+            const int h = row % G;
+            const int tok_t = row / G;
+            // scores in "exponent units": x = s * ce - m_ref.  With a positive
+            // scale the raw scores are used as they are (ce = c2); a zero or
+            // negative scale first multiplies them in (ce = 1).
+            const bool pos_scale = c2 > 0.f;
+            const float ce = pos_scale ? c2 : 1.f;
+            const float2 ce2 = make_float2(ce, ce);
+            int scnt = 0, pcnt = 0, tcount = 0;
+            const uint32_t tm_sp = tmem + lane_off + (pp ? p.tm_s[1] : p.tm_s[0]);
+            const uint32_t tm_op = tmem + lane_off + (pp ? p.tm_o[1] : p.tm_o[0]);
+
+            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+                const AttnTile t = p.tiles[tile];
+                const int tok = pp * TT + tok_t;
+                const bool valid = (row < TT * G) && (tok < t.ntok);
+                const int tpos = t.t0 + tok;
+                const int nvis = valid ? nvis_of(tpos, p.l, p.d, t.n_cmp) : 0;
+                const int slot = tcount & 1;
+                const uint8_t* arow = nullptr;
+                if constexpr (kMask)
+                    arow = (valid && p.amask != nullptr) ? p.amask + (long long)(t.tloc0 + tok) * p.am_s2 : nullptr;
+                // this slot's scratch: banded values [chunk][row][NJC], then the chunk
+                // references [row][chunk]
+                float* sbase_g = p.band + (((size_t)blockIdx.x * npipe + pp) * 2 + slot) * (size_t)p.region;
+                float* wrow = sbase_g + p.capj + (size_t)row * p.capc;
+                // the epilogue has finished with this slot (item tcount - 2)
+                mbar_wait(bar(B_SCR_EMPTY + 2 * pp + slot), ((tcount >> 1) & 1) ^ 1, abort_flag, p.err,
+                          kErrTimeoutBase + 13);
+
+                float m_ref = -INFINITY, m_true = -INFINITY, L = 0.f;
+                float carry[NCARRY];   // carry[k] = P of the column 1 + k before the chunk
+#pragma unroll
+                for (int k = 0; k < NCARRY; ++k) carry[k] = 0.f;
+
+                for (int i = 0; i < t.nkv; ++i) {
+                    const int sb = scnt % nsb;
+                    mbar_wait(bar(B_S_FULL + 2 * pp + sb), (scnt / nsb) & 1, abort_flag, p.err,
+                              kErrTimeoutBase + 10);
+                    tc_fence_after();
+                    const uint32_t sbase = tm_sp + sb * 128;
+                    const int lim = nvis - i * NKV;   // visible columns of this tile
+                    uint32_t rb[CH];
+                    float mrc[NCH];   // reference of each chunk of the tile
+                    if constexpr (kPrefetch) tmem_ld_n<CH>(sbase, rb);
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) {
+                        float s[CH];
+                        if constexpr (!kPrefetch) tmem_ld_n<CH>(sbase + c * CH, rb);
+                        tmem_wait_ld_regs<CH>(rb);
+#pragma unroll
+                        for (int e = 0; e < CH; ++e) s[e] = __uint_as_float(rb[e]);
+                        const int cl = lim - c * CH;   // visible columns of this chunk
+                        if (!pos_scale) {
+#pragma unroll
+                            for (int e = 0; e < CH; ++e) s[e] *= c2;
+                        }
+                        if (cl < CH) {
+#pragma unroll
+                            for (int e = 0; e < CH; ++e) s[e] = (e < cl) ? s[e] : -INFINITY;
+                        }
+                        if constexpr (kMask) {
+                            // atten_mask (step 1): a set byte removes a visible block
+                            if (arow != nullptr) {
+                                const uint8_t* mr = arow + (long long)i * NKV + c * CH;
+#pragma unroll
+                                for (int e = 0; e < CH; ++e)
+                                    if (e < cl && mr[e]) s[e] = -INFINITY;
+                            }
+                        }
+                        // chunk maximum: independent chains of 3-input max
+                        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                        for (int e = 0; e + 8 <= CH; e += 8) {
+                            mx4[0] = fmax3(mx4[0], s[e + 0], s[e + 1]);
+                            mx4[1] = fmax3(mx4[1], s[e + 2], s[e + 3]);
+                            mx4[2] = fmax3(mx4[2], s[e + 4], s[e + 5]);
+                            mx4[3] = fmax3(mx4[3], s[e + 6], s[e + 7]);
+                        }
+                        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
+                        m_true = fmaxf(m_true, mx);
+                        const bool need = (m_ref == -INFINITY) ? (mx > -INFINITY) : (mx > m_ref + kRescaleLog2);
+                        if (__any_sync(0xffffffffu, need)) {
+                            // move the reference maximum: everything summed or written
+                            // relative to the old one is scaled by 2^(old - new)
+                            const float m_new = need ? mx : m_ref;
+                            const float f = need ? ((m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new)) : 1.f;
+                            L *= f;
+#pragma unroll
+                            for (int k = 0; k < NCARRY; ++k) carry[k] *= f;
+                            if (c > 0) {
+                                tmem_wait_st();
+#pragma unroll
+                                for (int c0 = 0; c0 < NCH; ++c0)
+                                    if (c0 < c) tmem_scale_packed<T, CH / 2>(sbase + c0 * (CH / 2), f);
+                            }
+                            if (i > 0) {
+                                // P V of the previous tile has completed before O is touched
+                                mbar_wait(bar(B_P_EMPTY + pp), (pcnt - 1) & 1, abort_flag, p.err,
+                                          kErrTimeoutBase + 11);
+                                tc_fence_after();
+                                tmem_scale_f32(tm_op, p.d2, f);
+                            }
+                            m_ref = m_new;
+                        }
+                        // the next chunk's load runs while this one's P and band values
+                        // are computed (issued after the scaling above, which waits for
+                        // its own tensor-memory loads)
+                        if constexpr (kPrefetch) {
+                            if (c + 1 < NCH) tmem_ld_n<CH>(sbase + (c + 1) * CH, rb);
+                        }
+                        const float mr = (m_ref == -INFINITY) ? 0.f : m_ref;
+                        const float2 nm2 = make_float2(-mr, -mr);
+                        // P = 2^(x - m_ref) in fp32; partial sums in pairs
+                        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                          make_float2(0.f, 0.f)};
+#pragma unroll
+                        for (int e = 0; e < CH; e += 2) {
+                            const float2 x = ffma2(make_float2(s[e], s[e + 1]), ce2, nm2);
+                            s[e] = ex2(x.x);
+                            s[e + 1] = ex2(x.y);
+                            acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], make_float2(s[e], s[e + 1]));
+                        }
+                        const float2 t01 = fadd2(acc2[0], acc2[1]), t23 = fadd2(acc2[2], acc2[3]);
+                        L += (t01.x + t01.y) + (t23.x + t23.y);
+                        // P in the storage dtype over the score columns it came from
+                        {
+                            uint32_t pk[CH / 2];
+#pragma unroll
+                            for (int e = 0; e < CH / 2; ++e) pk[e] = pack2<T>(s[2 * e], s[2 * e + 1]);
+                            tmem_st_n<CH / 2>(sbase + c * (CH / 2), pk);
+                        }
+                        // step 4 on the fp32 P: anchors A*jj of this chunk; taps reach
+                        // back into the previous chunk through `carry`
+                        float v[NJC];
+#pragma unroll
+                        for (int jj = 0; jj < NJC; ++jj) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int u = 0; u < NTAP; ++u) {
+                                const int x = A * jj - u;
+                                const float pv = (x >= 0) ? s[x >= 0 ? x : 0] : carry[x < 0 ? (-x - 1) : 0];
+                                acc = fmaf(wband[u], pv, acc);
+                            }
+                            v[jj] = acc;
+                        }
+#pragma unroll
+                        for (int k = 0; k < NCARRY; ++k) carry[k] = s[CH - 1 - k];
+                        mrc[c] = mr;
+                        if (valid) {
+                            // a warp writes its 32 rows' values of the chunk contiguously
+                            float4* bd = reinterpret_cast<float4*>(
+                                sbase_g + ((size_t)(i * NCH + c) * 128 + row) * NJC);
+#pragma unroll
+                            for (int q4 = 0; q4 < NJC / 4; ++q4)
+                                __stcg(bd + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
+                        }
+                    }
+                    if (valid) {
+                        if constexpr (NCH == 4)
+                            __stcg(reinterpret_cast<float4*>(wrow + i * 4), make_float4(mrc[0], mrc[1], mrc[2], mrc[3]));
+                        else if constexpr (NCH == 2)
+                            __stcg(reinterpret_cast<float2*>(wrow + i * 2), make_float2(mrc[0], mrc[1]));
+                        else
+#pragma unroll
+                            for (int c = 0; c < NCH; ++c) __stcg(wrow + i * NCH + c, mrc[c]);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_P_FULL + pp));
+                    ++scnt;
+                    ++pcnt;
+                }
+                const float mr = (m_ref == -INFINITY) ? 0.f : m_ref;
+                if (t.nkv > 0 && valid) {
+                    // the first anchors past the last tile still collect taps from it
+                    float v[NJC];
+#pragma unroll
+                    for (int jj = 0; jj < NJC; ++jj) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int u = 0; u < NTAP; ++u) {
+                            const int x = A * jj - u;
+                            if (x < 0) acc = fmaf(wband[u], carry[-x - 1 >= 0 ? -x - 1 : 0], acc);
+                        }
+                        v[jj] = acc;
+                    }
+                    float4* bd = reinterpret_cast<float4*>(sbase_g + ((size_t)t.nkv * NCH * 128 + row) * NJC);
+#pragma unroll
+                    for (int q4 = 0; q4 < NJC / 4; ++q4)
+                        __stcg(bd + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
+                    __stcg(wrow + t.nkv * NCH, mr);
+                }
+                if (valid) {
+                    // softmax_max / softmax_sum: exact maximum (natural units) and the
+                    // sum of exp(s - max)
+                    const size_t si = ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * 8;
+                    const float mo = (m_true == -INFINITY) ? -INFINITY : m_true * 0.69314718055994530942f;
+                    const float lt = (L > 0.f) ? L * ex2(mr - m_true) : 0.f;
+                    const float4 mv = make_float4(mo, mo, mo, mo);
+                    const float4 lv = make_float4(lt, lt, lt, lt);
+                    reinterpret_cast<float4*>(p.smax + si)[0] = mv;
+                    reinterpret_cast<float4*>(p.smax + si)[1] = mv;
+                    reinterpret_cast<float4*>(p.ssum + si)[0] = lv;
+                    reinterpret_cast<float4*>(p.ssum + si)[1] = lv;
+                }
+                rowstat[((pp * 2 + slot) * 2 + 0) * 128 + row] = mr;
+                rowstat[((pp * 2 + slot) * 2 + 1) * 128 + row] = L;
+                __threadfence_block();   // scratch rows and statistics before the hand-off
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_ROW_DONE + 2 * pp + slot));
+            }
         }
     }
 
@@ -843,7 +878,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     }
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -39,31 +39,35 @@ cudaError_t launch_compress(const CompressParams& p, dim3 grid, int threads, siz
 cudaError_t read_compress_error(int* out, cudaStream_t st);
 
 // ----------------------------------------------------------- attention
-// Warp roles: warps 0-3 softmax (TMEM lanes 32w..32w+31), warps 4-7 epilogue
-// (group sum, output, top-k), warp 8 TMA producer, warp 9 MMA issuer, warps
-// 10-11 idle.  Launched at 168 registers per thread (384 x 168 = 64512); the
-// warpgroups then rebalance to 232 / 152 / 120, whose sum x 128 threads is
-// the same 64512.
-constexpr int kAttnThreads = 384;
-constexpr int kRegsSoftmax = 232;
-constexpr int kRegsEpilogue = 152;
-constexpr int kRegsCtl = 120;
-static_assert((kRegsSoftmax + kRegsEpilogue + kRegsCtl) * 128 <= kAttnThreads * 168,
+// One pass of online softmax per M-tile.  Warp roles (512 threads, four
+// warpgroups): warps 0-3 softmax of pipeline 0, warps 4-7 softmax of
+// pipeline 1 (idle when the launch runs one pipeline), warps 8-11 epilogue
+// (output, group sums, top-k), warp 12 TMA producer, warp 13 MMA issuer,
+// warps 14-15 idle.  Launched at 128 registers per thread (512 x 128 =
+// 65536); setmaxnreg then moves registers to the softmax warpgroups.
+constexpr int kAttnThreads = 512;
+constexpr int kRegsSoftmax = 176;
+constexpr int kRegsEpilogue = 96;
+constexpr int kRegsCtl = 64;
+static_assert((2 * kRegsSoftmax + kRegsEpilogue + kRegsCtl) * 128 <= kAttnThreads * 128,
               "register split exceeds the launch allocation");
 constexpr int kRows = 128;          // M of one tile: (tokens x heads of one KV group)
-constexpr int kEntryMax = 32;       // importance anchors per staging entry
+constexpr float kRescaleLog2 = 8.f; // a row's reference maximum moves only when a
+                                    // chunk's maximum exceeds it by more than this
 
-// One M-tile: up to 128/G consecutive query tokens of one sequence x the G
-// heads of one KV group.
+// One work item: up to npipe x (128/G) consecutive query tokens of one
+// sequence x the G heads of one KV group.  Pipeline p takes the tokens
+// [p*TT, (p+1)*TT) of the item (TT = 128/G), one 128-row M-tile each; both
+// read the same K/V tiles.
 struct AttnTile {
     int q_row0;     // first query row (T1 index)
-    int ntok;       // tokens in the tile (<= tokens per tile)
+    int ntok;       // tokens in the item (<= npipe * TT)
     int group;      // KV head g
     int cmp_row0;   // first compressed row of the sequence (Tc index)
     int n_cmp;      // compressed blocks of the sequence
     int n_sel;      // selection blocks of the sequence
     int t0;         // position of the first token (query offset applied)
-    int nkv;        // KV tiles to visit (both passes)
+    int nkv;        // KV tiles to visit
     int tloc0;      // query index of the first token inside its sequence (mask rows)
 };
 
@@ -71,8 +75,15 @@ struct AttnParams {
     const AttnTile* tiles;
     int num_tiles;
     int* err;               // device error word (workspace)
-    float* score_gmem;      // per-CTA score buffers when they do not fit on chip
-    int score_cap;          // floats per token in a score buffer
+    // per-CTA scratch for the per-head importance values: for each pipeline,
+    // two slots (consecutive items alternate) of `region` floats each.  A slot
+    // holds the banded values chunk-major, [chunk][row 0..127][anchor of the
+    // chunk] (capj floats), then the reference maximum each chunk was written
+    // against, row-major, [row][chunk] with row stride capc.
+    float* band;
+    int capj, capc, region;
+    float* score_gmem;      // per-warp score rows when they do not fit on chip
+    int score_cap;          // floats per score row
     int score_in_smem;
     void* out;
     int32_t* topk;
@@ -84,12 +95,12 @@ struct AttnParams {
     float scale_log2;       // scale * log2(e)
     int nkv_cols;           // compressed blocks per KV tile
     int nslot;              // K/V ring depth
-    int nqbuf;              // Q buffers (1 or 2)
-    int nsbuf;              // S buffers in tensor memory (1 or 2)
-    int tm_o, tm_p;         // tensor-memory columns of O and of P
+    int nqbuf;              // Q buffers (each holds npipe M-tiles of Q)
+    int npipe;              // M-tiles per item (1 or 2)
+    int nsb;                // score buffers per pipeline in tensor memory
+    int tm_s[2], tm_o[2];   // tensor-memory columns: score buffer 0 and O of each pipeline
     // shared-memory layout (byte offsets from a 1024-aligned base)
-    int off_q, q_bytes, off_ring, slot_bytes, off_stage, stage_entry_bytes, off_score, off_bar,
-        smem_bytes;
+    int off_q, q_bytes, off_ring, slot_bytes, off_rowstat, off_score, off_bar, smem_bytes;
     // optional masks (null = none): bool bytes (S1, row stride), one matrix for
     // every sequence and head, row = query index inside the sequence
     const uint8_t* amask;   // (S1, >= n_cmp): true removes the compressed block (step 1)
@@ -100,7 +111,8 @@ struct AttnParams {
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, int grid, cudaStream_t st);
-int attention_kv_cols(int a);   // compressed blocks per KV tile for band factor a
+int attention_kv_cols(int a);     // compressed blocks per KV tile for band factor a
+int attention_chunk_cols(int a);  // score columns per softmax chunk for band factor a
 
 // ------------------------------------------------ selection attention
 // Attention over the raw K/V blocks of l' tokens that the compressed branch's

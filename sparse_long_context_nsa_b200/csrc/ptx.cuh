@@ -102,6 +102,33 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Tiled 3D tensor copy global -> shared with an L2 cache policy (no multicast).
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                                 uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+        : "memory");
+}
+// L2 policy: lines touched under it are evicted first (data read or written once).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// 16-byte global store under an L2 policy.
+__device__ __forceinline__ void st_global_v4_hint(void* p, uint4 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w), "l"(policy)
+                 : "memory");
+}
+// Drops one 128-byte line from L2 without writing it back (its contents
+// become undefined): for scratch data that is dead once read.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -276,6 +303,92 @@ template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// tcgen05.ld / tcgen05.st of 32 lanes x 32 bits over 1..32 consecutive
+// columns (one register per column), and of any N of them in pieces.
+#define NSA_TMEM_LD_X(N, ...)                                                                        \
+    __device__ __forceinline__ void tmem_ld_x##N(uint32_t taddr, uint32_t* r) {                       \
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x" #N ".b32 " __VA_ARGS__ : NSA_OUT##N(r)        \
+                     : "r"(taddr));                                                                    \
+    }
+#define NSA_TMEM_ST_X(N, ...)                                                                        \
+    __device__ __forceinline__ void tmem_st_x##N(uint32_t taddr, const uint32_t* r) {                 \
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x" #N ".b32 [%0], " __VA_ARGS__ ::"r"(taddr),     \
+                     NSA_IN##N(r)                                                                      \
+                     : "memory");                                                                      \
+    }
+#define NSA_OUT1(r) "=r"(r[0])
+#define NSA_OUT2(r) NSA_OUT1(r), "=r"(r[1])
+#define NSA_OUT4(r) NSA_OUT2(r), "=r"(r[2]), "=r"(r[3])
+#define NSA_OUT8(r) NSA_OUT4(r), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+#define NSA_IN1(r) "r"(r[0])
+#define NSA_IN2(r) NSA_IN1(r), "r"(r[1])
+#define NSA_IN4(r) NSA_IN2(r), "r"(r[2]), "r"(r[3])
+#define NSA_IN8(r) NSA_IN4(r), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+NSA_TMEM_LD_X(1, "{%0}, [%1];")
+NSA_TMEM_LD_X(2, "{%0,%1}, [%2];")
+NSA_TMEM_LD_X(4, "{%0,%1,%2,%3}, [%4];")
+NSA_TMEM_LD_X(8, "{%0,%1,%2,%3,%4,%5,%6,%7}, [%8];")
+NSA_TMEM_ST_X(1, "{%1};")
+NSA_TMEM_ST_X(2, "{%1,%2};")
+NSA_TMEM_ST_X(4, "{%1,%2,%3,%4};")
+NSA_TMEM_ST_X(8, "{%1,%2,%3,%4,%5,%6,%7,%8};")
+#undef NSA_TMEM_LD_X
+#undef NSA_TMEM_ST_X
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+// N consecutive columns into r[0..N), in pieces of 32/16/8/4/2/1 columns.
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* r) {
+    if constexpr (N >= 32) {
+        tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+        if constexpr (N > 32) tmem_ld_n<N - 32>(taddr + 32, r + 32);
+    } else if constexpr (N >= 16) {
+        tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+        if constexpr (N > 16) tmem_ld_n<N - 16>(taddr + 16, r + 16);
+    } else if constexpr (N >= 8) {
+        tmem_ld_x8(taddr, r);
+        if constexpr (N > 8) tmem_ld_n<N - 8>(taddr + 8, r + 8);
+    } else if constexpr (N >= 4) {
+        tmem_ld_x4(taddr, r);
+        if constexpr (N > 4) tmem_ld_n<N - 4>(taddr + 4, r + 4);
+    } else if constexpr (N >= 2) {
+        tmem_ld_x2(taddr, r);
+        if constexpr (N > 2) tmem_ld_n<N - 2>(taddr + 2, r + 2);
+    } else if constexpr (N == 1) {
+        tmem_ld_x1(taddr, r);
+    }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+    if constexpr (N >= 32) {
+        tmem_st32(taddr, r);
+        if constexpr (N > 32) tmem_st_n<N - 32>(taddr + 32, r + 32);
+    } else if constexpr (N >= 16) {
+        tmem_st16(taddr, r);
+        if constexpr (N > 16) tmem_st_n<N - 16>(taddr + 16, r + 16);
+    } else if constexpr (N >= 8) {
+        tmem_st_x8(taddr, r);
+        if constexpr (N > 8) tmem_st_n<N - 8>(taddr + 8, r + 8);
+    } else if constexpr (N >= 4) {
+        tmem_st_x4(taddr, r);
+        if constexpr (N > 4) tmem_st_n<N - 4>(taddr + 4, r + 4);
+    } else if constexpr (N >= 2) {
+        tmem_st_x2(taddr, r);
+        if constexpr (N > 2) tmem_st_n<N - 2>(taddr + 2, r + 2);
+    } else if constexpr (N == 1) {
+        tmem_st_x1(taddr, r);
+    }
+}
+
 __device__ __forceinline__ float lg2(float x) {
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -8,7 +8,11 @@ Tolerances (written here once, used by every parity test):
                  differ by at most one unit in the last place; near a
                  cancelling sum the fp32 accumulation error bound (l terms,
                  unit roundoff 2^-24, times the sum of magnitudes) decides.
-  attention_out  max |gpu - oracle| <= 1e-2 (the stated bar for bf16 inputs)
+  attention_out  max |gpu - oracle| <= 1e-2 (the stated bar for bf16 inputs);
+                 constructed cases whose rows put nearly all weight on one
+                 value row add 2^-7 |oracle|: the output's own rounding to
+                 bf16 is up to 2^-8 |out| (0.0156 at |out| = 4, above 1e-2)
+                 and P in bf16 adds up to 2^-9 relative per term
   softmax stats  relative error <= 1e-3, absolute floor 1e-6 where
                  |oracle| < 1e-3; empty rows exactly -inf / 0; all 8 copies
                  equal.
@@ -43,8 +47,11 @@ def check_compress(got: torch.Tensor, x, w, l, d, cu, dtype):
     return float(err.max())
 
 
-def check_attention(res, ref, count, rows=None, tie_rel=1e-4, out_tol=1e-2, stat_rel=1e-3):
-    """res: GPU outputs (att, topk, smax, ssum); ref: oracle dict for `rows`."""
+def check_attention(res, ref, count, rows=None, tie_rel=1e-4, out_tol=1e-2, stat_rel=1e-3, out_rel=0.0):
+    """res: GPU outputs (att, topk, smax, ssum); ref: oracle dict for `rows`.
+
+    attention_out must satisfy |gpu - oracle| <= out_tol + out_rel * |oracle|
+    element-wise; out_rel = 0 is the plain max-abs bar."""
     att, tk, smax, ssum = res
     if rows is None:
         rows = ref["rows"]
@@ -59,7 +66,9 @@ def check_attention(res, ref, count, rows=None, tie_rel=1e-4, out_tol=1e-2, stat
     assert np.isfinite(g_out).all(), "non-finite attention_out"
     err = np.abs(g_out - ref["out"])
     report["out_max_abs"] = float(err.max()) if err.size else 0.0
-    assert report["out_max_abs"] <= out_tol, f"attention_out max abs err {report['out_max_abs']}"
+    excess = err - (out_tol + out_rel * np.abs(ref["out"]))
+    assert not (excess > 0).any(), (f"attention_out max abs err {report['out_max_abs']}, "
+                                    f"worst excess over the bound {float(excess.max())}")
 
     # stats: 8 equal copies, empty rows exact
     assert (g_max == g_max[..., :1]).all() and (g_sum == g_sum[..., :1]).all()

@@ -96,8 +96,11 @@ def test_band_parameters(nsa, l, d, lp):
     check_attention(res, ref, wl.count)
 
 
+# D2 > 128 runs one M-tile per work item (two score buffers and O of up to 256
+# columns in tensor memory); the others run two M-tiles per item
 @pytest.mark.parametrize("d1,d2,dtype", [(64, 64, "fp16"), (128, 128, "bf16"), (192, 128, "fp16"),
-                                         (96, 48, "bf16"), (128, 64, "bf16"), (32, 16, "fp16")])
+                                         (96, 48, "bf16"), (128, 64, "bf16"), (32, 16, "fp16"),
+                                         (256, 256, "bf16"), (160, 144, "fp16")])
 def test_head_dims_and_dtypes(nsa, d1, d2, dtype):
     wl = _wl([1800, 333], 8, 2, d1, d2, 64, 32, 64, 16, dtype=dtype)
     res, ref, _, _ = _run_both(nsa, wl)
@@ -130,6 +133,57 @@ def test_score_buffer_in_global_memory(nsa):
     res, ref, _, _ = _run_both(nsa, wl, rows=workloads.sample_rows(np.array([20000], np.int32),
                                                                       first=300, last=300, every=37))
     check_attention(res, ref, wl.count)
+
+
+def _direct(nsa, q, kc, vc, scale, l, d, lp, count, seqs, out_rel=0.0):
+    """GPU vs oracle on given q / kcmp / vcmp (storage dtype, CPU tensors)."""
+    cu = np.cumsum(seqs).astype(np.int32)
+    cuc = oracle.compress_len(cu, l, d)
+    cus = np.cumsum([-(-s_ // lp) for s_ in seqs]).astype(np.int32)
+    n1, n2 = q.shape[1], kc.shape[1]
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(n1, n2, q.shape[2], vc.shape[2], l, d, lp, count,
+                                                               cu, cuc, cus), dtype=torch.uint8, device="cuda")
+    res = nsa.nsa_compress_attention(q.cuda(), kc.cuda(), vc.cuda(), scale, n1, l, d, lp, count, cu, cuc, cus,
+                                     workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0, hex(int(ws[:4].view(torch.int32).item()))
+    ref = oracle.compress_attention(q, kc, vc, scale, l, d, lp, count, cu, cuc, cus)
+    return check_attention(res, ref, count, out_rel=out_rel)
+
+
+@pytest.mark.parametrize("step,dd", [(40, 64), (7, 64), (7, 256)], ids=["s40", "s7", "s7_d256"])
+def test_reference_maximum_moves(nsa, step, dd):
+    """Scores with a staircase offset: every `step` compressed blocks the
+    largest score of a row jumps by 10 (natural units, about 14 in log2), more
+    than the kernel lets P grow over its reference maximum, so the reference
+    moves inside KV tiles (chunks after the first), across KV tiles (O and L
+    rescaled) and, with step 7, several times per tile; D = 256 runs the
+    one-pipeline form, whose O rescale waits for the previous P V."""
+    g = torch.Generator().manual_seed(11)
+    S, n1, n2, l, d, lp, count = 3000, 16, 2, 32, 16, 64, 8
+    n_cmp = (S - l) // d + 1
+    scale = dd ** -0.5
+    q = torch.randn(S, n1, dd, generator=g)
+    q[:, :, 0] = 1.0
+    kc = torch.randn(n_cmp, n2, dd, generator=g)
+    kc[:, :, 0] = (10.0 / scale) * torch.div(torch.arange(n_cmp), step, rounding_mode="floor")[:, None].float() \
+        / max(1, (n_cmp // step) // 8)
+    vc = torch.randn(n_cmp, n2, dd, generator=g)
+    # rows end up on one or two value rows (|v| up to about 4.5): the bf16
+    # rounding of the output itself exceeds 1e-2 there, hence the relative term
+    rep = _direct(nsa, q.to(torch.bfloat16), kc.to(torch.bfloat16), vc.to(torch.bfloat16), scale, l, d, lp,
+                  count, [S], out_rel=2.0 ** -7)
+    print(rep)
+
+
+@pytest.mark.parametrize("scale", [-0.125, 0.0])
+def test_non_positive_scale(nsa, scale):
+    g = torch.Generator().manual_seed(12)
+    S, n1, n2, dd, l, d, lp, count = 1500, 8, 2, 64, 32, 16, 64, 8
+    n_cmp = (S - l) // d + 1
+    q = torch.randn(S, n1, dd, generator=g).to(torch.bfloat16)
+    kc = (torch.randn(n_cmp, n2, dd, generator=g) * 0.3).to(torch.bfloat16)
+    vc = torch.randn(n_cmp, n2, dd, generator=g).to(torch.bfloat16)
+    _direct(nsa, q, kc, vc, scale, l, d, lp, count, [S])
 
 
 def test_deterministic_and_status(nsa):

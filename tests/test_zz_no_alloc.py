@@ -79,17 +79,17 @@ def test_noalloc_matches_regular_entry_point_twice(nsa, wl):
 
 
 def test_noalloc_refuses_problems_beyond_the_fixed_scratch(nsa):
-    # one head per group and many selection blocks: per-CTA score buffers far
-    # beyond 16 MiB; refused before anything is enqueued
-    wl = workloads.Workload("big", (40000,), 64, 64, 64, 64, 16, 16, 16, 8, 0.125)
-    need = nsa.nsa_compress_attention_workspace_size(64, 64, 64, 64, 16, 16, 16, 8, [40000],
-                                                     nsa.nsa_compress_out_len([40000], 16, 16),
-                                                     [2500])
+    # l' = d = 16 over 300000 tokens: 18750 compressed blocks, each a
+    # selection anchor, so one CTA's importance scratch (two slots of 128 rows
+    # of ~19000 floats) alone exceeds 16 MiB; refused before anything is
+    # enqueued
+    S, n, dd = 300000, 1, 16
+    cuc = nsa.nsa_compress_out_len([S], 16, 16)
+    wl = workloads.Workload("big", (S,), n, n, dd, dd, 16, 16, 16, 8, 0.25)
+    need = nsa.nsa_compress_attention_workspace_size(n, n, dd, dd, 16, 16, 16, 8, [S], cuc, [S // 16])
     assert need > (16 << 20)
-    q = torch.zeros(40000, 64, 64, dtype=torch.bfloat16, device="cuda")
-    kv = torch.zeros(2500, 64, 64, dtype=torch.bfloat16, device="cuda")
-    outs = _empty_outputs(wl, 40000)
+    q = torch.zeros(S, n, dd, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(int(cuc[-1]), n, dd, dtype=torch.bfloat16, device="cuda")
+    outs = _empty_outputs(wl, S)
     with pytest.raises(Exception, match="NSA_ERR_WORKSPACE"):
-        nsa.nsa_compress_attention_noalloc(q, kv, kv, 0.125, 64, 16, 16, 16, 8, [40000],
-                                           nsa.nsa_compress_out_len([40000], 16, 16), [2500],
-                                           out=outs)
+        nsa.nsa_compress_attention_noalloc(q, kv, kv, 0.25, n, 16, 16, 16, 8, [S], cuc, [S // 16], out=outs)
