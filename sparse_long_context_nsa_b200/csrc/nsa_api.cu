@@ -187,12 +187,21 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
         pl.score_in_smem = in_smem;
         return pl.smem_bytes <= kSmemLimit;
     };
-    // preference: two pipelines, then a deeper K/V ring, a second Q buffer,
-    // on-chip score rows
-    static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}, {2, 2}, {1, 2}};
+    // preference: a K/V ring of at least three slots, then two pipelines, a
+    // deeper ring, a second Q buffer, on-chip score rows.  Measured on B200:
+    // with D1 = 192 two pipelines leave two ring slots and run slower than one
+    // pipeline with three (varlen workload 7.2 vs 6.6 ms)
+    static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}};
+    static const int kOrder2[][2] = {{2, 2}, {1, 2}};
     bool fits = false;
-    for (int np = std::min(npipe_max, d2 <= 128 ? 2 : 1); np >= 1 && !fits; --np)
+    const int np_hi = std::min(npipe_max, d2 <= 128 ? 2 : 1);
+    for (int np = np_hi; np >= 1 && !fits; --np)
         for (const auto& o : kOrder) {
+            if ((fits = layout(np, o[0], o[1], true))) break;
+            if ((fits = layout(np, o[0], o[1], false))) break;
+        }
+    for (int np = np_hi; np >= 1 && !fits; --np)
+        for (const auto& o : kOrder2) {
             if ((fits = layout(np, o[0], o[1], true))) break;
             if ((fits = layout(np, o[0], o[1], false))) break;
         }

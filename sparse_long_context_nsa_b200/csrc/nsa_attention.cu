@@ -146,6 +146,10 @@ __device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int
         }
         const int c = __reduce_add_sync(0xffffffffu, c0 + c1);
         if (c >= k) thr = trial;
+        // exactly k keys at or above the trial threshold: they are the top-k
+        // (the selection below takes the keys above thr, none of which is equal
+        // to a threshold that no key reaches exactly, plus none of the ties)
+        if (c == k) break;
     }
     return thr;
 }
@@ -195,6 +199,7 @@ __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, 
             for (int j = lane; j < lim; j += 32) c += (!masked(j) && __float_as_uint(sc[j]) >= trial) ? 1 : 0;
             c = __reduce_add_sync(0xffffffffu, c);
             if (c >= k) thr = trial;
+            if (c == k) break;   // exactly k keys at or above it: the top-k
         }
     }
     int ngt = 0;
@@ -573,6 +578,9 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // Lane l takes anchors 4l..4l+3 of every 128 (in one chunk, NJC % 4 == 0)
                 // and loops over the heads, eight at a time for loads in flight.
                 const float* wbase = base + p.capj + (size_t)(tl * G) * p.capc;
+                // (measured on B200: the chunk weights computed here, with their
+                // references loaded next to the banded values, beat a per-step weight
+                // table filled first, which serialises two L2 round trips per step)
                 for (int j0 = 0; j0 < jn; j0 += 128) {
                     const int j4 = j0 + 4 * lane;
                     const bool live = j4 < jn;
