@@ -704,9 +704,11 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const uint32_t sbase = tm_sp + sb * 128;
                     const int lim = nvis - i * NKV;   // visible columns of this tile
                     uint32_t rb[CH];
-                    float mrc[NCH];   // reference of each chunk of the tile
                     if constexpr (kPrefetch) tmem_ld_n<CH>(sbase, rb);
-#pragma unroll
+                    // a rolled loop: measured on B200, unrolling the chunks grows the
+                    // hot code past what the instruction caches hold with the other
+                    // roles running on the same SM (128K workload 46.7 -> 41.9 ms rolled)
+#pragma unroll 1
                     for (int c = 0; c < NCH; ++c) {
                         float s[CH];
                         if constexpr (!kPrefetch) tmem_ld_n<CH>(sbase + c * CH, rb);
@@ -809,7 +811,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
 #pragma unroll
                         for (int k = 0; k < NCARRY; ++k) carry[k] = s[CH - 1 - k];
-                        mrc[c] = mr;
+                        if (valid) __stcg(wrow + i * NCH + c, mr);
                         if (valid) {
                             // a warp writes its 32 rows' values of the chunk contiguously
                             float4* bd = reinterpret_cast<float4*>(
@@ -819,15 +821,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                 __stcg(bd + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
                         }
                     }
-                    if (valid) {
-                        if constexpr (NCH == 4)
-                            __stcg(reinterpret_cast<float4*>(wrow + i * 4), make_float4(mrc[0], mrc[1], mrc[2], mrc[3]));
-                        else if constexpr (NCH == 2)
-                            __stcg(reinterpret_cast<float2*>(wrow + i * 2), make_float2(mrc[0], mrc[1]));
-                        else
-#pragma unroll
-                            for (int c = 0; c < NCH; ++c) __stcg(wrow + i * NCH + c, mrc[c]);
-                    }
+
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
