@@ -180,6 +180,60 @@ nsa_status_t nsa_compress_attention_masked(
     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sharding one problem by KV-head group, with no communication: every
+ * (token, KV group) pair of steps 1-7 is independent, and a group's G query
+ * heads, its K/V head and its top-k row are read and written by it alone.
+ * A rank that computes groups [group_begin, group_begin + group_count) of
+ * the problem needs only those heads' data and writes only those outputs.
+ *
+ * nsa_shard_groups: the balanced contiguous split of n2 groups over `world`
+ * ranks (the first n2 % world ranks take one group more).  Pure host
+ * function; NSA_ERR_INVALID_ARG for n2 < 1, world < 1, rank outside
+ * [0, world) or NULL outputs.
+ */
+nsa_status_t nsa_shard_groups(int n2, int world, int rank, int* group_begin, int* group_count);
+
+/*
+ * Workspace bytes of nsa_compress_attention_shard for these arguments (a
+ * shard needs less than the whole problem).  Pure host function.
+ */
+nsa_status_t nsa_compress_attention_shard_workspace_size(
+    int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int group_begin, int group_count, size_t* bytes);
+
+/*
+ * nsa_compress_attention restricted to the KV groups [group_begin,
+ * group_begin + group_count): the query heads h with h / G in that range,
+ * their attention_out / softmax_max / softmax_sum rows, and topk_indices
+ * [t, g, :] for g in that range.  Tensors are the whole problem's (same
+ * shapes and layout as nsa_compress_attention); only the shard's heads are
+ * read and only the shard's outputs are written, everything else is left
+ * untouched.  The results are bitwise those of nsa_compress_attention for
+ * the same heads.  NSA_ERR_INVALID_ARG when the range is not inside [0, n2);
+ * other arguments and errors as nsa_compress_attention.
+ */
+nsa_status_t nsa_compress_attention_shard(
+    const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
+    int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int n2, int d1, int d2, nsa_dtype_t dtype, int group_begin, int group_count,
+    void* attention_out, int32_t* topk_indices, float* softmax_max, float* softmax_sum,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The work items a shard's launch runs, for inspection on the host (no CUDA
+ * call): each item is (first query row, tokens, KV group) as three int32 in
+ * `items` (capacity items fit); *n_items receives the total.  The items of
+ * the shards of nsa_shard_groups cover every (query row, KV group) pair of
+ * the problem exactly once.
+ */
+nsa_status_t nsa_compress_attention_shard_plan(
+    int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int group_begin, int group_count, int32_t* items, int64_t capacity, int64_t* n_items);
+
+/*
  * Bytes of device workspace nsa_select_attention needs for these shapes
  * (same arguments; a pure host computation).
  */

@@ -41,6 +41,10 @@ EXPORTED = (
     "nsa_noalloc_status",
     "nsa_select_attention_workspace_size",
     "nsa_select_attention",
+    "nsa_shard_groups",
+    "nsa_compress_attention_shard_workspace_size",
+    "nsa_compress_attention_shard",
+    "nsa_compress_attention_shard_plan",
 )
 
 _lib = None
@@ -103,6 +107,17 @@ def load(path: Optional[str] = None):
     lib.nsa_select_attention.argtypes = [vp, vp, vp, vp, ctypes.c_float, ci, ci, ci, i32p, i32p, ci, ci, ci,
                                          ci, ci, vp, vp, vp, cs, vp]
     lib.nsa_select_attention.restype = ci
+    lib.nsa_shard_groups.argtypes = [ci, ci, ci, ctypes.POINTER(ci), ctypes.POINTER(ci)]
+    lib.nsa_shard_groups.restype = ci
+    lib.nsa_compress_attention_shard_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p, i32p, i32p,
+                                                                ci, ci, ci, ctypes.POINTER(cs)]
+    lib.nsa_compress_attention_shard_workspace_size.restype = ci
+    lib.nsa_compress_attention_shard.argtypes = [vp, vp, vp, ctypes.c_float, ci, ci, ci, ci, ci, i32p, i32p, i32p,
+                                                 ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, cs, vp]
+    lib.nsa_compress_attention_shard.restype = ci
+    lib.nsa_compress_attention_shard_plan.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p, i32p, i32p, ci, ci, ci,
+                                                      vp, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+    lib.nsa_compress_attention_shard_plan.restype = ci
     if path is None:
         _lib = lib
     return lib
@@ -452,3 +467,96 @@ def nsa_select_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk
         workspace.data_ptr(), workspace.numel(), _stream(stream))
     _raise(st, "nsa_select_attention")
     return att, lse
+
+
+# ------------------------------------------------------------ head-group shards
+def nsa_shard_groups(n2: int, world: int, rank: int):
+    """(group_begin, group_count) of `rank` in the balanced contiguous split of
+    n2 KV groups over `world` ranks."""
+    b, c = ctypes.c_int(0), ctypes.c_int(0)
+    _raise(load().nsa_shard_groups(int(n2), int(world), int(rank), ctypes.byref(b), ctypes.byref(c)),
+           "nsa_shard_groups")
+    return int(b.value), int(c.value)
+
+
+def nsa_compress_attention_shard_workspace_size(head_num: int, n2: int, d1: int, d2: int, l: int, d: int, lp: int,
+                                                count: int, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                                group_begin: int, group_count: int) -> int:
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size):
+        raise ValueError("the three prefix-sum lists need one entry per sequence")
+    out = ctypes.c_size_t(0)
+    _raise(load().nsa_compress_attention_shard_workspace_size(
+        int(head_num), int(n2), int(d1), int(d2), int(l), int(d), int(lp), int(count), _ip(cq), _ip(cc), _ip(cs),
+        cq.size, int(group_begin), int(group_count), ctypes.byref(out)),
+        "nsa_compress_attention_shard_workspace_size")
+    return int(out.value)
+
+
+def nsa_compress_attention_shard_plan(head_num: int, n2: int, d1: int, d2: int, l: int, d: int, lp: int,
+                                      count: int, cu_seqlens_q, cu_cmp_kv, cu_sel_kv, group_begin: int,
+                                      group_count: int) -> np.ndarray:
+    """Work items of a shard's launch, (n_items, 3) int32: first query row,
+    tokens, KV group.  Host only."""
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    args = (int(head_num), int(n2), int(d1), int(d2), int(l), int(d), int(lp), int(count), _ip(cq), _ip(cc),
+            _ip(cs), cq.size, int(group_begin), int(group_count))
+    n = ctypes.c_int64(0)
+    _raise(load().nsa_compress_attention_shard_plan(*args, None, 0, ctypes.byref(n)),
+           "nsa_compress_attention_shard_plan")
+    items = np.zeros((max(int(n.value), 1), 3), dtype=np.int32)
+    _raise(load().nsa_compress_attention_shard_plan(*args, items.ctypes.data_as(ctypes.c_void_p), int(n.value),
+                                                    ctypes.byref(n)), "nsa_compress_attention_shard_plan")
+    return items[:int(n.value)]
+
+
+def nsa_compress_attention_shard(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tensor, scale: float,
+                                 head_num: int, l: int, d: int, lp: int, count: int, cu_seqlens_q, cu_cmp_kv,
+                                 cu_sel_kv, group_begin: int, group_count: int, out=None,
+                                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """nsa_compress_attention for the KV groups [group_begin, group_begin +
+    group_count) only.  Tensors are the whole problem's; the shard's heads are
+    read and the shard's outputs written (``out`` may pass the four output
+    tensors; rows of other groups are left as they are)."""
+    for t, nm in ((q, "q"), (kcmp, "kcmp"), (vcmp, "vcmp")):
+        _dev(t, nm)
+        if t.dim() != 3:
+            raise ValueError(f"{nm} must be 3-D (TND)")
+    dt = _dtype_code(q)
+    if kcmp.dtype != q.dtype or vcmp.dtype != q.dtype:
+        raise TypeError("q, kcmp and vcmp must share one dtype")
+    t1, n1, d1 = q.shape
+    tc, n2, d1k = kcmp.shape
+    d2 = vcmp.shape[2]
+    if int(head_num) != n1:
+        raise ValueError("head_num must equal the number of query heads")
+    if d1k != d1 or tuple(vcmp.shape[:2]) != (tc, n2):
+        raise ValueError("kcmp must be (Tc, N2, D1) and vcmp (Tc, N2, D2)")
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size):
+        raise ValueError("the three prefix-sum lists need one entry per sequence")
+    if int(cq[-1]) > t1 or int(cc[-1]) > tc:
+        raise ValueError("prefix sums run past the rows of q / kcmp")
+    dev = q.device
+    _same_device(q, (kcmp, "kcmp"), (vcmp, "vcmp"))
+    if out is None:
+        att = torch.zeros(t1, n1, d2, dtype=q.dtype, device=dev)
+        tk = torch.full((t1, n2, count), -1, dtype=torch.int32, device=dev)
+        smax = torch.zeros(t1, n1, 8, dtype=torch.float32, device=dev)
+        ssum = torch.zeros(t1, n1, 8, dtype=torch.float32, device=dev)
+    else:
+        att, tk, smax, ssum = out
+        _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
+        _out(tk, (t1, n2, count), torch.int32, dev, "topk_indices")
+        _out(smax, (t1, n1, 8), torch.float32, dev, "softmax_max")
+        _out(ssum, (t1, n1, 8), torch.float32, dev, "softmax_sum")
+    ws_bytes = nsa_compress_attention_shard_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs,
+                                                           group_begin, group_count)
+    workspace = _workspace(workspace, ws_bytes, dev)
+    st = load().nsa_compress_attention_shard(
+        q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d), int(lp),
+        int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, int(group_begin), int(group_count),
+        att.data_ptr(), tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        _stream(stream))
+    _raise(st, "nsa_compress_attention_shard")
+    return att, tk, smax, ssum

@@ -115,9 +115,13 @@ nsa_status_t validate_attention(int head_num, int n2, int d1, int d2, int l, int
 // M-tile per item.
 nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
                             const int32_t* cu_q, const int32_t* cu_cmp, const int32_t* cu_sel, int batch,
-                            bool build_tiles, AttnPlan& pl, int grid_cap = kMaxGrid, int npipe_max = 2) {
+                            bool build_tiles, AttnPlan& pl, int grid_cap = kMaxGrid, int npipe_max = 2,
+                            int group_begin = 0, int group_count = -1) {
     nsa_status_t s = validate_attention(head_num, n2, d1, d2, l, d, lp, count, cu_q, cu_cmp, cu_sel, batch);
     if (s != NSA_OK) return s;
+    if (group_count < 0) group_count = n2 - group_begin;
+    if (group_begin < 0 || group_count < 0 || group_begin + group_count > n2) return NSA_ERR_INVALID_ARG;
+    const int g_end = group_begin + group_count;
     pl.G = head_num / n2;
     pl.TT = kRows / pl.G;
     pl.a = lp / d;
@@ -226,7 +230,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
         int32_t pq = 0;
         for (int bq = 0; bq < batch; ++bq) {
             const int64_t Sq = cu_q[bq] - pq;
-            ntiles += ((Sq + run - 1) / run) * (int64_t)n2;
+            ntiles += ((Sq + run - 1) / run) * (int64_t)group_count;
             pq = cu_q[bq];
         }
     }
@@ -253,7 +257,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
                 t.tloc0 = (int)tok0;
                 const int nv = nvis_host(t.t0 + t.ntok - 1, l, d, n_cmp);
                 t.nkv = (nv + NKV - 1) / NKV;
-                for (int g = 0; g < n2; ++g) {
+                for (int g = group_begin; g < g_end; ++g) {
                     t.group = g;
                     pl.tiles.push_back(t);
                 }
@@ -548,7 +552,8 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
                                             const uint8_t* topk_mask, int tm_s2, void* attention_out,
                                             int32_t* topk_indices, float* softmax_max, float* softmax_sum,
                                             void* workspace, size_t workspace_bytes, void* stream,
-                                            int grid_cap = kMaxGrid, int npipe_max = 2) {
+                                            int grid_cap = kMaxGrid, int npipe_max = 2, int group_begin = 0,
+                                            int group_count = -1) {
     if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
     if (!q || !kcmp || !vcmp || !attention_out || !topk_indices || !softmax_max || !softmax_sum)
@@ -558,7 +563,7 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
         return NSA_ERR_INVALID_ARG;
     AttnPlan pl;
     nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
-                                    batch, true, pl, grid_cap, npipe_max);
+                                    batch, true, pl, grid_cap, npipe_max, group_begin, group_count);
     if (s != NSA_OK) return s;
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         workspace_bytes < pl.ws_total)
@@ -679,6 +684,66 @@ nsa_status_t nsa_compress_attention_masked(const void* q, const void* kcmp, cons
                                    cu_sel_kv, batch, n2, d1, d2, dtype, atten_mask, am_cols, topk_mask, tm_cols,
                                    attention_out, topk_indices, softmax_max, softmax_sum, workspace,
                                    workspace_bytes, stream);
+}
+
+nsa_status_t nsa_shard_groups(int n2, int world, int rank, int* group_begin, int* group_count) {
+    if (n2 < 1 || world < 1 || rank < 0 || rank >= world || !group_begin || !group_count)
+        return NSA_ERR_INVALID_ARG;
+    // contiguous, balanced: the first n2 % world ranks take one group more
+    const int q = n2 / world, r = n2 % world;
+    *group_count = q + (rank < r ? 1 : 0);
+    *group_begin = rank * q + std::min(rank, r);
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention_shard_workspace_size(int head_num, int n2, int d1, int d2, int l, int d,
+                                                         int lp, int count, const int32_t* cu_seqlens_q,
+                                                         const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+                                                         int batch, int group_begin, int group_count,
+                                                         size_t* bytes) {
+    if (bytes == nullptr || group_begin < 0 || group_count < 0) return NSA_ERR_INVALID_ARG;
+    AttnPlan pl;
+    nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                    batch, false, pl, kMaxGrid, 2, group_begin, group_count);
+    if (s != NSA_OK) return s;
+    *bytes = pl.ws_total;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention_shard(const void* q, const void* kcmp, const void* vcmp, float scale,
+                                          int head_num, int l, int d, int lp, int count,
+                                          const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv,
+                                          const int32_t* cu_sel_kv, int batch, int n2, int d1, int d2,
+                                          nsa_dtype_t dtype, int group_begin, int group_count,
+                                          void* attention_out, int32_t* topk_indices, float* softmax_max,
+                                          float* softmax_sum, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+    if (group_begin < 0 || group_count < 0) return NSA_ERR_INVALID_ARG;
+    return compress_attention_impl(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
+                                   cu_sel_kv, batch, n2, d1, d2, dtype, nullptr, 0, nullptr, 0, attention_out,
+                                   topk_indices, softmax_max, softmax_sum, workspace, workspace_bytes, stream,
+                                   kMaxGrid, 2, group_begin, group_count);
+}
+
+nsa_status_t nsa_compress_attention_shard_plan(int head_num, int n2, int d1, int d2, int l, int d, int lp,
+                                               int count, const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv,
+                                               const int32_t* cu_sel_kv, int batch, int group_begin,
+                                               int group_count, int32_t* items, int64_t capacity,
+                                               int64_t* n_items) {
+    if (n_items == nullptr || (capacity > 0 && items == nullptr)) return NSA_ERR_INVALID_ARG;
+    if (group_begin < 0 || group_count < 0) return NSA_ERR_INVALID_ARG;
+    AttnPlan pl;
+    nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                    batch, true, pl, kMaxGrid, 2, group_begin, group_count);
+    if (s != NSA_OK) return s;
+    *n_items = (int64_t)pl.tiles.size();
+    const int64_t n = std::min<int64_t>(capacity, (int64_t)pl.tiles.size());
+    for (int64_t i = 0; i < n; ++i) {
+        items[3 * i + 0] = pl.tiles[i].q_row0;
+        items[3 * i + 1] = pl.tiles[i].ntok;
+        items[3 * i + 2] = pl.tiles[i].group;
+    }
+    return NSA_OK;
 }
 
 nsa_status_t nsa_select_attention_workspace_size(int head_num, int n2, int d1, int d2, int lp, int count,
