@@ -11,7 +11,10 @@
  *   nsa_compress_attention_masked  the same with the optional atten_mask /
  *                           topk_mask of the page's keyword arguments
  *   nsa_select_attention    attention over the raw K/V blocks that top-k lists
- *                           ("lite_boost.ops.rain_fusion_attention").
+ *                           ("lite_boost.ops.rain_fusion_attention");
+ *   nsa_compress_attention_backward, nsa_compress_backward
+ *                           gradients of the compressed attention and of the
+ *                           compression (training scenario).
  *
  * Conventions shared by every entry point
  *   - Layout is TND ("mindspore.ops.nsa_compress_attention", note list):
@@ -280,9 +283,79 @@ nsa_status_t nsa_select_attention(
     void* attention_out, float* softmax_lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of device workspace nsa_compress_attention_backward needs (a pure
+ * host computation; same shape arguments as the backward call).
+ */
+nsa_status_t nsa_compress_attention_backward_workspace_size(
+    int head_num, int n2, int d1, int d2, int l, int d,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, int batch, size_t* bytes);
+
+/*
+ * Gradient of attention_out of nsa_compress_attention (its steps 1-3) with
+ * respect to q, kcmp and vcmp.  The page returns softmax_max / softmax_sum
+ * for gradient back-propagation ("mindspore.ops.nsa_compress_attention",
+ * Returns) and prints no backward formulas; they follow from the forward
+ * definition, with P_i = exp(s_i - m) / L over the visible blocks:
+ *   dvcmp_i = sum over rows and the G heads of group g of P_i dout
+ *   dS_i    = P_i (dout . vcmp_i - dout . attention_out)
+ *   dq      = scale sum_i dS_i kcmp_i
+ *   dkcmp_i = scale sum over rows and heads of dS_i q
+ * The importance scores and topk_indices are index outputs: no gradient.
+ * Arguments
+ *   q, kcmp, vcmp      the forward's inputs (device, TND, dtype)
+ *   attention_out      device (T1, N1, D2) dtype, the forward's output
+ *   dout               device (T1, N1, D2) dtype, gradient of attention_out
+ *   softmax_max, softmax_sum  device (T1, N1, 8) fp32, the forward's statistics
+ *   scale, head_num, l, d, cu_seqlens_q, cu_cmp_kv, batch, n2, d1, d2, dtype
+ *                      as in the forward call
+ *   dq                 device (T1, N1, D1) fp32, overwritten
+ *   dkcmp, dvcmp       device (Tc, N2, D1) / (Tc, N2, D2) fp32, overwritten
+ *   workspace          device, >= the size above, 256-byte aligned; first 16
+ *                      bytes: error word (nsa_workspace_status)
+ * Constraints: those of the forward without lp / count, and
+ * ceil(D1/64) + ceil(D2/64) <= 6 (Q, dO, K, V tiles on chip together:
+ * NSA_ERR_UNSUPPORTED beyond).  No atten_mask.  Deterministic: each dkcmp /
+ * dvcmp row is the sum of per-run partials in a fixed order, no atomics.
+ * Launches on `stream`: statistics prep, dq, dkcmp/dvcmp runs (one launch,
+ * or two when D2 > 128), partial reduction.
+ */
+nsa_status_t nsa_compress_attention_backward(
+    const void* q, const void* kcmp, const void* vcmp, const void* attention_out, const void* dout,
+    const float* softmax_max, const float* softmax_sum, float scale, int head_num, int l, int d,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, int batch, int n2, int d1, int d2,
+    nsa_dtype_t dtype, float* dq, float* dkcmp, float* dvcmp, void* workspace, size_t workspace_bytes,
+    void* stream);
+
+/*
+ * Bytes of device workspace nsa_compress_backward needs (host computation).
+ */
+nsa_status_t nsa_compress_backward_workspace_size(const int32_t* cu_seqlens, int batch, int l, int d,
+                                                  size_t* bytes);
+
+/*
+ * Gradient of nsa_compress ("aclnnNsaCompress", Formula: kcmp_i = sum_j
+ * w[j] k[i d + j], per head; training scenario).  The compression is linear:
+ *   dk[p]   = sum over the windows i that cover p of w[p - i d] dkcmp_i
+ *   dw[j,n] = sum_i dkcmp_i . k[i d + j] + dvcmp_i . v[i d + j]   (one w for K and V)
+ * Raw rows that no window covers get dk = 0.
+ * Arguments
+ *   k, v, w            the forward's inputs (device; v may be NULL, then dvcmp and dv too)
+ *   dkcmp, dvcmp       device (Tc, N2, D1) / (Tc, N2, D2) fp32, incoming gradients
+ *   dk, dv             device (T, N2, D1) / (T, N2, D2) fp32, overwritten
+ *   dw                 device (l, N2) fp32, overwritten
+ *   workspace          device, >= the size above, 256-byte aligned
+ * Constraints: those of nsa_compress.  Deterministic: dw is reduced per (j, n)
+ * by one CTA in a fixed order.
+ */
+nsa_status_t nsa_compress_backward(
+    const void* k, const void* v, const void* w, const float* dkcmp, const float* dvcmp, int l, int d,
+    const int32_t* cu_seqlens, int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+    float* dk, float* dv, float* dw, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream` and reads the device error word of `workspace`
- * (written by the last nsa_compress_attention or nsa_select_attention that
- * used it).  Returns NSA_OK,
+ * (written by the last nsa_compress_attention, nsa_select_attention or
+ * nsa_compress_attention_backward that used it).  Returns NSA_OK,
  * NSA_ERR_TIMEOUT when a device-side wait gave up, or NSA_ERR_CUDA.
  */
 nsa_status_t nsa_workspace_status(const void* workspace, void* stream);

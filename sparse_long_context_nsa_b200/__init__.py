@@ -45,6 +45,10 @@ EXPORTED = (
     "nsa_compress_attention_shard_workspace_size",
     "nsa_compress_attention_shard",
     "nsa_compress_attention_shard_plan",
+    "nsa_compress_attention_backward_workspace_size",
+    "nsa_compress_attention_backward",
+    "nsa_compress_backward_workspace_size",
+    "nsa_compress_backward",
 )
 
 _lib = None
@@ -118,6 +122,17 @@ def load(path: Optional[str] = None):
     lib.nsa_compress_attention_shard_plan.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p, i32p, i32p, ci, ci, ci,
                                                       vp, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
     lib.nsa_compress_attention_shard_plan.restype = ci
+    lib.nsa_compress_attention_backward_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, i32p, i32p, ci,
+                                                                   ctypes.POINTER(ctypes.c_size_t)]
+    lib.nsa_compress_attention_backward_workspace_size.restype = ci
+    lib.nsa_compress_attention_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, ci, ci, ci, i32p,
+                                                    i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.nsa_compress_attention_backward.restype = ci
+    lib.nsa_compress_backward_workspace_size.argtypes = [i32p, ci, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
+    lib.nsa_compress_backward_workspace_size.restype = ci
+    lib.nsa_compress_backward.argtypes = [vp, vp, vp, vp, vp, ci, ci, i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp,
+                                          ctypes.c_size_t, vp]
+    lib.nsa_compress_backward.restype = ci
     if path is None:
         _lib = lib
     return lib
@@ -560,3 +575,130 @@ def nsa_compress_attention_shard(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torc
         _stream(stream))
     _raise(st, "nsa_compress_attention_shard")
     return att, tk, smax, ssum
+
+
+def nsa_compress_attention_backward_workspace_size(head_num: int, n2: int, d1: int, d2: int, l: int, d: int,
+                                                   cu_seqlens_q, cu_cmp_kv) -> int:
+    cq, cc = _cu(cu_seqlens_q), _cu(cu_cmp_kv)
+    if cq.size != cc.size:
+        raise ValueError("the prefix-sum lists need one entry per sequence")
+    out = ctypes.c_size_t(0)
+    _raise(load().nsa_compress_attention_backward_workspace_size(
+        int(head_num), int(n2), int(d1), int(d2), int(l), int(d), _ip(cq), _ip(cc), cq.size, ctypes.byref(out)),
+        "nsa_compress_attention_backward_workspace_size")
+    return int(out.value)
+
+
+def nsa_compress_attention_backward(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tensor,
+                                    attention_out: torch.Tensor, dout: torch.Tensor, softmax_max: torch.Tensor,
+                                    softmax_sum: torch.Tensor, scale: float, head_num: int, l: int, d: int,
+                                    cu_seqlens_q, cu_cmp_kv, grads=None, workspace: Optional[torch.Tensor] = None,
+                                    stream=None):
+    """Gradient of attention_out of nsa_compress_attention with respect to q,
+    kcmp and vcmp for the incoming ``dout``, from the forward's inputs, output
+    and statistics.  Returns (dq (T1,N1,D1), dkcmp (Tc,N2,D1), dvcmp
+    (Tc,N2,D2)), fp32; ``grads`` may pass the three tensors preallocated."""
+    for t, nm in ((q, "q"), (kcmp, "kcmp"), (vcmp, "vcmp"), (attention_out, "attention_out"), (dout, "dout")):
+        _dev(t, nm)
+        if t.dim() != 3:
+            raise ValueError(f"{nm} must be 3-D (TND)")
+    dt = _dtype_code(q)
+    for t, nm in ((kcmp, "kcmp"), (vcmp, "vcmp"), (attention_out, "attention_out"), (dout, "dout")):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{nm} must have the dtype of q")
+    t1, n1, d1 = q.shape
+    tc, n2, _ = kcmp.shape
+    d2 = vcmp.shape[2]
+    dev = q.device
+    if int(head_num) != n1:
+        raise ValueError("head_num must equal the number of query heads")
+    if kcmp.shape[2] != d1 or tuple(vcmp.shape[:2]) != (tc, n2):
+        raise ValueError("kcmp must be (Tc, N2, D1) and vcmp (Tc, N2, D2)")
+    for t, nm in ((attention_out, "attention_out"), (dout, "dout")):
+        if tuple(t.shape) != (t1, n1, d2):
+            raise ValueError(f"{nm} must be (T1, N1, D2)")
+    for t, nm in ((softmax_max, "softmax_max"), (softmax_sum, "softmax_sum")):
+        _out(t, (t1, n1, 8), torch.float32, dev, nm)
+    _same_device(q, (kcmp, "kcmp"), (vcmp, "vcmp"), (attention_out, "attention_out"), (dout, "dout"))
+    cq, cc = _cu(cu_seqlens_q), _cu(cu_cmp_kv)
+    if cq.size != cc.size:
+        raise ValueError("the prefix-sum lists need one entry per sequence")
+    if int(cq[-1]) > t1 or int(cc[-1]) > tc:
+        raise ValueError("prefix sums run past the rows of q / kcmp")
+    if grads is None:
+        dq = torch.empty(t1, n1, d1, dtype=torch.float32, device=dev)
+        dk = torch.empty(tc, n2, d1, dtype=torch.float32, device=dev)
+        dv = torch.empty(tc, n2, d2, dtype=torch.float32, device=dev)
+    else:
+        dq, dk, dv = grads
+        _out(dq, (t1, n1, d1), torch.float32, dev, "dq")
+        _out(dk, (tc, n2, d1), torch.float32, dev, "dkcmp")
+        _out(dv, (tc, n2, d2), torch.float32, dev, "dvcmp")
+    nbytes = nsa_compress_attention_backward_workspace_size(n1, n2, d1, d2, l, d, cq, cc)
+    workspace = _workspace(workspace, nbytes, dev)
+    st = load().nsa_compress_attention_backward(
+        q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), attention_out.data_ptr(), dout.data_ptr(),
+        softmax_max.data_ptr(), softmax_sum.data_ptr(), float(scale), n1, int(l), int(d), _ip(cq), _ip(cc),
+        cq.size, n2, d1, d2, dt, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+        workspace.numel(), _stream(stream))
+    _raise(st, "nsa_compress_attention_backward")
+    return dq, dk, dv
+
+
+def nsa_compress_backward_workspace_size(cu_seqlens, l: int, d: int) -> int:
+    cu = _cu(cu_seqlens)
+    out = ctypes.c_size_t(0)
+    _raise(load().nsa_compress_backward_workspace_size(_ip(cu), cu.size, int(l), int(d), ctypes.byref(out)),
+           "nsa_compress_backward_workspace_size")
+    return int(out.value)
+
+
+def nsa_compress_backward(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tensor, dkcmp: torch.Tensor,
+                          dvcmp: Optional[torch.Tensor], l: int, d: int, cu_seqlens, grads=None,
+                          workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradient of nsa_compress: returns (dk (T2,N2,D1), dv (T2,N2,D2) or None,
+    dw (l,N2)), fp32, for the incoming fp32 dkcmp / dvcmp."""
+    _dev(k, "k")
+    _dev(w, "w")
+    _dev(dkcmp, "dkcmp")
+    dt = _dtype_code(k)
+    if w.dtype != k.dtype or (v is not None and v.dtype != k.dtype):
+        raise TypeError("k, v and w must share one dtype")
+    if (v is None) != (dvcmp is None):
+        raise ValueError("v and dvcmp go together")
+    t2, n2, d1 = k.shape
+    d2 = 0
+    cu = _cu(cu_seqlens)
+    tc = int(nsa_compress_out_len(cu, l, d)[-1])
+    _out(dkcmp, (tc, n2, d1), torch.float32, k.device, "dkcmp")
+    if v is not None:
+        _dev(v, "v")
+        d2 = v.shape[2]
+        if tuple(v.shape[:2]) != (t2, n2):
+            raise ValueError("v must be (T2, N2, D2) with the T2, N2 of k")
+        _out(dvcmp, (tc, n2, d2), torch.float32, k.device, "dvcmp")
+    if tuple(w.shape) != (l, n2):
+        raise ValueError("w must have shape (l, N2)")
+    if int(cu[-1]) > t2:
+        raise ValueError("cu_seqlens runs past the rows of k")
+    _same_device(k, (w, "w"), (v, "v"), (dkcmp, "dkcmp"), (dvcmp, "dvcmp"))
+    dev = k.device
+    if grads is None:
+        dk = torch.zeros(t2, n2, d1, dtype=torch.float32, device=dev)
+        dv = torch.zeros(t2, n2, d2, dtype=torch.float32, device=dev) if v is not None else None
+        dw = torch.empty(l, n2, dtype=torch.float32, device=dev)
+    else:
+        dk, dv, dw = grads
+        _out(dk, (t2, n2, d1), torch.float32, dev, "dk")
+        if v is not None:
+            _out(dv, (t2, n2, d2), torch.float32, dev, "dv")
+        _out(dw, (l, n2), torch.float32, dev, "dw")
+    nbytes = nsa_compress_backward_workspace_size(cu, l, d)
+    workspace = _workspace(workspace, nbytes, dev)
+    st = load().nsa_compress_backward(
+        k.data_ptr(), v.data_ptr() if v is not None else None, w.data_ptr(), dkcmp.data_ptr(),
+        dvcmp.data_ptr() if v is not None else None, int(l), int(d), _ip(cu), cu.size, n2, d1, d2, dt,
+        dk.data_ptr(), dv.data_ptr() if v is not None else None, dw.data_ptr(), workspace.data_ptr(),
+        workspace.numel(), _stream(stream))
+    _raise(st, "nsa_compress_backward")
+    return dk, dv, dw

@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libnsa_b200.so")
-SOURCES = ["nsa_api.cu", "nsa_compress.cu", "nsa_attention.cu", "nsa_select.cu"]
+SOURCES = ["nsa_api.cu", "nsa_compress.cu", "nsa_attention.cu", "nsa_select.cu", "nsa_backward.cu"]
 HEADERS = ["nsa_internal.h", "ptx.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

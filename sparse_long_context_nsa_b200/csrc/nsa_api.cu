@@ -398,6 +398,153 @@ nsa_status_t plan_select(int head_num, int n2, int d1, int d2, int lp, int count
     return NSA_OK;
 }
 
+// ------------------------------------------------------------------------
+// backward plan: dQ items, dK/dV runs and their partial slots
+// ------------------------------------------------------------------------
+struct BwdPlan {
+    int G = 0, TT = 0;
+    std::vector<bwd::QItem> qitems;
+    std::vector<bwd::KVItem> kvitems;
+    std::vector<bwd::KVTile> kvtiles;
+    int nslots = 0;
+    bool one_pass = true;   // dV and dK in one tensor-memory allocation
+    int off_q = 0, off_do = 0, off_k = 0, off_v = 0, off_row = 0, off_bar = 0, smem_bytes = 0;
+    size_t off_qitems = 0, off_kvitems = 0, off_kvtiles = 0, off_rowinfo = 0, off_part = 0, ws_total = 0;
+};
+
+nsa_status_t plan_backward(int head_num, int n2, int d1, int d2, int l, int d, const int32_t* cu_q,
+                           const int32_t* cu_cmp, int batch, bool build, BwdPlan& pl) {
+    // the forward's constraints (note list of mindspore.ops.nsa_compress_attention)
+    if (l % 16 || d % 16 || l < 16 || l > 128 || d < 16 || d > 64 || l < d) return NSA_ERR_INVALID_ARG;
+    if (d1 < 16 || d2 < 16 || d1 % 16 || d2 % 16 || d1 < d2) return NSA_ERR_INVALID_ARG;
+    if (n2 < 1 || head_num < n2 || head_num % n2) return NSA_ERR_INVALID_ARG;
+    nsa_status_t s;
+    if ((s = check_prefix(cu_q, batch)) != NSA_OK) return s;
+    if ((s = check_prefix(cu_cmp, batch)) != NSA_OK) return s;
+    // what the kernels hold: Q, dO, K, V tiles on chip together
+    const int nqc = (d1 + 63) / 64, nvc = (d2 + 63) / 64;
+    if (d1 > 256 || d2 > 256 || nqc + nvc > 6) return NSA_ERR_UNSUPPORTED;
+    if (head_num / n2 > kRows) return NSA_ERR_UNSUPPORTED;
+    pl.G = head_num / n2;
+    pl.TT = kRows / pl.G;
+    pl.one_pass = d2 <= 128;
+    const int TT = pl.TT, KV = bwd::kKV;
+
+    // shared memory (one CTA per SM: the kernels take all 512 tensor-memory columns)
+    int off = 0;
+    pl.off_q = off;
+    off += nqc * 16384;
+    pl.off_do = off;
+    off += nvc * 16384;
+    pl.off_k = off;
+    off += nqc * 16384;
+    pl.off_v = off;
+    off += nvc * 16384;
+    pl.off_row = off;
+    off += kRows * 12;
+    pl.off_bar = (off + 127) & ~127;
+    pl.smem_bytes = std::max(pl.off_bar + 128 + 1024, 116 * 1024);
+    if (pl.smem_bytes > kSmemLimit) return NSA_ERR_UNSUPPORTED;
+
+    // total dK/dV work in M-tile steps, to size the runs: about four runs per SM
+    auto first_row = [&](int kt, int64_t off_b) { return (int64_t)kt * KV * d + l - 1 - off_b; };
+    int64_t steps = 0, nq = 0;
+    {
+        int32_t pq = 0, pc = 0;
+        for (int b = 0; b < batch; ++b) {
+            const int64_t Sq = cu_q[b] - pq;
+            const int n_cmp = cu_cmp[b] - pc;
+            const int64_t off_b = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
+            nq += (Sq + TT - 1) / TT;
+            for (int kt = 0; kt * KV < n_cmp; ++kt) {
+                const int64_t rows = Sq - std::max<int64_t>(0, first_row(kt, off_b));
+                if (rows > 0) steps += (rows + TT - 1) / TT;
+            }
+            pq = cu_q[b];
+            pc = cu_cmp[b];
+        }
+    }
+    steps *= n2;
+    nq *= n2;
+    if (nq > ((int64_t)1 << 30)) return NSA_ERR_UNSUPPORTED;
+    const int64_t run = std::max<int64_t>(8, (steps + 4 * kMaxGrid - 1) / (4 * kMaxGrid));   // M-tiles per run
+
+    pl.qitems.clear();
+    pl.kvitems.clear();
+    pl.kvtiles.clear();
+    pl.nslots = 0;
+    int64_t nkvitems = 0, nkvtiles = 0, nslots = 0;
+    {
+        int32_t pq = 0, pc = 0;
+        for (int b = 0; b < batch; ++b) {
+            const int Sq = cu_q[b] - pq;
+            const int n_cmp = cu_cmp[b] - pc;
+            const int64_t off_b = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
+            for (int g = 0; g < n2; ++g) {
+                if (build)
+                    for (int tok0 = 0; tok0 < Sq; tok0 += TT) {
+                        bwd::QItem it;
+                        it.q_row0 = pq + tok0;
+                        it.ntok = std::min(TT, Sq - tok0);
+                        it.group = g;
+                        it.cmp_row0 = pc;
+                        it.n_cmp = n_cmp;
+                        it.t0 = (int)(tok0 + off_b);
+                        const int nv = nvis_host(it.t0 + it.ntok - 1, l, d, n_cmp);
+                        it.nkv = (nv + KV - 1) / KV;
+                        pl.qitems.push_back(it);
+                    }
+                for (int kt = 0; kt * KV < n_cmp; ++kt) {
+                    const int64_t tl0 = std::max<int64_t>(0, first_row(kt, off_b));
+                    const int64_t rows = std::max<int64_t>(0, Sq - tl0);
+                    const int64_t nmt = (rows + TT - 1) / TT;
+                    const int64_t nrun = (nmt + run - 1) / run;
+                    if (build) {
+                        bwd::KVTile t{pc, kt, n_cmp, g, (int)nslots, (int)nrun};
+                        pl.kvtiles.push_back(t);
+                        for (int64_t r = 0; r < nrun; ++r) {
+                            bwd::KVItem it;
+                            it.cmp_row0 = pc;
+                            it.kt = kt;
+                            it.n_cmp = n_cmp;
+                            it.group = g;
+                            it.q_row0 = (int)(pq + tl0 + r * run * TT);
+                            it.q_end = (int)std::min<int64_t>(pq + Sq, it.q_row0 + run * TT);
+                            it.t0 = (int)(tl0 + r * run * TT + off_b);
+                            it.slot = (int)(nslots + r);
+                            pl.kvitems.push_back(it);
+                        }
+                    }
+                    nslots += nrun;
+                    nkvitems += nrun;
+                    ++nkvtiles;
+                }
+            }
+            pq = cu_q[b];
+            pc = cu_cmp[b];
+        }
+    }
+    if (nslots > ((int64_t)1 << 24)) return NSA_ERR_UNSUPPORTED;
+    pl.nslots = (int)nslots;
+    if (build) {
+        // longest first (the hardware hands CTAs out roughly in index order)
+        std::stable_sort(pl.qitems.begin(), pl.qitems.end(),
+                         [](const bwd::QItem& x, const bwd::QItem& y) { return x.nkv > y.nkv; });
+        std::stable_sort(pl.kvitems.begin(), pl.kvitems.end(), [](const bwd::KVItem& x, const bwd::KVItem& y) {
+            return x.q_end - x.q_row0 > y.q_end - y.q_row0;
+        });
+    }
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const int64_t t1 = cu_q[batch - 1];
+    pl.off_qitems = kWsHeader;
+    pl.off_kvitems = pl.off_qitems + up((size_t)nq * sizeof(bwd::QItem));
+    pl.off_kvtiles = pl.off_kvitems + up((size_t)nkvitems * sizeof(bwd::KVItem));
+    pl.off_rowinfo = pl.off_kvtiles + up((size_t)nkvtiles * sizeof(bwd::KVTile));
+    pl.off_part = pl.off_rowinfo + up((size_t)t1 * head_num * sizeof(float2));
+    pl.ws_total = pl.off_part + up((size_t)nslots * bwd::kKV * (d1 + d2) * sizeof(float));
+    return NSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -830,6 +977,204 @@ nsa_status_t nsa_select_attention(const void* q, const void* k, const void* v, c
     if (sel::launch_plan(p, pl.max_words, st) != cudaSuccess) return NSA_ERR_CUDA;
     const int grid = std::min(pl.grid, nsm);
     if (sel::launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention_backward_workspace_size(int head_num, int n2, int d1, int d2, int l, int d,
+                                                            const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv,
+                                                            int batch, size_t* bytes) {
+    if (bytes == nullptr) return NSA_ERR_INVALID_ARG;
+    BwdPlan pl;
+    nsa_status_t s = plan_backward(head_num, n2, d1, d2, l, d, cu_seqlens_q, cu_cmp_kv, batch, false, pl);
+    if (s != NSA_OK) return s;
+    *bytes = pl.ws_total;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_attention_backward(const void* q, const void* kcmp, const void* vcmp,
+                                             const void* attention_out, const void* dout, const float* softmax_max,
+                                             const float* softmax_sum, float scale, int head_num, int l, int d,
+                                             const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, int batch,
+                                             int n2, int d1, int d2, nsa_dtype_t dtype, float* dq, float* dkcmp,
+                                             float* dvcmp, void* workspace, size_t workspace_bytes, void* stream) {
+    if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, kcmp, vcmp, attention_out, dout, softmax_max, softmax_sum, dq, dkcmp, dvcmp};
+    for (const void* ptr : ptrs)
+        if (ptr == nullptr || !aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+    BwdPlan pl;
+    nsa_status_t s = plan_backward(head_num, n2, d1, d2, l, d, cu_seqlens_q, cu_cmp_kv, batch, true, pl);
+    if (s != NSA_OK) return s;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < pl.ws_total)
+        return NSA_ERR_WORKSPACE;
+    const int64_t t1 = cu_seqlens_q[batch - 1];
+    const int64_t tc = cu_cmp_kv[batch - 1];
+    if (t1 == 0 && tc == 0) return NSA_OK;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    CUtensorMap tq, tdo, tk, tv;
+    if (!encode_tnd(&tq, q, dtype, d1, head_num, t1, pl.G, pl.TT) ||
+        !encode_tnd(&tdo, dout, dtype, d2, head_num, t1, pl.G, pl.TT) ||
+        !encode_tnd(&tk, kcmp, dtype, d1, n2, tc, 1, bwd::kKV) ||
+        !encode_tnd(&tv, vcmp, dtype, d2, n2, tc, 1, bwd::kKV))
+        return NSA_ERR_UNSUPPORTED;
+
+    // workspace: [header: error word][dQ items][dK/dV runs][KV tiles][row info][partial slots]
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    std::vector<uint8_t> host(pl.off_rowinfo, 0);
+    auto put = [&](size_t at, const void* src, size_t n) {
+        if (n) std::memcpy(host.data() + at, src, n);
+    };
+    put(pl.off_qitems, pl.qitems.data(), pl.qitems.size() * sizeof(bwd::QItem));
+    put(pl.off_kvitems, pl.kvitems.data(), pl.kvitems.size() * sizeof(bwd::KVItem));
+    put(pl.off_kvtiles, pl.kvtiles.data(), pl.kvtiles.size() * sizeof(bwd::KVTile));
+    if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+
+    bwd::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.qitems = reinterpret_cast<const bwd::QItem*>(ws + pl.off_qitems);
+    p.n_qitems = (int)pl.qitems.size();
+    p.kvitems = reinterpret_cast<const bwd::KVItem*>(ws + pl.off_kvitems);
+    p.n_kvitems = (int)pl.kvitems.size();
+    p.err = reinterpret_cast<int*>(ws);
+    p.rowinfo = reinterpret_cast<const float2*>(ws + pl.off_rowinfo);
+    p.dq = dq;
+    p.part = reinterpret_cast<float*>(ws + pl.off_part);
+    p.dtype = dtype == NSA_BF16 ? 0 : 1;
+    p.n1 = head_num;
+    p.n2 = n2;
+    p.d1 = d1;
+    p.d2 = d2;
+    p.G = pl.G;
+    p.tok_per_tile = pl.TT;
+    p.l = l;
+    p.d = d;
+    p.scale = scale;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.off_q = pl.off_q;
+    p.off_do = pl.off_do;
+    p.off_k = pl.off_k;
+    p.off_v = pl.off_v;
+    p.off_row = pl.off_row;
+    p.off_bar = pl.off_bar;
+    p.smem_bytes = pl.smem_bytes;
+
+    if (bwd::launch_prep(attention_out, dout, softmax_max, softmax_sum,
+                         reinterpret_cast<float2*>(ws + pl.off_rowinfo), t1 * head_num, d2, p.dtype,
+                         st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    if (bwd::launch_dq(p, tq, tdo, tk, tv, st) != cudaSuccess) return NSA_ERR_CUDA;
+    // dV and dK together when both accumulators fit beside the 128 score
+    // columns; else one pass for each
+    const int npass = pl.one_pass ? 1 : 2;
+    for (int i = 0; i < npass; ++i) {
+        p.mode = pl.one_pass ? 3 : 1 + i;   // bit 0 dV, bit 1 dK
+        p.col_dk = pl.one_pass ? 128 : 0;
+        if (bwd::launch_dkdv(p, tq, tdo, tk, tv, st) != cudaSuccess) return NSA_ERR_CUDA;
+    }
+    if (bwd::launch_reduce(reinterpret_cast<const bwd::KVTile*>(ws + pl.off_kvtiles), (int)pl.kvtiles.size(),
+                           p.part, dkcmp, dvcmp, n2, d1, d2, scale, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_backward_workspace_size(const int32_t* cu_seqlens, int batch, int l, int d,
+                                                  size_t* bytes) {
+    if (bytes == nullptr || l < 1 || d < 1) return NSA_ERR_INVALID_ARG;
+    nsa_status_t s = check_prefix(cu_seqlens, batch);
+    if (s != NSA_OK) return s;
+    int64_t tc = 0;
+    int32_t prev = 0;
+    for (int b = 0; b < batch; ++b) {
+        tc += ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
+        prev = cu_seqlens[b];
+    }
+    *bytes = kWsHeader + (((size_t)tc * 4 + 255) & ~(size_t)255);
+    return NSA_OK;
+}
+
+nsa_status_t nsa_compress_backward(const void* k, const void* v, const void* w, const float* dkcmp,
+                                   const float* dvcmp, int l, int d, const int32_t* cu_seqlens, int batch, int n2,
+                                   int d1, int d2, nsa_dtype_t dtype, float* dk, float* dv, float* dw,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    // the forward's constraints (aclnnNsaCompress)
+    if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
+    if (!k || !w || !dkcmp || !dk || !dw) return NSA_ERR_INVALID_ARG;
+    const bool has_v = v != nullptr;
+    if (has_v != (dvcmp != nullptr) || has_v != (dv != nullptr)) return NSA_ERR_INVALID_ARG;
+    if (l % 16 || d % 16 || d < 16 || l < d || l > 128) return NSA_ERR_INVALID_ARG;
+    if (n2 < 1 || d1 < 16 || d1 % 16 || d1 > 256) return NSA_ERR_INVALID_ARG;
+    if (has_v && (d2 < 16 || d2 % 16 || d2 > 256)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(dkcmp) || !aligned16(dk) ||
+        (has_v && (!aligned16(v) || !aligned16(dvcmp) || !aligned16(dv))))
+        return NSA_ERR_INVALID_ARG;
+    size_t need = 0;
+    nsa_status_t s = nsa_compress_backward_workspace_size(cu_seqlens, batch, l, d, &need);
+    if (s != NSA_OK) return s;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return NSA_ERR_WORKSPACE;
+    if ((int64_t)cu_seqlens[batch - 1] * n2 * std::max(d1, has_v ? d2 : 0) > ((int64_t)1 << 40))
+        return NSA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // first raw row of every compressed row, for the dw reduction
+    std::vector<int32_t> cmp_raw;
+    int32_t prev = 0;
+    for (int b = 0; b < batch; ++b) {
+        const int64_t nc = ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
+        for (int64_t i = 0; i < nc; ++i) cmp_raw.push_back((int32_t)(prev + i * d));
+        prev = cu_seqlens[b];
+    }
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    std::vector<uint8_t> host(kWsHeader + cmp_raw.size() * 4, 0);
+    if (!cmp_raw.empty()) std::memcpy(host.data() + kWsHeader, cmp_raw.data(), cmp_raw.size() * 4);
+    if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+
+    bwd::CompressBwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k;
+    p.v = v;
+    p.w = w;
+    p.dkcmp = dkcmp;
+    p.dvcmp = dvcmp;
+    p.dk = dk;
+    p.dv = dv;
+    p.dw = dw;
+    p.cmp_raw = reinterpret_cast<const int*>(ws + kWsHeader);
+    p.tc = (long long)cmp_raw.size();
+    p.l = l;
+    p.d = d;
+    p.n2 = n2;
+    p.d1 = d1;
+    p.d2 = has_v ? d2 : 0;
+    p.dtype = dtype == NSA_BF16 ? 0 : 1;
+
+    // dk, dv: sequences in batches of the parameter block's capacity
+    prev = 0;
+    int64_t cmp_prev = 0;
+    int b = 0;
+    while (b < batch) {
+        p.nseq = 0;
+        int blocks = 0;
+        for (; b < batch && p.nseq < kCompressMaxSeq; ++b) {
+            const int64_t S = (int64_t)cu_seqlens[b] - prev;
+            const int64_t nc = ncmp_of(S, l, d);
+            bwd::CompressBwdSeq& q = p.seq[p.nseq];
+            q.raw_start = prev;
+            q.raw_len = (int)S;
+            q.cmp_start = (int)cmp_prev;
+            q.n_cmp = (int)nc;
+            blocks += (int)((S + bwd::kRowsPerCta - 1) / bwd::kRowsPerCta);
+            q.blk_end = blocks;
+            prev = cu_seqlens[b];
+            cmp_prev += nc;
+            ++p.nseq;
+        }
+        if (blocks > 0 && bwd::launch_compress_bwd_dx(p, blocks, st) != cudaSuccess) return NSA_ERR_CUDA;
+    }
+    if (bwd::launch_compress_bwd_dw(p, st) != cudaSuccess) return NSA_ERR_CUDA;
     return NSA_OK;
 }
 

@@ -1,0 +1,633 @@
+// nsa_backward.cu -- gradients of compressed attention and of the compression
+// (sm_100a).
+//
+// The pages return softmax_max / softmax_sum "for gradient backprop"
+// ("mindspore.ops.nsa_compress_attention", Returns list; the softmax_lse of
+// "lite_boost.ops.rain_fusion_attention") and place the compression in the
+// training scenario ("aclnnNsaCompress", operator description), but print no
+// backward formulas.  They follow from the forward definition (steps 1-3; the
+// importance scores and the top-k are index outputs and carry no gradient):
+//   P_i  = exp(s_i - m) / L,  s_i = scale q . kcmp_i   (visible blocks)
+//   dV_i = sum over rows of P_i dout           (summed over the G heads of a group)
+//   dP_i = dout . vcmp_i,  delta = sum_i P_i dP_i = dout . out
+//   dS_i = P_i (dP_i - delta)
+//   dq   = scale sum_i dS_i kcmp_i,   dK_i = scale sum over rows of dS_i q
+// and for the compression kcmp_i = sum_j w_j k[i d + j] (linear):
+//   dk[p] = sum_i w[p - i d] dkcmp_i,   dw_j = sum_i dkcmp_i . k[i d + j]  (+ the V terms).
+//
+// Kernels:
+//   prep     per (row, head): delta = out . dout and the log2 normaliser
+//            m log2e + log2 L from the saved statistics.
+//   dq       one query M-tile (TT tokens x G heads) over its visible KV tiles
+//            of 128 blocks: S = Q K^T and dP = dO V^T by tcgen05.mma into
+//            tensor memory; the softmax warps (one row each) write dS in the
+//            storage dtype over S; dQ += dS K with dS read from tensor memory.
+//   dkdv     one KV tile of one group over the query M-tiles that see it, in
+//            halves of 64 rows: S^T = K Q^T and dP^T = V dO^T; P^T and dS^T
+//            over them; dV += P^T dO and dK += dS^T Q.  The rows of an M-tile
+//            are the G heads of the group, so the sums over the heads come out
+//            of the contraction.  Each tile's dK, dV are written once: no
+//            atomics, deterministic.
+//   dx / dw  the compression transposed: dk / dv gathered per raw row from the
+//            windows that cover it; dw reduced per (window position, head) over
+//            every compressed row in a fixed order.
+// One work item per CTA, the MMA steps issued in order and waited for (a first
+// form, correct before fast).  Every mbarrier wait is bounded and reports a
+// timeout in the workspace error word.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "nsa_internal.h"
+#include "ptx.cuh"
+
+namespace nsa {
+namespace bwd {
+
+template <typename T>
+__device__ __forceinline__ uint32_t pk2(float lo, float hi);
+template <>
+__device__ __forceinline__ uint32_t pk2<__nv_bfloat16>(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pk2<__half>(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <typename T>
+__device__ __forceinline__ float2 up2(uint32_t w);
+template <>
+__device__ __forceinline__ float2 up2<__nv_bfloat16>(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w));
+}
+template <>
+__device__ __forceinline__ float2 up2<__half>(uint32_t w) {
+    return __half22float2(*reinterpret_cast<__half2*>(&w));
+}
+
+__device__ __forceinline__ int nvis_at(int t, int l, int d, int n_cmp) {
+    // compressed block i is visible to position t iff i*d + l - 1 <= t
+    if (t < l - 1) return 0;
+    return min(n_cmp, (t - l + 1) / d + 1);
+}
+
+enum Bar { B_Q = 0, B_KV, B_S, B_P, B_MMA, B_DONE, B_N };
+
+// ------------------------------------------------------------------- prep
+// One warp per row: delta = sum_e out * dout (fp32) and the row's log2
+// normaliser; rows that attended to nothing (L = 0) get +inf, so P = 0.
+template <typename T>
+__global__ void prep_kernel(const T* __restrict__ out, const T* __restrict__ dout, const float* __restrict__ smax,
+                            const float* __restrict__ ssum, float2* __restrict__ rowinfo, long long rows, int d2) {
+    const int lane = threadIdx.x & 31;
+    const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    for (long long r = w0; r < rows; r += nw) {
+        float acc = 0.f;
+        for (int e = lane * 8; e < d2; e += 256) {
+            const uint4 ov = *reinterpret_cast<const uint4*>(out + r * d2 + e);
+            const uint4 gv = *reinterpret_cast<const uint4*>(dout + r * d2 + e);
+            const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 a = up2<T>(ow[k]), b = up2<T>(gw[k]);
+                acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            const float m = smax[r * 8], L = ssum[r * 8];
+            const float mb = (L > 0.f && m > -INFINITY) ? m * 1.4426950408889634f + log2f(L) : INFINITY;
+            rowinfo[r] = make_float2(mb, acc);
+        }
+    }
+}
+
+cudaError_t launch_prep(const void* out, const void* dout, const float* smax, const float* ssum, float2* rowinfo,
+                        long long rows, int d2, int dtype, cudaStream_t st) {
+    if (rows <= 0) return cudaSuccess;
+    const int threads = 256;   // eight rows at a time per CTA
+    const int blocks = (int)std::min<long long>((rows + 7) / 8, 148LL * 16);
+    if (dtype == 0)
+        prep_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(out), reinterpret_cast<const __nv_bfloat16*>(dout), smax, ssum,
+            rowinfo, rows, d2);
+    else
+        prep_kernel<__half><<<blocks, threads, 0, st>>>(reinterpret_cast<const __half*>(out),
+                                                        reinterpret_cast<const __half*>(dout), smax, ssum, rowinfo,
+                                                        rows, d2);
+    return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- shared
+struct Smem {
+    uint8_t* base;
+    uint64_t* bars;
+    uint32_t* tmem_slot;
+    volatile int* abort_flag;
+};
+
+__device__ __forceinline__ Smem smem_setup(const Params& p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem s;
+    s.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    s.bars = reinterpret_cast<uint64_t*>(s.base + p.off_bar);
+    s.tmem_slot = reinterpret_cast<uint32_t*>(s.base + p.off_bar + 8 * B_N);
+    s.abort_flag = reinterpret_cast<volatile int*>(s.base + p.off_bar + 8 * B_N + 4);
+    return s;
+}
+
+// 128 rows x 16 fp32 columns of this warp's lanes -> fp32 global row (x mul)
+__device__ __forceinline__ void store_row_f32(uint32_t taddr, int ncols, float mul, float* dst, bool valid) {
+    for (int c = 0; c < ncols; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c, r);
+        tmem_wait_ld_regs<16>(r);
+        if (valid) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                d4[q] = make_float4(__uint_as_float(r[4 * q]) * mul, __uint_as_float(r[4 * q + 1]) * mul,
+                                    __uint_as_float(r[4 * q + 2]) * mul, __uint_as_float(r[4 * q + 3]) * mul);
+        }
+    }
+}
+
+// --------------------------------------------------------------------- dQ
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    Smem sm = smem_setup(p);
+    auto bar = [&](int id) { return smem_u32(&sm.bars[id]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const QItem it = p.qitems[blockIdx.x];
+    const int G = p.G, TT = p.tok_per_tile;
+    const int nqc = (p.d1 + 63) / 64, nvc = (p.d2 + 63) / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P) ? 4 : 1);
+        *sm.abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 4) {
+        tmem_alloc(smem_u32(sm.tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sm.tmem_slot;   // S at 0, dP at 128, dQ at 256
+    const uint32_t qa = smem_u32(sm.base + p.off_q), doa = smem_u32(sm.base + p.off_do);
+    const uint32_t ka = smem_u32(sm.base + p.off_k), va = smem_u32(sm.base + p.off_v);
+
+    if (warp == 4) {
+        if (lane == 0) {
+            const uint32_t qbytes = nqc * 64 * G * TT * 2, dobytes = nvc * 64 * G * TT * 2;
+            const uint32_t kbytes = nqc * 64 * kKV * 2, vbytes = nvc * 64 * kKV * 2;
+            constexpr uint32_t id_s = idesc_f16(kBF16, 128, kKV, false, false);
+            const uint32_t id_q = idesc_f16(kBF16, 128, p.d1, false, true);
+            bool ok = true;
+            mbar_arrive_expect_tx(bar(B_Q), qbytes + dobytes);
+            for (int c = 0; c < nqc; ++c) tma_load_3d(qa + c * 16384, &tm_q, c * 64, it.group * G, it.q_row0, bar(B_Q));
+            for (int c = 0; c < nvc; ++c)
+                tma_load_3d(doa + c * 16384, &tm_do, c * 64, it.group * G, it.q_row0, bar(B_Q));
+            for (int i = 0; i < it.nkv && ok; ++i) {
+                const int row = it.cmp_row0 + i * kKV;
+                mbar_arrive_expect_tx(bar(B_KV), kbytes + vbytes);
+                for (int c = 0; c < nqc; ++c) tma_load_3d(ka + c * 16384, &tm_k, c * 64, it.group, row, bar(B_KV));
+                for (int c = 0; c < nvc; ++c) tma_load_3d(va + c * 16384, &tm_v, c * 64, it.group, row, bar(B_KV));
+                ok = mbar_wait(bar(B_KV), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x21);
+                if (i == 0) ok = ok && mbar_wait(bar(B_Q), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x22);
+                if (!ok) break;
+                tc_fence_after();
+                for (int ks = 0; ks < p.d1 / 16; ++ks) {   // S = Q K^T
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_ss(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id_s,
+                            ks > 0 ? 1u : 0u);
+                }
+                for (int ks = 0; ks < p.d2 / 16; ++ks) {   // dP = dO V^T
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_ss(tmem + 128, sdesc_sw128(doa + off, 16, 1024), sdesc_sw128(va + off, 16, 1024), id_s,
+                            ks > 0 ? 1u : 0u);
+                }
+                umma_commit(bar(B_S));
+                ok = mbar_wait(bar(B_P), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x23);
+                if (!ok) break;
+                tc_fence_after();
+                for (int ks = 0; ks < kKV / 16; ++ks)   // dQ += dS K (dS from tensor memory)
+                    umma_ts(tmem + 256, tmem + ks * 8, sdesc_sw128(ka + ks * 2048, kKV * 128, 1024), id_q,
+                            (i > 0 || ks > 0) ? 1u : 0u);
+                umma_commit(bar(B_MMA));
+                ok = mbar_wait(bar(B_MMA), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x24);
+            }
+        }
+    } else {
+        // one query row per thread
+        const int row = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int tok = row / G, h = row % G;
+        const bool valid = row < TT * G && tok < it.ntok;
+        const int nv = valid ? nvis_at(it.t0 + tok, p.l, p.d, it.n_cmp) : 0;
+        const size_t ri = ((size_t)(it.q_row0 + tok) * p.n1 + (size_t)it.group * G + h);
+        const float2 info = valid ? p.rowinfo[ri] : make_float2(INFINITY, 0.f);
+        const float c2 = p.scale_log2;
+        for (int i = 0; i < it.nkv; ++i) {
+            mbar_wait(bar(B_S), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x25);
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < kKV / 32; ++c) {
+                uint32_t rs[32], rp[32];
+                tmem_ld32(tmem + lane_off + c * 32, rs);
+                tmem_ld32(tmem + lane_off + 128 + c * 32, rp);
+                tmem_wait_ld_regs<32>(rs);
+                tmem_wait_ld_regs<32>(rp);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int kb = i * kKV + c * 32 + e;
+                    const bool v0 = kb < nv, v1 = kb + 1 < nv;
+                    const float p0 = v0 ? ex2(__uint_as_float(rs[e]) * c2 - info.x) : 0.f;
+                    const float p1 = v1 ? ex2(__uint_as_float(rs[e + 1]) * c2 - info.x) : 0.f;
+                    pk[e >> 1] = pk2<T>(v0 ? p0 * (__uint_as_float(rp[e]) - info.y) : 0.f,
+                                        v1 ? p1 * (__uint_as_float(rp[e + 1]) - info.y) : 0.f);
+                }
+                tmem_st16(tmem + lane_off + c * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_P));
+        }
+        float* dst = p.dq + ri * p.d1;
+        if (it.nkv > 0) {
+            mbar_wait(bar(B_MMA), (it.nkv - 1) & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x26);
+            tc_fence_after();
+            store_row_f32(tmem + lane_off + 256, p.d1, p.scale, dst, valid);
+        } else if (valid) {
+            for (int e = 0; e < p.d1; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*sm.abort_flag && threadIdx.x == 0) {
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {
+        }
+    }
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ dK, dV
+// Query rows are the contraction dimension of dV += P^T dO and dK += dS^T Q,
+// so every row that takes part must hold finite values: rows of the box past
+// G x TT are zeroed once, rows outside the run get P = dS = 0 by selection.
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    Smem sm = smem_setup(p);
+    auto bar = [&](int id) { return smem_u32(&sm.bars[id]); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const KVItem it = p.kvitems[blockIdx.x];
+    const int G = p.G, TT = p.tok_per_tile;
+    const int nqc = (p.d1 + 63) / 64, nvc = (p.d2 + 63) / 64;
+    const bool do_dv = p.mode & 1, do_dk = (p.mode >> 1) & 1;
+    const int n_mt = (it.q_end - it.q_row0 + TT - 1) / TT;   // query M-tiles of the run
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P) ? 4 : 1);
+        *sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    {
+        // rows G*TT..127 of every Q / dO chunk: never written by the copies
+        const int r0 = G * TT;
+        const int nch = nqc + nvc;
+        const int per = (128 - r0) * 8;   // 16-byte pieces per chunk
+        for (int x = threadIdx.x; x < nch * per; x += blockDim.x) {
+            const int c = x / per, o = x % per;
+            uint8_t* base = sm.base + (c < nqc ? p.off_q + c * 16384 : p.off_do + (c - nqc) * 16384);
+            *reinterpret_cast<uint4*>(base + r0 * 128 + o * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
+    if (warp == 4) {
+        tmem_alloc(smem_u32(sm.tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sm.tmem_slot;   // dV at 0, dK at col_dk, S^T at 384, dP^T at 448
+    const uint32_t qa = smem_u32(sm.base + p.off_q), doa = smem_u32(sm.base + p.off_do);
+    const uint32_t ka = smem_u32(sm.base + p.off_k), va = smem_u32(sm.base + p.off_v);
+    float2* rinfo = reinterpret_cast<float2*>(sm.base + p.off_row);   // the M-tile's 128 rows
+    int* rnv = reinterpret_cast<int*>(sm.base + p.off_row + 128 * sizeof(float2));
+
+    if (warp == 4) {
+        if (lane == 0) {
+            const uint32_t qbytes = nqc * 64 * G * TT * 2, dobytes = nvc * 64 * G * TT * 2;
+            const uint32_t kbytes = nqc * 64 * kKV * 2, vbytes = do_dk ? nvc * 64 * kKV * 2 : 0;
+            constexpr uint32_t id_s = idesc_f16(kBF16, 128, 64, false, false);
+            const uint32_t id_v = idesc_f16(kBF16, 128, p.d2, false, true);
+            const uint32_t id_k = idesc_f16(kBF16, 128, p.d1, false, true);
+            bool ok = true;
+            const int krow = it.cmp_row0 + it.kt * kKV;
+            mbar_arrive_expect_tx(bar(B_KV), kbytes + vbytes);
+            for (int c = 0; c < nqc; ++c) tma_load_3d(ka + c * 16384, &tm_k, c * 64, it.group, krow, bar(B_KV));
+            if (do_dk)
+                for (int c = 0; c < nvc; ++c) tma_load_3d(va + c * 16384, &tm_v, c * 64, it.group, krow, bar(B_KV));
+            ok = mbar_wait(bar(B_KV), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x31);
+            for (int mi = 0; mi < n_mt && ok; ++mi) {
+                const int row0 = it.q_row0 + mi * TT;
+                mbar_arrive_expect_tx(bar(B_Q), qbytes + dobytes);
+                for (int c = 0; c < nqc; ++c) tma_load_3d(qa + c * 16384, &tm_q, c * 64, it.group * G, row0, bar(B_Q));
+                for (int c = 0; c < nvc; ++c)
+                    tma_load_3d(doa + c * 16384, &tm_do, c * 64, it.group * G, row0, bar(B_Q));
+                ok = mbar_wait(bar(B_Q), mi & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x32);
+                for (int hf = 0; hf < 2 && ok; ++hf) {
+                    const int step = mi * 2 + hf;
+                    tc_fence_after();
+                    for (int ks = 0; ks < p.d1 / 16; ++ks) {   // S^T = K Q^T over 64 query rows
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        umma_ss(tmem + 384, sdesc_sw128(ka + off, 16, 1024),
+                                sdesc_sw128(qa + off + hf * 8192, 16, 1024), id_s, ks > 0 ? 1u : 0u);
+                    }
+                    if (do_dk)
+                        for (int ks = 0; ks < p.d2 / 16; ++ks) {   // dP^T = V dO^T
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            umma_ss(tmem + 448, sdesc_sw128(va + off, 16, 1024),
+                                    sdesc_sw128(doa + off + hf * 8192, 16, 1024), id_s, ks > 0 ? 1u : 0u);
+                        }
+                    umma_commit(bar(B_S));
+                    ok = mbar_wait(bar(B_P), step & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x33);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 64 / 16; ++ks) {
+                        // the 64 query rows of the half are the contraction dimension: the
+                        // row-major dO / Q chunks serve as MN-major operands
+                        if (do_dv)
+                            umma_ts(tmem, tmem + 384 + ks * 8, sdesc_sw128(doa + hf * 8192 + ks * 2048, 16384, 1024),
+                                    id_v, (step > 0 || ks > 0) ? 1u : 0u);
+                        if (do_dk)
+                            umma_ts(tmem + p.col_dk, tmem + 448 + ks * 8,
+                                    sdesc_sw128(qa + hf * 8192 + ks * 2048, 16384, 1024), id_k,
+                                    (step > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar(B_MMA));
+                    ok = mbar_wait(bar(B_MMA), step & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x34);
+                }
+            }
+            mbar_arrive(bar(B_DONE));
+        }
+    } else {
+        // one key (compressed block) of the tile per thread
+        const int kr = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int kb = it.kt * kKV + kr;   // block index inside the sequence
+        const bool kvalid = kb < it.n_cmp;
+        const float c2 = p.scale_log2;
+        for (int mi = 0; mi < n_mt; ++mi) {
+            const int row0 = it.q_row0 + mi * TT;
+            named_bar_sync(1, 128);   // the previous M-tile's rows are no longer read
+            {
+                const int tok = kr / G, h = kr % G;
+                const bool valid = kr < TT * G && row0 + tok < it.q_end;
+                const int tpos = it.t0 + (row0 - it.q_row0) + tok;
+                rinfo[kr] = valid ? p.rowinfo[(size_t)(row0 + tok) * p.n1 + (size_t)it.group * G + h]
+                                  : make_float2(INFINITY, 0.f);
+                rnv[kr] = valid ? nvis_at(tpos, p.l, p.d, it.n_cmp) : 0;
+            }
+            named_bar_sync(1, 128);
+            for (int hf = 0; hf < 2; ++hf) {
+                const int step = mi * 2 + hf;
+                mbar_wait(bar(B_S), step & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x35);
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t rs[32], rp[32];
+                    tmem_ld32(tmem + lane_off + 384 + c * 32, rs);
+                    if (do_dk) tmem_ld32(tmem + lane_off + 448 + c * 32, rp);
+                    tmem_wait_ld_regs<32>(rs);
+                    if (do_dk) tmem_wait_ld_regs<32>(rp);
+                    uint32_t ppk[16], dpk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int r = hf * 64 + c * 32 + e;
+                        const float2 i0 = rinfo[r], i1 = rinfo[r + 1];
+                        const bool v0 = kvalid && kb < rnv[r], v1 = kvalid && kb < rnv[r + 1];
+                        const float p0 = v0 ? ex2(__uint_as_float(rs[e]) * c2 - i0.x) : 0.f;
+                        const float p1 = v1 ? ex2(__uint_as_float(rs[e + 1]) * c2 - i1.x) : 0.f;
+                        ppk[e >> 1] = pk2<T>(p0, p1);
+                        if (do_dk)
+                            dpk[e >> 1] = pk2<T>(v0 ? p0 * (__uint_as_float(rp[e]) - i0.y) : 0.f,
+                                                 v1 ? p1 * (__uint_as_float(rp[e + 1]) - i1.y) : 0.f);
+                    }
+                    if (do_dv) tmem_st16(tmem + lane_off + 384 + c * 16, ppk);
+                    if (do_dk) tmem_st16(tmem + lane_off + 448 + c * 16, dpk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_P));
+            }
+        }
+        mbar_wait(bar(B_DONE), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x36);
+        tc_fence_after();
+        // the run's partial sums; a run with no M-tile leaves zeros
+        float* dst = p.part + ((size_t)it.slot * 128 + kr) * (p.d1 + p.d2);
+        if (n_mt > 0) {
+            if (do_dv) store_row_f32(tmem + lane_off, p.d2, 1.f, dst, true);
+            if (do_dk) store_row_f32(tmem + lane_off + p.col_dk, p.d1, 1.f, dst + p.d2, true);
+        } else {
+            if (do_dv)
+                for (int e = 0; e < p.d2; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (do_dk)
+                for (int e = 0; e < p.d1; e += 4)
+                    *reinterpret_cast<float4*>(dst + p.d2 + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*sm.abort_flag && threadIdx.x == 0) {
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {
+        }
+    }
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// dkcmp / dvcmp of one KV tile: its partial slots summed in slot order (a
+// fixed order, so the result does not depend on the schedule); dK x scale.
+__global__ void reduce_kernel(const KVTile* __restrict__ tiles, const float* __restrict__ part,
+                              float* __restrict__ dkcmp, float* __restrict__ dvcmp, int n2, int d1, int d2,
+                              float scale) {
+    const KVTile t = tiles[blockIdx.x];
+    const int w = d1 + d2, w4 = w / 4;
+    const int rows = min(kKV, t.n_cmp - t.kt * kKV);
+    for (int x = threadIdx.x; x < rows * w4; x += blockDim.x) {
+        const int r = x / w4, c = (x % w4) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < t.nslots; ++s) {
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(part + ((size_t)(t.slot0 + s) * 128 + r) * w + c));
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        const size_t row = (size_t)(t.cmp_row0 + t.kt * kKV + r) * n2 + t.group;
+        if (c < d2) {
+            *reinterpret_cast<float4*>(dvcmp + row * d2 + c) = acc;
+        } else {
+            acc = make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
+            *reinterpret_cast<float4*>(dkcmp + row * d1 + (c - d2)) = acc;
+        }
+    }
+}
+
+cudaError_t launch_reduce(const KVTile* tiles, int ntiles, const float* part, float* dkcmp, float* dvcmp, int n2,
+                          int d1, int d2, float scale, cudaStream_t st) {
+    if (ntiles <= 0) return cudaSuccess;
+    reduce_kernel<<<ntiles, 256, 0, st>>>(tiles, part, dkcmp, dvcmp, n2, d1, d2, scale);
+    return cudaGetLastError();
+}
+
+template <typename K>
+static cudaError_t launch_mma_kernel(K kern, const Params& p, int n, const CUtensorMap& tq, const CUtensorMap& tdo,
+                                     const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<n, kThreads, p.smem_bytes, st>>>(tq, tdo, tk, tv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dq(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                      const CUtensorMap& tv, cudaStream_t st) {
+    return p.dtype == 0 ? launch_mma_kernel(dq_kernel<__nv_bfloat16>, p, p.n_qitems, tq, tdo, tk, tv, st)
+                        : launch_mma_kernel(dq_kernel<__half>, p, p.n_qitems, tq, tdo, tk, tv, st);
+}
+
+cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                        const CUtensorMap& tv, cudaStream_t st) {
+    return p.dtype == 0 ? launch_mma_kernel(dkdv_kernel<__nv_bfloat16>, p, p.n_kvitems, tq, tdo, tk, tv, st)
+                        : launch_mma_kernel(dkdv_kernel<__half>, p, p.n_kvitems, tq, tdo, tk, tv, st);
+}
+
+// ---------------------------------------------------- compression transposed
+template <typename T>
+__device__ __forceinline__ float ld_elem(const void* base, size_t idx) {
+    return static_cast<float>(reinterpret_cast<const T*>(base)[idx]);
+}
+
+// dk[p] = sum_i w[p - i d] dkcmp_i over the windows i covering raw row p
+// (dv likewise).  A CTA takes kRowsPerCta raw rows of one sequence; a thread
+// one (head, 4 consecutive dims) column.
+template <typename T>
+__global__ void compress_dx_kernel(const CompressBwdParams p) {
+    int s = 0;
+    while (s + 1 < p.nseq && (int)blockIdx.x >= p.seq[s].blk_end) ++s;
+    const CompressBwdSeq q = p.seq[s];
+    const int blk0 = s ? p.seq[s - 1].blk_end : 0;
+    const int r0 = ((int)blockIdx.x - blk0) * kRowsPerCta;
+    const bool is_v = blockIdx.y == 1;
+    const int dim = is_v ? p.d2 : p.d1;
+    const float* g = is_v ? p.dvcmp : p.dkcmp;
+    float* dx = is_v ? p.dv : p.dk;
+    const int ncol = p.n2 * dim / 4;
+    for (int rr = 0; rr < kRowsPerCta; ++rr) {
+        const int pr = r0 + rr;   // raw row inside the sequence
+        if (pr >= q.raw_len) break;
+        // windows i with i d <= pr < i d + l
+        int i_lo = pr - p.l + 1 <= 0 ? 0 : (pr - p.l + 1 + p.d - 1) / p.d;
+        int i_hi = min(pr / p.d, q.n_cmp - 1);
+        for (int col = threadIdx.x; col < ncol; col += blockDim.x) {
+            const int n = (col * 4) / dim, e = (col * 4) % dim;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = i_lo; i <= i_hi; ++i) {
+                const float wv = ld_elem<T>(p.w, (size_t)(pr - i * p.d) * p.n2 + n);
+                const float4 gv = *reinterpret_cast<const float4*>(g + ((size_t)(q.cmp_start + i) * p.n2 + n) * dim + e);
+                acc.x = fmaf(wv, gv.x, acc.x);
+                acc.y = fmaf(wv, gv.y, acc.y);
+                acc.z = fmaf(wv, gv.z, acc.z);
+                acc.w = fmaf(wv, gv.w, acc.w);
+            }
+            *reinterpret_cast<float4*>(dx + ((size_t)(q.raw_start + pr) * p.n2 + n) * dim + e) = acc;
+        }
+    }
+}
+
+// dw[j, n] = sum_i (dkcmp_i . k[i d + j] + dvcmp_i . v[i d + j]) over every
+// compressed row, one CTA per (j, n), fixed-order block reduction.
+template <typename T>
+__global__ void compress_dw_kernel(const CompressBwdParams p) {
+    const int j = blockIdx.x, n = blockIdx.y;
+    const int c4k = p.d1 / 4, c4v = p.d2 / 4;
+    float acc = 0.f;
+    const long long total = p.tc * (c4k + c4v);
+    for (long long x = threadIdx.x; x < total; x += blockDim.x) {
+        const long long i = x / (c4k + c4v);
+        const int c = (int)(x - i * (c4k + c4v));
+        const bool is_v = c >= c4k;
+        const int dim = is_v ? p.d2 : p.d1;
+        const int e = (is_v ? c - c4k : c) * 4;
+        const float* g = (is_v ? p.dvcmp : p.dkcmp) + ((size_t)i * p.n2 + n) * dim + e;
+        const size_t raw = (size_t)p.cmp_raw[i] + j;
+        const void* src = is_v ? p.v : p.k;
+        const float4 gv = *reinterpret_cast<const float4*>(g);
+        const size_t xi = (raw * p.n2 + n) * dim + e;
+        acc = fmaf(gv.x, ld_elem<T>(src, xi), acc);
+        acc = fmaf(gv.y, ld_elem<T>(src, xi + 1), acc);
+        acc = fmaf(gv.z, ld_elem<T>(src, xi + 2), acc);
+        acc = fmaf(gv.w, ld_elem<T>(src, xi + 3), acc);
+    }
+    __shared__ float red[32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = (threadIdx.x < blockDim.x / 32) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (threadIdx.x == 0) p.dw[(size_t)j * p.n2 + n] = v;
+    }
+}
+
+cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaStream_t st) {
+    if (blocks <= 0) return cudaSuccess;
+    dim3 grid(blocks, p.dvcmp ? 2 : 1);
+    if (p.dtype == 0)
+        compress_dx_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);
+    else
+        compress_dx_kernel<__half><<<grid, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, cudaStream_t st) {
+    dim3 grid(p.l, p.n2);
+    if (p.dtype == 0)
+        compress_dw_kernel<__nv_bfloat16><<<grid, 512, 0, st>>>(p);
+    else
+        compress_dw_kernel<__half><<<grid, 512, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace bwd
+}  // namespace nsa

@@ -114,6 +114,86 @@ cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const C
 int attention_kv_cols(int a);     // compressed blocks per KV tile for band factor a
 int attention_chunk_cols(int a);  // score columns per softmax chunk for band factor a
 
+// ------------------------------------------------------------ backward
+// Gradients of steps 1-3 (attention_out) with respect to q, kcmp and vcmp,
+// and of the compression with respect to the raw K/V rows and w.
+namespace bwd {
+constexpr int kThreads = 160;    // warps 0-3 softmax (TMEM lane quadrants), warp 4 TMA + MMA
+constexpr int kKV = 128;         // compressed blocks per KV tile
+
+// dQ: one query M-tile (TT tokens x G heads of one group) over its KV tiles
+struct QItem {
+    int q_row0, ntok, group, cmp_row0, n_cmp, t0, nkv;
+};
+// dK/dV: one KV tile of one group over a run of the query M-tiles that see
+// it; the run's partial sums go to partial slot `slot`
+struct KVItem {
+    int cmp_row0;   // first compressed row of the sequence
+    int kt;         // KV tile index inside the sequence
+    int n_cmp;      // compressed blocks of the sequence
+    int group;
+    int q_row0;     // first query row of the run
+    int q_end;      // end of the run's query rows
+    int t0;         // position of query row q_row0 (query offset applied)
+    int slot;       // partial slot: 128 rows x (D2 + D1) fp32
+};
+// One KV tile's partial slots [slot0, slot0 + nslots), summed in order
+struct KVTile {
+    int cmp_row0, kt, n_cmp, group, slot0, nslots;
+};
+
+struct Params {
+    const QItem* qitems;
+    int n_qitems;
+    const KVItem* kvitems;
+    int n_kvitems;
+    int* err;
+    const float2* rowinfo;   // (T1, N1): log2 normaliser m*log2e + log2 L (inf: row sees nothing), delta
+    float* dq;               // (T1, N1, D1) fp32
+    float* part;             // partial slots of dK/dV: [slot][128][D2 | D1] fp32
+    int mode;                // dK/dV kernel: bit 0 dV, bit 1 dK
+    int col_dk;              // tensor-memory column of the dK accumulator
+    int dtype, n1, n2, d1, d2, G, tok_per_tile, l, d;
+    float scale, scale_log2;
+    int off_q, off_do, off_k, off_v, off_row, off_bar, smem_bytes;
+};
+
+cudaError_t launch_prep(const void* out, const void* dout, const float* smax, const float* ssum, float2* rowinfo,
+                        long long rows, int d2, int dtype, cudaStream_t st);
+cudaError_t launch_dq(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                      const CUtensorMap& tv, cudaStream_t st);
+cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                        const CUtensorMap& tv, cudaStream_t st);
+// dkcmp / dvcmp rows of every KV tile from its partial slots (dK scaled)
+cudaError_t launch_reduce(const KVTile* tiles, int ntiles, const float* part, float* dkcmp, float* dvcmp, int n2,
+                          int d1, int d2, float scale, cudaStream_t st);
+
+constexpr int kRowsPerCta = 32;   // raw rows per CTA of the compression transpose
+struct CompressBwdSeq {
+    int raw_start, raw_len, cmp_start, n_cmp;
+    int blk_end;                  // inclusive prefix of the sequences' row blocks in this launch
+};
+struct CompressBwdParams {
+    const void* k;
+    const void* v;
+    const void* w;
+    const float* dkcmp;
+    const float* dvcmp;
+    float* dk;
+    float* dv;
+    float* dw;
+    const int* cmp_raw;           // per compressed row: its first raw row (T2 index)
+    long long tc;
+    int l, d, n2, d1, d2, dtype;
+    int nseq;
+    CompressBwdSeq seq[kCompressMaxSeq];
+};
+// dk, dv for the launch's sequences (one call per batch of sequences)
+cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaStream_t st);
+// dw over every compressed row (one call)
+cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, cudaStream_t st);
+}  // namespace bwd
+
 // ------------------------------------------------ selection attention
 // Attention over the raw K/V blocks of l' tokens that the compressed branch's
 // top-k lists per (query row, KV group).  Same warp roles and register split

@@ -20,6 +20,21 @@ Tolerances (written here once, used by every parity test):
                  indices; the two index sets may differ only in indices whose
                  oracle score is within 1e-4 (relative) of the oracle's k-th
                  largest score (several answers are correct at near-ties).
+  gradients      (backward of the compressed attention) per tensor:
+                 ||gpu - oracle||_F <= 2^-7 ||oracle||_F and
+                 max |gpu - oracle| <= 2^-6 max |oracle|.
+                 The kernels recompute P in fp32 and feed P and
+                 dS = P (dP - delta) to the tensor cores in the storage dtype
+                 (relative rounding 2^-9 in bf16, 2^-12 in fp16); delta is
+                 taken from the forward's attention_out, itself rounded to the
+                 storage dtype (2^-9).  These errors are independent across
+                 the terms of each contraction, so the tensor-wide relative
+                 error stays near 2^-9; the bounds leave a factor of 4 (norm)
+                 and 8 (max) for the elements where cancellation concentrates.
+  compress grads dk, dv: at most l/d fp32 terms per element,
+                 |gpu - oracle| <= 2^-20 sum |w dkcmp|; dw: a fixed-order fp32
+                 reduction of Tc * D terms, |gpu - oracle| <= 2^-14 sum |terms|
+                 (sums of magnitudes from the oracle on |inputs|).
 """
 import numpy as np
 import torch
@@ -115,3 +130,41 @@ def check_attention(res, ref, count, rows=None, tie_rel=1e-4, out_tol=1e-2, stat
             n_tie_diff += 1
     report["topk_tie_rows"] = n_tie_diff
     return report
+
+
+def check_grad(got, ref: np.ndarray, name: str, fro: float = 2.0 ** -7, mx: float = 2.0 ** -6) -> dict:
+    """One gradient tensor against the oracle (rules in the module docstring)."""
+    g = got.double().cpu().numpy() if hasattr(got, "cpu") else np.asarray(got, dtype=np.float64)
+    assert g.shape == ref.shape, (name, g.shape, ref.shape)
+    assert np.isfinite(g).all(), f"{name}: non-finite values"
+    err = g - ref
+    nr = float(np.linalg.norm(ref))
+    rel_f = float(np.linalg.norm(err)) / max(nr, 1e-30)
+    amax = float(np.abs(ref).max()) if ref.size else 0.0
+    rel_m = float(np.abs(err).max()) / max(amax, 1e-30) if ref.size else 0.0
+    if nr == 0.0:
+        assert float(np.abs(g).max(initial=0.0)) == 0.0, f"{name}: oracle is zero, gpu is not"
+    else:
+        assert rel_f <= fro, f"{name}: relative Frobenius error {rel_f:.3e} > {fro:.3e}"
+        assert rel_m <= mx, f"{name}: max error {rel_m:.3e} of max|oracle| > {mx:.3e}"
+    return {"name": name, "rel_fro": rel_f, "rel_max": rel_m}
+
+
+def check_compress_dx(dx, x, w, dcmp, l, d, cu):
+    """dx (T, N2, D) of the compression of x for the incoming dcmp.  Returns
+    the oracle's dw of this input and its sum of magnitudes, for check_dw."""
+    ref_dx, ref_dw = oracle.compress_backward(x, w, dcmp, l, d, cu)
+    abs_dx, abs_dw = oracle.compress_backward(np.abs(oracle._f64(x)), np.abs(oracle._f64(w)),
+                                              np.abs(oracle._f64(dcmp)), l, d, cu)
+    g = dx.double().cpu().numpy()
+    err = np.abs(g - ref_dx)
+    assert (err <= 2.0 ** -20 * abs_dx).all(), float(err.max())
+    return ref_dw, abs_dw
+
+
+def check_dw(dw, parts):
+    """dw (l, N2) against the sum of the oracle's per-input parts."""
+    ref = sum(p[0] for p in parts)
+    mag = sum(p[1] for p in parts)
+    err = np.abs(dw.double().cpu().numpy() - ref)
+    assert (err <= 2.0 ** -14 * mag).all(), float(err.max())

@@ -15,6 +15,8 @@ Recipe (stated once here, repeated in the design notes):
   * cu_sel_kv: prefix sums of ceil(S_b / l') (the number of selection blocks
     of each raw sequence).
   * Short-query workloads keep the last ``q_last`` tokens of each sequence.
+  * Backward: the incoming gradient of attention_out is ``randn`` (T1, N1, D2)
+    from a generator seeded with seed + 1000, cast to the storage dtype.
 The pages name no dataset or benchmark suite; these inputs stand alone.
 """
 from __future__ import annotations
@@ -116,6 +118,14 @@ class Workload:
         del kf
         return {"q": q, "k": k, "v": v, "w": w, "cu_seqlens": cu,
                 "cu_seqlens_q": self.cu_seqlens_q(), "cu_sel_kv": self.cu_sel_kv()}
+
+
+def grad_output(wl: Workload, device: str = "cpu") -> torch.Tensor:
+    """The seeded incoming gradient of attention_out, (T1, N1, D2)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(wl.seed + 1000)
+    t1 = int(sum(wl.q_lengths()))
+    return torch.randn(t1, wl.n1, wl.d2, generator=g, device=device, dtype=torch.float32).to(wl.torch_dtype)
 
 
 def _varlen_lengths() -> tuple:
