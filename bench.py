@@ -44,6 +44,7 @@ _CSRC = os.path.join(ROOT, "sparse_long_context_nsa_b200", "csrc")
 ATTN_SRC = [os.path.join(_CSRC, "nsa_attention.cu")]
 CMP_SRC = [os.path.join(_CSRC, "nsa_compress.cu")]
 SEL_SRC = [os.path.join(_CSRC, "nsa_select.cu")]
+BWD_SRC = [os.path.join(_CSRC, "nsa_backward.cu")]
 
 
 # ------------------------------------------------------------------ work
@@ -61,6 +62,27 @@ def visible_pairs(wl: workloads.Workload) -> int:
 
 def attention_flops(wl) -> float:
     return 2.0 * (wl.d1 + wl.d2) * wl.n1 * visible_pairs(wl)
+
+
+def backward_flops(wl) -> float:
+    """algorithmic FLOPs of the attention backward: the five contractions per
+    visible (row, block) pair and head -- S = q k (recomputed), dP = dout v,
+    dv += P dout, dq += dS k, dk += dS q -- 2 (3 D1 + 2 D2) each."""
+    return 2.0 * (3 * wl.d1 + 2 * wl.d2) * wl.n1 * visible_pairs(wl)
+
+
+def backward_executed_flops(wl) -> float:
+    """tensor FLOPs the kernels issue: the dq pass recomputes S and dP, the
+    dk/dv pass recomputes them again."""
+    return 2.0 * (4 * wl.d1 + 3 * wl.d2) * wl.n1 * visible_pairs(wl)
+
+
+def compress_backward_bytes(wl) -> float:
+    """bytes the compression backward must move once: raw k, v (storage dtype)
+    and w in, dkcmp / dvcmp (fp32) in, dk, dv (fp32) and dw out."""
+    tc = sum(0 if S < wl.l else (S - wl.l) // wl.d + 1 for S in wl.seqlens)
+    return float(wl.t2 * wl.n2 * (wl.d1 + wl.d2) * (2 + 4) + tc * wl.n2 * (wl.d1 + wl.d2) * 4
+                 + wl.l * wl.n2 * (2 + 4))
 
 
 def compress_bytes(wl) -> float:
@@ -119,7 +141,7 @@ def profile_traffic(kind, workload):
         return None
     with open(p) as f:
         d = json.load(f)
-    src = {"attention": ATTN_SRC, "compress": CMP_SRC, "select": SEL_SRC}[kind]
+    src = {"attention": ATTN_SRC, "compress": CMP_SRC, "select": SEL_SRC, "backward": BWD_SRC}[kind]
     if d.get("workload") != workload or d.get("source_sha256_16") != src_hash(src):
         return None
     return d.get("bytes_per_launch_full_workload")
@@ -402,13 +424,57 @@ def run_ours(args, rank, world, local_rank):
         sel = dict(ms=float(np.mean([e[0].elapsed_time(e[1]) for e in sev])), steps=ks,
                    keys=row_keys(tk_host, cuq, cu, wl.lp), topk=tk_host)
 
+    # ---------- backward: gradients of the step's attention and compression ----------
+    bwd = None
+    if not args.no_backward:
+        gout = workloads.grad_output(wl, device=str(dev))
+        att, _, smax, ssum = outs
+        bws = torch.empty(nsa.nsa_compress_attention_backward_workspace_size(
+            wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, cuq, cuc), dtype=torch.uint8, device=dev)
+        grads = (torch.empty(t1, wl.n1, wl.d1, dtype=torch.float32, device=dev),
+                 torch.empty(tc, wl.n2, wl.d1, dtype=torch.float32, device=dev),
+                 torch.empty(tc, wl.n2, wl.d2, dtype=torch.float32, device=dev))
+        cws = torch.empty(nsa.nsa_compress_backward_workspace_size(cu, wl.l, wl.d), dtype=torch.uint8, device=dev)
+        cgrads = (torch.empty(k.shape, dtype=torch.float32, device=dev),
+                  torch.empty(v.shape, dtype=torch.float32, device=dev),
+                  torch.empty(wl.l, wl.n2, dtype=torch.float32, device=dev))
+
+        def bwd_att():
+            nsa.nsa_compress_attention_backward(q, kc, vc, att, gout, smax, ssum, wl.scale, wl.n1, wl.l, wl.d,
+                                                cuq, cuc, grads=grads, workspace=bws)
+
+        def bwd_cmp():
+            nsa.nsa_compress_backward(k, v, w, grads[1], grads[2], wl.l, wl.d, cu, grads=cgrads, workspace=cws)
+
+        for _ in range(max(args.warmup, 0)):
+            flush.zero_()
+            bwd_att()
+            bwd_cmp()
+        kb = max(3, min(K, args.backward_steps))
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(kb)]
+        for i in range(kb):
+            flush.zero_()
+            bev[i][0].record()
+            bwd_att()
+            bev[i][1].record()
+            bwd_cmp()
+            bev[i][2].record()
+        torch.cuda.synchronize()
+        if nsa.nsa_workspace_status(bws) != 0 or nsa.nsa_workspace_status(cws) != 0:
+            raise RuntimeError("device-side timeout in the backward")
+        bwd = dict(att_ms=float(np.mean([e[0].elapsed_time(e[1]) for e in bev])),
+                   cmp_ms=float(np.mean([e[1].elapsed_time(e[2]) for e in bev])), steps=kb,
+                   launches=(5 if wl.d2 > 128 else 4) + 2 + (len(wl.seqlens) - 1) // 96,
+                   gsample=gout[:min(int(wl.seqlens[0]), 16384), :wl.n1 // wl.n2].cpu())
+        del grads, cgrads, bws, gout
+
     side = None
     if not args.no_side:
         del flush
         side = time_side_case(args, nsa, dev, rank)
 
     return dict(wl=wl, K=K, step_ms=step_ms, att_ms=att_ms, cmp_ms=cmp_ms, t1=t1, wall=t_wall,
-                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk, side=side, x=x,
+                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk, side=side, x=x, bwd=bwd,
                 launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
 
 
@@ -619,6 +685,41 @@ def masked_cpu_baseline(wl, x, am, tm, budget_s=8.0):
             "sample": f"{rows.size} of {T1} evenly spaced query rows, all heads, same masks, {dt_s:.1f} s"}
 
 
+def backward_cpu_baseline(wl, x, gsample, budget_s=10.0):
+    """The backward oracle as it stands on a bounded sample: KV group 0 of the
+    first sequence's leading S' tokens (S' doubled from 1024 until one call
+    takes a quarter of the budget), with its kcmp / vcmp from the oracle's
+    compression.  Throughput over the sample's algorithmic FLOPs.  gsample:
+    the incoming gradient of those rows and heads (the GPU run's own)."""
+    import oracle
+    G = wl.n1 // wl.n2
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.FP16
+    s0 = min(int(wl.seqlens[0]), gsample.shape[0])
+    if wl.q_last is not None:
+        return None
+    q0 = x["q"][:s0, :G].cpu()
+    k0, v0, w0 = x["k"][:s0, :1].cpu(), x["v"][:s0, :1].cpu(), x["w"][:, :1].cpu()
+    gout = gsample
+    S = min(1024, s0)
+    best = None
+    while True:
+        cu = np.array([S], dtype=np.int32)
+        kc, cuc = oracle.compress(k0[:S], w0, wl.l, wl.d, cu, dtype=dt)
+        vc, _ = oracle.compress(v0[:S], w0, wl.l, wl.d, cu, dtype=dt)
+        t = time.perf_counter()
+        oracle.compress_attention_backward(q0[:S], kc, vc, gout[:S], wl.scale, wl.l, wl.d, cu, cuc)
+        dt_s = time.perf_counter() - t
+        sw = wl.replace(seqlens=(S,), n1=G, n2=1, q_last=None)
+        best = (S, dt_s, backward_flops(sw))
+        if dt_s >= budget_s / 4 or S >= s0:
+            break
+        S = min(2 * S, s0)
+    S, dt_s, fl = best
+    return {"value": fl / dt_s / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"KV group 0 ({G} heads) of the first {S} tokens of sequence 0: attention backward in "
+                      f"fp64, {dt_s:.2f} s"}
+
+
 def run_reference(args, rank, world):
     """Reference arm: the fp64 CPU oracle (the pages publish no code to run)."""
     if rank != 0:
@@ -690,6 +791,8 @@ def main():
     ap.add_argument("--no-masks", action="store_true", help="skip the masked-attention measurement")
     ap.add_argument("--select-steps", type=int, default=20)
     ap.add_argument("--select-cpu-budget", type=float, default=8.0)
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--backward-steps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -736,6 +839,10 @@ def main():
         dev0 = torch.device("cuda", local_rank)
         sel_ms = max_over_ranks([r["sel"]["ms"]], dev0, world)[0]
         sel_flops_all = sum_over_ranks([select_flops(wl, r["sel"]["keys"])], dev0, world)[0]
+    bwd_att_ms = bwd_cmp_ms = None
+    if r["bwd"] is not None:
+        bwd_att_ms, bwd_cmp_ms = max_over_ranks([r["bwd"]["att_ms"], r["bwd"]["cmp_ms"]],
+                                                torch.device("cuda", local_rank), world)
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
@@ -827,6 +934,30 @@ def main():
                                  if (not args.no_cpu_baseline and world == 1) else None),
                 "gpu_launches": 2 * r["sel"]["steps"],
             }
+        if r["bwd"] is not None:
+            bf, bx = backward_flops(wl), backward_executed_flops(wl)
+            bt = bf / (bwd_att_ms * 1e-3) / 1e12
+            cb = compress_backward_bytes(wl)
+            cg = cb / (bwd_cmp_ms * 1e-3) / 1e9
+            line["backward"] = {
+                "what": "nsa_compress_attention_backward (dq, dkcmp, dvcmp from the step's output and "
+                        "statistics) then nsa_compress_backward (dk, dv, dw); L2 flushed before every call",
+                "steps": r["bwd"]["steps"], "ms": bwd_att_ms + bwd_cmp_ms,
+                "attention_backward": {
+                    "ms": bwd_att_ms, "tflops": bt, "pct_of_bf16_peak": 100.0 * bt / peak_t,
+                    "flops_per_launch": bf, "executed_flops": bx,
+                    "executed_tflops": bx / (bwd_att_ms * 1e-3) / 1e12,
+                    "roofline": {"bound": "tensor", "achieved": bt, "peak": peak_t, "unit": "TFLOP/s",
+                                 "frac": bt / peak_t, "traffic": profile_traffic("backward", wl.name),
+                                 "peak_source": f"{peak_src} bf16_tflops (burst)"}},
+                "compress_backward": {
+                    "ms": bwd_cmp_ms, "gbs": cg, "bytes": cb,
+                    "roofline": {"bound": "hbm", "achieved": cg, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": cg / peaks["hbm_gbs"], "traffic": None,
+                                 "peak_source": f"{peak_src} hbm_gbs"}},
+                "gpu_launches": r["bwd"]["launches"] * r["bwd"]["steps"],
+                "cpu_baseline": (backward_cpu_baseline(wl, r["x"], r["bwd"]["gsample"])
+                                 if (not args.no_cpu_baseline and world == 1) else None)}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()
