@@ -364,9 +364,12 @@ def run_ours(args, rank, world, local_rank):
         am_d, tm_d = torch.from_numpy(am).to(dev), torch.from_numpy(tm).to(dev)
         mouts = tuple(torch.empty_like(t) for t in outs)
 
+        mws = torch.empty(nsa.nsa_compress_attention_masked_workspace_size(
+            wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, cuq, cuc, cus), dtype=torch.uint8, device=dev)
+
         def masked_call():
             nsa.nsa_compress_attention(q, kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count, cuq, cuc, cus,
-                                       out=mouts, workspace=ws, atten_mask=am_d, topk_mask=tm_d)
+                                       out=mouts, workspace=mws, atten_mask=am_d, topk_mask=tm_d)
 
         for _ in range(max(args.warmup, 0)):
             flush.zero_()
@@ -379,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
             masked_call()
             mev[i][1].record()
         torch.cuda.synchronize()
-        if nsa.nsa_workspace_status(ws) != 0:
+        if nsa.nsa_workspace_status(mws) != 0:
             raise RuntimeError("device-side timeout in masked attention")
         # attended (row, block) pairs: visible by the causal rule and not masked
         pairs = 0

@@ -167,11 +167,24 @@ nsa_status_t nsa_compress_attention(
  *               am_cols >= every sequence's compressed block count.
  *   topk_mask   device bytes, tm_rows x tm_cols, NULL = no mask.  Needs
  *               tm_rows >= every S_q and tm_cols >= every n_sel.
- * Other arguments, outputs, workspace (nsa_compress_attention_workspace_size)
- * and errors as nsa_compress_attention; a mask too small for the batch is
+ * The call first packs each given mask into bit rows inside the workspace
+ * (one launch per mask), so the attention kernel reads 1 bit per (row,
+ * block).  Workspace: nsa_compress_attention_masked_workspace_size with the
+ * same masks present.  Other arguments, outputs and errors as
+ * nsa_compress_attention; a mask too small for the batch is
  * NSA_ERR_INVALID_ARG.  With both masks NULL the call is
  * nsa_compress_attention.
  */
+/*
+ * Workspace bytes of nsa_compress_attention_masked: that of the unmasked call
+ * plus the bit-packed rows of each mask that is present (with_* non-zero).
+ * Pure host function.
+ */
+nsa_status_t nsa_compress_attention_masked_workspace_size(
+    int head_num, int n2, int d1, int d2, int l, int d, int lp, int count,
+    const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+    int batch, int with_atten_mask, int with_topk_mask, size_t* bytes);
+
 nsa_status_t nsa_compress_attention_masked(
     const void* q, const void* kcmp, const void* vcmp, float scale, int head_num,
     int l, int d, int lp, int count,

@@ -35,6 +35,7 @@ EXPORTED = (
     "nsa_compress_attention_workspace_size",
     "nsa_compress_attention",
     "nsa_compress_attention_masked",
+    "nsa_compress_attention_masked_workspace_size",
     "nsa_workspace_status",
     "nsa_compress_status",
     "nsa_compress_attention_noalloc",
@@ -96,6 +97,9 @@ def load(path: Optional[str] = None):
                                                   i32p, ci, ci, ci, ci, ci, vp, ci, ci, vp, ci, ci, vp, vp, vp,
                                                   vp, vp, cs, vp]
     lib.nsa_compress_attention_masked.restype = ci
+    lib.nsa_compress_attention_masked_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p, i32p, i32p,
+                                                                 ci, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
+    lib.nsa_compress_attention_masked_workspace_size.restype = ci
     lib.nsa_workspace_status.argtypes = [vp, vp]
     lib.nsa_workspace_status.restype = ci
     lib.nsa_compress_status.argtypes = [vp]
@@ -285,6 +289,20 @@ def nsa_compress_attention_workspace_size(head_num: int, n2: int, d1: int, d2: i
     return int(out.value)
 
 
+def nsa_compress_attention_masked_workspace_size(head_num: int, n2: int, d1: int, d2: int, l: int, d: int,
+                                                 lp: int, count: int, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                                 atten_mask: bool = True, topk_mask: bool = True) -> int:
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size):
+        raise ValueError("the three prefix-sum lists need one entry per sequence")
+    out = ctypes.c_size_t(0)
+    _raise(load().nsa_compress_attention_masked_workspace_size(
+        int(head_num), int(n2), int(d1), int(d2), int(l), int(d), int(lp), int(count), _ip(cq), _ip(cc),
+        _ip(cs), cq.size, int(bool(atten_mask)), int(bool(topk_mask)), ctypes.byref(out)),
+        "nsa_compress_attention_masked_workspace_size")
+    return int(out.value)
+
+
 def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tensor, scale: float,
                            head_num: int, l: int, d: int, lp: int, count: int, cu_seqlens_q,
                            cu_cmp_kv, cu_sel_kv, out=None, workspace: Optional[torch.Tensor] = None,
@@ -331,7 +349,11 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
         _out(tk, (t1, n2, count), torch.int32, dev, "topk_indices")
         _out(smax, (t1, n1, 8), torch.float32, dev, "softmax_max")
         _out(ssum, (t1, n1, 8), torch.float32, dev, "softmax_sum")
-    ws_bytes = nsa_compress_attention_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs)
+    if atten_mask is None and topk_mask is None:
+        ws_bytes = nsa_compress_attention_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs)
+    else:
+        ws_bytes = nsa_compress_attention_masked_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs,
+                                                                atten_mask is not None, topk_mask is not None)
     workspace = _workspace(workspace, ws_bytes, dev)
     if atten_mask is None and topk_mask is None:
         st = load().nsa_compress_attention(

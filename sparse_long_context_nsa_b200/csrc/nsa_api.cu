@@ -284,6 +284,36 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
     return NSA_OK;
 }
 
+// Bit-packed copies of the optional masks, placed after the attention
+// workspace: max_q rows each; atten_mask rows cover every column a KV tile
+// walk reads (plus a two-word window tail), topk_mask rows every candidate.
+struct MaskPack {
+    int64_t rows = 0, max_c = 0, max_s = 0;
+    int am_words = 0, tm_words = 0;
+    size_t am_bytes = 0, tm_bytes = 0;
+};
+
+MaskPack plan_masks(const AttnPlan& pl, const int32_t* cu_q, const int32_t* cu_cmp, const int32_t* cu_sel,
+                    int batch, bool am, bool tm) {
+    MaskPack m;
+    for (int b = 0; b < batch; ++b) {
+        m.rows = std::max<int64_t>(m.rows, cu_q[b] - (b ? cu_q[b - 1] : 0));
+        m.max_c = std::max<int64_t>(m.max_c, cu_cmp[b] - (b ? cu_cmp[b - 1] : 0));
+        m.max_s = std::max<int64_t>(m.max_s, cu_sel[b] - (b ? cu_sel[b - 1] : 0));
+    }
+    auto words = [](int64_t cols) { return (int)((((cols + 31) / 32 + 2) + 1) & ~int64_t(1)); };
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    if (am) {
+        m.am_words = words((int64_t)pl.max_nkv * pl.nkv_cols);
+        m.am_bytes = up((size_t)m.rows * m.am_words * 4);
+    }
+    if (tm) {
+        m.tm_words = words(m.max_s);
+        m.tm_bytes = up((size_t)m.rows * m.tm_words * 4);
+    }
+    return m;
+}
+
 // ------------------------------------------------------------------------
 // selection-attention plan
 // ------------------------------------------------------------------------
@@ -712,8 +742,10 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
                                     batch, true, pl, grid_cap, npipe_max, group_begin, group_count);
     if (s != NSA_OK) return s;
+    const MaskPack mp = plan_masks(pl, cu_seqlens_q, cu_cmp_kv, cu_sel_kv, batch, atten_mask != nullptr,
+                                   topk_mask != nullptr);
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-        workspace_bytes < pl.ws_total)
+        workspace_bytes < pl.ws_total + mp.am_bytes + mp.tm_bytes)
         return NSA_ERR_WORKSPACE;
     if (pl.tiles.empty()) return NSA_OK;
 
@@ -785,10 +817,19 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     p.off_score = pl.off_score;
     p.off_bar = pl.off_bar;
     p.smem_bytes = pl.smem_bytes;
-    p.amask = atten_mask;
-    p.am_s2 = am_s2;
-    p.tmask = topk_mask;
-    p.tm_s2 = tm_s2;
+    // the masks as bit rows (one launch each, before the attention)
+    uint32_t* am_bits = reinterpret_cast<uint32_t*>(ws + pl.ws_total);
+    uint32_t* tm_bits = reinterpret_cast<uint32_t*>(ws + pl.ws_total + mp.am_bytes);
+    if (atten_mask && launch_pack_mask(atten_mask, am_s2, (int)std::min<int64_t>(am_s2, mp.max_c), (int)mp.rows,
+                                       mp.am_words, am_bits, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    if (topk_mask && launch_pack_mask(topk_mask, tm_s2, (int)std::min<int64_t>(tm_s2, mp.max_s), (int)mp.rows,
+                                      mp.tm_words, tm_bits, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    p.am_bits = atten_mask ? am_bits : nullptr;
+    p.am_words = mp.am_words;
+    p.tm_bits = topk_mask ? tm_bits : nullptr;
+    p.tm_words = mp.tm_words;
     const int grid = std::min(pl.grid, nsm);   // the workspace holds pl.grid CTAs' scratch
     if (launch_attention(p, tq, tk, tv, grid, st) != cudaSuccess) return NSA_ERR_CUDA;
     return NSA_OK;
@@ -803,6 +844,22 @@ nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void*
     return compress_attention_impl(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
                                    cu_sel_kv, batch, n2, d1, d2, dtype, nullptr, 0, nullptr, 0, attention_out,
                                    topk_indices, softmax_max, softmax_sum, workspace, workspace_bytes, stream);
+}
+
+nsa_status_t nsa_compress_attention_masked_workspace_size(int head_num, int n2, int d1, int d2, int l, int d,
+                                                          int lp, int count, const int32_t* cu_seqlens_q,
+                                                          const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv,
+                                                          int batch, int with_atten_mask, int with_topk_mask,
+                                                          size_t* bytes) {
+    if (bytes == nullptr) return NSA_ERR_INVALID_ARG;
+    AttnPlan pl;
+    nsa_status_t s = plan_attention(head_num, n2, d1, d2, l, d, lp, count, cu_seqlens_q, cu_cmp_kv, cu_sel_kv,
+                                    batch, false, pl);
+    if (s != NSA_OK) return s;
+    const MaskPack mp = plan_masks(pl, cu_seqlens_q, cu_cmp_kv, cu_sel_kv, batch, with_atten_mask != 0,
+                                   with_topk_mask != 0);
+    *bytes = pl.ws_total + mp.am_bytes + mp.tm_bytes;
+    return NSA_OK;
 }
 
 nsa_status_t nsa_compress_attention_masked(const void* q, const void* kcmp, const void* vcmp, float scale,

@@ -123,15 +123,18 @@ __device__ __forceinline__ int nvis_of(int t, int l, int d, int n_cmp) {
 // k-th largest key (fp32 bit pattern) of sc[0 .. ncand) held in registers,
 // NR keys per lane (key i of a lane belongs to j = lane + 32 i); keys at
 // j >= lim are 0.  Bitwise search from the top bit down.
+// Bit j of a packed mask row (bit j % 32 of word j / 32; set = removed).
+__device__ __forceinline__ bool mask_bit(const uint32_t* row, int j) { return (row[j >> 5] >> (j & 31)) & 1u; }
+
 template <int NR, bool kMask>
 __device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int lim, int k, int lane,
-                                                 const uint8_t* trow) {
+                                                 const uint32_t* trow) {
     uint32_t key[NR];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
         const int j = lane + 32 * i;
         bool in = j < lim;
-        if constexpr (kMask) in = in && !(trow && trow[j]);
+        if constexpr (kMask) in = in && !(trow && mask_bit(trow, j));
         key[i] = in ? __float_as_uint(sc[j]) : 0u;
     }
     uint32_t thr = 0;
@@ -159,20 +162,25 @@ __device__ __forceinline__ uint32_t kth_key_regs(const float* sc, int ncand, int
 // Exact k-th largest key by a bitwise search over the fp32 bit patterns
 // (scores are >= 0, so the bit patterns order like the values), then an
 // ordered ballot scan keeps every key above it plus the earliest ties, which
-// also lists the indices in ascending order.  With a topk_mask row (kMask),
-// candidates whose mask byte is set are out of the set (step 6).
+// also lists the indices in ascending order.  With a topk_mask row (kMask,
+// bit-packed), candidates whose bit is set are out of the set (step 6).
 template <bool kMask>
 __device__ __forceinline__ void warp_topk(const float* sc, int ncand, int jcov, int count,
-                                          int32_t* dst, int lane, const uint8_t* trow) {
+                                          int32_t* dst, int lane, const uint32_t* trow) {
     auto masked = [&](int j) {
-        if constexpr (kMask) return trow != nullptr && trow[j] != 0;
+        if constexpr (kMask) return trow != nullptr && mask_bit(trow, j);
         return false;
     };
     int n_in = ncand;
     if constexpr (kMask) {
         if (trow) {
+            // set bits among the candidates, a word per lane
             int nm = 0;
-            for (int j = lane; j < ncand; j += 32) nm += trow[j] ? 1 : 0;
+            for (int w = lane; w * 32 < ncand; w += 32) {
+                const int left = ncand - w * 32;
+                const uint32_t keep = left >= 32 ? 0xffffffffu : ((1u << left) - 1u);
+                nm += __popc(trow[w] & keep);
+            }
             n_in = ncand - __reduce_add_sync(0xffffffffu, nm);
         }
     }
@@ -547,16 +555,13 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 int32_t* dst = p.topk + ((size_t)(t.q_row0 + tau) * p.n2 + t.group) * p.count;
                 const int nv = nvis_of(tp, p.l, p.d, t.n_cmp);
                 bool empty = nv == 0;
-                const uint8_t* trow = nullptr;
+                const uint32_t* trow = nullptr;
                 if constexpr (kMask) {
-                    // a token whose visible blocks are all masked attends to nothing
-                    if (!empty && p.amask != nullptr) {
-                        const uint8_t* ar = p.amask + (long long)(t.tloc0 + tau) * p.am_s2;
-                        int keep = 0;
-                        for (int c = lane; c < nv; c += 32) keep |= (ar[c] == 0) ? 1 : 0;
-                        empty = !__any_sync(0xffffffffu, keep);
-                    }
-                    if (p.tmask != nullptr) trow = p.tmask + (long long)(t.tloc0 + tau) * p.tm_s2;
+                    // a token whose visible blocks are all masked attends to nothing; its
+                    // heads share the mask row, so its first head's softmax sum is 0
+                    if (!empty && p.am_bits != nullptr)
+                        empty = rowstat[((pp * 2 + slot) * 2 + 1) * 128 + tl * G] == 0.f;
+                    if (p.tm_bits != nullptr) trow = p.tm_bits + (size_t)(t.tloc0 + tau) * p.tm_words;
                 }
                 if (empty) {
                     for (int j = lane; j < p.count; j += 32) dst[j] = -1;
@@ -680,9 +685,10 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int tpos = t.t0 + tok;
                 const int nvis = valid ? nvis_of(tpos, p.l, p.d, t.n_cmp) : 0;
                 const int slot = tcount & 1;
-                const uint8_t* arow = nullptr;
+                const uint32_t* arow = nullptr;
                 if constexpr (kMask)
-                    arow = (valid && p.amask != nullptr) ? p.amask + (long long)(t.tloc0 + tok) * p.am_s2 : nullptr;
+                    arow = (valid && p.am_bits != nullptr) ? p.am_bits + (size_t)(t.tloc0 + tok) * p.am_words
+                                                           : nullptr;
                 // this slot's scratch: banded values [chunk][row][NJC], then the chunk
                 // references [row][chunk]
                 float* sbase_g = p.band + (((size_t)blockIdx.x * npipe + pp) * 2 + slot) * (size_t)p.region;
@@ -725,12 +731,16 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             for (int e = 0; e < CH; ++e) s[e] = (e < cl) ? s[e] : -INFINITY;
                         }
                         if constexpr (kMask) {
-                            // atten_mask (step 1): a set byte removes a visible block
+                            // atten_mask (step 1), bit-packed: a set bit removes a visible
+                            // block; the chunk's CH <= 64 bits from a three-word window
                             if (arow != nullptr) {
-                                const uint8_t* mr = arow + (long long)i * NKV + c * CH;
+                                const int col0 = i * NKV + c * CH;
+                                const int w0 = col0 >> 5, b0 = col0 & 31;
+                                const uint32_t a0 = arow[w0], a1 = arow[w0 + 1], a2 = arow[w0 + 2];
+                                const uint32_t lo = __funnelshift_r(a0, a1, b0), hi = __funnelshift_r(a1, a2, b0);
 #pragma unroll
                                 for (int e = 0; e < CH; ++e)
-                                    if (e < cl && mr[e]) s[e] = -INFINITY;
+                                    if (((e < 32 ? lo >> e : hi >> (e - 32)) & 1u) != 0u) s[e] = -INFINITY;
                             }
                         }
                         // chunk maximum: independent chains of 3-input max
@@ -886,6 +896,35 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 }
 
+// A byte mask (rows x s2, nonzero = set) to bit rows of `words` 32-bit words:
+// bit j of row r = src[r][j] for j < ncols, 0 beyond.  One warp per (row,
+// 32 words): lane k reads byte 32 w + k of each word w in turn (coalesced),
+// a ballot forms the word, and lane w % 32 stores it.
+__global__ void pack_mask_kernel(const uint8_t* __restrict__ src, long long s2, int ncols, int rows, int words,
+                                 uint32_t* __restrict__ dst) {
+    const int lane = threadIdx.x & 31;
+    const long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int wbase = blockIdx.y * 32;
+    const uint8_t* row = src + r * s2;
+    uint32_t mine = 0;
+    for (int k = 0; k < 32; ++k) {
+        const int col = (wbase + k) * 32 + lane;
+        const bool set = col < ncols && row[col] != 0;
+        const uint32_t word = __ballot_sync(0xffffffffu, set);
+        if (lane == k) mine = word;
+    }
+    if (wbase + lane < words) dst[r * words + wbase + lane] = mine;
+}
+
+cudaError_t launch_pack_mask(const uint8_t* src, long long s2, int ncols, int rows, int words, uint32_t* dst,
+                             cudaStream_t st) {
+    if (rows <= 0 || words <= 0) return cudaSuccess;
+    dim3 grid((rows + 7) / 8, (words + 31) / 32);
+    pack_mask_kernel<<<grid, 256, 0, st>>>(src, s2, ncols, rows, words, dst);
+    return cudaGetLastError();
+}
+
 template <typename T, int A, bool kMask>
 static cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, int grid, cudaStream_t st) {
@@ -915,7 +954,7 @@ static cudaError_t launch_a(const AttnParams& p, const CUtensorMap& tq, const CU
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, int grid, cudaStream_t st) {
     // the masked kernel only where a mask is given: the unmasked one is unchanged
-    if (p.amask != nullptr || p.tmask != nullptr)
+    if (p.am_bits != nullptr || p.tm_bits != nullptr)
         return p.dtype == 0 ? launch_a<__nv_bfloat16, true>(p, tq, tk, tv, grid, st)
                             : launch_a<__half, true>(p, tq, tk, tv, grid, st);
     return p.dtype == 0 ? launch_a<__nv_bfloat16, false>(p, tq, tk, tv, grid, st)

@@ -103,12 +103,15 @@ struct AttnParams {
     int off_q, q_bytes, off_ring, slot_bytes, off_rowstat, off_score, off_bar, smem_bytes;
     // optional masks (null = none): bool bytes (S1, row stride), one matrix for
     // every sequence and head, row = query index inside the sequence
-    const uint8_t* amask;   // (S1, >= n_cmp): true removes the compressed block (step 1)
-    long long am_s2;
-    const uint8_t* tmask;   // (S1, >= n_sel): true removes the top-k candidate (step 6)
-    long long tm_s2;
+    const uint32_t* am_bits;   // atten_mask bit-packed, am_words words per mask row (step 1)
+    int am_words;
+    const uint32_t* tm_bits;   // topk_mask bit-packed, tm_words words per mask row (step 6)
+    int tm_words;
 };
 
+// byte mask (rows x s2) -> bit rows of `words` words, columns >= ncols cleared
+cudaError_t launch_pack_mask(const uint8_t* src, long long s2, int ncols, int rows, int words, uint32_t* dst,
+                             cudaStream_t st);
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, int grid, cudaStream_t st);
 int attention_kv_cols(int a);     // compressed blocks per KV tile for band factor a

@@ -44,9 +44,9 @@ def _masks(wl, x, cuc, p_att, p_topk, seed):
 
 
 def _gpu(nsa, wl, x, kc, vc, cuc, am, tm):
-    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
-        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"]),
-        dtype=torch.uint8, device="cuda")
+    ws = torch.empty(nsa.nsa_compress_attention_masked_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"],
+        am is not None, tm is not None), dtype=torch.uint8, device="cuda")
     res = nsa.nsa_compress_attention(
         x["q"].cuda(), kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
         x["cu_sel_kv"], workspace=ws,
@@ -171,7 +171,7 @@ def test_masks_on_the_16k_workload_sampled_rows(nsa):
     cuc = nsa.nsa_compress_out_len(x["cu_seqlens"], wl.l, wl.d)
     kc, vc = nsa.nsa_compress(x["k"], x["v"], x["w"], wl.l, wl.d, x["cu_seqlens"])
     am, tm = _masks(wl, x, cuc, 0.3, 0.3, seed=5)
-    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+    ws = torch.empty(nsa.nsa_compress_attention_masked_workspace_size(
         wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"]),
         dtype=torch.uint8, device="cuda")
     res = nsa.nsa_compress_attention(x["q"], kc, vc, wl.scale, wl.n1, wl.l, wl.d, wl.lp, wl.count,
@@ -184,3 +184,19 @@ def test_masks_on_the_16k_workload_sampled_rows(nsa):
                                     vc.float().cpu(), wl.scale, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
                                     x["cu_sel_kv"], rows=rows, q_rows_only=True, atten_mask=am, topk_mask=tm)
     _check([t.cpu() for t in res], ref, wl, x, tm)
+
+
+def test_masked_call_needs_the_masked_workspace(nsa):
+    wl = _wl([700], 8, 2, 64, 32, 16, 64, 5, seed=26)
+    x, kc, vc, cuc = _inputs(wl)
+    am, tm = _masks(wl, x, cuc, 0.3, 0.3, seed=7)
+    small = nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    need = nsa.nsa_compress_attention_masked_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+    assert need > small
+    with pytest.raises(ValueError):
+        nsa.nsa_compress_attention(x["q"].cuda(), kc.cuda(), vc.cuda(), wl.scale, wl.n1, wl.l, wl.d, wl.lp,
+                                   wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"],
+                                   workspace=torch.empty(small, dtype=torch.uint8, device="cuda"),
+                                   atten_mask=torch.from_numpy(am).cuda(), topk_mask=torch.from_numpy(tm).cuda())
