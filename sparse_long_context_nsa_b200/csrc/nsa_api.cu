@@ -438,7 +438,7 @@ struct BwdPlan {
     std::vector<bwd::KVTile> kvtiles;
     int nslots = 0;
     bool one_pass = true;   // dV and dK in one tensor-memory allocation
-    int off_q = 0, off_do = 0, off_k = 0, off_v = 0, off_row = 0, off_bar = 0, smem_bytes = 0;
+    int nst = 1, stage_bytes = 0, off_row = 0, off_bar = 0, smem_bytes = 0;
     size_t off_qitems = 0, off_kvitems = 0, off_kvtiles = 0, off_rowinfo = 0, off_part = 0, ws_total = 0;
 };
 
@@ -460,21 +460,18 @@ nsa_status_t plan_backward(int head_num, int n2, int d1, int d2, int l, int d, c
     pl.one_pass = d2 <= 128;
     const int TT = pl.TT, KV = bwd::kKV;
 
-    // shared memory (one CTA per SM: the kernels take all 512 tensor-memory columns)
-    int off = 0;
-    pl.off_q = off;
-    off += nqc * 16384;
-    pl.off_do = off;
-    off += nvc * 16384;
-    pl.off_k = off;
-    off += nqc * 16384;
-    pl.off_v = off;
-    off += nvc * 16384;
-    pl.off_row = off;
-    off += kRows * 12;
-    pl.off_bar = (off + 127) & ~127;
-    pl.smem_bytes = std::max(pl.off_bar + 128 + 1024, 116 * 1024);
-    if (pl.smem_bytes > kSmemLimit) return NSA_ERR_UNSUPPORTED;
+    // shared memory (one CTA per SM: the kernels take all 512 tensor-memory columns): the
+    // fixed operands (Q/dO of a dQ item, K/V of a dK/dV tile), then one or two stages of the
+    // streamed ones, the rows' statistics (two M-tile buffers) and the barriers
+    pl.stage_bytes = (nqc + nvc) * 16384;
+    auto fits = [&](int nst) {
+        pl.nst = nst;
+        pl.off_row = (1 + nst) * pl.stage_bytes;
+        pl.off_bar = (pl.off_row + 2 * kRows * 12 + 127) & ~127;
+        pl.smem_bytes = std::max(pl.off_bar + 128 + 1024, 116 * 1024);
+        return pl.smem_bytes <= kSmemLimit;
+    };
+    if (!fits(2) && !fits(1)) return NSA_ERR_UNSUPPORTED;
 
     // total dK/dV work in M-tile steps, to size the runs: about four runs per SM
     auto first_row = [&](int kt, int64_t off_b) { return (int64_t)kt * KV * d + l - 1 - off_b; };
@@ -1109,25 +1106,37 @@ nsa_status_t nsa_compress_attention_backward(const void* q, const void* kcmp, co
     p.d = d;
     p.scale = scale;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    p.off_q = pl.off_q;
-    p.off_do = pl.off_do;
-    p.off_k = pl.off_k;
-    p.off_v = pl.off_v;
     p.off_row = pl.off_row;
     p.off_bar = pl.off_bar;
     p.smem_bytes = pl.smem_bytes;
+    p.nst = pl.nst;
+    p.stage_bytes = pl.stage_bytes;
+    const int qc_bytes = ((d1 + 63) / 64) * 16384;
 
     if (bwd::launch_prep(attention_out, dout, softmax_max, softmax_sum,
                          reinterpret_cast<float2*>(ws + pl.off_rowinfo), t1 * head_num, d2, p.dtype,
                          st) != cudaSuccess)
         return NSA_ERR_CUDA;
+    // dQ: Q and dO fixed, K/V streamed
+    p.off_q = 0;
+    p.off_do = qc_bytes;
+    p.off_k = pl.stage_bytes;
+    p.off_v = pl.stage_bytes + qc_bytes;
     if (bwd::launch_dq(p, tq, tdo, tk, tv, st) != cudaSuccess) return NSA_ERR_CUDA;
+    // dK/dV: Q and dO streamed, K/V fixed
+    p.off_q = 0;
+    p.off_do = qc_bytes;
+    p.off_k = pl.nst * pl.stage_bytes;
+    p.off_v = pl.nst * pl.stage_bytes + qc_bytes;
     // dV and dK together when both accumulators fit beside the 128 score
     // columns; else one pass for each
     const int npass = pl.one_pass ? 1 : 2;
     for (int i = 0; i < npass; ++i) {
         p.mode = pl.one_pass ? 3 : 1 + i;   // bit 0 dV, bit 1 dK
         p.col_dk = pl.one_pass ? 128 : 0;
+        // a second score buffer at columns 256..383 when the accumulators end by column 256
+        const int acc_end = pl.one_pass ? 128 + d1 : (i == 0 ? d2 : d1);
+        p.nsb = acc_end <= 256 ? 2 : 1;
         if (bwd::launch_dkdv(p, tq, tdo, tk, tv, st) != cudaSuccess) return NSA_ERR_CUDA;
     }
     if (bwd::launch_reduce(reinterpret_cast<const bwd::KVTile*>(ws + pl.off_kvtiles), (int)pl.kvtiles.size(),

@@ -74,7 +74,9 @@ __device__ __forceinline__ int nvis_at(int t, int l, int d, int n_cmp) {
     return min(n_cmp, (t - l + 1) / d + 1);
 }
 
-enum Bar { B_Q = 0, B_KV, B_S, B_P, B_MMA, B_DONE, B_N };
+// B_Q0/1 and B_KV0/1: one barrier per stage of the two-stage rings; B_S0/1, B_P0/1: one per
+// score buffer; B_QE0/1: a Q/dO stage's last reader has retired
+enum Bar { B_Q0 = 0, B_Q1, B_KV0, B_KV1, B_S0, B_S1, B_P0, B_P1, B_QE0, B_QE1, B_MMA, B_DONE, B_N };
 
 // ------------------------------------------------------------------- prep
 // One warp per row: delta = sum_e out * dout (fp32) and the row's log2
@@ -171,7 +173,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     const int nqc = (p.d1 + 63) / 64, nvc = (p.d2 + 63) / 64;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P) ? 4 : 1);
+        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P0 || i == B_P1) ? 4 : 1);
         *sm.abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -194,38 +196,50 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             constexpr uint32_t id_s = idesc_f16(kBF16, 128, kKV, false, false);
             const uint32_t id_q = idesc_f16(kBF16, 128, p.d1, false, true);
             bool ok = true;
-            mbar_arrive_expect_tx(bar(B_Q), qbytes + dobytes);
-            for (int c = 0; c < nqc; ++c) tma_load_3d(qa + c * 16384, &tm_q, c * 64, it.group * G, it.q_row0, bar(B_Q));
+            mbar_arrive_expect_tx(bar(B_Q0), qbytes + dobytes);
+            for (int c = 0; c < nqc; ++c)
+                tma_load_3d(qa + c * 16384, &tm_q, c * 64, it.group * G, it.q_row0, bar(B_Q0));
             for (int c = 0; c < nvc; ++c)
-                tma_load_3d(doa + c * 16384, &tm_do, c * 64, it.group * G, it.q_row0, bar(B_Q));
-            for (int i = 0; i < it.nkv && ok; ++i) {
+                tma_load_3d(doa + c * 16384, &tm_do, c * 64, it.group * G, it.q_row0, bar(B_Q0));
+            // K/V tiles through a ring of p.nst stages: with two, tile i + 1 loads while
+            // tile i computes (its stage was last read by tile i - 1, retired below)
+            auto load_kv = [&](int i) {
+                const int st = i % p.nst;
+                const uint32_t ks0 = ka + st * p.stage_bytes, vs0 = va + st * p.stage_bytes;
                 const int row = it.cmp_row0 + i * kKV;
-                mbar_arrive_expect_tx(bar(B_KV), kbytes + vbytes);
-                for (int c = 0; c < nqc; ++c) tma_load_3d(ka + c * 16384, &tm_k, c * 64, it.group, row, bar(B_KV));
-                for (int c = 0; c < nvc; ++c) tma_load_3d(va + c * 16384, &tm_v, c * 64, it.group, row, bar(B_KV));
-                ok = mbar_wait(bar(B_KV), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x21);
-                if (i == 0) ok = ok && mbar_wait(bar(B_Q), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x22);
+                mbar_arrive_expect_tx(bar(B_KV0 + st), kbytes + vbytes);
+                for (int c = 0; c < nqc; ++c) tma_load_3d(ks0 + c * 16384, &tm_k, c * 64, it.group, row, bar(B_KV0 + st));
+                for (int c = 0; c < nvc; ++c) tma_load_3d(vs0 + c * 16384, &tm_v, c * 64, it.group, row, bar(B_KV0 + st));
+            };
+            if (it.nkv > 0) load_kv(0);
+            for (int i = 0; i < it.nkv && ok; ++i) {
+                const int st = i % p.nst;
+                const uint32_t kst = ka + st * p.stage_bytes, vst = va + st * p.stage_bytes;
+                ok = mbar_wait(bar(B_KV0 + st), (i / p.nst) & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x21);
+                if (i == 0) ok = ok && mbar_wait(bar(B_Q0), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x22);
                 if (!ok) break;
+                if (p.nst == 2 && i + 1 < it.nkv) load_kv(i + 1);
                 tc_fence_after();
                 for (int ks = 0; ks < p.d1 / 16; ++ks) {   // S = Q K^T
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    umma_ss(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id_s,
+                    umma_ss(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kst + off, 16, 1024), id_s,
                             ks > 0 ? 1u : 0u);
                 }
                 for (int ks = 0; ks < p.d2 / 16; ++ks) {   // dP = dO V^T
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    umma_ss(tmem + 128, sdesc_sw128(doa + off, 16, 1024), sdesc_sw128(va + off, 16, 1024), id_s,
+                    umma_ss(tmem + 128, sdesc_sw128(doa + off, 16, 1024), sdesc_sw128(vst + off, 16, 1024), id_s,
                             ks > 0 ? 1u : 0u);
                 }
-                umma_commit(bar(B_S));
-                ok = mbar_wait(bar(B_P), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x23);
+                umma_commit(bar(B_S0));
+                ok = mbar_wait(bar(B_P0), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x23);
                 if (!ok) break;
                 tc_fence_after();
                 for (int ks = 0; ks < kKV / 16; ++ks)   // dQ += dS K (dS from tensor memory)
-                    umma_ts(tmem + 256, tmem + ks * 8, sdesc_sw128(ka + ks * 2048, kKV * 128, 1024), id_q,
+                    umma_ts(tmem + 256, tmem + ks * 8, sdesc_sw128(kst + ks * 2048, kKV * 128, 1024), id_q,
                             (i > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(bar(B_MMA));
                 ok = mbar_wait(bar(B_MMA), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x24);
+                if (ok && p.nst == 1 && i + 1 < it.nkv) load_kv(i + 1);
             }
         }
     } else {
@@ -239,7 +253,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const float2 info = valid ? p.rowinfo[ri] : make_float2(INFINITY, 0.f);
         const float c2 = p.scale_log2;
         for (int i = 0; i < it.nkv; ++i) {
-            mbar_wait(bar(B_S), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x25);
+            mbar_wait(bar(B_S0), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x25);
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < kKV / 32; ++c) {
@@ -263,7 +277,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_P));
+            if (lane == 0) mbar_arrive(bar(B_P0));
         }
         float* dst = p.dq + ri * p.d1;
         if (it.nkv > 0) {
@@ -307,18 +321,20 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int n_mt = (it.q_end - it.q_row0 + TT - 1) / TT;   // query M-tiles of the run
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P) ? 4 : 1);
+        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P0 || i == B_P1) ? 4 : 1);
         *sm.abort_flag = 0;
         fence_mbar_init();
     }
     {
-        // rows G*TT..127 of every Q / dO chunk: never written by the copies
+        // rows G*TT..127 of every Q / dO chunk of every stage: never written by the copies
         const int r0 = G * TT;
         const int nch = nqc + nvc;
         const int per = (128 - r0) * 8;   // 16-byte pieces per chunk
-        for (int x = threadIdx.x; x < nch * per; x += blockDim.x) {
-            const int c = x / per, o = x % per;
-            uint8_t* base = sm.base + (c < nqc ? p.off_q + c * 16384 : p.off_do + (c - nqc) * 16384);
+        for (int x = threadIdx.x; x < p.nst * nch * per; x += blockDim.x) {
+            const int sc = x / per, o = x % per;
+            const int st = sc / nch, c = sc % nch;
+            uint8_t* base = sm.base + st * p.stage_bytes +
+                            (c < nqc ? p.off_q + c * 16384 : p.off_do + (c - nqc) * 16384);
             *reinterpret_cast<uint4*>(base + r0 * 128 + o * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
@@ -333,8 +349,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = *sm.tmem_slot;   // dV at 0, dK at col_dk, S^T at 384, dP^T at 448
     const uint32_t qa = smem_u32(sm.base + p.off_q), doa = smem_u32(sm.base + p.off_do);
     const uint32_t ka = smem_u32(sm.base + p.off_k), va = smem_u32(sm.base + p.off_v);
-    float2* rinfo = reinterpret_cast<float2*>(sm.base + p.off_row);   // the M-tile's 128 rows
-    int* rnv = reinterpret_cast<int*>(sm.base + p.off_row + 128 * sizeof(float2));
+    // the rows' statistics and visible counts, one buffer per M-tile parity
+    float2* rinfo2 = reinterpret_cast<float2*>(sm.base + p.off_row);
+    int* rnv2 = reinterpret_cast<int*>(sm.base + p.off_row + 2 * 128 * sizeof(float2));
 
     if (warp == 4) {
         if (lane == 0) {
@@ -345,52 +362,97 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const uint32_t id_k = idesc_f16(kBF16, 128, p.d1, false, true);
             bool ok = true;
             const int krow = it.cmp_row0 + it.kt * kKV;
-            mbar_arrive_expect_tx(bar(B_KV), kbytes + vbytes);
-            for (int c = 0; c < nqc; ++c) tma_load_3d(ka + c * 16384, &tm_k, c * 64, it.group, krow, bar(B_KV));
+            mbar_arrive_expect_tx(bar(B_KV0), kbytes + vbytes);
+            for (int c = 0; c < nqc; ++c) tma_load_3d(ka + c * 16384, &tm_k, c * 64, it.group, krow, bar(B_KV0));
             if (do_dk)
-                for (int c = 0; c < nvc; ++c) tma_load_3d(va + c * 16384, &tm_v, c * 64, it.group, krow, bar(B_KV));
-            ok = mbar_wait(bar(B_KV), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x31);
-            for (int mi = 0; mi < n_mt && ok; ++mi) {
+                for (int c = 0; c < nvc; ++c) tma_load_3d(va + c * 16384, &tm_v, c * 64, it.group, krow, bar(B_KV0));
+            // Q / dO M-tiles through a ring of p.nst stages.  A stage is refilled once the
+            // dV/dK MMAs of the M-tile that last used it have retired (B_QE).
+            auto load_q = [&](int mi) {
+                const int st = mi % p.nst;
                 const int row0 = it.q_row0 + mi * TT;
-                mbar_arrive_expect_tx(bar(B_Q), qbytes + dobytes);
-                for (int c = 0; c < nqc; ++c) tma_load_3d(qa + c * 16384, &tm_q, c * 64, it.group * G, row0, bar(B_Q));
+                const uint32_t qs0 = qa + st * p.stage_bytes, ds0 = doa + st * p.stage_bytes;
+                mbar_arrive_expect_tx(bar(B_Q0 + st), qbytes + dobytes);
+                for (int c = 0; c < nqc; ++c)
+                    tma_load_3d(qs0 + c * 16384, &tm_q, c * 64, it.group * G, row0, bar(B_Q0 + st));
                 for (int c = 0; c < nvc; ++c)
-                    tma_load_3d(doa + c * 16384, &tm_do, c * 64, it.group * G, row0, bar(B_Q));
-                ok = mbar_wait(bar(B_Q), mi & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x32);
-                for (int hf = 0; hf < 2 && ok; ++hf) {
-                    const int step = mi * 2 + hf;
-                    tc_fence_after();
-                    for (int ks = 0; ks < p.d1 / 16; ++ks) {   // S^T = K Q^T over 64 query rows
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        umma_ss(tmem + 384, sdesc_sw128(ka + off, 16, 1024),
-                                sdesc_sw128(qa + off + hf * 8192, 16, 1024), id_s, ks > 0 ? 1u : 0u);
-                    }
-                    if (do_dk)
-                        for (int ks = 0; ks < p.d2 / 16; ++ks) {   // dP^T = V dO^T
-                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            umma_ss(tmem + 448, sdesc_sw128(va + off, 16, 1024),
-                                    sdesc_sw128(doa + off + hf * 8192, 16, 1024), id_s, ks > 0 ? 1u : 0u);
-                        }
-                    umma_commit(bar(B_S));
-                    ok = mbar_wait(bar(B_P), step & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x33);
+                    tma_load_3d(ds0 + c * 16384, &tm_do, c * 64, it.group * G, row0, bar(B_Q0 + st));
+            };
+            int loaded = 0;   // M-tiles whose loads have been issued
+            auto ensure_loaded = [&](int m) {
+                while (ok && loaded <= m && loaded < n_mt) {
+                    const int st = loaded % p.nst;
+                    if (loaded >= p.nst)
+                        ok = mbar_wait(bar(B_QE0 + st), ((loaded / p.nst) - 1) & 1, sm.abort_flag, p.err,
+                                       kErrTimeoutBase + 0x37);
                     if (!ok) break;
-                    tc_fence_after();
-                    for (int ks = 0; ks < 64 / 16; ++ks) {
-                        // the 64 query rows of the half are the contraction dimension: the
-                        // row-major dO / Q chunks serve as MN-major operands
-                        if (do_dv)
-                            umma_ts(tmem, tmem + 384 + ks * 8, sdesc_sw128(doa + hf * 8192 + ks * 2048, 16384, 1024),
-                                    id_v, (step > 0 || ks > 0) ? 1u : 0u);
-                        if (do_dk)
-                            umma_ts(tmem + p.col_dk, tmem + 448 + ks * 8,
-                                    sdesc_sw128(qa + hf * 8192 + ks * 2048, 16384, 1024), id_k,
-                                    (step > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    umma_commit(bar(B_MMA));
-                    ok = mbar_wait(bar(B_MMA), step & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x34);
+                    load_q(loaded++);
                 }
+            };
+            ok = mbar_wait(bar(B_KV0), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x31);
+            // Steps s = 2 mi + hf (halves of 64 query rows).  Step s uses score buffer
+            // s % nsb (S^T at sb_col, dP^T at sb_col + 64).  With two buffers, S of step s + 1
+            // is issued before the dV/dK of step s, so it runs while step s's softmax works;
+            // the tensor core executes one thread's MMAs in issue order, so S of step s + 2
+            // cannot overwrite P / dS of step s before its dV/dK has read them.
+            const int nsb = p.nsb;
+            auto sb_col = [&](int b) { return b == 0 ? 384u : 256u; };
+            auto issue_s = [&](int step) {
+                const int mi = step >> 1, hf = step & 1, st = mi % p.nst, b = step % nsb;
+                if (hf == 0) {
+                    ensure_loaded(mi);
+                    ok = ok && mbar_wait(bar(B_Q0 + st), (mi / p.nst) & 1, sm.abort_flag, p.err,
+                                         kErrTimeoutBase + 0x32);
+                }
+                if (!ok) return;
+                const uint32_t qs = qa + st * p.stage_bytes, ds = doa + st * p.stage_bytes;
+                tc_fence_after();
+                for (int ks = 0; ks < p.d1 / 16; ++ks) {   // S^T = K Q^T over 64 query rows
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_ss(tmem + sb_col(b), sdesc_sw128(ka + off, 16, 1024),
+                            sdesc_sw128(qs + off + hf * 8192, 16, 1024), id_s, ks > 0 ? 1u : 0u);
+                }
+                if (do_dk)
+                    for (int ks = 0; ks < p.d2 / 16; ++ks) {   // dP^T = V dO^T
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        umma_ss(tmem + sb_col(b) + 64, sdesc_sw128(va + off, 16, 1024),
+                                sdesc_sw128(ds + off + hf * 8192, 16, 1024), id_s, ks > 0 ? 1u : 0u);
+                    }
+                umma_commit(bar(B_S0 + b));
+            };
+            auto issue_d = [&](int step) {
+                const int mi = step >> 1, hf = step & 1, st = mi % p.nst, b = step % nsb;
+                ok = ok && mbar_wait(bar(B_P0 + b), (step / nsb) & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x33);
+                if (!ok) return;
+                const uint32_t qs = qa + st * p.stage_bytes, ds = doa + st * p.stage_bytes;
+                tc_fence_after();
+                for (int ks = 0; ks < 64 / 16; ++ks) {
+                    // the 64 query rows of the half are the contraction dimension: the
+                    // row-major dO / Q chunks serve as MN-major operands
+                    if (do_dv)
+                        umma_ts(tmem, tmem + sb_col(b) + ks * 8, sdesc_sw128(ds + hf * 8192 + ks * 2048, 16384, 1024),
+                                id_v, (step > 0 || ks > 0) ? 1u : 0u);
+                    if (do_dk)
+                        umma_ts(tmem + p.col_dk, tmem + sb_col(b) + 64 + ks * 8,
+                                sdesc_sw128(qs + hf * 8192 + ks * 2048, 16384, 1024), id_k,
+                                (step > 0 || ks > 0) ? 1u : 0u);
+                }
+                if (hf == 1) umma_commit(bar(B_QE0 + st));
+                // the next M-tile's load: its stage's last reader was issued a step ago
+                if (p.nst == 2 && hf == 0) ensure_loaded(mi + 1);
+            };
+            const int total = 2 * n_mt;
+            if (total > 0 && ok) issue_s(0);
+            for (int step = 0; step < total && ok; ++step) {
+                // S of the next step goes first when a second buffer holds it, except that with
+                // one Q/dO stage the next M-tile's load waits for this step's dV/dK to retire
+                const bool ahead = nsb == 2 && !(p.nst == 1 && ((step + 1) & 1) == 0);
+                if (ahead && step + 1 < total) issue_s(step + 1);
+                issue_d(step);
+                if (!ahead && step + 1 < total) issue_s(step + 1);
             }
-            mbar_arrive(bar(B_DONE));
+            // arrives once every MMA issued above has retired
+            umma_commit(bar(B_DONE));
         }
     } else {
         // one key (compressed block) of the tile per thread
@@ -399,27 +461,38 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int kb = it.kt * kKV + kr;   // block index inside the sequence
         const bool kvalid = kb < it.n_cmp;
         const float c2 = p.scale_log2;
-        for (int mi = 0; mi < n_mt; ++mi) {
+        // this thread's row kr of M-tile mi: its statistics and visible count
+        auto row_of = [&](int mi, float2& info, int& nv) {
             const int row0 = it.q_row0 + mi * TT;
-            named_bar_sync(1, 128);   // the previous M-tile's rows are no longer read
-            {
-                const int tok = kr / G, h = kr % G;
-                const bool valid = kr < TT * G && row0 + tok < it.q_end;
-                const int tpos = it.t0 + (row0 - it.q_row0) + tok;
-                rinfo[kr] = valid ? p.rowinfo[(size_t)(row0 + tok) * p.n1 + (size_t)it.group * G + h]
-                                  : make_float2(INFINITY, 0.f);
-                rnv[kr] = valid ? nvis_at(tpos, p.l, p.d, it.n_cmp) : 0;
-            }
+            const int tok = kr / G, h = kr % G;
+            const bool valid = kr < TT * G && row0 + tok < it.q_end;
+            const int tpos = it.t0 + (row0 - it.q_row0) + tok;
+            info = valid ? p.rowinfo[(size_t)(row0 + tok) * p.n1 + (size_t)it.group * G + h]
+                         : make_float2(INFINITY, 0.f);
+            nv = valid ? nvis_at(tpos, p.l, p.d, it.n_cmp) : 0;
+        };
+        if (n_mt > 0) row_of(0, rinfo2[kr], rnv2[kr]);
+        for (int mi = 0; mi < n_mt; ++mi) {
+            // buffer mi & 1 is complete, and M-tile mi - 1 (the other buffer) is no
+            // longer read by anyone
             named_bar_sync(1, 128);
+            const float2* rinfo = rinfo2 + (mi & 1) * 128;
+            const int* rnv = rnv2 + (mi & 1) * 128;
+            // the next M-tile's row, loaded now and stored after this M-tile's work
+            float2 nxt_info = make_float2(INFINITY, 0.f);
+            int nxt_nv = 0;
+            if (mi + 1 < n_mt) row_of(mi + 1, nxt_info, nxt_nv);
             for (int hf = 0; hf < 2; ++hf) {
                 const int step = mi * 2 + hf;
-                mbar_wait(bar(B_S), step & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x35);
+                const int b = step % p.nsb;
+                const uint32_t scol = b == 0 ? 384u : 256u;   // S^T of this step's buffer, dP^T at + 64
+                mbar_wait(bar(B_S0 + b), (step / p.nsb) & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x35);
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < 2; ++c) {
                     uint32_t rs[32], rp[32];
-                    tmem_ld32(tmem + lane_off + 384 + c * 32, rs);
-                    if (do_dk) tmem_ld32(tmem + lane_off + 448 + c * 32, rp);
+                    tmem_ld32(tmem + lane_off + scol + c * 32, rs);
+                    if (do_dk) tmem_ld32(tmem + lane_off + scol + 64 + c * 32, rp);
                     tmem_wait_ld_regs<32>(rs);
                     if (do_dk) tmem_wait_ld_regs<32>(rp);
                     uint32_t ppk[16], dpk[16];
@@ -435,13 +508,17 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                             dpk[e >> 1] = pk2<T>(v0 ? p0 * (__uint_as_float(rp[e]) - i0.y) : 0.f,
                                                  v1 ? p1 * (__uint_as_float(rp[e + 1]) - i1.y) : 0.f);
                     }
-                    if (do_dv) tmem_st16(tmem + lane_off + 384 + c * 16, ppk);
-                    if (do_dk) tmem_st16(tmem + lane_off + 448 + c * 16, dpk);
+                    if (do_dv) tmem_st16(tmem + lane_off + scol + c * 16, ppk);
+                    if (do_dk) tmem_st16(tmem + lane_off + scol + 64 + c * 16, dpk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_P));
+                if (lane == 0) mbar_arrive(bar(B_P0 + b));
+            }
+            if (mi + 1 < n_mt) {
+                rinfo2[((mi + 1) & 1) * 128 + kr] = nxt_info;
+                rnv2[((mi + 1) & 1) * 128 + kr] = nxt_nv;
             }
         }
         mbar_wait(bar(B_DONE), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x36);

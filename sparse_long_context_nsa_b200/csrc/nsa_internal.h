@@ -156,9 +156,13 @@ struct Params {
     float* part;             // partial slots of dK/dV: [slot][128][D2 | D1] fp32
     int mode;                // dK/dV kernel: bit 0 dV, bit 1 dK
     int col_dk;              // tensor-memory column of the dK accumulator
+    int nsb;                 // dK/dV kernel: score buffers (2 when the accumulators end by column 256)
     int dtype, n1, n2, d1, d2, G, tok_per_tile, l, d;
     float scale, scale_log2;
+    // shared memory (byte offsets from a 1024-aligned base) of the launched kernel: stage 0 of
+    // each operand; the ring's stages (Q/dO for dK/dV, K/V for dQ) are stage_bytes apart
     int off_q, off_do, off_k, off_v, off_row, off_bar, smem_bytes;
+    int nst, stage_bytes;
 };
 
 cudaError_t launch_prep(const void* out, const void* dout, const float* smax, const float* ssum, float2* rowinfo,
