@@ -10,6 +10,8 @@
  *                           ("mindspore.ops.nsa_compress_attention", steps 1-7);
  *   nsa_compress_attention_masked  the same with the optional atten_mask /
  *                           topk_mask of the page's keyword arguments
+ *   nsa_compress_attention_paged   the same over a paged compressed K/V cache
+ *                           (decode)
  *   nsa_select_attention    attention over the raw K/V blocks that top-k lists
  *                           ("lite_boost.ops.rain_fusion_attention");
  *   nsa_compress_attention_backward, nsa_compress_backward
@@ -175,6 +177,34 @@ nsa_status_t nsa_compress_attention(
  * NSA_ERR_INVALID_ARG.  With both masks NULL the call is
  * nsa_compress_attention.
  */
+/*
+ * nsa_compress_attention over a paged compressed K/V cache (the block_table of
+ * "lite_boost.ops.rain_fusion_attention", applied to the compressed blocks):
+ * sequence b's compressed block i lives in row i % page_size of pool page
+ * block_table[b * max_pages_per_seq + i / page_size].  The decode shape -- one
+ * query per sequence (cu_seqlens_q = 1, 2, ..., batch), which by the query
+ * offset of step 1 sits at the last raw position the blocks cover -- is the
+ * main use; any query counts are accepted.  Outputs, workspace
+ * (nsa_compress_attention_workspace_size with the same arguments) and errors as
+ * nsa_compress_attention, whose results it reproduces bit for bit when the
+ * pages hold the same rows.
+ *   kcmp_pages, vcmp_pages  device (num_pages, page_size, N2, D1 / D2) dtype
+ *   block_table   device int32 (batch, max_pages_per_seq), 4-byte aligned.  An
+ *                 entry outside [0, num_pages) reads zeros (never faults).
+ *   cu_cmp_kv     host prefix sums of the sequences' compressed block counts
+ * Rows of a sequence's last page past its block count must hold finite values
+ * (they meet zero weights in P . V).  Constraints: page_size a multiple of 8
+ * that divides the KV tile (128 blocks when l'/d is 1, 2, 4 or 8; 96, 80 or
+ * 112 otherwise) -- NSA_ERR_UNSUPPORTED; a block table row too short for a
+ * sequence -- NSA_ERR_INVALID_ARG.
+ */
+nsa_status_t nsa_compress_attention_paged(
+    const void* q, const void* kcmp_pages, const void* vcmp_pages, int64_t num_pages, int page_size,
+    const int32_t* block_table, int max_pages_per_seq, float scale, int head_num, int l, int d, int lp,
+    int count, const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv, const int32_t* cu_sel_kv, int batch,
+    int n2, int d1, int d2, nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
+    float* softmax_max, float* softmax_sum, void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Workspace bytes of nsa_compress_attention_masked: that of the unmasked call
  * plus the bit-packed rows of each mask that is present (with_* non-zero).

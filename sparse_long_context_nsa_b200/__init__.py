@@ -36,6 +36,7 @@ EXPORTED = (
     "nsa_compress_attention",
     "nsa_compress_attention_masked",
     "nsa_compress_attention_masked_workspace_size",
+    "nsa_compress_attention_paged",
     "nsa_workspace_status",
     "nsa_compress_status",
     "nsa_compress_attention_noalloc",
@@ -100,6 +101,10 @@ def load(path: Optional[str] = None):
     lib.nsa_compress_attention_masked_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p, i32p, i32p,
                                                                  ci, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
     lib.nsa_compress_attention_masked_workspace_size.restype = ci
+    lib.nsa_compress_attention_paged.argtypes = [vp, vp, vp, ctypes.c_int64, ci, vp, ci, ctypes.c_float, ci, ci, ci,
+                                                 ci, ci, i32p, i32p, i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp,
+                                                 ctypes.c_size_t, vp]
+    lib.nsa_compress_attention_paged.restype = ci
     lib.nsa_workspace_status.argtypes = [vp, vp]
     lib.nsa_workspace_status.restype = ci
     lib.nsa_compress_status.argtypes = [vp]
@@ -724,3 +729,58 @@ def nsa_compress_backward(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.T
         workspace.numel(), _stream(stream))
     _raise(st, "nsa_compress_backward")
     return dk, dv, dw
+
+
+def nsa_compress_attention_paged(q: torch.Tensor, kcmp_pages: torch.Tensor, vcmp_pages: torch.Tensor,
+                                 block_table: torch.Tensor, scale: float, head_num: int, l: int, d: int, lp: int,
+                                 count: int, cu_seqlens_q, cu_cmp_kv, cu_sel_kv, out=None,
+                                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """nsa_compress_attention over a paged compressed K/V cache.
+
+    kcmp_pages (num_pages, page_size, N2, D1), vcmp_pages (num_pages, page_size,
+    N2, D2), block_table (batch, max_pages) int32 on the device: sequence b's
+    compressed block i is row i % page_size of page block_table[b, i // page_size].
+    Returns (attention_out, topk_indices, softmax_max, softmax_sum)."""
+    for t, nm in ((q, "q"), (kcmp_pages, "kcmp_pages"), (vcmp_pages, "vcmp_pages"), (block_table, "block_table")):
+        _dev(t, nm)
+    dt = _dtype_code(q)
+    if kcmp_pages.dtype != q.dtype or vcmp_pages.dtype != q.dtype:
+        raise TypeError("q and the page pools must share one dtype")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise TypeError("block_table must be a 2-D int32 tensor (batch, max_pages)")
+    if q.dim() != 3 or kcmp_pages.dim() != 4 or vcmp_pages.dim() != 4:
+        raise ValueError("q must be (T1, N1, D1) and the pools (num_pages, page_size, N2, D)")
+    t1, n1, d1 = q.shape
+    num_pages, page_size, n2, d1k = kcmp_pages.shape
+    d2 = vcmp_pages.shape[3]
+    if d1k != d1 or tuple(vcmp_pages.shape[:3]) != (num_pages, page_size, n2):
+        raise ValueError("kcmp_pages must be (P, page_size, N2, D1) and vcmp_pages (P, page_size, N2, D2)")
+    if int(head_num) != n1:
+        raise ValueError("head_num must equal the number of query heads")
+    cq, cc, cs = _cu(cu_seqlens_q), _cu(cu_cmp_kv), _cu(cu_sel_kv)
+    if not (cq.size == cc.size == cs.size == block_table.shape[0]):
+        raise ValueError("one prefix-sum entry and one block-table row per sequence")
+    if int(cq[-1]) > t1:
+        raise ValueError("cu_seqlens_q runs past the rows of q")
+    dev = q.device
+    _same_device(q, (kcmp_pages, "kcmp_pages"), (vcmp_pages, "vcmp_pages"), (block_table, "block_table"))
+    if out is None:
+        att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
+        tk = torch.empty(t1, n2, count, dtype=torch.int32, device=dev)
+        smax = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
+        ssum = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
+    else:
+        att, tk, smax, ssum = out
+        _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
+        _out(tk, (t1, n2, count), torch.int32, dev, "topk_indices")
+        _out(smax, (t1, n1, 8), torch.float32, dev, "softmax_max")
+        _out(ssum, (t1, n1, 8), torch.float32, dev, "softmax_sum")
+    ws_bytes = nsa_compress_attention_workspace_size(n1, n2, d1, d2, l, d, lp, count, cq, cc, cs)
+    workspace = _workspace(workspace, ws_bytes, dev)
+    st = load().nsa_compress_attention_paged(
+        q.data_ptr(), kcmp_pages.data_ptr(), vcmp_pages.data_ptr(), int(num_pages), int(page_size),
+        block_table.data_ptr(), int(block_table.shape[1]), float(scale), n1, int(l), int(d), int(lp), int(count),
+        _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(), tk.data_ptr(), smax.data_ptr(),
+        ssum.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _raise(st, "nsa_compress_attention_paged")
+    return att, tk, smax, ssum

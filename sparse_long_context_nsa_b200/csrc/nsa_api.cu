@@ -135,6 +135,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
 
     // score-row capacity (largest candidate count) and the longest KV walk
     int cap = 1, max_nkv = 0;
+    int64_t max_sq = 0;
     {
         int32_t pq = 0, pc = 0, ps = 0;
         for (int bq = 0; bq < batch; ++bq) {
@@ -142,6 +143,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
             const int n_cmp = cu_cmp[bq] - pc;
             const int n_sel = cu_sel[bq] - ps;
             const int64_t off = n_cmp > 0 ? std::max<int64_t>(0, (int64_t)(n_cmp - 1) * d + l - Sq) : 0;
+            max_sq = std::max(max_sq, Sq);
             if (Sq > 0) {
                 const int64_t tlast = Sq - 1 + off;
                 const int nv = nvis_host(tlast, l, d, n_cmp);
@@ -198,7 +200,9 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
     static const int kOrder[][2] = {{2, 4}, {2, 3}, {1, 4}, {1, 3}};
     static const int kOrder2[][2] = {{2, 2}, {1, 2}};
     bool fits = false;
-    const int np_hi = std::min(npipe_max, d2 <= 128 ? 2 : 1);
+    // a second pipeline needs a second M-tile of tokens: when every sequence's queries
+    // fit one M-tile (decode, few queries), one pipeline with two score buffers
+    const int np_hi = std::min(npipe_max, (d2 <= 128 && max_sq > pl.TT) ? 2 : 1);
     for (int np = np_hi; np >= 1 && !fits; --np)
         for (const auto& o : kOrder) {
             if ((fits = layout(np, o[0], o[1], true))) break;
@@ -255,6 +259,7 @@ nsa_status_t plan_attention(int head_num, int n2, int d1, int d2, int l, int d, 
                 t.n_sel = n_sel;
                 t.t0 = (int)(tok0 + off);
                 t.tloc0 = (int)tok0;
+                t.seq = bq;
                 const int nv = nvis_host(t.t0 + t.ntok - 1, l, d, n_cmp);
                 t.nkv = (nv + NKV - 1) / NKV;
                 for (int g = group_begin; g < g_end; ++g) {
@@ -727,7 +732,8 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
                                             int32_t* topk_indices, float* softmax_max, float* softmax_sum,
                                             void* workspace, size_t workspace_bytes, void* stream,
                                             int grid_cap = kMaxGrid, int npipe_max = 2, int group_begin = 0,
-                                            int group_count = -1) {
+                                            int group_count = -1, const int32_t* block_table = nullptr,
+                                            int bt_stride = 0, int page_rows = 0, int64_t num_pages = 0) {
     if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return NSA_ERR_INVALID_ARG;
     if (!q || !kcmp || !vcmp || !attention_out || !topk_indices || !softmax_max || !softmax_sum)
@@ -750,10 +756,19 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     const int64_t t1 = cu_seqlens_q[batch - 1];
     const int64_t tc = cu_cmp_kv[batch - 1];
     CUtensorMap tq, tk, tv;
-    if (!encode_tnd(&tq, q, dtype, d1, head_num, t1, pl.G, pl.TT) ||
-        !encode_tnd(&tk, kcmp, dtype, d1, n2, tc, 1, pl.nkv_cols) ||
-        !encode_tnd(&tv, vcmp, dtype, d2, n2, tc, 1, pl.nkv_cols))
+    if (block_table != nullptr) {
+        // pools of pages: boxes of one page; a KV tile is NKV / page_rows pages
+        if (page_rows < 8 || page_rows % 8 || pl.nkv_cols % page_rows) return NSA_ERR_UNSUPPORTED;
+        if (num_pages < 1 || num_pages * page_rows >= ((int64_t)1 << 31)) return NSA_ERR_INVALID_ARG;
+        if (!encode_tnd(&tq, q, dtype, d1, head_num, t1, pl.G, pl.TT) ||
+            !encode_tnd(&tk, kcmp, dtype, d1, n2, num_pages * page_rows, 1, page_rows) ||
+            !encode_tnd(&tv, vcmp, dtype, d2, n2, num_pages * page_rows, 1, page_rows))
+            return NSA_ERR_UNSUPPORTED;
+    } else if (!encode_tnd(&tq, q, dtype, d1, head_num, t1, pl.G, pl.TT) ||
+               !encode_tnd(&tk, kcmp, dtype, d1, n2, tc, 1, pl.nkv_cols) ||
+               !encode_tnd(&tv, vcmp, dtype, d2, n2, tc, 1, pl.nkv_cols)) {
         return NSA_ERR_UNSUPPORTED;
+    }
 
     // workspace: [header: error word][item list][score rows][importance scratch]
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
@@ -772,6 +787,10 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     p.tiles = reinterpret_cast<const AttnTile*>(ws + kWsHeader);
     p.num_tiles = (int)pl.tiles.size();
     p.err = reinterpret_cast<int*>(ws);
+    p.block_table = block_table;
+    p.bt_stride = bt_stride;
+    p.page_rows = page_rows;
+    p.pool_rows = (int)(num_pages * page_rows);
     p.score_gmem = pl.score_in_smem ? nullptr : reinterpret_cast<float*>(ws + off_score);
     p.band = reinterpret_cast<float*>(ws + off_score + pl.ws_score);
     p.capj = pl.capj;
@@ -841,6 +860,30 @@ nsa_status_t nsa_compress_attention(const void* q, const void* kcmp, const void*
     return compress_attention_impl(q, kcmp, vcmp, scale, head_num, l, d, lp, count, cu_seqlens_q, cu_cmp_kv,
                                    cu_sel_kv, batch, n2, d1, d2, dtype, nullptr, 0, nullptr, 0, attention_out,
                                    topk_indices, softmax_max, softmax_sum, workspace, workspace_bytes, stream);
+}
+
+nsa_status_t nsa_compress_attention_paged(const void* q, const void* kcmp_pages, const void* vcmp_pages,
+                                          int64_t num_pages, int page_size, const int32_t* block_table,
+                                          int max_pages_per_seq, float scale, int head_num, int l, int d, int lp,
+                                          int count, const int32_t* cu_seqlens_q, const int32_t* cu_cmp_kv,
+                                          const int32_t* cu_sel_kv, int batch, int n2, int d1, int d2,
+                                          nsa_dtype_t dtype, void* attention_out, int32_t* topk_indices,
+                                          float* softmax_max, float* softmax_sum, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+    if (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u)) return NSA_ERR_INVALID_ARG;
+    if (page_size < 1 || max_pages_per_seq < 1 || num_pages < 1) return NSA_ERR_INVALID_ARG;
+    nsa_status_t s = check_prefix(cu_cmp_kv, batch);
+    if (s != NSA_OK) return s;
+    // every sequence's compressed blocks must fit its row of the block table
+    for (int b = 0; b < batch; ++b) {
+        const int64_t nc = cu_cmp_kv[b] - (b ? cu_cmp_kv[b - 1] : 0);
+        if ((nc + page_size - 1) / page_size > max_pages_per_seq) return NSA_ERR_INVALID_ARG;
+    }
+    return compress_attention_impl(q, kcmp_pages, vcmp_pages, scale, head_num, l, d, lp, count, cu_seqlens_q,
+                                   cu_cmp_kv, cu_sel_kv, batch, n2, d1, d2, dtype, nullptr, 0, nullptr, 0,
+                                   attention_out, topk_indices, softmax_max, softmax_sum, workspace,
+                                   workspace_bytes, stream, kMaxGrid, 2, 0, -1, block_table, max_pages_per_seq,
+                                   page_size, num_pages);
 }
 
 nsa_status_t nsa_compress_attention_masked_workspace_size(int head_num, int n2, int d1, int d2, int l, int d,

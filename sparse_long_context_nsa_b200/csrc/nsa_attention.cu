@@ -344,7 +344,11 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t k_bytes = (uint32_t)(nqc * 64 * NKV * 2);
             const uint32_t v_bytes = (uint32_t)(nvc * 64 * NKV * 2);
             bool ok = true;
-            auto load_kv = [&](bool is_v, int g, int row) {
+            // K or V tile kt of item t: NKV compressed rows from the sequence's contiguous
+            // rows, or, with a block table, page by page (an entry past the sequence's pages
+            // reads rows beyond the pool, which the copy fills with zeros)
+            auto load_kv = [&](bool is_v, const AttnTile& t, int kt) {
+                const int g = t.group;
                 const int slot = item % nslot;
                 const uint32_t ph = (item / nslot) & 1;
                 ok = ok && mbar_wait(bar(B_SLOT_EMPTY0 + slot), ph ^ 1, abort_flag, p.err, kErrTimeoutBase + 2);
@@ -353,8 +357,20 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t dst = ring_addr + slot * p.slot_bytes;
                 mbar_arrive_expect_tx(fb, is_v ? v_bytes : k_bytes);
                 const int nc = is_v ? nvc : nqc;
-                for (int c = 0; c < nc; ++c)
-                    tma_load_3d(dst + c * NKV * 128, is_v ? &tm_v : &tm_k, c * 64, g, row, fb);
+                const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+                if (p.block_table == nullptr) {
+                    const int row = t.cmp_row0 + kt * NKV;
+                    for (int c = 0; c < nc; ++c) tma_load_3d(dst + c * NKV * 128, map, c * 64, g, row, fb);
+                } else {
+                    const int pr = p.page_rows, npg = (t.n_cmp + pr - 1) / pr;
+                    for (int pg = 0; pg < NKV / pr; ++pg) {
+                        const int logical = kt * (NKV / pr) + pg;
+                        const int row = logical < npg ? p.block_table[(size_t)t.seq * p.bt_stride + logical] * pr
+                                                      : p.pool_rows;
+                        for (int c = 0; c < nc; ++c)
+                            tma_load_3d(dst + c * NKV * 128 + pg * pr * 128, map, c * 64, g, row, fb);
+                    }
+                }
                 ++item;
             };
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
@@ -371,10 +387,10 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tma_load_3d_hint(qdst + pp * q_tile_stride + c * 16384, &tm_q, c * 64, t.group * G,
                                          t.q_row0 + pp * TT, bar(B_Q_FULL0 + qb), q_policy);
                 // K_0, then K_{i+1} ahead of V_i: the order the MMA issuer consumes them
-                if (t.nkv > 0 && ok) load_kv(false, t.group, t.cmp_row0);
+                if (t.nkv > 0 && ok) load_kv(false, t, 0);
                 for (int i = 0; i < t.nkv && ok; ++i) {
-                    if (i + 1 < t.nkv) load_kv(false, t.group, t.cmp_row0 + (i + 1) * NKV);
-                    load_kv(true, t.group, t.cmp_row0 + i * NKV);
+                    if (i + 1 < t.nkv) load_kv(false, t, i + 1);
+                    load_kv(true, t, i);
                 }
             }
         } else if (warp == 13 && lane == 0) {

@@ -69,12 +69,18 @@ struct AttnTile {
     int t0;         // position of the first token (query offset applied)
     int nkv;        // KV tiles to visit
     int tloc0;      // query index of the first token inside its sequence (mask rows)
+    int seq;        // sequence index (block-table row)
 };
 
 struct AttnParams {
     const AttnTile* tiles;
     int num_tiles;
     int* err;               // device error word (workspace)
+    // paged compressed K/V: when block_table is set, sequence b's compressed rows
+    // j*page_rows .. live in pool page block_table[b * bt_stride + j] (the tensor
+    // maps cover the pools, pool_rows rows, with boxes of page_rows rows)
+    const int32_t* block_table;
+    int bt_stride, page_rows, pool_rows;
     // per-CTA scratch for the per-head importance values: for each pipeline,
     // two slots (consecutive items alternate) of `region` floats each.  A slot
     // holds the banded values chunk-major, [chunk][row 0..127][anchor of the
