@@ -20,6 +20,7 @@ independent batch, no collective on the data path).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -471,14 +472,75 @@ def run_ours(args, rank, world, local_rank):
                    gsample=gout[:min(int(wl.seqlens[0]), 16384), :wl.n1 // wl.n2].cpu())
         del grads, cgrads, bws, gout
 
+    dec = None
+    if not args.no_decode:
+        dec = time_decode(args, nsa, dev, rank, flush)
+
     side = None
     if not args.no_side:
         del flush
         side = time_side_case(args, nsa, dev, rank)
 
     return dict(wl=wl, K=K, step_ms=step_ms, att_ms=att_ms, cmp_ms=cmp_ms, t1=t1, wall=t_wall,
-                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk, side=side, x=x, bwd=bwd,
+                clocks=clk.result(), e2e=e2e, sel=sel, msk=msk, side=side, x=x, bwd=bwd, dec=dec,
                 launches_per_step=1 + 1 + (len(wl.seqlens) - 1) // 96)
+
+
+def decode_bytes(dw) -> float:
+    """bytes a decode step must move: every sequence's compressed K/V once, plus
+    q, attention_out, the statistics and the top-k lists."""
+    e = 2
+    kv = dw.batch * dw.n_cmp * dw.n2 * (dw.d1 + dw.d2) * e
+    io = dw.batch * dw.n1 * (dw.d1 + dw.d2) * e + dw.batch * dw.n1 * 16 * 4 + dw.batch * dw.n2 * dw.count * 4
+    return float(kv + io)
+
+
+def time_decode(args, nsa, dev, rank, flush):
+    """One decode step over a paged compressed cache (one query per sequence),
+    L2 flushed before every call."""
+    dw = workloads.DECODE_64x64K
+    dw = dataclasses.replace(dw, seed=dw.seed + rank)
+    x = dw.generate(device=str(dev))
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        dw.n1, dw.n2, dw.d1, dw.d2, dw.l, dw.d, dw.lp, dw.count, x["cu_seqlens_q"], x["cu_cmp_kv"], x["cu_sel_kv"]),
+        dtype=torch.uint8, device=dev)
+
+    def call():
+        return nsa.nsa_compress_attention_paged(x["q"], x["kcmp_pages"], x["vcmp_pages"], x["block_table"], dw.scale,
+                                                dw.n1, dw.l, dw.d, dw.lp, dw.count, x["cu_seqlens_q"],
+                                                x["cu_cmp_kv"], x["cu_sel_kv"], workspace=ws)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        call()
+    n = max(3, min(args.steps, args.decode_steps))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        evs[i][0].record()
+        res = call()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    if nsa.nsa_workspace_status(ws) != 0:
+        raise RuntimeError("device-side timeout in paged decode")
+    return dict(wl=dw, ms=float(np.mean([e[0].elapsed_time(e[1]) for e in evs])), steps=n, x=x, res=res)
+
+
+def decode_cpu_baseline(dw, x, nseq=16):
+    """The oracle as it stands on the first nseq sequences of the decode step
+    (their pages gathered into contiguous compressed tensors on the host)."""
+    import oracle
+    bt = x["block_table"].cpu().numpy()
+    kp, vp = x["kcmp_pages"].cpu(), x["vcmp_pages"].cpu()
+    kc = torch.cat([kp[bt[b]].reshape(-1, dw.n2, dw.d1)[:dw.n_cmp] for b in range(nseq)])
+    vc = torch.cat([vp[bt[b]].reshape(-1, dw.n2, dw.d2)[:dw.n_cmp] for b in range(nseq)])
+    q = x["q"][:nseq].cpu()
+    t = time.perf_counter()
+    oracle.compress_attention(q, kc, vc, dw.scale, dw.l, dw.d, dw.lp, dw.count, x["cu_seqlens_q"][:nseq],
+                              x["cu_cmp_kv"][:nseq], x["cu_sel_kv"][:nseq])
+    sec = time.perf_counter() - t
+    return {"value": nseq / sec, "unit": "decode tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{nseq} of {dw.batch} sequences, all heads, {sec:.2f} s"}
 
 
 def time_side_case(args, nsa, dev, rank):
@@ -795,6 +857,8 @@ def main():
     ap.add_argument("--select-steps", type=int, default=20)
     ap.add_argument("--select-cpu-budget", type=float, default=8.0)
     ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--no-decode", action="store_true", help="skip the paged decode measurement")
+    ap.add_argument("--decode-steps", type=int, default=20)
     ap.add_argument("--backward-steps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -842,6 +906,9 @@ def main():
         dev0 = torch.device("cuda", local_rank)
         sel_ms = max_over_ranks([r["sel"]["ms"]], dev0, world)[0]
         sel_flops_all = sum_over_ranks([select_flops(wl, r["sel"]["keys"])], dev0, world)[0]
+    dec_ms = None
+    if r["dec"] is not None:
+        dec_ms = max_over_ranks([r["dec"]["ms"]], torch.device("cuda", local_rank), world)[0]
     bwd_att_ms = bwd_cmp_ms = None
     if r["bwd"] is not None:
         bwd_att_ms, bwd_cmp_ms = max_over_ranks([r["bwd"]["att_ms"], r["bwd"]["cmp_ms"]],
@@ -960,6 +1027,23 @@ def main():
                                  "peak_source": f"{peak_src} hbm_gbs"}},
                 "gpu_launches": r["bwd"]["launches"] * r["bwd"]["steps"],
                 "cpu_baseline": (backward_cpu_baseline(wl, r["x"], r["bwd"]["gsample"])
+                                 if (not args.no_cpu_baseline and world == 1) else None)}
+        if r["dec"] is not None:
+            dw = r["dec"]["wl"]
+            db = decode_bytes(dw)
+            dg = db / (dec_ms * 1e-3) / 1e9
+            dfl = 2.0 * (dw.d1 + dw.d2) * dw.n1 * dw.n_cmp * dw.batch
+            line["paged_decode"] = {
+                "what": f"nsa_compress_attention_paged: {dw.batch} sequences x 1 query against {dw.n_cmp} compressed "
+                        f"blocks each ({dw.raw_len} raw tokens), N1={dw.n1}, N2={dw.n2}, D={dw.d1}, pages of "
+                        f"{dw.page_size} blocks in a permuted pool; L2 flushed before every call",
+                "workload": dw.name, "ms": dec_ms, "steps": r["dec"]["steps"],
+                "decode_tok_s": world * dw.batch / (dec_ms * 1e-3), "gbs": dg, "bytes": db,
+                "tflops": dfl / (dec_ms * 1e-3) / 1e12,
+                "roofline": {"bound": "hbm", "achieved": dg, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": dg / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} hbm_gbs"},
+                "gpu_launches": r["dec"]["steps"],
+                "cpu_baseline": (decode_cpu_baseline(dw, r["dec"]["x"])
                                  if (not args.no_cpu_baseline and world == 1) else None)}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -146,3 +146,24 @@ def test_paged_refuses_bad_arguments(nsa):
     with pytest.raises(ValueError):   # a block-table row too short for the sequence's pages
         nsa.nsa_compress_attention_paged(q, kp.cuda(), vp.cuda(), bt[:, :-1].contiguous().cuda(), wl.scale,
                                          wl.n1, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+
+
+def test_decode_workload_full_size_sampled_sequences(nsa):
+    # the bench's decode step at full size; 8 of its 64 sequences against the oracle
+    dw = workloads.DECODE_64x64K
+    x = dw.generate(device="cuda")
+    res = nsa.nsa_compress_attention_paged(x["q"], x["kcmp_pages"], x["vcmp_pages"], x["block_table"], dw.scale,
+                                           dw.n1, dw.l, dw.d, dw.lp, dw.count, x["cu_seqlens_q"], x["cu_cmp_kv"],
+                                           x["cu_sel_kv"])
+    picks = [0, 9, 17, 31, 40, 52, 60, 63]
+    bt = x["block_table"].cpu().numpy()
+    kp, vp = x["kcmp_pages"].cpu(), x["vcmp_pages"].cpu()
+    kc = torch.cat([kp[bt[b]].reshape(-1, dw.n2, dw.d1)[:dw.n_cmp] for b in picks])
+    vc = torch.cat([vp[bt[b]].reshape(-1, dw.n2, dw.d2)[:dw.n_cmp] for b in picks])
+    n = len(picks)
+    ref = oracle.compress_attention(x["q"][picks].cpu(), kc, vc, dw.scale, dw.l, dw.d, dw.lp, dw.count,
+                                    np.arange(1, n + 1, dtype=np.int32),
+                                    (np.arange(1, n + 1) * dw.n_cmp).astype(np.int32),
+                                    x["cu_sel_kv"][:n])
+    sub = [t[picks] for t in res]
+    check_attention(sub, ref, dw.count)

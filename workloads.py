@@ -128,6 +128,53 @@ def grad_output(wl: Workload, device: str = "cpu") -> torch.Tensor:
     return torch.randn(t1, wl.n1, wl.d2, generator=g, device=device, dtype=torch.float32).to(wl.torch_dtype)
 
 
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """One query per sequence against a paged compressed K/V cache."""
+    name: str
+    batch: int
+    raw_len: int            # raw tokens of every sequence
+    n1: int
+    n2: int
+    d1: int
+    d2: int
+    l: int
+    d: int
+    lp: int
+    count: int
+    page_size: int
+    scale: float
+    dtype: str = "bf16"
+    seed: int = 6
+    std: float = 0.25       # of the compressed keys and values drawn directly
+
+    @property
+    def n_cmp(self) -> int:
+        return 0 if self.raw_len < self.l else (self.raw_len - self.l) // self.d + 1
+
+    def generate(self, device: str = "cpu"):
+        """q (batch, N1, D1); page pools kcmp / vcmp (pages, page_size, N2, D); a
+        block table (batch, pages per sequence) int32 whose pages are a seeded
+        permutation of the pool; host prefix sums cu_seqlens_q (1 .. batch),
+        cu_cmp_kv and cu_sel_kv.  The compressed cache is drawn directly
+        (randn * std): its values play no part in the work done."""
+        g = torch.Generator(device=device)
+        g.manual_seed(self.seed)
+        dt = torch.bfloat16 if self.dtype == "bf16" else torch.float16
+        ppseq = -(-self.n_cmp // self.page_size)
+        npages = self.batch * ppseq
+        q = torch.randn(self.batch, self.n1, self.d1, generator=g, device=device).to(dt)
+        kp = (torch.randn(npages, self.page_size, self.n2, self.d1, generator=g, device=device) * self.std).to(dt)
+        vp = (torch.randn(npages, self.page_size, self.n2, self.d2, generator=g, device=device) * self.std).to(dt)
+        perm = torch.randperm(npages, generator=g, device=device).to(torch.int32)
+        table = perm.view(self.batch, ppseq).contiguous()
+        b = np.arange(1, self.batch + 1, dtype=np.int64)
+        nsel = -(-self.raw_len // self.lp)
+        return {"q": q, "kcmp_pages": kp, "vcmp_pages": vp, "block_table": table,
+                "cu_seqlens_q": b.astype(np.int32), "cu_cmp_kv": (b * self.n_cmp).astype(np.int32),
+                "cu_sel_kv": (b * nsel).astype(np.int32)}
+
+
 def _varlen_lengths() -> tuple:
     lens = np.random.default_rng(1).integers(2048, 32768, 8, endpoint=True)
     return tuple(int(x) for x in lens)
@@ -152,6 +199,11 @@ SHORTQ_4x64K = Workload("compress_t262144_shortq_4x128_n64_n8_d128",
 # a device footprint near 1 GB, small enough for a full ncu capture.
 PROFILE_32K = Workload("single_s32768_n64_n4_d128", (32768,), 64, 4, 128, 128,
                        32, 16, 64, 16, 128 ** -0.5, "bf16", seed=5)
+
+# Decode: 64 sequences of 65536 raw tokens (1023 compressed blocks each, the
+# short-query workload's block geometry), one query each, 64-block pages.
+DECODE_64x64K = DecodeWorkload("decode_b64_s65536_n64_n8_d128_page64", 64, 65536, 64, 8, 128, 128, 128, 64, 128,
+                               32, 64, 128 ** -0.5)
 
 WORKLOADS = {w.name: w for w in (TINY, SINGLE_16K, VARLEN_8, LONG_128K, SHORTQ_4x64K, PROFILE_32K)}
 BY_INDEX = [TINY, SINGLE_16K, VARLEN_8, LONG_128K, SHORTQ_4x64K]
