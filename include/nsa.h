@@ -10,8 +10,9 @@
  *                           ("mindspore.ops.nsa_compress_attention", steps 1-7);
  *   nsa_compress_attention_masked  the same with the optional atten_mask /
  *                           topk_mask of the page's keyword arguments
- *   nsa_compress_attention_paged   the same over a paged compressed K/V cache
- *                           (decode)
+ *   nsa_compress_paged, nsa_compress_attention_paged
+ *                           the compression into, and the attention over, a
+ *                           paged compressed K/V cache (decode)
  *   nsa_select_attention    attention over the raw K/V blocks that top-k lists
  *                           ("lite_boost.ops.rain_fusion_attention");
  *   nsa_compress_attention_backward, nsa_compress_backward
@@ -95,6 +96,28 @@ nsa_status_t nsa_compress_out_len(const int32_t* cu_seqlens, int batch, int l, i
 nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, int d,
                           const int32_t* cu_seqlens, int batch, int n2, int d1, int d2,
                           nsa_dtype_t dtype, void* kcmp, void* vcmp, void* stream);
+
+/*
+ * nsa_compress into a paged compressed cache: block i of sequence b goes to row
+ * i % page_size of pool page block_table[b * max_pages_per_seq + i / page_size].
+ * Only blocks first_block[b] .. n_cmp_b - 1 are computed (first_block NULL: all),
+ * so a decode step compresses just the window its new token completed
+ * (first_block[b] = n_cmp_b - 1 when (S_b - l) % d == 0, else n_cmp_b) and
+ * nsa_compress_attention_paged then reads the cache.  Same arithmetic as
+ * nsa_compress (bitwise equal rows).
+ *   kcmp_pages, vcmp_pages  device (num_pages, page_size, N2, D1 / D2), written
+ *   block_table   device int32 (batch, max_pages_per_seq); an entry outside
+ *                 [0, num_pages) is never written through: the store is skipped
+ *                 and nsa_compress_status reports NSA_ERR_INVALID_ARG
+ *   first_block   host int32 [batch] or NULL; 0 <= first_block[b] <= n_cmp_b
+ * Other arguments and constraints as nsa_compress; a block table row too short
+ * for a sequence's blocks is NSA_ERR_INVALID_ARG.
+ */
+nsa_status_t nsa_compress_paged(const void* k, const void* v, const void* w, int l, int d,
+                                const int32_t* cu_seqlens, int batch, int n2, int d1, int d2,
+                                nsa_dtype_t dtype, void* kcmp_pages, void* vcmp_pages, int64_t num_pages,
+                                int page_size, const int32_t* block_table, int max_pages_per_seq,
+                                const int32_t* first_block, void* stream);
 
 /*
  * Workspace bytes that nsa_compress_attention needs for these arguments.
@@ -405,7 +428,9 @@ nsa_status_t nsa_workspace_status(const void* workspace, void* stream);
 
 /*
  * Device-side error word of the compress kernel on the current device
- * (0 = none).  Synchronises `stream`.  NSA_ERR_TIMEOUT when a wait gave up.
+ * (0 = none).  Synchronises `stream`.  NSA_ERR_TIMEOUT when a wait gave up,
+ * NSA_ERR_INVALID_ARG when nsa_compress_paged met a block-table entry outside
+ * its pool.
  */
 nsa_status_t nsa_compress_status(void* stream);
 

@@ -37,6 +37,7 @@ EXPORTED = (
     "nsa_compress_attention_masked",
     "nsa_compress_attention_masked_workspace_size",
     "nsa_compress_attention_paged",
+    "nsa_compress_paged",
     "nsa_workspace_status",
     "nsa_compress_status",
     "nsa_compress_attention_noalloc",
@@ -105,6 +106,9 @@ def load(path: Optional[str] = None):
                                                  ci, ci, i32p, i32p, i32p, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp,
                                                  ctypes.c_size_t, vp]
     lib.nsa_compress_attention_paged.restype = ci
+    lib.nsa_compress_paged.argtypes = [vp, vp, vp, ci, ci, i32p, ci, ci, ci, ci, ci, vp, vp, ctypes.c_int64, ci, vp,
+                                       ci, i32p, vp]
+    lib.nsa_compress_paged.restype = ci
     lib.nsa_workspace_status.argtypes = [vp, vp]
     lib.nsa_workspace_status.restype = ci
     lib.nsa_compress_status.argtypes = [vp]
@@ -784,3 +788,44 @@ def nsa_compress_attention_paged(q: torch.Tensor, kcmp_pages: torch.Tensor, vcmp
         ssum.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream))
     _raise(st, "nsa_compress_attention_paged")
     return att, tk, smax, ssum
+
+
+def nsa_compress_paged(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tensor, l: int, d: int, cu_seqlens,
+                       kcmp_pages: torch.Tensor, vcmp_pages: Optional[torch.Tensor], block_table: torch.Tensor,
+                       first_block=None, stream=None):
+    """Compress windows first_block[b] .. n_cmp_b - 1 of every sequence (all when
+    first_block is None) into the paged pools kcmp_pages / vcmp_pages
+    (num_pages, page_size, N2, D), in place, through block_table (batch,
+    max_pages) int32."""
+    for t, nm in ((k, "k"), (w, "w"), (kcmp_pages, "kcmp_pages"), (block_table, "block_table")):
+        _dev(t, nm)
+    dt = _dtype_code(k)
+    if w.dtype != k.dtype or kcmp_pages.dtype != k.dtype or (v is not None and v.dtype != k.dtype):
+        raise TypeError("k, v, w and the pools must share one dtype")
+    if (v is None) != (vcmp_pages is None):
+        raise ValueError("v and vcmp_pages go together")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise TypeError("block_table must be a 2-D int32 tensor (batch, max_pages)")
+    t2, n2, d1 = k.shape
+    num_pages, page_size = int(kcmp_pages.shape[0]), int(kcmp_pages.shape[1])
+    if tuple(kcmp_pages.shape[2:]) != (n2, d1):
+        raise ValueError("kcmp_pages must be (num_pages, page_size, N2, D1)")
+    d2 = d1
+    if v is not None:
+        _dev(v, "v")
+        _dev(vcmp_pages, "vcmp_pages")
+        d2 = v.shape[2]
+        if tuple(vcmp_pages.shape) != (num_pages, page_size, n2, d2):
+            raise ValueError("vcmp_pages must be (num_pages, page_size, N2, D2)")
+    cu = _cu(cu_seqlens)
+    if int(cu[-1]) > t2 or block_table.shape[0] != cu.size:
+        raise ValueError("cu_seqlens runs past k, or the block table has the wrong number of rows")
+    fb = None if first_block is None else _cu(first_block)
+    _same_device(k, (w, "w"), (v, "v"), (kcmp_pages, "kcmp_pages"), (vcmp_pages, "vcmp_pages"),
+                 (block_table, "block_table"))
+    st = load().nsa_compress_paged(
+        k.data_ptr(), v.data_ptr() if v is not None else None, w.data_ptr(), int(l), int(d), _ip(cu), cu.size, n2,
+        d1, d2, dt, kcmp_pages.data_ptr(), vcmp_pages.data_ptr() if v is not None else None, num_pages, page_size,
+        block_table.data_ptr(), int(block_table.shape[1]), _ip(fb) if fb is not None else None, _stream(stream))
+    _raise(st, "nsa_compress_paged")
+    return kcmp_pages, vcmp_pages

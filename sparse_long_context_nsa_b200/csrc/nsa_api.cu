@@ -610,9 +610,16 @@ nsa_status_t nsa_compress_out_len(const int32_t* cu_seqlens, int batch, int l, i
     return NSA_OK;
 }
 
-nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, int d, const int32_t* cu_seqlens,
-                          int batch, int n2, int d1, int d2, nsa_dtype_t dtype, void* kcmp, void* vcmp,
-                          void* stream) {
+}  // extern "C"
+
+// Compression of blocks first_block[b] .. n_cmp_b - 1 of every sequence (all
+// of them when first_block is null), into contiguous rows or, with a block
+// table, into pages.
+static nsa_status_t compress_impl(const void* k, const void* v, const void* w, int l, int d,
+                                  const int32_t* cu_seqlens, int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+                                  void* kcmp, void* vcmp, void* stream, const int32_t* first_block = nullptr,
+                                  const int32_t* block_table = nullptr, int bt_stride = 0, int page_rows = 0,
+                                  int64_t num_pages = 0) {
     // constraint lists of aclnnNsaCompress and mindspore.ops.nsa_compress_attention
     if (dtype != NSA_BF16 && dtype != NSA_FP16) return NSA_ERR_INVALID_ARG;
     if (k == nullptr || w == nullptr || kcmp == nullptr) return NSA_ERR_INVALID_ARG;
@@ -649,7 +656,11 @@ nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, in
     {
         int32_t prev = 0;
         for (int b = 0; b < batch; ++b) {
-            total_out += ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
+            const int64_t nc = ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
+            const int64_t f = first_block ? first_block[b] : 0;
+            if (f < 0 || f > nc) return NSA_ERR_INVALID_ARG;
+            if (block_table && (nc + page_rows - 1) / page_rows > bt_stride) return NSA_ERR_INVALID_ARG;
+            total_out += nc - f;
             prev = cu_seqlens[b];
         }
     }
@@ -673,6 +684,10 @@ nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, in
     p.dtype = dtype == NSA_BF16 ? 0 : 1;
     p.chunk = chunk;
     p.rows_per_stage = rs;
+    p.block_table = block_table;
+    p.bt_stride = bt_stride;
+    p.page_rows = page_rows;
+    p.num_pages = (int)num_pages;
     const int threads = (int)(((rowelems / 8) + 31) / 32 * 32);
 
     int32_t prev_raw = 0;
@@ -688,7 +703,9 @@ nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, in
             q.raw_start = prev_raw;
             q.cmp_start = (int)cmp_prev;
             q.ncmp = (int)nc;
-            q.nchunks = (int)((nc + chunk - 1) / chunk);
+            q.first = first_block ? first_block[b] : 0;
+            q.seq = b;
+            q.nchunks = (int)((nc - q.first + chunk - 1) / chunk);
             chunks += q.nchunks;
             q.chunk_end = chunks;
             prev_raw = cu_seqlens[b];
@@ -702,9 +719,30 @@ nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, in
     return NSA_OK;
 }
 
+extern "C" {
+
+nsa_status_t nsa_compress(const void* k, const void* v, const void* w, int l, int d, const int32_t* cu_seqlens,
+                          int batch, int n2, int d1, int d2, nsa_dtype_t dtype, void* kcmp, void* vcmp,
+                          void* stream) {
+    return compress_impl(k, v, w, l, d, cu_seqlens, batch, n2, d1, d2, dtype, kcmp, vcmp, stream);
+}
+
+nsa_status_t nsa_compress_paged(const void* k, const void* v, const void* w, int l, int d,
+                                const int32_t* cu_seqlens, int batch, int n2, int d1, int d2, nsa_dtype_t dtype,
+                                void* kcmp_pages, void* vcmp_pages, int64_t num_pages, int page_size,
+                                const int32_t* block_table, int max_pages_per_seq, const int32_t* first_block,
+                                void* stream) {
+    if (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u)) return NSA_ERR_INVALID_ARG;
+    if (page_size < 1 || max_pages_per_seq < 1 || num_pages < 1) return NSA_ERR_INVALID_ARG;
+    if (num_pages * page_size >= ((int64_t)1 << 31)) return NSA_ERR_INVALID_ARG;
+    return compress_impl(k, v, w, l, d, cu_seqlens, batch, n2, d1, d2, dtype, kcmp_pages, vcmp_pages, stream,
+                         first_block, block_table, max_pages_per_seq, page_size, num_pages);
+}
+
 nsa_status_t nsa_compress_status(void* stream) {
     int err = 0;
     if (read_compress_error(&err, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NSA_ERR_CUDA;
+    if (err == kErrBadPage) return NSA_ERR_INVALID_ARG;   // a block-table entry outside the pool
     return err ? NSA_ERR_TIMEOUT : NSA_OK;
 }
 

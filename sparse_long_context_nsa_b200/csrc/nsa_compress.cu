@@ -95,7 +95,7 @@ nsa_compress_kernel(const CompressParams p) {
     }
     const CompressSeq sq = p.seq[lo];
     const int chunk = blockIdx.x - (sq.chunk_end - sq.nchunks);
-    const int i0 = chunk * p.chunk;
+    const int i0 = sq.first + chunk * p.chunk;
     const int i1 = min(i0 + p.chunk, sq.ncmp);
     if (i0 >= i1) return;
 
@@ -196,8 +196,20 @@ nsa_compress_kernel(const CompressParams p) {
                             if (kk == nb - 1)
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) o[e] = acc[kk][e];
-                        T* out = dst + ((int64_t)sq.cmp_start + i) * rowelems + cv * 8;
-                        *reinterpret_cast<uint4*>(out) = pack8<T>(o);
+                        int64_t orow = (int64_t)sq.cmp_start + i;
+                        bool ok_row = true;
+                        if (p.block_table != nullptr) {
+                            // the page comes from the caller's table: out-of-pool entries
+                            // are reported, never written through
+                            const int pg = p.block_table[(size_t)sq.seq * p.bt_stride + i / p.page_rows];
+                            ok_row = pg >= 0 && pg < p.num_pages;
+                            orow = (int64_t)pg * p.page_rows + i % p.page_rows;
+                            if (!ok_row) atomicCAS(&g_compress_err, 0, kErrBadPage);
+                        }
+                        if (ok_row) {
+                            T* out = dst + orow * rowelems + cv * 8;
+                            *reinterpret_cast<uint4*>(out) = pack8<T>(o);
+                        }
                     }
 #pragma unroll
                     for (int kk = BMAX - 1; kk >= 1; --kk)

@@ -12,10 +12,16 @@ constexpr int kCompressStages = 4;        // shared-memory ring depth
 constexpr int kCompressMaxThreads = 512;  // one thread per 16-byte column vector
 constexpr int kCompressMaxSeq = 96;       // sequences per launch (kernel-parameter space)
 
+// Device error word value: a block-table entry outside the page pool (the
+// store it addressed was skipped).
+constexpr int kErrBadPage = 0x200;
+
 struct CompressSeq {
     int raw_start;   // first raw row of the sequence (T2 index)
     int cmp_start;   // first compressed row (Tc index)
     int ncmp;        // compressed blocks of the sequence
+    int first;       // first block computed (blocks first .. ncmp-1)
+    int seq;         // sequence index (block-table row)
     int nchunks;     // CTAs given to the sequence
     int chunk_end;   // inclusive prefix of nchunks over the launch's sequences
 };
@@ -30,6 +36,10 @@ struct CompressParams {
     int dtype;            // 0 bf16, 1 fp16
     int chunk;            // output blocks per CTA
     int rows_per_stage;   // raw rows per bulk copy
+    // paged output: block i of sequence b goes to row i % page_rows of pool page
+    // block_table[b * bt_stride + i / page_rows] (null: contiguous, row cmp_start + i)
+    const int32_t* block_table;
+    int bt_stride, page_rows, num_pages;
     int nseq;
     CompressSeq seq[kCompressMaxSeq];
 };

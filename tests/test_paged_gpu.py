@@ -167,3 +167,55 @@ def test_decode_workload_full_size_sampled_sequences(nsa):
                                     x["cu_sel_kv"][:n])
     sub = [t[picks] for t in res]
     check_attention(sub, ref, dw.count)
+
+
+def _gather(pool, table, n_cmp_list):
+    out = []
+    for b, n in enumerate(n_cmp_list):
+        out.append(pool[table[b].long()].reshape(-1, *pool.shape[2:])[:n])
+    return torch.cat(out)
+
+
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_paged_compress_equals_contiguous(nsa, page_size):
+    wl = _wl([300, 0, 40, 777, 2100], 8, 4, 64, 32, 16, 64, 8, seed=41)
+    x = wl.generate(device="cuda")
+    cu = x["cu_seqlens"]
+    kc, vc = nsa.nsa_compress(x["k"], x["v"], x["w"], wl.l, wl.d, cu)
+    cuc = nsa.nsa_compress_out_len(cu, wl.l, wl.d)
+    ncs = [int(n) for n in np.diff(np.concatenate([[0], cuc]))]
+    npg = [-(-n // page_size) for n in ncs]
+    total = sum(npg) + 2
+    perm = torch.randperm(total, generator=torch.Generator().manual_seed(page_size)).to(torch.int32)
+    table = torch.full((len(ncs), max(npg) + 1), -1, dtype=torch.int32)
+    o = 0
+    for b, n in enumerate(npg):
+        table[b, :n] = perm[o:o + n]
+        o += n
+    kp = torch.zeros(total, page_size, wl.n2, wl.d1, dtype=kc.dtype, device="cuda")
+    vp = torch.zeros_like(kp)
+    nsa.nsa_compress_paged(x["k"], x["v"], x["w"], wl.l, wl.d, cu, kp, vp, table.cuda())
+    assert nsa.nsa_compress_status() == 0
+    assert torch.equal(_gather(kp.cpu(), table, ncs).view(torch.int16), kc.cpu().view(torch.int16))
+    assert torch.equal(_gather(vp.cpu(), table, ncs).view(torch.int16), vc.cpu().view(torch.int16))
+    # a decode step: only the last block of each sequence, into a pool holding the others
+    kp2, vp2 = kp.clone(), vp.clone()
+    for b, n in enumerate(ncs):
+        if n:
+            pg, r = int(table[b, (n - 1) // page_size]), (n - 1) % page_size
+            kp2[pg, r] = 0
+            vp2[pg, r] = 0
+    nsa.nsa_compress_paged(x["k"], x["v"], x["w"], wl.l, wl.d, cu, kp2, vp2, table.cuda(),
+                           first_block=[max(0, n - 1) for n in ncs])
+    assert nsa.nsa_compress_status() == 0
+    assert torch.equal(kp2, kp) and torch.equal(vp2, vp)
+
+
+def test_paged_compress_reports_out_of_pool_pages(nsa):
+    wl = _wl([900], 8, 2, 64, 32, 16, 64, 8, seed=42)   # 55 blocks: pages 0..3
+    x = wl.generate(device="cuda")
+    kp = torch.zeros(4, 16, wl.n2, wl.d1, dtype=x["k"].dtype, device="cuda")
+    table = torch.tensor([[0, 1, 2, 99]], dtype=torch.int32, device="cuda")   # blocks 48..54 -> page 99: outside
+    nsa.nsa_compress_paged(x["k"], None, x["w"], wl.l, wl.d, x["cu_seqlens"], kp, None, table)
+    assert nsa.nsa_compress_status() == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_compress_status() == 0                                      # reported once
