@@ -23,6 +23,14 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnsa_b200.so")
+# NSA_DEBUG=1: load the debug build (device bounds checks) and put a guard band
+# with a canary pattern after every output and workspace this binding allocates,
+# checked after every call.
+LIB_DEBUG_PATH = os.path.join(_PKG, "libnsa_b200_debug.so")
+DEBUG = os.environ.get("NSA_DEBUG") == "1"
+_GUARD_BYTES = 4096
+_CANARY = 0xA5
+_guards = []   # (name, guard bytes) of the allocations made for the current call
 
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED = 0, 1, 2
 NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = 3, 4, 5
@@ -77,7 +85,7 @@ def load(path: Optional[str] = None):
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIB_PATH
+    p = path or (LIB_DEBUG_PATH if DEBUG else LIB_PATH)
     if not os.path.exists(p):
         raise ImportError(f"{p} is missing: build it with sparse_long_context_nsa_b200._build.build()")
     lib = ctypes.CDLL(p)
@@ -151,7 +159,50 @@ def load(path: Optional[str] = None):
     return lib
 
 
-def _raise(status: int, what: str):
+def _alloc(fill, *shape, dtype, device) -> torch.Tensor:
+    """An output or workspace tensor; in debug mode followed by a guard band of
+    canary bytes that _raise checks once the call has run."""
+    if not DEBUG:
+        return (torch.zeros if fill else torch.empty)(*shape, dtype=dtype, device=device)
+    n = 1
+    for x in shape:
+        n *= int(x)
+    esize = torch.empty((), dtype=dtype).element_size()
+    flat = torch.empty(n * esize + _GUARD_BYTES, dtype=torch.uint8, device=device)
+    if fill:
+        flat[:n * esize].zero_()
+    flat[n * esize:].fill_(_CANARY)
+    _guards.append((f"{tuple(shape)} {dtype}", flat[n * esize:]))
+    return flat[:n * esize].view(dtype).view(*shape)
+
+
+def _empty(*shape, dtype, device) -> torch.Tensor:
+    return _alloc(False, *shape, dtype=dtype, device=device)
+
+
+def _zeros(*shape, dtype, device) -> torch.Tensor:
+    return _alloc(True, *shape, dtype=dtype, device=device)
+
+
+def _check_guards(what: str):
+    """Debug mode: every guard band allocated for this call still holds its
+    canary pattern (a write past the end of an output would have changed it)."""
+    if not _guards:
+        return
+    torch.cuda.synchronize()
+    bad = [name for name, g in _guards if not bool((g == _CANARY).all())]
+    _guards.clear()
+    if bad:
+        raise NsaError(NSA_ERR_INVALID_ARG, f"{what}: guard band overwritten after {', '.join(bad)}")
+
+
+def _raise(status: int, what: str, guards: bool = False):
+    """Maps a status to an exception; after a compute call (guards=True) also
+    checks the debug guard bands of the call's allocations."""
+    if guards:
+        if status == NSA_OK:
+            _check_guards(what)
+        _guards.clear()
     if status == NSA_OK:
         return
     if status in (NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED):
@@ -202,7 +253,7 @@ def _workspace(ws: torch.Tensor, nbytes: int, device) -> torch.Tensor:
     replaced: the kernel writes its error word into the workspace it runs
     on, and the caller reads that word back from its own tensor."""
     if ws is None:
-        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return _empty(max(nbytes, 256), dtype=torch.uint8, device=device)
     _dev(ws, "workspace")
     if ws.device != device or ws.dtype != torch.uint8:
         raise ValueError(f"workspace must be a uint8 tensor on {device}")
@@ -271,17 +322,17 @@ def nsa_compress(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tensor, l:
     cuc = nsa_compress_out_len(cu, l, d)
     tc = int(cuc[-1])
     if kcmp is None:
-        kcmp = torch.empty(tc, n2, d1, dtype=k.dtype, device=k.device)
+        kcmp = _empty(tc, n2, d1, dtype=k.dtype, device=k.device)
     else:
         _out(kcmp, (tc, n2, d1), k.dtype, k.device, "kcmp")
     if v is not None and vcmp is None:
-        vcmp = torch.empty(tc, n2, d2, dtype=k.dtype, device=k.device)
+        vcmp = _empty(tc, n2, d2, dtype=k.dtype, device=k.device)
     elif v is not None:
         _out(vcmp, (tc, n2, d2), k.dtype, k.device, "vcmp")
     st = load().nsa_compress(k.data_ptr(), v.data_ptr() if v is not None else None, w.data_ptr(),
                              int(l), int(d), _ip(cu), cu.size, n2, d1, d2, dt, kcmp.data_ptr(),
                              vcmp.data_ptr() if v is not None else None, _stream(stream))
-    _raise(st, "nsa_compress")
+    _raise(st, "nsa_compress", guards=True)
     return kcmp, vcmp
 
 
@@ -348,10 +399,10 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
     dev = q.device
     _same_device(q, (kcmp, "kcmp"), (vcmp, "vcmp"))
     if out is None:
-        att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
-        tk = torch.empty(t1, n2, count, dtype=torch.int32, device=dev)
-        smax = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
-        ssum = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
+        att = _empty(t1, n1, d2, dtype=q.dtype, device=dev)
+        tk = _empty(t1, n2, count, dtype=torch.int32, device=dev)
+        smax = _empty(t1, n1, 8, dtype=torch.float32, device=dev)
+        ssum = _empty(t1, n1, 8, dtype=torch.float32, device=dev)
     else:
         att, tk, smax, ssum = out
         _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
@@ -370,7 +421,7 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
             int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
             tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
             _stream(stream))
-        _raise(st, "nsa_compress_attention")
+        _raise(st, "nsa_compress_attention", guards=True)
         return att, tk, smax, ssum
     masks = []
     for mk, nm in ((atten_mask, "atten_mask"), (topk_mask, "topk_mask")):
@@ -390,7 +441,7 @@ def nsa_compress_attention(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torch.Tens
         am.data_ptr() if am is not None else None, ar, ac, tm.data_ptr() if tm is not None else None, tr, tc_,
         att.data_ptr(), tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
         _stream(stream))
-    _raise(st, "nsa_compress_attention_masked")
+    _raise(st, "nsa_compress_attention_masked", guards=True)
     return att, tk, smax, ssum
 
 
@@ -432,7 +483,7 @@ def nsa_compress_attention_noalloc(q: torch.Tensor, kcmp: torch.Tensor, vcmp: to
         q.data_ptr(), kcmp.data_ptr(), vcmp.data_ptr(), float(scale), int(head_num), int(l), int(d),
         int(lp), int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(),
         tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), _stream(stream))
-    _raise(st, "nsa_compress_attention_noalloc")
+    _raise(st, "nsa_compress_attention_noalloc", guards=True)
     return att, tk, smax, ssum
 
 
@@ -499,8 +550,8 @@ def nsa_select_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk
     dev = q.device
     _same_device(q, (k, "k"), (v, "v"), (topk_indices, "topk_indices"))
     if out is None:
-        att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
-        lse = torch.empty(t1, n1, dtype=torch.float32, device=dev)
+        att = _empty(t1, n1, d2, dtype=q.dtype, device=dev)
+        lse = _empty(t1, n1, dtype=torch.float32, device=dev)
     else:
         att, lse = out
         _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
@@ -511,7 +562,7 @@ def nsa_select_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk
         q.data_ptr(), k.data_ptr(), v.data_ptr(), topk_indices.data_ptr(), float(scale), int(head_num),
         int(lp), int(count), _ip(cq), _ip(ck), cq.size, n2, d1, d2, dt, att.data_ptr(), lse.data_ptr(),
         workspace.data_ptr(), workspace.numel(), _stream(stream))
-    _raise(st, "nsa_select_attention")
+    _raise(st, "nsa_select_attention", guards=True)
     return att, lse
 
 
@@ -586,10 +637,10 @@ def nsa_compress_attention_shard(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torc
     dev = q.device
     _same_device(q, (kcmp, "kcmp"), (vcmp, "vcmp"))
     if out is None:
-        att = torch.zeros(t1, n1, d2, dtype=q.dtype, device=dev)
+        att = _zeros(t1, n1, d2, dtype=q.dtype, device=dev)
         tk = torch.full((t1, n2, count), -1, dtype=torch.int32, device=dev)
-        smax = torch.zeros(t1, n1, 8, dtype=torch.float32, device=dev)
-        ssum = torch.zeros(t1, n1, 8, dtype=torch.float32, device=dev)
+        smax = _zeros(t1, n1, 8, dtype=torch.float32, device=dev)
+        ssum = _zeros(t1, n1, 8, dtype=torch.float32, device=dev)
     else:
         att, tk, smax, ssum = out
         _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
@@ -604,7 +655,7 @@ def nsa_compress_attention_shard(q: torch.Tensor, kcmp: torch.Tensor, vcmp: torc
         int(count), _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, int(group_begin), int(group_count),
         att.data_ptr(), tk.data_ptr(), smax.data_ptr(), ssum.data_ptr(), workspace.data_ptr(), workspace.numel(),
         _stream(stream))
-    _raise(st, "nsa_compress_attention_shard")
+    _raise(st, "nsa_compress_attention_shard", guards=True)
     return att, tk, smax, ssum
 
 
@@ -657,9 +708,9 @@ def nsa_compress_attention_backward(q: torch.Tensor, kcmp: torch.Tensor, vcmp: t
     if int(cq[-1]) > t1 or int(cc[-1]) > tc:
         raise ValueError("prefix sums run past the rows of q / kcmp")
     if grads is None:
-        dq = torch.empty(t1, n1, d1, dtype=torch.float32, device=dev)
-        dk = torch.empty(tc, n2, d1, dtype=torch.float32, device=dev)
-        dv = torch.empty(tc, n2, d2, dtype=torch.float32, device=dev)
+        dq = _empty(t1, n1, d1, dtype=torch.float32, device=dev)
+        dk = _empty(tc, n2, d1, dtype=torch.float32, device=dev)
+        dv = _empty(tc, n2, d2, dtype=torch.float32, device=dev)
     else:
         dq, dk, dv = grads
         _out(dq, (t1, n1, d1), torch.float32, dev, "dq")
@@ -672,7 +723,7 @@ def nsa_compress_attention_backward(q: torch.Tensor, kcmp: torch.Tensor, vcmp: t
         softmax_max.data_ptr(), softmax_sum.data_ptr(), float(scale), n1, int(l), int(d), _ip(cq), _ip(cc),
         cq.size, n2, d1, d2, dt, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
         workspace.numel(), _stream(stream))
-    _raise(st, "nsa_compress_attention_backward")
+    _raise(st, "nsa_compress_attention_backward", guards=True)
     return dq, dk, dv
 
 
@@ -715,9 +766,9 @@ def nsa_compress_backward(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.T
     _same_device(k, (w, "w"), (v, "v"), (dkcmp, "dkcmp"), (dvcmp, "dvcmp"))
     dev = k.device
     if grads is None:
-        dk = torch.zeros(t2, n2, d1, dtype=torch.float32, device=dev)
-        dv = torch.zeros(t2, n2, d2, dtype=torch.float32, device=dev) if v is not None else None
-        dw = torch.empty(l, n2, dtype=torch.float32, device=dev)
+        dk = _zeros(t2, n2, d1, dtype=torch.float32, device=dev)
+        dv = _zeros(t2, n2, d2, dtype=torch.float32, device=dev) if v is not None else None
+        dw = _empty(l, n2, dtype=torch.float32, device=dev)
     else:
         dk, dv, dw = grads
         _out(dk, (t2, n2, d1), torch.float32, dev, "dk")
@@ -731,7 +782,7 @@ def nsa_compress_backward(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.T
         dvcmp.data_ptr() if v is not None else None, int(l), int(d), _ip(cu), cu.size, n2, d1, d2, dt,
         dk.data_ptr(), dv.data_ptr() if v is not None else None, dw.data_ptr(), workspace.data_ptr(),
         workspace.numel(), _stream(stream))
-    _raise(st, "nsa_compress_backward")
+    _raise(st, "nsa_compress_backward", guards=True)
     return dk, dv, dw
 
 
@@ -769,10 +820,10 @@ def nsa_compress_attention_paged(q: torch.Tensor, kcmp_pages: torch.Tensor, vcmp
     dev = q.device
     _same_device(q, (kcmp_pages, "kcmp_pages"), (vcmp_pages, "vcmp_pages"), (block_table, "block_table"))
     if out is None:
-        att = torch.empty(t1, n1, d2, dtype=q.dtype, device=dev)
-        tk = torch.empty(t1, n2, count, dtype=torch.int32, device=dev)
-        smax = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
-        ssum = torch.empty(t1, n1, 8, dtype=torch.float32, device=dev)
+        att = _empty(t1, n1, d2, dtype=q.dtype, device=dev)
+        tk = _empty(t1, n2, count, dtype=torch.int32, device=dev)
+        smax = _empty(t1, n1, 8, dtype=torch.float32, device=dev)
+        ssum = _empty(t1, n1, 8, dtype=torch.float32, device=dev)
     else:
         att, tk, smax, ssum = out
         _out(att, (t1, n1, d2), q.dtype, dev, "attention_out")
@@ -786,7 +837,7 @@ def nsa_compress_attention_paged(q: torch.Tensor, kcmp_pages: torch.Tensor, vcmp
         block_table.data_ptr(), int(block_table.shape[1]), float(scale), n1, int(l), int(d), int(lp), int(count),
         _ip(cq), _ip(cc), _ip(cs), cq.size, n2, d1, d2, dt, att.data_ptr(), tk.data_ptr(), smax.data_ptr(),
         ssum.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream))
-    _raise(st, "nsa_compress_attention_paged")
+    _raise(st, "nsa_compress_attention_paged", guards=True)
     return att, tk, smax, ssum
 
 
@@ -827,5 +878,5 @@ def nsa_compress_paged(k: torch.Tensor, v: Optional[torch.Tensor], w: torch.Tens
         k.data_ptr(), v.data_ptr() if v is not None else None, w.data_ptr(), int(l), int(d), _ip(cu), cu.size, n2,
         d1, d2, dt, kcmp_pages.data_ptr(), vcmp_pages.data_ptr() if v is not None else None, num_pages, page_size,
         block_table.data_ptr(), int(block_table.shape[1]), _ip(fb) if fb is not None else None, _stream(stream))
-    _raise(st, "nsa_compress_paged")
+    _raise(st, "nsa_compress_paged", guards=True)
     return kcmp_pages, vcmp_pages

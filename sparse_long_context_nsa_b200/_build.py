@@ -12,6 +12,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libnsa_b200.so")
+# The debug build: kernels check their computed global indices (NSA_DEBUG) and
+# record a violation in the error word instead of writing outside a tensor.
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libnsa_b200_debug.so")
 SOURCES = ["nsa_api.cu", "nsa_compress.cu", "nsa_attention.cu", "nsa_select.cu", "nsa_backward.cu"]
 HEADERS = ["nsa_internal.h", "ptx.cuh"]
 
@@ -34,17 +38,20 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(dep) > t for dep in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile every CUDA source for sm_100a and link the shared library."""
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA source for sm_100a and link the shared library (with
+    debug=True the NSA_DEBUG library with device bounds checks)."""
+    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    extra = ["-DNSA_DEBUG"] if debug else []
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "nsa.h")]
     jobs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD, src.replace(".cu", ".o"))
+        o = os.path.join(build_dir, src.replace(".cu", ".o"))
         if force or _stale(o, [s] + hdrs):
-            cmd = [nvcc] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose_ptxas else []) + ["-c", s, "-o", o]
+            cmd = [nvcc] + ARCH + FLAGS + extra + (["-Xptxas", "-v"] if verbose_ptxas else []) + ["-c", s, "-o", o]
             jobs.append(cmd)
     if jobs:
         with concurrent.futures.ThreadPoolExecutor(max_workers=len(jobs)) as ex:
@@ -54,14 +61,13 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
-    objs = [os.path.join(BUILD, s.replace(".cu", ".o")) for s in SOURCES]
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    objs = [os.path.join(build_dir, s.replace(".cu", ".o")) for s in SOURCES]
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call([nvcc] + ARCH + ["-shared", "-o", tmp] + objs + ["-cudart", "static"])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -33,6 +33,14 @@ nsa_status_t check_prefix(const int32_t* cu, int batch) {
     return NSA_OK;
 }
 
+// Status of a device error word: a timed-out wait, a block-table entry outside
+// its pool, or (debug builds) a computed index outside its tensor.
+nsa_status_t error_status(int err) {
+    if (err == 0) return NSA_OK;
+    if (err == kErrBadPage || (err >= kErrBounds && err < kErrBounds + 0x100)) return NSA_ERR_INVALID_ARG;
+    return NSA_ERR_TIMEOUT;
+}
+
 int64_t ncmp_of(int64_t S, int l, int d) {
     // aclnnNsaCompress Formula: blocks i = 0 .. floor((S-l)/d); none when S < l
     return S < l ? 0 : (S - l) / d + 1;
@@ -688,6 +696,7 @@ static nsa_status_t compress_impl(const void* k, const void* v, const void* w, i
     p.bt_stride = bt_stride;
     p.page_rows = page_rows;
     p.num_pages = (int)num_pages;
+    p.tc_rows = total_out;   // rows of the contiguous outputs (all blocks when no table)
     const int threads = (int)(((rowelems / 8) + 31) / 32 * 32);
 
     int32_t prev_raw = 0;
@@ -742,8 +751,7 @@ nsa_status_t nsa_compress_paged(const void* k, const void* v, const void* w, int
 nsa_status_t nsa_compress_status(void* stream) {
     int err = 0;
     if (read_compress_error(&err, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NSA_ERR_CUDA;
-    if (err == kErrBadPage) return NSA_ERR_INVALID_ARG;   // a block-table entry outside the pool
-    return err ? NSA_ERR_TIMEOUT : NSA_OK;
+    return error_status(err);
 }
 
 nsa_status_t nsa_compress_attention_workspace_size(int head_num, int n2, int d1, int d2, int l, int d, int lp,
@@ -829,6 +837,7 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     p.bt_stride = bt_stride;
     p.page_rows = page_rows;
     p.pool_rows = (int)(num_pages * page_rows);
+    p.rows_q = t1;
     p.score_gmem = pl.score_in_smem ? nullptr : reinterpret_cast<float*>(ws + off_score);
     p.band = reinterpret_cast<float*>(ws + off_score + pl.ws_score);
     p.capj = pl.capj;
@@ -1080,6 +1089,7 @@ nsa_status_t nsa_select_attention(const void* q, const void* k, const void* v, c
     p.tiles = reinterpret_cast<const sel::Tile*>(ws + kWsHeader);
     p.num_tiles = (int)pl.tiles.size();
     p.err = reinterpret_cast<int*>(ws);
+    p.rows_q = t1;
     p.topk = topk_indices;
     p.count = count;
     p.list_n = reinterpret_cast<int*>(ws + kWsHeader + pl.ws_tiles);
@@ -1176,6 +1186,9 @@ nsa_status_t nsa_compress_attention_backward(const void* q, const void* kcmp, co
     p.rowinfo = reinterpret_cast<const float2*>(ws + pl.off_rowinfo);
     p.dq = dq;
     p.part = reinterpret_cast<float*>(ws + pl.off_part);
+    p.rows_q = t1;
+    p.rows_c = tc;
+    p.n_slots = pl.nslots;
     p.dtype = dtype == NSA_BF16 ? 0 : 1;
     p.n1 = head_num;
     p.n2 = n2;
@@ -1221,7 +1234,7 @@ nsa_status_t nsa_compress_attention_backward(const void* q, const void* kcmp, co
         if (bwd::launch_dkdv(p, tq, tdo, tk, tv, st) != cudaSuccess) return NSA_ERR_CUDA;
     }
     if (bwd::launch_reduce(reinterpret_cast<const bwd::KVTile*>(ws + pl.off_kvtiles), (int)pl.kvtiles.size(),
-                           p.part, dkcmp, dvcmp, n2, d1, d2, scale, st) != cudaSuccess)
+                           p.part, dkcmp, dvcmp, n2, d1, d2, scale, tc, p.err, st) != cudaSuccess)
         return NSA_ERR_CUDA;
     return NSA_OK;
 }
@@ -1291,6 +1304,7 @@ nsa_status_t nsa_compress_backward(const void* k, const void* v, const void* w, 
     p.dw = dw;
     p.cmp_raw = reinterpret_cast<const int*>(ws + kWsHeader);
     p.tc = (long long)cmp_raw.size();
+    p.t2 = cu_seqlens[batch - 1];
     p.l = l;
     p.d = d;
     p.n2 = n2;
@@ -1331,7 +1345,7 @@ nsa_status_t nsa_workspace_status(const void* workspace, void* stream) {
     if (cudaStreamSynchronize(st) != cudaSuccess) return NSA_ERR_CUDA;
     int err = 0;
     if (cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NSA_ERR_CUDA;
-    return err ? NSA_ERR_TIMEOUT : NSA_OK;
+    return error_status(err);
 }
 
 }  // extern "C"
@@ -1415,5 +1429,5 @@ extern "C" nsa_status_t nsa_noalloc_status(void* stream) {
     int err = 0;
     if (cudaMemcpyFromSymbol(&err, g_static_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost) != cudaSuccess)
         return NSA_ERR_CUDA;
-    return err ? NSA_ERR_TIMEOUT : NSA_OK;
+    return error_status(err);
 }

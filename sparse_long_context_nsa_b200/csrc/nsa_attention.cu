@@ -527,7 +527,8 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc_fence_after();
                 // O (tensor memory) / L -> attention_out
                 const int tok = pp * TT + etok;
-                const bool valid = (erow < TT * G) && (tok < t.ntok);
+                const bool valid = (erow < TT * G) && (tok < t.ntok) &&
+                                   nsa_index_ok(t.q_row0 + tok < p.rows_q, p.err, 1);
                 const int nvis = valid ? nvis_of(t.t0 + tok, p.l, p.d, t.n_cmp) : 0;
                 const float Lr = rowstat[((pp * 2 + slot) * 2 + 1) * 128 + erow];
                 // rows that attend to nothing write zeros (their O may never have been
@@ -568,6 +569,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int pp = tau / TT;
                 const int tl = tau - pp * TT;
                 const int tp = t.t0 + tau;
+                if (!nsa_index_ok(t.q_row0 + tau < p.rows_q && t.group < p.n2, p.err, 2)) continue;
                 int32_t* dst = p.topk + ((size_t)(t.q_row0 + tau) * p.n2 + t.group) * p.count;
                 const int nv = nvis_of(tp, p.l, p.d, t.n_cmp);
                 bool empty = nv == 0;
@@ -837,8 +839,11 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
 #pragma unroll
                         for (int k = 0; k < NCARRY; ++k) carry[k] = s[CH - 1 - k];
-                        if (valid) __stcg(wrow + i * NCH + c, mr);
-                        if (valid) {
+                        // (debug builds: the chunk stays inside the slot's scratch)
+                        const bool in_slot =
+                            nsa_index_ok((i * NCH + c + 1) * 128 * NJC <= p.capj && i * NCH + c < p.capc, p.err, 4);
+                        if (valid && in_slot) __stcg(wrow + i * NCH + c, mr);
+                        if (valid && in_slot) {
                             // a warp writes its 32 rows' values of the chunk contiguously
                             float4* bd = reinterpret_cast<float4*>(
                                 sbase_g + ((size_t)(i * NCH + c) * 128 + row) * NJC);
@@ -875,7 +880,7 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         __stcg(bd + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
                     __stcg(wrow + t.nkv * NCH, mr);
                 }
-                if (valid) {
+                if (valid && nsa_index_ok(t.q_row0 + tok < p.rows_q, p.err, 3)) {
                     // softmax_max / softmax_sum: exact maximum (natural units) and the
                     // sum of exp(s - max)
                     const size_t si = ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * 8;

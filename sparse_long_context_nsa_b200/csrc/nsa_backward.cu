@@ -247,7 +247,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const int row = warp * 32 + lane;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const int tok = row / G, h = row % G;
-        const bool valid = row < TT * G && tok < it.ntok;
+        const bool valid = row < TT * G && tok < it.ntok && nsa_index_ok(it.q_row0 + tok < p.rows_q, p.err, 8);
         const int nv = valid ? nvis_at(it.t0 + tok, p.l, p.d, it.n_cmp) : 0;
         const size_t ri = ((size_t)(it.q_row0 + tok) * p.n1 + (size_t)it.group * G + h);
         const float2 info = valid ? p.rowinfo[ri] : make_float2(INFINITY, 0.f);
@@ -525,7 +525,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tc_fence_after();
         // the run's partial sums; a run with no M-tile leaves zeros
         float* dst = p.part + ((size_t)it.slot * 128 + kr) * (p.d1 + p.d2);
-        if (n_mt > 0) {
+        if (!nsa_index_ok(it.slot < p.n_slots, p.err, 9)) {
+        } else if (n_mt > 0) {
             if (do_dv) store_row_f32(tmem + lane_off, p.d2, 1.f, dst, true);
             if (do_dk) store_row_f32(tmem + lane_off + p.col_dk, p.d1, 1.f, dst + p.d2, true);
         } else {
@@ -554,10 +555,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // fixed order, so the result does not depend on the schedule); dK x scale.
 __global__ void reduce_kernel(const KVTile* __restrict__ tiles, const float* __restrict__ part,
                               float* __restrict__ dkcmp, float* __restrict__ dvcmp, int n2, int d1, int d2,
-                              float scale) {
+                              float scale, long long rows_c, int* err) {
     const KVTile t = tiles[blockIdx.x];
     const int w = d1 + d2, w4 = w / 4;
-    const int rows = min(kKV, t.n_cmp - t.kt * kKV);
+    int rows = min(kKV, t.n_cmp - t.kt * kKV);
+    if (!nsa_index_ok(t.cmp_row0 + t.kt * kKV + rows <= rows_c, err, 10)) rows = 0;
     for (int x = threadIdx.x; x < rows * w4; x += blockDim.x) {
         const int r = x / w4, c = (x % w4) * 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -579,9 +581,9 @@ __global__ void reduce_kernel(const KVTile* __restrict__ tiles, const float* __r
 }
 
 cudaError_t launch_reduce(const KVTile* tiles, int ntiles, const float* part, float* dkcmp, float* dvcmp, int n2,
-                          int d1, int d2, float scale, cudaStream_t st) {
+                          int d1, int d2, float scale, long long rows_c, int* err, cudaStream_t st) {
     if (ntiles <= 0) return cudaSuccess;
-    reduce_kernel<<<ntiles, 256, 0, st>>>(tiles, part, dkcmp, dvcmp, n2, d1, d2, scale);
+    reduce_kernel<<<ntiles, 256, 0, st>>>(tiles, part, dkcmp, dvcmp, n2, d1, d2, scale, rows_c, err);
     return cudaGetLastError();
 }
 
@@ -631,6 +633,7 @@ __global__ void compress_dx_kernel(const CompressBwdParams p) {
     for (int rr = 0; rr < kRowsPerCta; ++rr) {
         const int pr = r0 + rr;   // raw row inside the sequence
         if (pr >= q.raw_len) break;
+        if (!nsa_index_ok(q.raw_start + pr < p.t2, nullptr, 11)) break;
         // windows i with i d <= pr < i d + l
         int i_lo = pr - p.l + 1 <= 0 ? 0 : (pr - p.l + 1 + p.d - 1) / p.d;
         int i_hi = min(pr / p.d, q.n_cmp - 1);

@@ -197,7 +197,8 @@ nsa_compress_kernel(const CompressParams p) {
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) o[e] = acc[kk][e];
                         int64_t orow = (int64_t)sq.cmp_start + i;
-                        bool ok_row = true;
+                        bool ok_row = p.block_table != nullptr ||
+                                      nsa_index_ok(orow < p.tc_rows, &g_compress_err, 6);
                         if (p.block_table != nullptr) {
                             // the page comes from the caller's table: out-of-pool entries
                             // are reported, never written through

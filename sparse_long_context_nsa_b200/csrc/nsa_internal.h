@@ -15,6 +15,25 @@ constexpr int kCompressMaxSeq = 96;       // sequences per launch (kernel-parame
 // Device error word value: a block-table entry outside the page pool (the
 // store it addressed was skipped).
 constexpr int kErrBadPage = 0x200;
+// Debug builds (NSA_DEBUG): a computed global index outside its tensor; the
+// access was skipped.  kErrBounds + the id of the checking site.
+constexpr int kErrBounds = 0x300;
+
+#ifdef __CUDACC__
+// Debug-build bounds check of a computed global index: false (and the first
+// such site recorded in *err) when `ok` fails; release builds compile it away.
+__device__ __forceinline__ bool nsa_index_ok(bool ok, int* err, int site) {
+#ifdef NSA_DEBUG
+    if (!ok && err != nullptr) atomicCAS(err, 0, kErrBounds + site);
+    return ok;
+#else
+    (void)err;
+    (void)site;
+    (void)ok;
+    return true;
+#endif
+}
+#endif
 
 struct CompressSeq {
     int raw_start;   // first raw row of the sequence (T2 index)
@@ -40,6 +59,7 @@ struct CompressParams {
     // block_table[b * bt_stride + i / page_rows] (null: contiguous, row cmp_start + i)
     const int32_t* block_table;
     int bt_stride, page_rows, num_pages;
+    long long tc_rows;    // rows of the contiguous outputs (debug bounds checks)
     int nseq;
     CompressSeq seq[kCompressMaxSeq];
 };
@@ -91,6 +111,7 @@ struct AttnParams {
     // maps cover the pools, pool_rows rows, with boxes of page_rows rows)
     const int32_t* block_table;
     int bt_stride, page_rows, pool_rows;
+    long long rows_q;       // rows of q and of the outputs (debug bounds checks)
     // per-CTA scratch for the per-head importance values: for each pipeline,
     // two slots (consecutive items alternate) of `region` floats each.  A slot
     // holds the banded values chunk-major, [chunk][row 0..127][anchor of the
@@ -170,6 +191,7 @@ struct Params {
     const float2* rowinfo;   // (T1, N1): log2 normaliser m*log2e + log2 L (inf: row sees nothing), delta
     float* dq;               // (T1, N1, D1) fp32
     float* part;             // partial slots of dK/dV: [slot][128][D2 | D1] fp32
+    long long rows_q, rows_c, n_slots;   // extents for debug bounds checks
     int mode;                // dK/dV kernel: bit 0 dV, bit 1 dK
     int col_dk;              // tensor-memory column of the dK accumulator
     int nsb;                 // dK/dV kernel: score buffers (2 when the accumulators end by column 256)
@@ -189,7 +211,7 @@ cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMa
                         const CUtensorMap& tv, cudaStream_t st);
 // dkcmp / dvcmp rows of every KV tile from its partial slots (dK scaled)
 cudaError_t launch_reduce(const KVTile* tiles, int ntiles, const float* part, float* dkcmp, float* dvcmp, int n2,
-                          int d1, int d2, float scale, cudaStream_t st);
+                          int d1, int d2, float scale, long long rows_c, int* err, cudaStream_t st);
 
 constexpr int kRowsPerCta = 32;   // raw rows per CTA of the compression transpose
 struct CompressBwdSeq {
@@ -207,6 +229,7 @@ struct CompressBwdParams {
     float* dw;
     const int* cmp_raw;           // per compressed row: its first raw row (T2 index)
     long long tc;
+    long long t2;                 // raw rows (debug bounds checks)
     int l, d, n2, d1, d2, dtype;
     int nseq;
     CompressBwdSeq seq[kCompressMaxSeq];
@@ -247,6 +270,7 @@ struct Params {
     const Tile* tiles;
     int num_tiles;
     int* err;                   // device error word (workspace)
+    long long rows_q;           // rows of q and of the outputs (debug bounds checks)
     const int32_t* topk;        // (T1, N2, count) block lists
     int count;
     int* list_n;                // per tile: blocks in the union of its tokens' lists

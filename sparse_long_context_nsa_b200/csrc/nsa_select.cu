@@ -398,7 +398,8 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             const Tile t = p.tiles[tile];
             const int n = list_n(tile);
-            const bool valid = (row < TT * G) && (tok < t.ntok);
+            const bool valid = (row < TT * G) && (tok < t.ntok) &&
+                               nsa_index_ok(t.q_row0 + tok < p.rows_q, p.err, 7);
             const size_t ridx = (size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h;
             T* orow = reinterpret_cast<T*>(p.out) + ridx * p.d2;
             if (n == 0) {

@@ -256,3 +256,11 @@ def _call_masked(lib, **kw):
 ])
 def test_masked_attention_rejects_before_launch(lib, kw, status):
     assert _call_masked(lib, **kw) == status
+
+
+def test_debug_library_exports_every_declared_symbol():
+    # the NSA_DEBUG build (device bounds checks) offers the same C ABI
+    path = _build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(dbg, name), name
