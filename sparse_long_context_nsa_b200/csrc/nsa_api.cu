@@ -838,6 +838,7 @@ static nsa_status_t compress_attention_impl(const void* q, const void* kcmp, con
     p.page_rows = page_rows;
     p.pool_rows = (int)(num_pages * page_rows);
     p.rows_q = t1;
+    p.two_pass = ((pl.G & (pl.G - 1)) == 0 && pl.G <= 32 && pl.nkv_cols == 128) ? 1 : 0;
     p.score_gmem = pl.score_in_smem ? nullptr : reinterpret_cast<float*>(ws + off_score);
     p.band = reinterpret_cast<float*>(ws + off_score + pl.ws_score);
     p.capj = pl.capj;

@@ -260,7 +260,7 @@ __device__ __noinline__ void tmem_scale_packed(uint32_t taddr, float f) {
     tmem_st_n<NP>(taddr, r);
 }
 
-template <typename T, int A, bool kMask>
+template <typename T, int A, bool kMask, bool kTwoPass>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -386,6 +386,9 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int c = 0; c < nqc; ++c)
                         tma_load_3d_hint(qdst + pp * q_tile_stride + c * 16384, &tm_q, c * 64, t.group * G,
                                          t.q_row0 + pp * TT, bar(B_Q_FULL0 + qb), q_policy);
+                // two passes: first every K tile alone (the row maxima and sums)
+                if constexpr (kTwoPass)
+                    for (int i = 0; i < t.nkv && ok; ++i) load_kv(false, t, i);
                 // K_0, then K_{i+1} ahead of V_i: the order the MMA issuer consumes them
                 if (t.nkv > 0 && ok) load_kv(false, t, 0);
                 for (int i = 0; i < t.nkv && ok; ++i) {
@@ -453,6 +456,36 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t qaddr = q_addr0 + qb * p.q_bytes;
+                if constexpr (kTwoPass) {
+                    // pass 1: S_i = Q K_i^T for every tile; the softmax reads each S and
+                    // hands its buffer back through P_FULL (there is no P V in this pass).
+                    // A buffer is reissued only once the S it held has been read.
+                    auto consume = [&](int pp) {
+                        int& pc = pp ? pvc1 : pvc0;
+                        ok = ok && mbar_wait(bar(B_P_FULL + pp), pc & 1, abort_flag, p.err, kErrTimeoutBase + 15);
+                        // the softmax's reads of the buffer are ordered before the next MMA into it
+                        tc_fence_after();
+                        ++pc;
+                    };
+                    // With two buffers (one pipeline) S_i goes into the buffer that S_{i-2}
+                    // left, and the hand-back of S_{i-1} is waited for right after S_i is
+                    // issued: nothing may block in between, or the softmax could hand back
+                    // two buffers before the first wait and P_FULL would alias a phase.
+                    for (int i = 0; i < t.nkv && ok; ++i) {
+                        const int ks = wait_slot();
+                        if (!ok) break;
+                        tc_fence_after();
+                        for (int pp = 0; pp < npipe && ok; ++pp) {
+                            if (nsb == 1 && i >= 1) consume(pp);
+                            if (ok) qk(pp, qaddr, ks);
+                        }
+                        umma_commit(bar(B_SLOT_EMPTY0 + ks));
+                        if (nsb == 2 && i >= 1) consume(0);
+                    }
+                    if (t.nkv > 0)
+                        for (int pp = 0; pp < npipe; ++pp) consume(pp);   // the last S of each pipeline
+                    if (!ok) break;
+                }
                 if (t.nkv > 0) {
                     const int k0 = wait_slot();
                     if (!ok) break;
@@ -589,58 +622,72 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // anchors past nkv*NJ + NJC collect no tap from a visible block
                 const int jn = min(ncand, t.nkv * NJ + NJC);
                 const float* base = p.band + (((size_t)blockIdx.x * npipe + pp) * 2 + slot) * (size_t)p.region;
-                const float* rs = rowstat + (pp * 2 + slot) * 2 * 128 + tl * G;
-                // the token's heads' normalisers m_ref + log2 L, once
-                for (int hh = lane; hh < G; hh += 32) {
-                    const float Lh = rs[128 + hh];
-                    mbw[hh] = (Lh > 0.f) ? rs[hh] + lg2(Lh) : INFINITY;
-                }
-                __syncwarp();
-                // P_slc'[j] = sum_h 2^(m_c - m_ref - log2 L) x banded value, where m_c
-                // is the reference the value's chunk was written against (steps 4-5).
-                // Lane l takes anchors 4l..4l+3 of every 128 (in one chunk, NJC % 4 == 0)
-                // and loops over the heads, eight at a time for loads in flight.
-                const float* wbase = base + p.capj + (size_t)(tl * G) * p.capc;
-                // (measured on B200: the chunk weights computed here, with their
-                // references loaded next to the banded values, beat a per-step weight
-                // table filled first, which serialises two L2 round trips per step)
-                for (int j0 = 0; j0 < jn; j0 += 128) {
-                    const int j4 = j0 + 4 * lane;
-                    const bool live = j4 < jn;
-                    const int c = j4 / NJC;                     // chunk of the four anchors
-                    const float* bp = base + ((size_t)c * 128 + tl * G) * NJC + (j4 - c * NJC);
-                    const float* wp = wbase + c;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    int hh = 0;
-                    for (; hh + 8 <= G; hh += 8) {
-                        float4 bv[8];
-                        float mv[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            bv[u] = live ? __ldcg(reinterpret_cast<const float4*>(bp + (size_t)(hh + u) * NJC))
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                            mv[u] = live ? __ldcg(wp + (size_t)(hh + u) * p.capc) : 0.f;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float w = live ? ex2(mv[u] - mbw[hh + u]) : 0.f;
-                            acc.x = fmaf(w, bv[u].x, acc.x);
-                            acc.y = fmaf(w, bv[u].y, acc.y);
-                            acc.z = fmaf(w, bv[u].z, acc.z);
-                            acc.w = fmaf(w, bv[u].w, acc.w);
+                if constexpr (kTwoPass) {
+                    // the token's scores were summed over its heads by the softmax warps:
+                    // [chunk][token][NJC] in the slot; lane l takes anchors 4l..4l+3 of every 128
+                    for (int j0 = 0; j0 < jn; j0 += 128) {
+                        const int j4 = j0 + 4 * lane;
+                        if (j4 < jn) {
+                            const int c = j4 / NJC;
+                            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(
+                                base + ((size_t)c * TT + tl) * NJC + (j4 - c * NJC)));
+                            *reinterpret_cast<float4*>(score + j4) = v4;
                         }
                     }
-                    for (; hh < G; ++hh) {
-                        if (live) {
-                            const float4 b1 = __ldcg(reinterpret_cast<const float4*>(bp + (size_t)hh * NJC));
-                            const float w = ex2(__ldcg(wp + (size_t)hh * p.capc) - mbw[hh]);
-                            acc.x = fmaf(w, b1.x, acc.x);
-                            acc.y = fmaf(w, b1.y, acc.y);
-                            acc.z = fmaf(w, b1.z, acc.z);
-                            acc.w = fmaf(w, b1.w, acc.w);
-                        }
+                } else {
+                    const float* rs = rowstat + (pp * 2 + slot) * 2 * 128 + tl * G;
+                    // the token's heads' normalisers m_ref + log2 L, once
+                    for (int hh = lane; hh < G; hh += 32) {
+                        const float Lh = rs[128 + hh];
+                        mbw[hh] = (Lh > 0.f) ? rs[hh] + lg2(Lh) : INFINITY;
                     }
-                    if (live) *reinterpret_cast<float4*>(score + j4) = acc;
+                    __syncwarp();
+                    // P_slc'[j] = sum_h 2^(m_c - m_ref - log2 L) x banded value, where m_c
+                    // is the reference the value's chunk was written against (steps 4-5).
+                    // Lane l takes anchors 4l..4l+3 of every 128 (in one chunk, NJC % 4 == 0)
+                    // and loops over the heads, eight at a time for loads in flight.
+                    const float* wbase = base + p.capj + (size_t)(tl * G) * p.capc;
+                    // (measured on B200: the chunk weights computed here, with their
+                    // references loaded next to the banded values, beat a per-step weight
+                    // table filled first, which serialises two L2 round trips per step)
+                    for (int j0 = 0; j0 < jn; j0 += 128) {
+                        const int j4 = j0 + 4 * lane;
+                        const bool live = j4 < jn;
+                        const int c = j4 / NJC;                     // chunk of the four anchors
+                        const float* bp = base + ((size_t)c * 128 + tl * G) * NJC + (j4 - c * NJC);
+                        const float* wp = wbase + c;
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        int hh = 0;
+                        for (; hh + 8 <= G; hh += 8) {
+                            float4 bv[8];
+                            float mv[8];
+    #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                bv[u] = live ? __ldcg(reinterpret_cast<const float4*>(bp + (size_t)(hh + u) * NJC))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                                mv[u] = live ? __ldcg(wp + (size_t)(hh + u) * p.capc) : 0.f;
+                            }
+    #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const float w = live ? ex2(mv[u] - mbw[hh + u]) : 0.f;
+                                acc.x = fmaf(w, bv[u].x, acc.x);
+                                acc.y = fmaf(w, bv[u].y, acc.y);
+                                acc.z = fmaf(w, bv[u].z, acc.z);
+                                acc.w = fmaf(w, bv[u].w, acc.w);
+                            }
+                        }
+                        for (; hh < G; ++hh) {
+                            if (live) {
+                                const float4 b1 = __ldcg(reinterpret_cast<const float4*>(bp + (size_t)hh * NJC));
+                                const float w = ex2(__ldcg(wp + (size_t)hh * p.capc) - mbw[hh]);
+                                acc.x = fmaf(w, b1.x, acc.x);
+                                acc.y = fmaf(w, b1.y, acc.y);
+                                acc.z = fmaf(w, b1.z, acc.z);
+                                acc.w = fmaf(w, b1.w, acc.w);
+                            }
+                        }
+                        if (live) *reinterpret_cast<float4*>(score + j4) = acc;
+                    }
                 }
                 __syncwarp();
                 warp_topk<kMask>(score, ncand, jn, p.count, dst, lane, trow);
@@ -651,13 +698,14 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // are free
             named_bar_sync(2, 128);
             if (t.nkv > 0) {
-                const size_t band_bytes = (size_t)(t.nkv * NCH + 1) * 128 * NJC * 4;
+                // (two passes: one row of scores per token, no chunk references)
+                const size_t band_bytes = (size_t)(t.nkv * NCH + 1) * (kTwoPass ? TT : 128) * NJC * 4;
                 for (int pp = 0; pp < npipe; ++pp) {
                     const char* sb0 = reinterpret_cast<const char*>(
                         p.band + (((size_t)blockIdx.x * npipe + pp) * 2 + slot) * (size_t)p.region);
                     for (size_t o = (size_t)(warp - 8) * 32 + lane; o * 128 < band_bytes; o += 128)
                         discard_l2_line(sb0 + o * 128);
-                    const size_t mref_bytes = (size_t)128 * p.capc * 4;
+                    const size_t mref_bytes = kTwoPass ? 0 : (size_t)128 * p.capc * 4;
                     const char* mb0 = sb0 + (size_t)p.capj * 4;
                     for (size_t o = (size_t)(warp - 8) * 32 + lane; o * 128 < mref_bytes; o += 128)
                         discard_l2_line(mb0 + o * 128);
@@ -714,6 +762,198 @@ nsa_cmp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // the epilogue has finished with this slot (item tcount - 2)
                 mbar_wait(bar(B_SCR_EMPTY + 2 * pp + slot), ((tcount >> 1) & 1) ^ 1, abort_flag, p.err,
                           kErrTimeoutBase + 13);
+
+                if constexpr (kTwoPass) {
+                    // a score chunk in exponent units (x = s * ce), masked columns -inf
+                    auto load_chunk = [&](uint32_t sbase, int i, int c, int lim, float (&sx)[CH]) {
+                        uint32_t rb[CH];
+                        tmem_ld_n<CH>(sbase + c * CH, rb);
+                        tmem_wait_ld_regs<CH>(rb);
+#pragma unroll
+                        for (int e = 0; e < CH; ++e) sx[e] = __uint_as_float(rb[e]) * (pos_scale ? 1.f : c2);
+                        const int cl = lim - c * CH;
+                        if (cl < CH) {
+#pragma unroll
+                            for (int e = 0; e < CH; ++e) sx[e] = (e < cl) ? sx[e] : -INFINITY;
+                        }
+                        if constexpr (kMask) {
+                            if (arow != nullptr) {
+                                const int col0 = i * NKV + c * CH;
+                                const int w0 = col0 >> 5, b0 = col0 & 31;
+                                const uint32_t a0 = arow[w0], a1 = arow[w0 + 1], a2 = arow[w0 + 2];
+                                const uint32_t lo = __funnelshift_r(a0, a1, b0), hi = __funnelshift_r(a1, a2, b0);
+#pragma unroll
+                                for (int e = 0; e < CH; ++e)
+                                    if (((e < 32 ? lo >> e : hi >> (e - 32)) & 1u) != 0u) sx[e] = -INFINITY;
+                            }
+                        }
+                    };
+                    // ---- pass 1: the row's exact maximum m and sum L = sum 2^(x - m) ----
+                    float m = -INFINITY, L = 0.f;
+                    for (int i = 0; i < t.nkv; ++i) {
+                        const int sb = scnt % nsb;
+                        mbar_wait(bar(B_S_FULL + 2 * pp + sb), (scnt / nsb) & 1, abort_flag, p.err,
+                                  kErrTimeoutBase + 10);
+                        tc_fence_after();
+                        const uint32_t sbase = tm_sp + sb * 128;
+                        const int lim = nvis - i * NKV;
+#pragma unroll 1
+                        for (int c = 0; c < NCH; ++c) {
+                            float sx[CH];
+                            load_chunk(sbase, i, c, lim, sx);
+                            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                            for (int e = 0; e + 8 <= CH; e += 8) {
+                                mx4[0] = fmax3(mx4[0], sx[e + 0], sx[e + 1]);
+                                mx4[1] = fmax3(mx4[1], sx[e + 2], sx[e + 3]);
+                                mx4[2] = fmax3(mx4[2], sx[e + 4], sx[e + 5]);
+                                mx4[3] = fmax3(mx4[3], sx[e + 6], sx[e + 7]);
+                            }
+                            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
+                            if (mx > m) {
+                                L = (m == -INFINITY) ? 0.f : L * ex2(m - mx);
+                                m = mx;
+                            }
+                            if (m > -INFINITY) {
+                                const float2 nm2 = make_float2(-m, -m);
+                                float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                                  make_float2(0.f, 0.f)};
+#pragma unroll
+                                for (int e = 0; e < CH; e += 2) {
+                                    const float2 x = ffma2(make_float2(sx[e], sx[e + 1]), ce2, nm2);
+                                    acc2[(e >> 1) & 3] = fadd2(acc2[(e >> 1) & 3], make_float2(ex2(x.x), ex2(x.y)));
+                                }
+                                const float2 t01 = fadd2(acc2[0], acc2[1]), t23 = fadd2(acc2[2], acc2[3]);
+                                L += (t01.x + t01.y) + (t23.x + t23.y);
+                            }
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_P_FULL + pp));   // the score buffer is read
+                        ++scnt;
+                        ++pcnt;
+                    }
+                    // P~ = 2^(x - m) relative to the exact maximum (the maximum itself is 1,
+                    // exact in the storage dtype) feeds P V; the band values take P~ / L in
+                    // fp32, the normalised P of step 2.  0 for a row that attends to nothing.
+                    const float mref = (L > 0.f) ? m : INFINITY;
+                    const float inv_l = (L > 0.f) ? 1.f / L : 0.f;
+                    const float2 nmb2 = make_float2(-mref, -mref);
+                    // ---- pass 2: P, P V, and the band values summed over the token's G heads ----
+                    // The heads of a token are G adjacent lanes (G a power of two <= 32): a
+                    // transposing butterfly leaves lane h with anchors [h NJC/G, (h+1) NJC/G)
+                    // of the token's sum, written to the slot as [chunk][token][NJC].
+                    auto reduce_store = [&](float (&v)[NJC], int q) {
+                        int off = 0;
+#pragma unroll
+                        for (int st = 0, half = NJC / 2; half >= 1; ++st, half >>= 1) {
+                            const int dist = G >> (st + 1);
+                            if (dist == 0) break;
+                            const bool upper = (lane & dist) != 0;
+#pragma unroll
+                            for (int e = 0; e < half; ++e) {
+                                const float send = upper ? v[e] : v[e + half];
+                                const float keep = upper ? v[e + half] : v[e];
+                                v[e] = keep + __shfl_xor_sync(0xffffffffu, send, dist);
+                            }
+                            if (upper) off += half;
+                        }
+                        // G > NJC: the lanes that share a set of anchors finish the sum
+                        for (int dist = G / (2 * NJC); dist >= 1; dist >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], dist);
+                        const int per = NJC >= G ? NJC / G : 1;
+                        const bool writer = NJC >= G || (h % (G / NJC)) == 0;
+                        const bool in_slot = nsa_index_ok((size_t)(q + 1) * TT * NJC <= (size_t)p.capj, p.err, 4);
+                        if (valid && writer && in_slot) {
+                            float* dst = sbase_g + ((size_t)q * TT + tok_t) * NJC + off;
+#pragma unroll
+                            for (int e = 0; e < NJC; ++e)
+                                if (e < per) __stcg(dst + e, v[e]);
+                        }
+                    };
+                    float carry[NCARRY];
+#pragma unroll
+                    for (int k = 0; k < NCARRY; ++k) carry[k] = 0.f;
+                    for (int i = 0; i < t.nkv; ++i) {
+                        const int sb = scnt % nsb;
+                        mbar_wait(bar(B_S_FULL + 2 * pp + sb), (scnt / nsb) & 1, abort_flag, p.err,
+                                  kErrTimeoutBase + 10);
+                        tc_fence_after();
+                        const uint32_t sbase = tm_sp + sb * 128;
+                        const int lim = nvis - i * NKV;
+#pragma unroll 1
+                        for (int c = 0; c < NCH; ++c) {
+                            float sx[CH];
+                            load_chunk(sbase, i, c, lim, sx);
+#pragma unroll
+                            for (int e = 0; e < CH; e += 2) {
+                                const float2 x = ffma2(make_float2(sx[e], sx[e + 1]), ce2, nmb2);
+                                sx[e] = ex2(x.x);
+                                sx[e + 1] = ex2(x.y);
+                            }
+                            {
+                                uint32_t pk[CH / 2];
+#pragma unroll
+                                for (int e = 0; e < CH / 2; ++e) pk[e] = pack2<T>(sx[2 * e], sx[2 * e + 1]);
+                                tmem_st_n<CH / 2>(sbase + c * (CH / 2), pk);
+                            }
+                            float v[NJC];
+#pragma unroll
+                            for (int jj = 0; jj < NJC; ++jj) {
+                                float acc = 0.f;
+#pragma unroll
+                                for (int u = 0; u < NTAP; ++u) {
+                                    const int x = A * jj - u;
+                                    const float pv = (x >= 0) ? sx[x >= 0 ? x : 0] : carry[x < 0 ? (-x - 1) : 0];
+                                    acc = fmaf(wband[u], pv, acc);
+                                }
+                                v[jj] = acc;
+                            }
+#pragma unroll
+                            for (int k = 0; k < NCARRY; ++k) carry[k] = sx[CH - 1 - k];
+#pragma unroll
+                            for (int jj = 0; jj < NJC; ++jj) v[jj] *= inv_l;
+                            reduce_store(v, i * NCH + c);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_P_FULL + pp));
+                        ++scnt;
+                        ++pcnt;
+                    }
+                    if (t.nkv > 0) {
+                        // the first anchors past the last tile still collect taps from it
+                        float v[NJC];
+#pragma unroll
+                        for (int jj = 0; jj < NJC; ++jj) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int u = 0; u < NTAP; ++u) {
+                                const int x = A * jj - u;
+                                if (x < 0) acc = fmaf(wband[u], carry[-x - 1 >= 0 ? -x - 1 : 0], acc);
+                            }
+                            v[jj] = acc * inv_l;
+                        }
+                        reduce_store(v, t.nkv * NCH);
+                    }
+                    if (valid && nsa_index_ok(t.q_row0 + tok < p.rows_q, p.err, 3)) {
+                        const size_t si = ((size_t)(t.q_row0 + tok) * p.n1 + (size_t)t.group * G + h) * 8;
+                        const float mo = (m == -INFINITY) ? -INFINITY : m * 0.69314718055994530942f;
+                        const float4 mv = make_float4(mo, mo, mo, mo);
+                        const float4 lv = make_float4(L, L, L, L);
+                        reinterpret_cast<float4*>(p.smax + si)[0] = mv;
+                        reinterpret_cast<float4*>(p.smax + si)[1] = mv;
+                        reinterpret_cast<float4*>(p.ssum + si)[0] = lv;
+                        reinterpret_cast<float4*>(p.ssum + si)[1] = lv;
+                    }
+                    // the epilogue divides O by L (0 for a row that attends to nothing)
+                    rowstat[((pp * 2 + slot) * 2 + 0) * 128 + row] = m;
+                    rowstat[((pp * 2 + slot) * 2 + 1) * 128 + row] = L;
+                    __threadfence_block();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_ROW_DONE + 2 * pp + slot));
+                    continue;
+                }
 
                 float m_ref = -INFINITY, m_true = -INFINITY, L = 0.f;
                 float carry[NCARRY];   // carry[k] = P of the column 1 + k before the chunk
@@ -946,10 +1186,10 @@ cudaError_t launch_pack_mask(const uint8_t* src, long long s2, int ncols, int ro
     return cudaGetLastError();
 }
 
-template <typename T, int A, bool kMask>
+template <typename T, int A, bool kMask, bool kTwoPass>
 static cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, int grid, cudaStream_t st) {
-    auto kern = nsa_cmp_attn_kernel<T, A, kMask>;
+    auto kern = nsa_cmp_attn_kernel<T, A, kMask, kTwoPass>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
     kern<<<grid, kAttnThreads, p.smem_bytes, st>>>(tq, tk, tv, p);
@@ -959,15 +1199,25 @@ static cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CU
 template <typename T, bool kMask>
 static cudaError_t launch_a(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, int grid, cudaStream_t st) {
+    // two passes (head sums on chip) for 128-block KV tiles and G a power of two <= 32
+    if (p.two_pass) {
+        switch (p.a) {
+            case 1: return launch_t<T, 1, kMask, true>(p, tq, tk, tv, grid, st);
+            case 2: return launch_t<T, 2, kMask, true>(p, tq, tk, tv, grid, st);
+            case 4: return launch_t<T, 4, kMask, true>(p, tq, tk, tv, grid, st);
+            case 8: return launch_t<T, 8, kMask, true>(p, tq, tk, tv, grid, st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (p.a) {
-        case 1: return launch_t<T, 1, kMask>(p, tq, tk, tv, grid, st);
-        case 2: return launch_t<T, 2, kMask>(p, tq, tk, tv, grid, st);
-        case 3: return launch_t<T, 3, kMask>(p, tq, tk, tv, grid, st);
-        case 4: return launch_t<T, 4, kMask>(p, tq, tk, tv, grid, st);
-        case 5: return launch_t<T, 5, kMask>(p, tq, tk, tv, grid, st);
-        case 6: return launch_t<T, 6, kMask>(p, tq, tk, tv, grid, st);
-        case 7: return launch_t<T, 7, kMask>(p, tq, tk, tv, grid, st);
-        case 8: return launch_t<T, 8, kMask>(p, tq, tk, tv, grid, st);
+        case 1: return launch_t<T, 1, kMask, false>(p, tq, tk, tv, grid, st);
+        case 2: return launch_t<T, 2, kMask, false>(p, tq, tk, tv, grid, st);
+        case 3: return launch_t<T, 3, kMask, false>(p, tq, tk, tv, grid, st);
+        case 4: return launch_t<T, 4, kMask, false>(p, tq, tk, tv, grid, st);
+        case 5: return launch_t<T, 5, kMask, false>(p, tq, tk, tv, grid, st);
+        case 6: return launch_t<T, 6, kMask, false>(p, tq, tk, tv, grid, st);
+        case 7: return launch_t<T, 7, kMask, false>(p, tq, tk, tv, grid, st);
+        case 8: return launch_t<T, 8, kMask, false>(p, tq, tk, tv, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -112,6 +112,10 @@ struct AttnParams {
     const int32_t* block_table;
     int bt_stride, page_rows, pool_rows;
     long long rows_q;       // rows of q and of the outputs (debug bounds checks)
+    // two passes: exact row maxima and sums first, then normalised P, whose band
+    // values the softmax sums over a token's G heads on chip (one score row per
+    // token in the scratch); for 128-block KV tiles and G a power of two <= 32
+    int two_pass;
     // per-CTA scratch for the per-head importance values: for each pipeline,
     // two slots (consecutive items alternate) of `region` floats each.  A slot
     // holds the banded values chunk-major, [chunk][row 0..127][anchor of the

@@ -113,8 +113,13 @@ def test_decode_one_query_per_sequence(nsa):
     x, kc, vc, cuc = _inputs(wl)
     assert list(x["cu_seqlens_q"]) == list(range(1, 13))
     kp, vp, bt = _paginate(kc, vc, cuc, 64, seed=35)
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        wl.n1, wl.n2, wl.d1, wl.d2, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"]),
+        dtype=torch.uint8, device="cuda")
     res = nsa.nsa_compress_attention_paged(x["q"].cuda(), kp.cuda(), vp.cuda(), bt.cuda(), wl.scale, wl.n1, wl.l,
-                                           wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"])
+                                           wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc, x["cu_sel_kv"],
+                                           workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0
     ref = oracle.compress_attention(x["q"], kc, vc, wl.scale, wl.l, wl.d, wl.lp, wl.count, x["cu_seqlens_q"], cuc,
                                     x["cu_sel_kv"])
     check_attention(res, ref, wl.count)
@@ -152,9 +157,13 @@ def test_decode_workload_full_size_sampled_sequences(nsa):
     # the bench's decode step at full size; 8 of its 64 sequences against the oracle
     dw = workloads.DECODE_64x64K
     x = dw.generate(device="cuda")
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(
+        dw.n1, dw.n2, dw.d1, dw.d2, dw.l, dw.d, dw.lp, dw.count, x["cu_seqlens_q"], x["cu_cmp_kv"], x["cu_sel_kv"]),
+        dtype=torch.uint8, device="cuda")
     res = nsa.nsa_compress_attention_paged(x["q"], x["kcmp_pages"], x["vcmp_pages"], x["block_table"], dw.scale,
                                            dw.n1, dw.l, dw.d, dw.lp, dw.count, x["cu_seqlens_q"], x["cu_cmp_kv"],
-                                           x["cu_sel_kv"])
+                                           x["cu_sel_kv"], workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0, hex(int(ws[:4].view(torch.int32).item()))
     picks = [0, 9, 17, 31, 40, 52, 60, 63]
     bt = x["block_table"].cpu().numpy()
     kp, vp = x["kcmp_pages"].cpu(), x["vcmp_pages"].cpu()
