@@ -9,7 +9,9 @@
 // and one tensor (K or V).  The raw rows of the run are contiguous in TND
 // layout, so they are streamed through a shared-memory ring with 1D bulk
 // copies (one copy moves a few rows of every head at once).  Every raw row is
-// read from HBM once per CTA; the windows overlap in shared memory only.
+// read from HBM once per CTA; the windows overlap in shared memory only, and the
+// l - d rows two neighbouring runs share are read by both at about the same time
+// (neighbours walk in opposite directions), the second read hitting L2.
 // Each thread owns one 16-byte column vector (8 elements of one head) and
 // keeps the partial sums of the <= ceil(l/d) windows that cover the current
 // row in registers, shifting them by one slot at each group of d rows.
@@ -76,6 +78,168 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return
 template <>
 __device__ __forceinline__ float to_f32<__half>(__half x) { return __half2float(x); }
 
+// The stage loop of one run.  REV = false walks rows first to last, REV = true
+// last to first.  In both directions the register slot k holds the window that
+// started k groups of d rows before the current group q (window q - k), and the
+// current row sits at position j = k d + (row mod d) inside it; walking forward a
+// window is complete when its group of last rows is done, walking backward when
+// its first row is.
+template <typename T, int BMAX, bool REV>
+__device__ __forceinline__ void compress_run(const CompressParams& p, const CompressSeq& sq, int i0, int i1,
+                                             int nrows, int rowbytes, int rowelems, int dim,
+                                             const char* gsrc, T* __restrict__ dst, const float* wsm,
+                                             uint64_t* bars, volatile int* abort_flag, uint8_t* stages) {
+    const int l = p.l, d = p.d;
+    const int nb = (l + d - 1) / d;                  // windows covering one row
+    const int nvec = rowelems / 8;                   // 16-byte vectors per row
+    const int rs = p.rows_per_stage;
+    const int nstage = (nrows + rs - 1) / rs;
+    const int stage_bytes = rs * rowbytes;
+    // stage n of the walk covers the run's stage REV ? nstage - 1 - n : n
+    auto stage_of = [&](int n) { return REV ? nstage - 1 - n : n; };
+    auto issue = [&](int n) {
+        const int slot = n % kCompressStages;
+        const int sg = stage_of(n);
+        const int rows = min(rs, nrows - sg * rs);
+        const uint32_t bytes = (uint32_t)(rows * rowbytes);
+        const uint32_t bar = smem_u32(&bars[slot]);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(smem_u32(stages + slot * stage_bytes), gsrc + (int64_t)sg * stage_bytes, bytes, bar);
+    };
+    if (threadIdx.x == 0) {
+        for (int n = 0; n < kCompressStages && n < nstage; ++n) issue(n);
+    }
+
+    const int cv = threadIdx.x;                      // column vector of this thread
+    const bool active = cv < nvec;
+    const int head = active ? (cv * 8) / dim : 0;
+    float acc[BMAX][8];
+#pragma unroll
+    for (int k = 0; k < BMAX; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+
+    // the store of window i (the slot kk that holds it)
+    auto store = [&](int i, int kk) {
+        if (i < i0 || i >= i1) return;
+        float o[8];
+#pragma unroll
+        for (int k = 0; k < BMAX; ++k)
+            if (k == kk)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = acc[k][e];
+        int64_t orow = (int64_t)sq.cmp_start + i;
+        bool ok_row = p.block_table != nullptr || nsa_index_ok(orow < p.tc_rows, &g_compress_err, 6);
+        if (p.block_table != nullptr) {
+            // the page comes from the caller's table: out-of-pool entries
+            // are reported, never written through
+            const int pg = p.block_table[(size_t)sq.seq * p.bt_stride + i / p.page_rows];
+            ok_row = pg >= 0 && pg < p.num_pages;
+            orow = (int64_t)pg * p.page_rows + i % p.page_rows;
+            if (!ok_row) atomicCAS(&g_compress_err, 0, kErrBadPage);
+        }
+        if (ok_row) {
+            T* out = dst + orow * rowelems + cv * 8;
+            *reinterpret_cast<uint4*>(out) = pack8<T>(o);
+        }
+    };
+    // one row at position j = k d + rin of window q - k, for every slot
+    auto add_row = [&](const uint4& u, int rin) {
+        float x[8];
+        cvt8<T>(u, x);
+#pragma unroll
+        for (int k = 0; k < BMAX; ++k) {
+            const int j = k * d + rin;
+            if (k < nb && j < l) {
+                const float wv = wsm[j * p.n2 + head];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wv, x[e], acc[k][e]);
+            }
+        }
+    };
+
+    // forward: the group of the first row and the row's place in it; backward: the
+    // same for the first of the last four rows (nrows, d and every stage's row
+    // count are multiples of 4, so four rows never straddle a group)
+    int q = REV ? i0 + (nrows - 4) / d : i0;
+    int rin = REV ? (nrows - 4) % d : 0;
+    int next_issue = min(kCompressStages, nstage);   // stages handed to the copy engine
+    int n = 0;
+    bool failed = false;
+    for (; n < nstage; ++n) {
+        const int slot = n % kCompressStages;
+        const uint32_t parity = (uint32_t)((n / kCompressStages) & 1);
+        const bool got = mbar_wait(smem_u32(&bars[slot]), parity, abort_flag, &g_compress_err,
+                                   kErrTimeoutBase + 1);
+        const int rows = min(rs, nrows - stage_of(n) * rs);
+        const uint8_t* base = stages + slot * stage_bytes;
+        if (active && got) {
+            if constexpr (!REV) {
+                // four rows per step: their loads are independent
+                for (int r = 0; r < rows; r += 4) {
+                    uint4 u[4];
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr)
+                        u[rr] = *reinterpret_cast<const uint4*>(base + (r + rr) * rowbytes + cv * 16);
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) add_row(u[rr], rin + rr);
+                    rin += 4;
+                    const bool last_row = (n == nstage - 1) && (r + 4 == rows);
+                    if (rin == d || last_row) {
+                        // window q-(nb-1) has seen its last row: store it, shift slots up
+                        store(q - (nb - 1), nb - 1);
+#pragma unroll
+                        for (int kk = BMAX - 1; kk >= 1; --kk)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[kk][e] = acc[kk - 1][e];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[0][e] = 0.f;
+                        rin = 0;
+                        ++q;
+                    }
+                }
+            } else {
+                for (int r = rows - 4; r >= 0; r -= 4) {
+                    uint4 u[4];
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr)
+                        u[rr] = *reinterpret_cast<const uint4*>(base + (r + rr) * rowbytes + cv * 16);
+#pragma unroll
+                    for (int rr = 3; rr >= 0; --rr) add_row(u[rr], rin + rr);
+                    if (rin == 0) {
+                        // window q has seen its first row: store it, shift slots down
+                        store(q, 0);
+#pragma unroll
+                        for (int kk = 0; kk + 1 < BMAX; ++kk)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[kk][e] = acc[kk + 1][e];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[BMAX - 1][e] = 0.f;
+                        rin = d - 4;
+                        --q;
+                    } else {
+                        rin -= 4;
+                    }
+                }
+            }
+        }
+        // every thread is done with this slot, and all agree whether the wait succeeded
+        if (!__syncthreads_and(got ? 1 : 0)) { failed = true; break; }
+        if (threadIdx.x == 0 && next_issue < nstage) issue(next_issue);
+        if (next_issue < nstage) ++next_issue;
+    }
+    if (failed && threadIdx.x == 0) {
+        // a wait gave up: let the copies still in flight land before the CTA exits
+        for (int u = n; u < next_issue; ++u) {
+            const uint32_t bar = smem_u32(&bars[u % kCompressStages]);
+            const uint32_t parity = (uint32_t)((u / kCompressStages) & 1);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < 100000000ull) {
+            }
+        }
+    }
+}
+
 // One CTA = one run of output blocks [i0, i1) of one sequence of one tensor.
 // BMAX >= ceil(l/d): number of register slots for overlapping windows.
 template <typename T, int BMAX>
@@ -100,14 +264,10 @@ nsa_compress_kernel(const CompressParams p) {
     if (i0 >= i1) return;
 
     const int l = p.l, d = p.d;
-    const int nb = (l + d - 1) / d;                  // windows covering one row
     const int rowelems = p.n2 * dim;
     const int rowbytes = rowelems * (int)sizeof(T);
-    const int nvec = rowelems / 8;                   // 16-byte vectors per row
     const int64_t rel0 = (int64_t)i0 * d;            // first raw row of the run (in seq)
     const int nrows = (i1 - 1 - i0) * d + l;         // raw rows of the run
-    const int rs = p.rows_per_stage;
-    const int nstage = (nrows + rs - 1) / rs;
     const char* gsrc = reinterpret_cast<const char*>(src) +
                        ((int64_t)sq.raw_start + rel0) * (int64_t)rowbytes;
 
@@ -117,7 +277,6 @@ nsa_compress_kernel(const CompressParams p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + wbytes);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + wbytes + 8 * kCompressStages);
     uint8_t* stages = smem_raw + wbytes + 128;
-    const int stage_bytes = rs * rowbytes;
 
     const T* wsrc = reinterpret_cast<const T*>(p.w);
     for (int i = threadIdx.x; i < l * p.n2; i += blockDim.x) wsm[i] = to_f32<T>(wsrc[i]);
@@ -129,115 +288,17 @@ nsa_compress_kernel(const CompressParams p) {
     }
     __syncthreads();
 
-    auto issue = [&](int s) {
-        const int slot = s % kCompressStages;
-        const int rows = min(rs, nrows - s * rs);
-        const uint32_t bytes = (uint32_t)(rows * rowbytes);
-        const uint32_t bar = smem_u32(&bars[slot]);
-        mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(smem_u32(stages + slot * stage_bytes), gsrc + (int64_t)s * stage_bytes, bytes, bar);
-    };
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kCompressStages && s < nstage; ++s) issue(s);
-    }
-
-    const int cv = threadIdx.x;                      // column vector of this thread
-    const bool active = cv < nvec;
-    const int head = active ? (cv * 8) / dim : 0;
-    float acc[BMAX][8];
-#pragma unroll
-    for (int k = 0; k < BMAX; ++k)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
-
-    int q = i0;                                      // rel / d
-    int rin = 0;                                     // rel % d
-    int next_issue = min(kCompressStages, nstage);   // stages handed to the copy engine
-    int s = 0;
-    bool failed = false;
-    for (; s < nstage; ++s) {
-        const int slot = s % kCompressStages;
-        const uint32_t parity = (uint32_t)((s / kCompressStages) & 1);
-        const bool got = mbar_wait(smem_u32(&bars[slot]), parity, abort_flag, &g_compress_err,
-                                   kErrTimeoutBase + 1);
-        const int rows = min(rs, nrows - s * rs);
-        const uint8_t* base = stages + slot * stage_bytes;
-        if (active && got) {
-            // four rows per step: their loads are independent (rows and d are
-            // multiples of 4, so a window group never ends inside a step)
-            for (int r = 0; r < rows; r += 4) {
-                uint4 u[4];
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-                    u[rr] = *reinterpret_cast<const uint4*>(base + (r + rr) * rowbytes + cv * 16);
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    float x[8];
-                    cvt8<T>(u[rr], x);
-#pragma unroll
-                    for (int k = 0; k < BMAX; ++k) {
-                        const int j = k * d + rin + rr;       // position inside window q-k
-                        if (k < nb && j < l) {
-                            const float wv = wsm[j * p.n2 + head];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wv, x[e], acc[k][e]);
-                        }
-                    }
-                }
-                rin += 4;
-                const bool last_row = (s == nstage - 1) && (r + 4 == rows);
-                if (rin == d || last_row) {
-                    // window q-(nb-1) has seen its last row: store it, shift slots
-                    const int i = q - (nb - 1);
-                    if (i >= i0 && i < i1) {
-                        float o[8];
-#pragma unroll
-                        for (int kk = 0; kk < BMAX; ++kk)
-                            if (kk == nb - 1)
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) o[e] = acc[kk][e];
-                        int64_t orow = (int64_t)sq.cmp_start + i;
-                        bool ok_row = p.block_table != nullptr ||
-                                      nsa_index_ok(orow < p.tc_rows, &g_compress_err, 6);
-                        if (p.block_table != nullptr) {
-                            // the page comes from the caller's table: out-of-pool entries
-                            // are reported, never written through
-                            const int pg = p.block_table[(size_t)sq.seq * p.bt_stride + i / p.page_rows];
-                            ok_row = pg >= 0 && pg < p.num_pages;
-                            orow = (int64_t)pg * p.page_rows + i % p.page_rows;
-                            if (!ok_row) atomicCAS(&g_compress_err, 0, kErrBadPage);
-                        }
-                        if (ok_row) {
-                            T* out = dst + orow * rowelems + cv * 8;
-                            *reinterpret_cast<uint4*>(out) = pack8<T>(o);
-                        }
-                    }
-#pragma unroll
-                    for (int kk = BMAX - 1; kk >= 1; --kk)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[kk][e] = acc[kk - 1][e];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[0][e] = 0.f;
-                    rin = 0;
-                    ++q;
-                }
-            }
-        }
-        // every thread is done with this slot, and all agree whether the wait succeeded
-        if (!__syncthreads_and(got ? 1 : 0)) { failed = true; break; }
-        if (threadIdx.x == 0 && next_issue < nstage) issue(next_issue);
-        if (next_issue < nstage) ++next_issue;
-    }
-    if (failed && threadIdx.x == 0) {
-        // a wait gave up: let the copies still in flight land before the CTA exits
-        for (int u = s; u < next_issue; ++u) {
-            const uint32_t bar = smem_u32(&bars[u % kCompressStages]);
-            const uint32_t parity = (uint32_t)((u / kCompressStages) & 1);
-            const unsigned long long t0 = globaltimer();
-            while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < 100000000ull) {
-            }
-        }
-    }
+    // Adjacent runs walk their rows in opposite directions: a run and its neighbour
+    // reach the l - d rows they share at about the same time (both at their ends, or
+    // both at their starts), so the second read of those rows is an L2 hit instead of
+    // a second trip to HBM.  (Up to four windows per row; with more, the backward
+    // form's registers would spill, and every run walks forward.)
+    if (BMAX <= 4 && (chunk & 1))
+        compress_run<T, BMAX, true>(p, sq, i0, i1, nrows, rowbytes, rowelems, dim, gsrc, dst, wsm, bars,
+                                     abort_flag, stages);
+    else
+        compress_run<T, BMAX, false>(p, sq, i0, i1, nrows, rowbytes, rowelems, dim, gsrc, dst, wsm, bars,
+                                      abort_flag, stages);
 }
 
 template <typename T, int BMAX>
