@@ -175,6 +175,43 @@ def test_reference_maximum_moves(nsa, step, dd):
     print(rep)
 
 
+def _staircase_short(nsa, n1, n2, dd, seqs, nq, step, l=32, d=16, lp=64, count=8):
+    """The last nq queries of each sequence against keys whose first component
+    climbs by 10/3 (natural units) every `step` blocks of a sequence."""
+    g = torch.Generator().manual_seed(11)
+    scale = dd ** -0.5
+    cu = np.cumsum(seqs).astype(np.int32)
+    cuc = oracle.compress_len(cu, l, d)
+    cus = np.cumsum([-(-s_ // lp) for s_ in seqs]).astype(np.int32)
+    cuq = np.cumsum([min(nq, s_) for s_ in seqs]).astype(np.int32)
+    q = torch.randn(int(cuq[-1]), n1, dd, generator=g)
+    q[:, :, 0] = 1.0
+    kc = torch.randn(int(cuc[-1]), n2, dd, generator=g)
+    pos = torch.cat([torch.arange(int(cuc[i]) - (int(cuc[i - 1]) if i else 0)) for i in range(len(seqs))])
+    kc[:, :, 0] = (10.0 / scale) * torch.div(pos, step, rounding_mode="floor")[:, None].float() / 3.0
+    vc = torch.randn(int(cuc[-1]), n2, dd, generator=g)
+    q, kc, vc = q.to(torch.bfloat16), kc.to(torch.bfloat16), vc.to(torch.bfloat16)
+    ws = torch.empty(nsa.nsa_compress_attention_workspace_size(n1, n2, dd, dd, l, d, lp, count, cuq, cuc, cus),
+                     dtype=torch.uint8, device="cuda")
+    res = nsa.nsa_compress_attention(q.cuda(), kc.cuda(), vc.cuda(), scale, n1, l, d, lp, count, cuq, cuc, cus,
+                                     workspace=ws)
+    assert nsa.nsa_workspace_status(ws) == 0
+    ref = oracle.compress_attention(q, kc, vc, scale, l, d, lp, count, cuq, cuc, cus)
+    return check_attention(res, ref, count, out_rel=2.0 ** -7)
+
+
+@pytest.mark.parametrize("n1,dd,nq", [(16, 256, 16), (128, 256, 3000), (24, 256, 3000)],
+                         ids=["g8_d256_16q", "g64_d256", "g12_d256"])
+def test_one_pass_one_pipeline(nsa, n1, dd, nq):
+    """The one-pass kernel with one pipeline and two score buffers (D2 > 128),
+    many items per CTA and a reference maximum that moves: G = 8 with at most
+    one M-tile of queries per sequence (300 sequences of 16 queries), G = 64
+    (above the two-pass range) and G = 12 (not a power of two) over whole
+    sequences."""
+    seqs = [3000 - 7 * (i % 50) for i in range(300)] if nq == 16 else [3000, 2500]
+    print(_staircase_short(nsa, n1, 2, dd, seqs, nq, step=7))
+
+
 @pytest.mark.parametrize("scale", [-0.125, 0.0])
 def test_non_positive_scale(nsa, scale):
     g = torch.Generator().manual_seed(12)
