@@ -654,8 +654,10 @@ static nsa_status_t compress_impl(const void* k, const void* v, const void* w, i
     // sizes of the per-CTA ring and the output run of one CTA
     const int rowbytes = (int)(rowelems * 2);
     // rows per bulk copy: about 8 KB, a multiple of 4 (the kernel steps 4 rows at a time).
-    // Measured on B200 against 16 KB and 32 KB stages and 3-8 deep rings: 8 KB x 4 gives
-    // the smallest CTAs (about 6 per SM) and the highest read rate.
+    // Measured on B200 against 16 KB and 32 KB stages and 3-8 deep rings, and, once
+    // neighbouring runs shared their overlap rows through L2, against 3, 4 and 6 deep
+    // rings of 8 KB: 8 KB x 2 gives the smallest CTAs (eight per SM, the register limit)
+    // and the highest read rate (262144 tokens: 219 us against 229 / 234 / 261 us).
     int rs = std::max(4, (8192 / rowbytes) & ~3);
     const int stage_bytes = rs * rowbytes;
     const int wbytes = ((l * n2 * 4) + 127) & ~127;

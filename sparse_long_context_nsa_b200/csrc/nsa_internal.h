@@ -8,7 +8,7 @@
 namespace nsa {
 
 // ------------------------------------------------------------ compress
-constexpr int kCompressStages = 4;        // shared-memory ring depth
+constexpr int kCompressStages = 2;        // shared-memory ring depth
 constexpr int kCompressMaxThreads = 512;  // one thread per 16-byte column vector
 constexpr int kCompressMaxSeq = 96;       // sequences per launch (kernel-parameter space)
 
