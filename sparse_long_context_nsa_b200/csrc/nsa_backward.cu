@@ -610,14 +610,11 @@ cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMa
 }
 
 // ---------------------------------------------------- compression transposed
-template <typename T>
-__device__ __forceinline__ float ld_elem(const void* base, size_t idx) {
-    return static_cast<float>(reinterpret_cast<const T*>(base)[idx]);
-}
 
 // dk[p] = sum_i w[p - i d] dkcmp_i over the windows i covering raw row p
 // (dv likewise).  A CTA takes kRowsPerCta raw rows of one sequence; a thread
-// one (head, 4 consecutive dims) column.
+// one (head, 4 consecutive dims) column, four rows at a time: the loads of
+// the four rows are issued before their sums and stores.
 template <typename T>
 __global__ void compress_dx_kernel(const CompressBwdParams p) {
     int s = 0;
@@ -627,55 +624,85 @@ __global__ void compress_dx_kernel(const CompressBwdParams p) {
     const int r0 = ((int)blockIdx.x - blk0) * kRowsPerCta;
     const bool is_v = blockIdx.y == 1;
     const int dim = is_v ? p.d2 : p.d1;
-    const float* g = is_v ? p.dvcmp : p.dkcmp;
-    float* dx = is_v ? p.dv : p.dk;
+    const float* __restrict__ g = is_v ? p.dvcmp : p.dkcmp;
+    float* __restrict__ dx = is_v ? p.dv : p.dk;
+    const T* __restrict__ w = reinterpret_cast<const T*>(p.w);
     const int ncol = p.n2 * dim / 4;
-    for (int rr = 0; rr < kRowsPerCta; ++rr) {
-        const int pr = r0 + rr;   // raw row inside the sequence
-        if (pr >= q.raw_len) break;
-        if (!nsa_index_ok(q.raw_start + pr < p.t2, nullptr, 11)) break;
-        // windows i with i d <= pr < i d + l
-        int i_lo = pr - p.l + 1 <= 0 ? 0 : (pr - p.l + 1 + p.d - 1) / p.d;
-        int i_hi = min(pr / p.d, q.n_cmp - 1);
-        for (int col = threadIdx.x; col < ncol; col += blockDim.x) {
-            const int n = (col * 4) / dim, e = (col * 4) % dim;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int i = i_lo; i <= i_hi; ++i) {
-                const float wv = ld_elem<T>(p.w, (size_t)(pr - i * p.d) * p.n2 + n);
-                const float4 gv = *reinterpret_cast<const float4*>(g + ((size_t)(q.cmp_start + i) * p.n2 + n) * dim + e);
-                acc.x = fmaf(wv, gv.x, acc.x);
-                acc.y = fmaf(wv, gv.y, acc.y);
-                acc.z = fmaf(wv, gv.z, acc.z);
-                acc.w = fmaf(wv, gv.w, acc.w);
+    const int nb = (p.l + p.d - 1) / p.d;   // windows covering a row, at most
+    for (int col = threadIdx.x; col < ncol; col += blockDim.x) {
+        const int n = (col * 4) / dim, e = (col * 4) % dim;
+        for (int rr = 0; rr < kRowsPerCta; rr += 4) {
+            float4 acc[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                const int pr = r0 + rr + u;   // raw row inside the sequence
+                if (pr >= q.raw_len) continue;
+                // windows i with i d <= pr < i d + l
+                const int i_lo = pr - p.l + 1 <= 0 ? 0 : (pr - p.l + 1 + p.d - 1) / p.d;
+                const int i_hi = min(pr / p.d, q.n_cmp - 1);
+                for (int k = 0; k < nb; ++k) {
+                    const int i = i_lo + k;
+                    if (i > i_hi) break;
+                    const float wv = static_cast<float>(w[(size_t)(pr - i * p.d) * p.n2 + n]);
+                    const float4 gv = __ldg(reinterpret_cast<const float4*>(
+                        g + ((size_t)(q.cmp_start + i) * p.n2 + n) * dim + e));
+                    acc[u].x = fmaf(wv, gv.x, acc[u].x);
+                    acc[u].y = fmaf(wv, gv.y, acc[u].y);
+                    acc[u].z = fmaf(wv, gv.z, acc[u].z);
+                    acc[u].w = fmaf(wv, gv.w, acc[u].w);
+                }
             }
-            *reinterpret_cast<float4*>(dx + ((size_t)(q.raw_start + pr) * p.n2 + n) * dim + e) = acc;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int pr = r0 + rr + u;
+                if (pr >= q.raw_len || !nsa_index_ok(q.raw_start + pr < p.t2, nullptr, 11)) continue;
+                // written once: stream past L2
+                __stcs(reinterpret_cast<float4*>(dx + ((size_t)(q.raw_start + pr) * p.n2 + n) * dim + e), acc[u]);
+            }
         }
     }
 }
 
 // dw[j, n] = sum_i (dkcmp_i . k[i d + j] + dvcmp_i . v[i d + j]) over every
-// compressed row, one CTA per (j, n), fixed-order block reduction.
+// compressed row, one CTA per (j, n), fixed-order block reduction.  A thread
+// reads four elements of k or v in one 8-byte load, four such loads in flight.
 template <typename T>
 __global__ void compress_dw_kernel(const CompressBwdParams p) {
     const int j = blockIdx.x, n = blockIdx.y;
     const int c4k = p.d1 / 4, c4v = p.d2 / 4;
     float acc = 0.f;
     const long long total = p.tc * (c4k + c4v);
-    for (long long x = threadIdx.x; x < total; x += blockDim.x) {
-        const long long i = x / (c4k + c4v);
-        const int c = (int)(x - i * (c4k + c4v));
-        const bool is_v = c >= c4k;
-        const int dim = is_v ? p.d2 : p.d1;
-        const int e = (is_v ? c - c4k : c) * 4;
-        const float* g = (is_v ? p.dvcmp : p.dkcmp) + ((size_t)i * p.n2 + n) * dim + e;
-        const size_t raw = (size_t)p.cmp_raw[i] + j;
-        const void* src = is_v ? p.v : p.k;
-        const float4 gv = *reinterpret_cast<const float4*>(g);
-        const size_t xi = (raw * p.n2 + n) * dim + e;
-        acc = fmaf(gv.x, ld_elem<T>(src, xi), acc);
-        acc = fmaf(gv.y, ld_elem<T>(src, xi + 1), acc);
-        acc = fmaf(gv.z, ld_elem<T>(src, xi + 2), acc);
-        acc = fmaf(gv.w, ld_elem<T>(src, xi + 3), acc);
+    constexpr int U = 4;   // elements of the stride loop whose loads are in flight together
+    for (long long x0 = threadIdx.x; x0 < total; x0 += (long long)U * blockDim.x) {
+        float4 gv[U];
+        uint2 u[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const long long x = x0 + (long long)k * blockDim.x;
+            gv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            u[k] = make_uint2(0u, 0u);
+            if (x >= total) continue;
+            const long long i = x / (c4k + c4v);
+            const int c = (int)(x - i * (c4k + c4v));
+            const bool is_v = c >= c4k;
+            const int dim = is_v ? p.d2 : p.d1;
+            const int e = (is_v ? c - c4k : c) * 4;
+            const float* g = (is_v ? p.dvcmp : p.dkcmp) + ((size_t)i * p.n2 + n) * dim + e;
+            const size_t raw = (size_t)p.cmp_raw[i] + j;
+            const T* src = reinterpret_cast<const T*>(is_v ? p.v : p.k);
+            gv[k] = __ldg(reinterpret_cast<const float4*>(g));
+            const size_t xi = (raw * p.n2 + n) * dim + e;   // a multiple of 4 elements: 8-byte aligned
+            u[k] = __ldg(reinterpret_cast<const uint2*>(src + xi));
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const float2 a = up2<T>(u[k].x), b = up2<T>(u[k].y);
+            acc = fmaf(gv[k].x, a.x, acc);
+            acc = fmaf(gv[k].y, a.y, acc);
+            acc = fmaf(gv[k].z, b.x, acc);
+            acc = fmaf(gv[k].w, b.y, acc);
+        }
     }
     __shared__ float red[32];
 #pragma unroll
