@@ -393,7 +393,8 @@ nsa_status_t nsa_compress_attention_backward(
     void* stream);
 
 /*
- * Bytes of device workspace nsa_compress_backward needs (host computation).
+ * Bytes of device workspace nsa_compress_backward needs (host computation): a
+ * header, one int per compressed row and 4 MiB for the dw partial sums.
  */
 nsa_status_t nsa_compress_backward_workspace_size(const int32_t* cu_seqlens, int batch, int l, int d,
                                                   size_t* bytes);
@@ -410,8 +411,10 @@ nsa_status_t nsa_compress_backward_workspace_size(const int32_t* cu_seqlens, int
  *   dk, dv             device (T, N2, D1) / (T, N2, D2) fp32, overwritten
  *   dw                 device (l, N2) fp32, overwritten
  *   workspace          device, >= the size above, 256-byte aligned
- * Constraints: those of nsa_compress.  Deterministic: dw is reduced per (j, n)
- * by one CTA in a fixed order.
+ * Constraints: those of nsa_compress; l * N2 * 4 bytes at most 4 MiB
+ * (NSA_ERR_UNSUPPORTED beyond).  Deterministic: dw is summed in partial sums
+ * over runs of consecutive compressed rows (in the workspace), then over the
+ * runs in run order.  Three launches for dk / dv, dw partials and their sum.
  */
 nsa_status_t nsa_compress_backward(
     const void* k, const void* v, const void* w, const float* dkcmp, const float* dvcmp, int l, int d,

@@ -1247,6 +1247,10 @@ nsa_status_t nsa_compress_attention_backward(const void* q, const void* kcmp, co
     return NSA_OK;
 }
 
+// the dw partial sums ([run][l][n2] fp32) get a fixed part of the workspace: as many runs as
+// fit, up to about eight CTAs per SM
+constexpr size_t kDwPartBytes = (size_t)4 << 20;
+
 nsa_status_t nsa_compress_backward_workspace_size(const int32_t* cu_seqlens, int batch, int l, int d,
                                                   size_t* bytes) {
     if (bytes == nullptr || l < 1 || d < 1) return NSA_ERR_INVALID_ARG;
@@ -1258,7 +1262,7 @@ nsa_status_t nsa_compress_backward_workspace_size(const int32_t* cu_seqlens, int
         tc += ncmp_of((int64_t)cu_seqlens[b] - prev, l, d);
         prev = cu_seqlens[b];
     }
-    *bytes = kWsHeader + (((size_t)tc * 4 + 255) & ~(size_t)255);
+    *bytes = kWsHeader + (((size_t)tc * 4 + 255) & ~(size_t)255) + kDwPartBytes;
     return NSA_OK;
 }
 
@@ -1312,6 +1316,23 @@ nsa_status_t nsa_compress_backward(const void* k, const void* v, const void* w, 
     p.dw = dw;
     p.cmp_raw = reinterpret_cast<const int*>(ws + kWsHeader);
     p.tc = (long long)cmp_raw.size();
+    // dw runs: about eight CTAs per SM over (runs x head groups), within the partial budget
+    int nruns = 0;
+    if (p.tc > 0) {
+        const size_t per_run = (size_t)l * n2 * 4;
+        if (per_run > kDwPartBytes) return NSA_ERR_UNSUPPORTED;
+        int dev = 0, nsm = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        const int hpc = bwd::compress_dw_heads_per_cta(l);
+        const int64_t ygroups = (n2 + hpc - 1) / hpc;
+        int64_t want = std::max<int64_t>(1, (int64_t)nsm * 8 / ygroups);
+        want = std::min<int64_t>(want, (int64_t)(kDwPartBytes / per_run));
+        want = std::min<int64_t>(want, p.tc);
+        p.dw_run = (int)((p.tc + want - 1) / want);
+        nruns = (int)((p.tc + p.dw_run - 1) / p.dw_run);
+    }
+    p.dw_part = reinterpret_cast<float*>(ws + kWsHeader + ((cmp_raw.size() * 4 + 255) & ~(size_t)255));
     p.t2 = cu_seqlens[batch - 1];
     p.l = l;
     p.d = d;
@@ -1343,7 +1364,7 @@ nsa_status_t nsa_compress_backward(const void* k, const void* v, const void* w, 
         }
         if (blocks > 0 && bwd::launch_compress_bwd_dx(p, blocks, st) != cudaSuccess) return NSA_ERR_CUDA;
     }
-    if (bwd::launch_compress_bwd_dw(p, st) != cudaSuccess) return NSA_ERR_CUDA;
+    if (bwd::launch_compress_bwd_dw(p, nruns, st) != cudaSuccess) return NSA_ERR_CUDA;
     return NSA_OK;
 }
 

@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include "nsa_internal.h"
@@ -665,56 +666,80 @@ __global__ void compress_dx_kernel(const CompressBwdParams p) {
 }
 
 // dw[j, n] = sum_i (dkcmp_i . k[i d + j] + dvcmp_i . v[i d + j]) over every
-// compressed row, one CTA per (j, n), fixed-order block reduction.  A thread
-// reads four elements of k or v in one 8-byte load, four such loads in flight.
+// compressed row i, in two steps.  Partial sums: a CTA takes a run of
+// consecutive compressed rows (p.dw_run of them, across sequence boundaries:
+// cmp_raw gives each row's first raw row) and heads [y hpc, (y+1) hpc); thread
+// (h, j) sums the dot products of window position j over the run, reading raw
+// row cmp_raw[i] + j (a warp reads 32 consecutive rows of one head, and
+// neighbouring windows' rows again from cache).  Then dw = the partials summed
+// over the runs in run order (deterministic).
 template <typename T>
-__global__ void compress_dw_kernel(const CompressBwdParams p) {
-    const int j = blockIdx.x, n = blockIdx.y;
-    const int c4k = p.d1 / 4, c4v = p.d2 / 4;
+__global__ void compress_dw_part_kernel(const CompressBwdParams p) {
+    const int hpc = blockDim.x / p.l;
+    const int h = threadIdx.x / p.l, j = threadIdx.x - h * p.l;
+    const int n = blockIdx.y * hpc + h;
+    if (h >= hpc) return;
+    const long long i0 = (long long)blockIdx.x * p.dw_run;
+    const long long i1 = min(i0 + p.dw_run, p.tc);
     float acc = 0.f;
-    const long long total = p.tc * (c4k + c4v);
-    constexpr int U = 4;   // elements of the stride loop whose loads are in flight together
-    for (long long x0 = threadIdx.x; x0 < total; x0 += (long long)U * blockDim.x) {
-        float4 gv[U];
-        uint2 u[U];
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const long long x = x0 + (long long)k * blockDim.x;
-            gv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            u[k] = make_uint2(0u, 0u);
-            if (x >= total) continue;
-            const long long i = x / (c4k + c4v);
-            const int c = (int)(x - i * (c4k + c4v));
-            const bool is_v = c >= c4k;
-            const int dim = is_v ? p.d2 : p.d1;
-            const int e = (is_v ? c - c4k : c) * 4;
-            const float* g = (is_v ? p.dvcmp : p.dkcmp) + ((size_t)i * p.n2 + n) * dim + e;
-            const size_t raw = (size_t)p.cmp_raw[i] + j;
-            const T* src = reinterpret_cast<const T*>(is_v ? p.v : p.k);
-            gv[k] = __ldg(reinterpret_cast<const float4*>(g));
-            const size_t xi = (raw * p.n2 + n) * dim + e;   // a multiple of 4 elements: 8-byte aligned
-            u[k] = __ldg(reinterpret_cast<const uint2*>(src + xi));
+    if (n < p.n2) {
+        const T* __restrict__ kk = reinterpret_cast<const T*>(p.k);
+        const T* __restrict__ vv = reinterpret_cast<const T*>(p.v);
+        for (long long i = i0; i < i1; ++i) {
+            const long long r = (long long)p.cmp_raw[i] + j;
+            if (!nsa_index_ok(r < p.t2, nullptr, 12)) continue;
+            const float* gk = p.dkcmp + ((size_t)i * p.n2 + n) * p.d1;
+            const T* xk = kk + ((size_t)r * p.n2 + n) * p.d1;
+#pragma unroll 2
+            for (int e = 0; e < p.d1; e += 8) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(xk + e));
+                const float4 g0 = __ldg(reinterpret_cast<const float4*>(gk + e));
+                const float4 g1 = __ldg(reinterpret_cast<const float4*>(gk + e + 4));
+                const float2 a0 = up2<T>(u.x), a1 = up2<T>(u.y), a2 = up2<T>(u.z), a3 = up2<T>(u.w);
+                acc = fmaf(g0.x, a0.x, acc);
+                acc = fmaf(g0.y, a0.y, acc);
+                acc = fmaf(g0.z, a1.x, acc);
+                acc = fmaf(g0.w, a1.y, acc);
+                acc = fmaf(g1.x, a2.x, acc);
+                acc = fmaf(g1.y, a2.y, acc);
+                acc = fmaf(g1.z, a3.x, acc);
+                acc = fmaf(g1.w, a3.y, acc);
+            }
+            if (p.dvcmp != nullptr) {
+                const float* gv = p.dvcmp + ((size_t)i * p.n2 + n) * p.d2;
+                const T* xv = vv + ((size_t)r * p.n2 + n) * p.d2;
+#pragma unroll 2
+                for (int e = 0; e < p.d2; e += 8) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(xv + e));
+                    const float4 g0 = __ldg(reinterpret_cast<const float4*>(gv + e));
+                    const float4 g1 = __ldg(reinterpret_cast<const float4*>(gv + e + 4));
+                    const float2 a0 = up2<T>(u.x), a1 = up2<T>(u.y), a2 = up2<T>(u.z), a3 = up2<T>(u.w);
+                    acc = fmaf(g0.x, a0.x, acc);
+                    acc = fmaf(g0.y, a0.y, acc);
+                    acc = fmaf(g0.z, a1.x, acc);
+                    acc = fmaf(g0.w, a1.y, acc);
+                    acc = fmaf(g1.x, a2.x, acc);
+                    acc = fmaf(g1.y, a2.y, acc);
+                    acc = fmaf(g1.z, a3.x, acc);
+                    acc = fmaf(g1.w, a3.y, acc);
+                }
+            }
         }
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const float2 a = up2<T>(u[k].x), b = up2<T>(u[k].y);
-            acc = fmaf(gv[k].x, a.x, acc);
-            acc = fmaf(gv[k].y, a.y, acc);
-            acc = fmaf(gv[k].z, b.x, acc);
-            acc = fmaf(gv[k].w, b.y, acc);
-        }
+        p.dw_part[((size_t)blockIdx.x * p.l + j) * p.n2 + n] = acc;
     }
-    __shared__ float red[32];
+}
+
+// one warp per (j, n) of dw: lane k sums runs k, k + 32, ... in order, then a
+// fixed butterfly sums the lanes
+__global__ void compress_dw_reduce_kernel(const CompressBwdParams p, int nruns) {
+    const int x = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // (j, n) of dw
+    const int lane = threadIdx.x & 31;
+    if (x >= p.l * p.n2) return;
+    float acc = 0.f;
+    for (int u = lane; u < nruns; u += 32) acc += p.dw_part[(size_t)u * p.l * p.n2 + x];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        float v = (threadIdx.x < blockDim.x / 32) ? red[threadIdx.x] : 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (threadIdx.x == 0) p.dw[(size_t)j * p.n2 + n] = v;
-    }
+    if (lane == 0) p.dw[x] = acc;
 }
 
 cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaStream_t st) {
@@ -727,12 +752,20 @@ cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaS
     return cudaGetLastError();
 }
 
-cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, cudaStream_t st) {
-    dim3 grid(p.l, p.n2);
-    if (p.dtype == 0)
-        compress_dw_kernel<__nv_bfloat16><<<grid, 512, 0, st>>>(p);
-    else
-        compress_dw_kernel<__half><<<grid, 512, 0, st>>>(p);
+int compress_dw_heads_per_cta(int l) { return std::max(1, 256 / l); }
+
+cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, int nruns, cudaStream_t st) {
+    const int hpc = compress_dw_heads_per_cta(p.l);
+    if (nruns > 0) {
+        dim3 grid(nruns, (p.n2 + hpc - 1) / hpc);
+        if (p.dtype == 0)
+            compress_dw_part_kernel<__nv_bfloat16><<<grid, hpc * p.l, 0, st>>>(p);
+        else
+            compress_dw_part_kernel<__half><<<grid, hpc * p.l, 0, st>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    compress_dw_reduce_kernel<<<(p.l * p.n2 + 7) / 8, 256, 0, st>>>(p, nruns);
     return cudaGetLastError();
 }
 

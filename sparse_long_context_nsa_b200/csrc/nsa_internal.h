@@ -232,6 +232,8 @@ struct CompressBwdParams {
     float* dv;
     float* dw;
     const int* cmp_raw;           // per compressed row: its first raw row (T2 index)
+    float* dw_part;               // dw partial sums, [run][l][n2]
+    int dw_run;                   // compressed rows per dw run
     long long tc;
     long long t2;                 // raw rows (debug bounds checks)
     int l, d, n2, d1, d2, dtype;
@@ -240,8 +242,10 @@ struct CompressBwdParams {
 };
 // dk, dv for the launch's sequences (one call per batch of sequences)
 cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaStream_t st);
-// dw over every compressed row (one call)
-cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, cudaStream_t st);
+// dw over every compressed row: partial sums per run of p.dw_run rows, then their
+// sum in run order (two launches)
+int compress_dw_heads_per_cta(int l);
+cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, int nruns, cudaStream_t st);
 }  // namespace bwd
 
 // ------------------------------------------------ selection attention
