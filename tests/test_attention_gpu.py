@@ -200,15 +200,20 @@ def _staircase_short(nsa, n1, n2, dd, seqs, nq, step, l=32, d=16, lp=64, count=8
     return check_attention(res, ref, count, out_rel=2.0 ** -7)
 
 
-@pytest.mark.parametrize("n1,dd,nq", [(16, 256, 16), (128, 256, 3000), (24, 256, 3000)],
-                         ids=["g8_d256_16q", "g64_d256", "g12_d256"])
-def test_one_pass_one_pipeline(nsa, n1, dd, nq):
+@pytest.mark.parametrize("n1,dd,nq,mixed", [(16, 256, 16, False), (16, 256, 16, True), (128, 256, 3000, False),
+                                             (24, 256, 3000, True)],
+                         ids=["g8_d256_16q", "g8_d256_16q_short_seqs", "g64_d256", "g12_d256"])
+def test_one_pass_one_pipeline(nsa, n1, dd, nq, mixed):
     """The one-pass kernel with one pipeline and two score buffers (D2 > 128),
     many items per CTA and a reference maximum that moves: G = 8 with at most
-    one M-tile of queries per sequence (300 sequences of 16 queries), G = 64
-    (above the two-pass range) and G = 12 (not a power of two) over whole
-    sequences."""
-    seqs = [3000 - 7 * (i % 50) for i in range(300)] if nq == 16 else [3000, 2500]
+    one M-tile of queries per sequence (300 sequences of 16 queries; or
+    sequences as short as 16 tokens, whose rows attend to nothing or to one
+    block), G = 64 (above the two-pass range) and G = 12 (not a power of two)
+    over whole sequences, short ones among them."""
+    if nq == 16:
+        seqs = [16, 31, 32, 40, 47, 100, 300, 1000, 3000] * 30 if mixed else [3000 - 7 * (i % 50) for i in range(300)]
+    else:
+        seqs = [3000, 700, 40, 16] if mixed else [3000, 2500]
     print(_staircase_short(nsa, n1, 2, dd, seqs, nq, step=7))
 
 
