@@ -614,9 +614,11 @@ cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMa
 
 // dk[p] = sum_i w[p - i d] dkcmp_i over the windows i covering raw row p
 // (dv likewise).  A CTA takes kRowsPerCta raw rows of one sequence; a thread
-// one (head, 4 consecutive dims) column, four rows at a time: the loads of
-// the four rows are issued before their sums and stores.
-template <typename T>
+// one (head, 4 consecutive dims) column.  Walking its rows, a thread keeps
+// the dkcmp values of the windows that cover the current row in registers
+// (slot k: window q - k, q the row's group of d rows, position j = k d +
+// row mod d in it) and loads one new window per group of d rows.
+template <typename T, int BMAX>
 __global__ void compress_dx_kernel(const CompressBwdParams p) {
     int s = 0;
     while (s + 1 < p.nseq && (int)blockIdx.x >= p.seq[s].blk_end) ++s;
@@ -629,37 +631,44 @@ __global__ void compress_dx_kernel(const CompressBwdParams p) {
     float* __restrict__ dx = is_v ? p.dv : p.dk;
     const T* __restrict__ w = reinterpret_cast<const T*>(p.w);
     const int ncol = p.n2 * dim / 4;
-    const int nb = (p.l + p.d - 1) / p.d;   // windows covering a row, at most
+    const int l = p.l, d = p.d;
+    const int nb = (l + d - 1) / d;   // windows covering a row, at most
+    const int rows = min(kRowsPerCta, q.raw_len - r0);
+    auto g_of = [&](int i, int n, int e) {   // dkcmp of window i (0 outside the sequence's windows)
+        return (i >= 0 && i < q.n_cmp)
+                   ? __ldg(reinterpret_cast<const float4*>(g + ((size_t)(q.cmp_start + i) * p.n2 + n) * dim + e))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
     for (int col = threadIdx.x; col < ncol; col += blockDim.x) {
         const int n = (col * 4) / dim, e = (col * 4) % dim;
-        for (int rr = 0; rr < kRowsPerCta; rr += 4) {
-            float4 acc[4];
+        int qg = r0 / d, rin = r0 - qg * d;
+        float4 gq[BMAX];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                const int pr = r0 + rr + u;   // raw row inside the sequence
-                if (pr >= q.raw_len) continue;
-                // windows i with i d <= pr < i d + l
-                const int i_lo = pr - p.l + 1 <= 0 ? 0 : (pr - p.l + 1 + p.d - 1) / p.d;
-                const int i_hi = min(pr / p.d, q.n_cmp - 1);
-                for (int k = 0; k < nb; ++k) {
-                    const int i = i_lo + k;
-                    if (i > i_hi) break;
-                    const float wv = static_cast<float>(w[(size_t)(pr - i * p.d) * p.n2 + n]);
-                    const float4 gv = __ldg(reinterpret_cast<const float4*>(
-                        g + ((size_t)(q.cmp_start + i) * p.n2 + n) * dim + e));
-                    acc[u].x = fmaf(wv, gv.x, acc[u].x);
-                    acc[u].y = fmaf(wv, gv.y, acc[u].y);
-                    acc[u].z = fmaf(wv, gv.z, acc[u].z);
-                    acc[u].w = fmaf(wv, gv.w, acc[u].w);
+        for (int k = 0; k < BMAX; ++k) gq[k] = (k < nb) ? g_of(qg - k, n, e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int rr = 0; rr < rows; ++rr) {
+            const int pr = r0 + rr;   // raw row inside the sequence
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < BMAX; ++k) {
+                const int j = k * d + rin;
+                if (k < nb && j < l) {
+                    const float wv = static_cast<float>(w[(size_t)j * p.n2 + n]);
+                    acc.x = fmaf(wv, gq[k].x, acc.x);
+                    acc.y = fmaf(wv, gq[k].y, acc.y);
+                    acc.z = fmaf(wv, gq[k].z, acc.z);
+                    acc.w = fmaf(wv, gq[k].w, acc.w);
                 }
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int pr = r0 + rr + u;
-                if (pr >= q.raw_len || !nsa_index_ok(q.raw_start + pr < p.t2, nullptr, 11)) continue;
+            if (nsa_index_ok(q.raw_start + pr < p.t2, nullptr, 11))
                 // written once: stream past L2
-                __stcs(reinterpret_cast<float4*>(dx + ((size_t)(q.raw_start + pr) * p.n2 + n) * dim + e), acc[u]);
+                __stcs(reinterpret_cast<float4*>(dx + ((size_t)(q.raw_start + pr) * p.n2 + n) * dim + e), acc);
+            if (++rin == d) {
+                // the next group: every window moves one slot up, window qg + 1 enters slot 0
+                rin = 0;
+                ++qg;
+#pragma unroll
+                for (int k = BMAX - 1; k >= 1; --k) gq[k] = gq[k - 1];
+                gq[0] = g_of(qg, n, e);
             }
         }
     }
@@ -745,11 +754,19 @@ __global__ void compress_dw_reduce_kernel(const CompressBwdParams p, int nruns) 
 cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaStream_t st) {
     if (blocks <= 0) return cudaSuccess;
     dim3 grid(blocks, p.dvcmp ? 2 : 1);
-    if (p.dtype == 0)
-        compress_dx_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);
-    else
-        compress_dx_kernel<__half><<<grid, 256, 0, st>>>(p);
-    return cudaGetLastError();
+    const int nb = (p.l + p.d - 1) / p.d;
+    const bool bf = p.dtype == 0;
+#define NSA_DX(BM)                                                                          \
+    {                                                                                      \
+        if (bf) compress_dx_kernel<__nv_bfloat16, BM><<<grid, 256, 0, st>>>(p);            \
+        else compress_dx_kernel<__half, BM><<<grid, 256, 0, st>>>(p);                      \
+        return cudaGetLastError();                                                         \
+    }
+    if (nb <= 1) NSA_DX(1)
+    if (nb <= 2) NSA_DX(2)
+    if (nb <= 4) NSA_DX(4)
+    NSA_DX(8)
+#undef NSA_DX
 }
 
 int compress_dw_heads_per_cta(int l) { return std::max(1, 256 / l); }

@@ -127,8 +127,12 @@ def test_deterministic(nsa):
 
 
 def test_compress_backward(nsa):
+    # ceil(l/d) = 2 windows per row (TINY, 64/32, 128/64), 1 (32/32), 4 (64/16), 8 (128/16) and
+    # l % d != 0 (48/32)
     for wl in (workloads.TINY, _wl([300, 0, 20, 777], 8, 4, 64, 32, l=64, d=32, dtype="fp16"),
-               _wl([1000], 8, 2, 128, 128, l=128, d=64)):
+               _wl([1000], 8, 2, 128, 128, l=128, d=64), _wl([700, 33], 8, 2, 64, 64, l=32, d=32),
+               _wl([900], 8, 2, 64, 64, l=64, d=16), _wl([1100, 200], 4, 2, 64, 32, l=128, d=16, lp=128),
+               _wl([650], 8, 2, 64, 64, l=48, d=32, lp=64)):
         x = wl.generate()
         tc = int(nsa.nsa_compress_out_len(x["cu_seqlens"], wl.l, wl.d)[-1])
         g = torch.Generator().manual_seed(wl.seed + 2000)
