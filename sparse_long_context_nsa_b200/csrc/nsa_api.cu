@@ -1324,7 +1324,7 @@ nsa_status_t nsa_compress_backward(const void* k, const void* v, const void* w, 
         int dev = 0, nsm = 148;
         if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-        const int hpc = bwd::compress_dw_heads_per_cta(l);
+        const int hpc = bwd::compress_dw_heads_per_cta(d, n2);
         const int64_t ygroups = (n2 + hpc - 1) / hpc;
         int64_t want = std::max<int64_t>(1, (int64_t)nsm * 8 / ygroups);
         want = std::min<int64_t>(want, (int64_t)(kDwPartBytes / per_run));

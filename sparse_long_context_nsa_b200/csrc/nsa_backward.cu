@@ -676,66 +676,92 @@ __global__ void compress_dx_kernel(const CompressBwdParams p) {
 
 // dw[j, n] = sum_i (dkcmp_i . k[i d + j] + dvcmp_i . v[i d + j]) over every
 // compressed row i, in two steps.  Partial sums: a CTA takes a run of
-// consecutive compressed rows (p.dw_run of them, across sequence boundaries:
-// cmp_raw gives each row's first raw row) and heads [y hpc, (y+1) hpc); thread
-// (h, j) sums the dot products of window position j over the run, reading raw
-// row cmp_raw[i] + j (a warp reads 32 consecutive rows of one head, and
-// neighbouring windows' rows again from cache).  Then dw = the partials summed
-// over the runs in run order (deterministic).
-template <typename T>
+// consecutive compressed rows [i0, i1) (p.dw_run of them, across sequence
+// boundaries: cmp_raw gives each row's first raw row) and heads [y hpc,
+// (y+1) hpc).  Thread (h, t) walks the run's groups of d raw rows, reading
+// row t of each group once and adding it to every window of the run that
+// covers it (window g - k at position j = k d + t, in slot k), as the forward
+// compress does with its window sums; group g < i1 is window g's first group,
+// the groups past i1 - 1 continue the last window's rows.  Then dw = the
+// partials summed over the runs in run order (deterministic).
+template <typename T, int BMAX>
 __global__ void compress_dw_part_kernel(const CompressBwdParams p) {
-    const int hpc = blockDim.x / p.l;
-    const int h = threadIdx.x / p.l, j = threadIdx.x - h * p.l;
+    const int d = p.d, l = p.l;
+    const int hpc = blockDim.x / d;
+    const int h = threadIdx.x / d, t = threadIdx.x - h * d;
     const int n = blockIdx.y * hpc + h;
-    if (h >= hpc) return;
+    if (h >= hpc || n >= p.n2) return;
+    const int nb = (l + d - 1) / d;
     const long long i0 = (long long)blockIdx.x * p.dw_run;
     const long long i1 = min(i0 + p.dw_run, p.tc);
-    float acc = 0.f;
-    if (n < p.n2) {
-        const T* __restrict__ kk = reinterpret_cast<const T*>(p.k);
-        const T* __restrict__ vv = reinterpret_cast<const T*>(p.v);
-        for (long long i = i0; i < i1; ++i) {
-            const long long r = (long long)p.cmp_raw[i] + j;
-            if (!nsa_index_ok(r < p.t2, nullptr, 12)) continue;
-            const float* gk = p.dkcmp + ((size_t)i * p.n2 + n) * p.d1;
-            const T* xk = kk + ((size_t)r * p.n2 + n) * p.d1;
-#pragma unroll 2
-            for (int e = 0; e < p.d1; e += 8) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4*>(xk + e));
-                const float4 g0 = __ldg(reinterpret_cast<const float4*>(gk + e));
-                const float4 g1 = __ldg(reinterpret_cast<const float4*>(gk + e + 4));
-                const float2 a0 = up2<T>(u.x), a1 = up2<T>(u.y), a2 = up2<T>(u.z), a3 = up2<T>(u.w);
-                acc = fmaf(g0.x, a0.x, acc);
-                acc = fmaf(g0.y, a0.y, acc);
-                acc = fmaf(g0.z, a1.x, acc);
-                acc = fmaf(g0.w, a1.y, acc);
-                acc = fmaf(g1.x, a2.x, acc);
-                acc = fmaf(g1.y, a2.y, acc);
-                acc = fmaf(g1.z, a3.x, acc);
-                acc = fmaf(g1.w, a3.y, acc);
+    const T* __restrict__ kk = reinterpret_cast<const T*>(p.k);
+    const T* __restrict__ vv = reinterpret_cast<const T*>(p.v);
+    float acc[BMAX];
+#pragma unroll
+    for (int k = 0; k < BMAX; ++k) acc[k] = 0.f;
+    const long long last = p.cmp_raw[i1 - 1];
+    for (long long g = i0; g < i1 + nb - 1; ++g) {
+        const long long base = g < i1 ? (long long)p.cmp_raw[g] : last + (g - i1 + 1) * d;
+        // the run's windows that hold row base + t, and where
+        bool any = false;
+        bool valid[BMAX];
+#pragma unroll
+        for (int k = 0; k < BMAX; ++k) {
+            const long long wdx = g - k;
+            valid[k] = k < nb && k * d + t < l && wdx >= i0 && wdx < i1 &&
+                       (long long)p.cmp_raw[wdx] + (long long)k * d == base;
+            any = any || valid[k];
+        }
+        if (!any) continue;
+        const long long r = base + t;
+        if (!nsa_index_ok(r < p.t2, nullptr, 12)) continue;
+        const T* xk = kk + ((size_t)r * p.n2 + n) * p.d1;
+        for (int e = 0; e < p.d1; e += 8) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(xk + e));
+            const float2 a0 = up2<T>(u.x), a1 = up2<T>(u.y), a2 = up2<T>(u.z), a3 = up2<T>(u.w);
+#pragma unroll
+            for (int k = 0; k < BMAX; ++k) {
+                if (!valid[k]) continue;
+                const float* gk = p.dkcmp + ((size_t)(g - k) * p.n2 + n) * p.d1 + e;
+                const float4 g0 = __ldg(reinterpret_cast<const float4*>(gk));
+                const float4 g1 = __ldg(reinterpret_cast<const float4*>(gk + 4));
+                acc[k] = fmaf(g0.x, a0.x, acc[k]);
+                acc[k] = fmaf(g0.y, a0.y, acc[k]);
+                acc[k] = fmaf(g0.z, a1.x, acc[k]);
+                acc[k] = fmaf(g0.w, a1.y, acc[k]);
+                acc[k] = fmaf(g1.x, a2.x, acc[k]);
+                acc[k] = fmaf(g1.y, a2.y, acc[k]);
+                acc[k] = fmaf(g1.z, a3.x, acc[k]);
+                acc[k] = fmaf(g1.w, a3.y, acc[k]);
             }
-            if (p.dvcmp != nullptr) {
-                const float* gv = p.dvcmp + ((size_t)i * p.n2 + n) * p.d2;
-                const T* xv = vv + ((size_t)r * p.n2 + n) * p.d2;
-#pragma unroll 2
-                for (int e = 0; e < p.d2; e += 8) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(xv + e));
-                    const float4 g0 = __ldg(reinterpret_cast<const float4*>(gv + e));
-                    const float4 g1 = __ldg(reinterpret_cast<const float4*>(gv + e + 4));
-                    const float2 a0 = up2<T>(u.x), a1 = up2<T>(u.y), a2 = up2<T>(u.z), a3 = up2<T>(u.w);
-                    acc = fmaf(g0.x, a0.x, acc);
-                    acc = fmaf(g0.y, a0.y, acc);
-                    acc = fmaf(g0.z, a1.x, acc);
-                    acc = fmaf(g0.w, a1.y, acc);
-                    acc = fmaf(g1.x, a2.x, acc);
-                    acc = fmaf(g1.y, a2.y, acc);
-                    acc = fmaf(g1.z, a3.x, acc);
-                    acc = fmaf(g1.w, a3.y, acc);
+        }
+        if (p.dvcmp != nullptr) {
+            const T* xv = vv + ((size_t)r * p.n2 + n) * p.d2;
+            for (int e = 0; e < p.d2; e += 8) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(xv + e));
+                const float2 a0 = up2<T>(u.x), a1 = up2<T>(u.y), a2 = up2<T>(u.z), a3 = up2<T>(u.w);
+#pragma unroll
+                for (int k = 0; k < BMAX; ++k) {
+                    if (!valid[k]) continue;
+                    const float* gv = p.dvcmp + ((size_t)(g - k) * p.n2 + n) * p.d2 + e;
+                    const float4 g0 = __ldg(reinterpret_cast<const float4*>(gv));
+                    const float4 g1 = __ldg(reinterpret_cast<const float4*>(gv + 4));
+                    acc[k] = fmaf(g0.x, a0.x, acc[k]);
+                    acc[k] = fmaf(g0.y, a0.y, acc[k]);
+                    acc[k] = fmaf(g0.z, a1.x, acc[k]);
+                    acc[k] = fmaf(g0.w, a1.y, acc[k]);
+                    acc[k] = fmaf(g1.x, a2.x, acc[k]);
+                    acc[k] = fmaf(g1.y, a2.y, acc[k]);
+                    acc[k] = fmaf(g1.z, a3.x, acc[k]);
+                    acc[k] = fmaf(g1.w, a3.y, acc[k]);
                 }
             }
         }
-        p.dw_part[((size_t)blockIdx.x * p.l + j) * p.n2 + n] = acc;
     }
+    // every position j = k d + t of the run's partial row is this thread's
+#pragma unroll
+    for (int k = 0; k < BMAX; ++k)
+        if (k < nb && k * d + t < l) p.dw_part[((size_t)blockIdx.x * l + k * d + t) * p.n2 + n] = acc[k];
 }
 
 // one warp per (j, n) of dw: lane k sums runs k, k + 32, ... in order, then a
@@ -769,16 +795,24 @@ cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaS
 #undef NSA_DX
 }
 
-int compress_dw_heads_per_cta(int l) { return std::max(1, 256 / l); }
+int compress_dw_heads_per_cta(int d, int n2) { return std::max(1, std::min(256 / d, n2)); }
 
 cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, int nruns, cudaStream_t st) {
-    const int hpc = compress_dw_heads_per_cta(p.l);
+    const int hpc = compress_dw_heads_per_cta(p.d, p.n2);
     if (nruns > 0) {
         dim3 grid(nruns, (p.n2 + hpc - 1) / hpc);
-        if (p.dtype == 0)
-            compress_dw_part_kernel<__nv_bfloat16><<<grid, hpc * p.l, 0, st>>>(p);
-        else
-            compress_dw_part_kernel<__half><<<grid, hpc * p.l, 0, st>>>(p);
+        const int nb = (p.l + p.d - 1) / p.d;
+        const bool bf = p.dtype == 0;
+#define NSA_DW(BM)                                                                          \
+    {                                                                                      \
+        if (bf) compress_dw_part_kernel<__nv_bfloat16, BM><<<grid, hpc * p.d, 0, st>>>(p); \
+        else compress_dw_part_kernel<__half, BM><<<grid, hpc * p.d, 0, st>>>(p);           \
+    }
+        if (nb <= 1) NSA_DW(1)
+        else if (nb <= 2) NSA_DW(2)
+        else if (nb <= 4) NSA_DW(4)
+        else NSA_DW(8)
+#undef NSA_DW
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -244,7 +244,7 @@ struct CompressBwdParams {
 cudaError_t launch_compress_bwd_dx(const CompressBwdParams& p, int blocks, cudaStream_t st);
 // dw over every compressed row: partial sums per run of p.dw_run rows, then their
 // sum in run order (two launches)
-int compress_dw_heads_per_cta(int l);
+int compress_dw_heads_per_cta(int d, int n2);   // heads of one dw partial-sum CTA
 cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, int nruns, cudaStream_t st);
 }  // namespace bwd
 
