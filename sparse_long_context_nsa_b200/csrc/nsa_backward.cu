@@ -162,7 +162,7 @@ __device__ __forceinline__ void store_row_f32(uint32_t taddr, int ncols, float m
 
 // --------------------------------------------------------------------- dQ
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsDq, 1)
 dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
           const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p) {
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
@@ -174,7 +174,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     const int nqc = (p.d1 + 63) / 64, nvc = (p.d2 + 63) / 64;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P0 || i == B_P1) ? 4 : 1);
+        // dS of a tile is written by eight warps (two per lane quadrant, one per column half)
+        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P0 || i == B_P1) ? 8 : 1);
         *sm.abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -235,18 +236,21 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 ok = mbar_wait(bar(B_P0), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x23);
                 if (!ok) break;
                 tc_fence_after();
-                for (int ks = 0; ks < kKV / 16; ++ks)   // dQ += dS K (dS from tensor memory)
-                    umma_ts(tmem + 256, tmem + ks * 8, sdesc_sw128(kst + ks * 2048, kKV * 128, 1024), id_q,
-                            (i > 0 || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < kKV / 16; ++ks)   // dQ += dS K (dS from tensor memory: each
+                                                        // half of the keys at the start of its half)
+                    umma_ts(tmem + 256, tmem + ks * 8 + (ks >= kKV / 32 ? kKV / 4 : 0),
+                            sdesc_sw128(kst + ks * 2048, kKV * 128, 1024), id_q, (i > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(bar(B_MMA));
                 ok = mbar_wait(bar(B_MMA), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x24);
                 if (ok && p.nst == 1 && i + 1 < it.nkv) load_kv(i + 1);
             }
         }
     } else {
-        // one query row per thread
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // one query row per thread; warps 0-3 take the first half of a tile's columns
+        // (and of dQ), warps 5-8 the second, each in its lane quadrant (warp % 4)
+        const int quad = warp & 3, half = warp > 4 ? 1 : 0;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const int tok = row / G, h = row % G;
         const bool valid = row < TT * G && tok < it.ntok && nsa_index_ok(it.q_row0 + tok < p.rows_q, p.err, 8);
         const int nv = valid ? nvis_at(it.t0 + tok, p.l, p.d, it.n_cmp) : 0;
@@ -257,7 +261,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             mbar_wait(bar(B_S0), i & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x25);
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kKV / 32; ++c) {
+            for (int c = half * (kKV / 64); c < (half + 1) * (kKV / 64); ++c) {
                 uint32_t rs[32], rp[32];
                 tmem_ld32(tmem + lane_off + c * 32, rs);
                 tmem_ld32(tmem + lane_off + 128 + c * 32, rp);
@@ -273,20 +277,25 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                     pk[e >> 1] = pk2<T>(v0 ? p0 * (__uint_as_float(rp[e]) - info.y) : 0.f,
                                         v1 ? p1 * (__uint_as_float(rp[e + 1]) - info.y) : 0.f);
                 }
-                tmem_st16(tmem + lane_off + c * 16, pk);
+                // dS of the chunk over S columns this warp has already read: the first 32
+                // columns of its own half (the other half's warp still reads its S)
+                tmem_st16(tmem + lane_off + c * 16 + half * (kKV / 4), pk);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_P0));
         }
+        // this warp's half of the row of dQ (16-column pieces)
+        const int c16 = (p.d1 / 16 + 1) / 2;
+        const int e0 = half * c16 * 16, e1 = min(p.d1, (half + 1) * c16 * 16);
         float* dst = p.dq + ri * p.d1;
         if (it.nkv > 0) {
             mbar_wait(bar(B_MMA), (it.nkv - 1) & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x26);
             tc_fence_after();
-            store_row_f32(tmem + lane_off + 256, p.d1, p.scale, dst, valid);
+            if (e1 > e0) store_row_f32(tmem + lane_off + 256 + e0, e1 - e0, p.scale, dst + e0, valid);
         } else if (valid) {
-            for (int e = 0; e < p.d1; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = e0; e < e1; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     tc_fence_before();
@@ -589,25 +598,26 @@ cudaError_t launch_reduce(const KVTile* tiles, int ntiles, const float* part, fl
 }
 
 template <typename K>
-static cudaError_t launch_mma_kernel(K kern, const Params& p, int n, const CUtensorMap& tq, const CUtensorMap& tdo,
-                                     const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+static cudaError_t launch_mma_kernel(K kern, const Params& p, int n, int threads, const CUtensorMap& tq,
+                                     const CUtensorMap& tdo, const CUtensorMap& tk, const CUtensorMap& tv,
+                                     cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
-    kern<<<n, kThreads, p.smem_bytes, st>>>(tq, tdo, tk, tv, p);
+    kern<<<n, threads, p.smem_bytes, st>>>(tq, tdo, tk, tv, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_dq(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                       const CUtensorMap& tv, cudaStream_t st) {
-    return p.dtype == 0 ? launch_mma_kernel(dq_kernel<__nv_bfloat16>, p, p.n_qitems, tq, tdo, tk, tv, st)
-                        : launch_mma_kernel(dq_kernel<__half>, p, p.n_qitems, tq, tdo, tk, tv, st);
+    return p.dtype == 0 ? launch_mma_kernel(dq_kernel<__nv_bfloat16>, p, p.n_qitems, kThreadsDq, tq, tdo, tk, tv, st)
+                        : launch_mma_kernel(dq_kernel<__half>, p, p.n_qitems, kThreadsDq, tq, tdo, tk, tv, st);
 }
 
 cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                         const CUtensorMap& tv, cudaStream_t st) {
-    return p.dtype == 0 ? launch_mma_kernel(dkdv_kernel<__nv_bfloat16>, p, p.n_kvitems, tq, tdo, tk, tv, st)
-                        : launch_mma_kernel(dkdv_kernel<__half>, p, p.n_kvitems, tq, tdo, tk, tv, st);
+    return p.dtype == 0 ? launch_mma_kernel(dkdv_kernel<__nv_bfloat16>, p, p.n_kvitems, kThreads, tq, tdo, tk, tv, st)
+                        : launch_mma_kernel(dkdv_kernel<__half>, p, p.n_kvitems, kThreads, tq, tdo, tk, tv, st);
 }
 
 // ---------------------------------------------------- compression transposed

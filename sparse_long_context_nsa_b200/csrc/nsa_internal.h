@@ -163,6 +163,7 @@ int attention_chunk_cols(int a);  // score columns per softmax chunk for band fa
 // and of the compression with respect to the raw K/V rows and w.
 namespace bwd {
 constexpr int kThreads = 160;    // warps 0-3 softmax (TMEM lane quadrants), warp 4 TMA + MMA
+constexpr int kThreadsDq = 288;  // dQ: warps 0-3 and 5-8 softmax (two per lane quadrant), warp 4 TMA + MMA
 constexpr int kKV = 128;         // compressed blocks per KV tile
 
 // dQ: one query M-tile (TT tokens x G heads of one group) over its KV tiles
