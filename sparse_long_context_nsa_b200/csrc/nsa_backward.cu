@@ -317,7 +317,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 // so every row that takes part must hold finite values: rows of the box past
 // G x TT are zeroed once, rows outside the run get P = dS = 0 by selection.
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsDq, 1)
 dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p) {
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
@@ -331,7 +331,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int n_mt = (it.q_end - it.q_row0 + TT - 1) / TT;   // query M-tiles of the run
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P0 || i == B_P1) ? 4 : 1);
+        // Pᵀ and dSᵀ of a step are written by eight warps (two per lane quadrant)
+        for (int i = 0; i < B_N; ++i) mbar_init(bar(i), (i == B_P0 || i == B_P1) ? 8 : 1);
         *sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -439,11 +440,14 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int ks = 0; ks < 64 / 16; ++ks) {
                     // the 64 query rows of the half are the contraction dimension: the
                     // row-major dO / Q chunks serve as MN-major operands
+                    // Pᵀ / dSᵀ of query rows 32c .. 32c + 31 sit at the start of chunk c's
+                    // columns (c = ks / 2), packed two to a column
+                    const uint32_t pc = ks * 8 + (ks >= 2 ? 16 : 0);
                     if (do_dv)
-                        umma_ts(tmem, tmem + sb_col(b) + ks * 8, sdesc_sw128(ds + hf * 8192 + ks * 2048, 16384, 1024),
+                        umma_ts(tmem, tmem + sb_col(b) + pc, sdesc_sw128(ds + hf * 8192 + ks * 2048, 16384, 1024),
                                 id_v, (step > 0 || ks > 0) ? 1u : 0u);
                     if (do_dk)
-                        umma_ts(tmem + p.col_dk, tmem + sb_col(b) + 64 + ks * 8,
+                        umma_ts(tmem + p.col_dk, tmem + sb_col(b) + 64 + pc,
                                 sdesc_sw128(qs + hf * 8192 + ks * 2048, 16384, 1024), id_k,
                                 (step > 0 || ks > 0) ? 1u : 0u);
                 }
@@ -465,9 +469,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             umma_commit(bar(B_DONE));
         }
     } else {
-        // one key (compressed block) of the tile per thread
-        const int kr = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // one key (compressed block) of the tile per thread; warps 0-3 take the first 32
+        // query rows of each half-step, warps 5-8 the second, each in its lane quadrant
+        const int quad = warp & 3, chalf = warp > 4 ? 1 : 0;
+        const int kr = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const int kb = it.kt * kKV + kr;   // block index inside the sequence
         const bool kvalid = kb < it.n_cmp;
         const float c2 = p.scale_log2;
@@ -481,11 +487,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                          : make_float2(INFINITY, 0.f);
             nv = valid ? nvis_at(tpos, p.l, p.d, it.n_cmp) : 0;
         };
-        if (n_mt > 0) row_of(0, rinfo2[kr], rnv2[kr]);
+        if (n_mt > 0 && chalf == 0) row_of(0, rinfo2[kr], rnv2[kr]);
         for (int mi = 0; mi < n_mt; ++mi) {
             // buffer mi & 1 is complete, and M-tile mi - 1 (the other buffer) is no
             // longer read by anyone
-            named_bar_sync(1, 128);
+            named_bar_sync(1, 256);
             const float2* rinfo = rinfo2 + (mi & 1) * 128;
             const int* rnv = rnv2 + (mi & 1) * 128;
             // the next M-tile's row, loaded now and stored after this M-tile's work
@@ -498,8 +504,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const uint32_t scol = b == 0 ? 384u : 256u;   // S^T of this step's buffer, dP^T at + 64
                 mbar_wait(bar(B_S0 + b), (step / p.nsb) & 1, sm.abort_flag, p.err, kErrTimeoutBase + 0x35);
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
+                {
+                    const int c = chalf;
                     uint32_t rs[32], rp[32];
                     tmem_ld32(tmem + lane_off + scol + c * 32, rs);
                     if (do_dk) tmem_ld32(tmem + lane_off + scol + 64 + c * 32, rp);
@@ -518,15 +524,16 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                             dpk[e >> 1] = pk2<T>(v0 ? p0 * (__uint_as_float(rp[e]) - i0.y) : 0.f,
                                                  v1 ? p1 * (__uint_as_float(rp[e + 1]) - i1.y) : 0.f);
                     }
-                    if (do_dv) tmem_st16(tmem + lane_off + scol + c * 16, ppk);
-                    if (do_dk) tmem_st16(tmem + lane_off + scol + 64 + c * 16, dpk);
+                    // over this chunk's own Sᵀ / dPᵀ columns (the other warp reads the rest)
+                    if (do_dv) tmem_st16(tmem + lane_off + scol + c * 32, ppk);
+                    if (do_dk) tmem_st16(tmem + lane_off + scol + 64 + c * 32, dpk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_P0 + b));
             }
-            if (mi + 1 < n_mt) {
+            if (mi + 1 < n_mt && chalf == 0) {
                 rinfo2[((mi + 1) & 1) * 128 + kr] = nxt_info;
                 rnv2[((mi + 1) & 1) * 128 + kr] = nxt_nv;
             }
@@ -534,17 +541,36 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_wait(bar(B_DONE), 0, sm.abort_flag, p.err, kErrTimeoutBase + 0x36);
         tc_fence_after();
         // the run's partial sums; a run with no M-tile leaves zeros
+        // (each of the quadrant's two warps stores half of the row's columns: dV then dK,
+        // in 16-column pieces)
         float* dst = p.part + ((size_t)it.slot * 128 + kr) * (p.d1 + p.d2);
+        const int ndv = do_dv ? p.d2 : 0, ndk = do_dk ? p.d1 : 0;
+        const int np16 = (ndv + ndk) / 16, mine0 = chalf * ((np16 + 1) / 2) * 16,
+                  mine1 = min(ndv + ndk, (chalf + 1) * ((np16 + 1) / 2) * 16);
+        // column x of the row: dV for x < ndv, dK after (tensor memory: 0 and col_dk)
+        auto seg = [&](int x0, int x1, bool zero) {
+            if (x1 <= x0) return;
+            const int xa = x0, xb = min(x1, ndv);
+            if (xb > xa) {
+                if (zero) {
+                    for (int e = xa; e < xb; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    store_row_f32(tmem + lane_off + xa, xb - xa, 1.f, dst + xa, true);
+                }
+            }
+            const int ya = max(x0, ndv) - ndv, yb = x1 - ndv;
+            if (yb > ya) {
+                float* dk = dst + p.d2 + ya;
+                if (zero) {
+                    for (int e = 0; e < yb - ya; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    store_row_f32(tmem + lane_off + p.col_dk + ya, yb - ya, 1.f, dk, true);
+                }
+            }
+        };
         if (!nsa_index_ok(it.slot < p.n_slots, p.err, 9)) {
-        } else if (n_mt > 0) {
-            if (do_dv) store_row_f32(tmem + lane_off, p.d2, 1.f, dst, true);
-            if (do_dk) store_row_f32(tmem + lane_off + p.col_dk, p.d1, 1.f, dst + p.d2, true);
         } else {
-            if (do_dv)
-                for (int e = 0; e < p.d2; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (do_dk)
-                for (int e = 0; e < p.d1; e += 4)
-                    *reinterpret_cast<float4*>(dst + p.d2 + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            seg(mine0, mine1, n_mt == 0);
         }
     }
     tc_fence_before();
@@ -616,8 +642,8 @@ cudaError_t launch_dq(const Params& p, const CUtensorMap& tq, const CUtensorMap&
 
 cudaError_t launch_dkdv(const Params& p, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                         const CUtensorMap& tv, cudaStream_t st) {
-    return p.dtype == 0 ? launch_mma_kernel(dkdv_kernel<__nv_bfloat16>, p, p.n_kvitems, kThreads, tq, tdo, tk, tv, st)
-                        : launch_mma_kernel(dkdv_kernel<__half>, p, p.n_kvitems, kThreads, tq, tdo, tk, tv, st);
+    return p.dtype == 0 ? launch_mma_kernel(dkdv_kernel<__nv_bfloat16>, p, p.n_kvitems, kThreadsDq, tq, tdo, tk, tv, st)
+                        : launch_mma_kernel(dkdv_kernel<__half>, p, p.n_kvitems, kThreadsDq, tq, tdo, tk, tv, st);
 }
 
 // ---------------------------------------------------- compression transposed
