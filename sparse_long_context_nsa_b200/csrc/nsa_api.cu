@@ -336,7 +336,7 @@ struct SelPlan {
     int G = 0, TT = 0, cap = 1, max_words = 1, grid = 0;
     std::vector<sel::Tile> tiles;
     int nslot = 0, nqbuf = 1, nsbuf = 2, tm_o = 0, tm_s = 0, s_stride = 0;
-    int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_bar = 0, smem_bytes = 0;
+    int off_q = 0, q_bytes = 0, off_ring = 0, slot_bytes = 0, off_bar = 0, off_x = 0, smem_bytes = 0;
     size_t ws_tiles = 0, ws_n = 0, ws_blk = 0, ws_mask = 0, ws_total = 0;
 };
 
@@ -393,6 +393,8 @@ nsa_status_t plan_select(int head_num, int n2, int d1, int d2, int lp, int count
         off += ns * pl.slot_bytes;
         pl.off_bar = off;
         off += sel::kBarBytes;
+        pl.off_x = off;
+        off += sel::kXchgBytes;
         pl.smem_bytes = off + 1024;   // slack for 1024-byte alignment of the base
         pl.nqbuf = nq;
         pl.nslot = ns;
@@ -1126,6 +1128,7 @@ nsa_status_t nsa_select_attention(const void* q, const void* k, const void* v, c
     p.off_ring = pl.off_ring;
     p.slot_bytes = pl.slot_bytes;
     p.off_bar = pl.off_bar;
+    p.off_x = pl.off_x;
     p.smem_bytes = pl.smem_bytes;
     if (sel::launch_plan(p, pl.max_words, st) != cudaSuccess) return NSA_ERR_CUDA;
     const int grid = std::min(pl.grid, nsm);

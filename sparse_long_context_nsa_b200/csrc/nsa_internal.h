@@ -255,12 +255,21 @@ cudaError_t launch_compress_bwd_dw(const CompressBwdParams& p, int nruns, cudaSt
 // as the compressed-attention kernel.
 namespace sel {
 constexpr int kThreads = 192;      // warps 0-3 softmax + output, 4 TMA, 5 MMA
+constexpr int kThreadsSplit = 320; // and warps 6-9 softmax when a KV tile splits in two halves
+constexpr int kXchgBytes = 3072;   // per-row maxima and sums exchanged by the two halves
 constexpr int kMaxSBuf = 8;        // score buffers in tensor memory
 constexpr int kBarBytes = 512;     // mbarriers, tensor-memory address, abort flag
 constexpr int kPlanThreads = 256;
 // listed blocks of lp keys placed side by side in one KV tile: 128 keys when
 // lp divides 128, else one block per tile
 constexpr int blocks_per_tile(int lp) { return (128 % lp == 0) ? 128 / lp : 1; }
+// whether the attention kernel for l' = lp splits a KV tile between two softmax warps per
+// lane quadrant: tiles of several listed blocks whose halves are whole tensor-memory pieces
+// (measured on B200: 16K and varlen workloads (l' = 64) 6-7 % faster; with one 128-key block
+// per tile (l' = 128) 3 % slower, the per-tile exchange of row maxima costing more than the
+// halved arithmetic saves)
+constexpr bool attn_split(int lp) { return blocks_per_tile(lp) >= 2 && (blocks_per_tile(lp) * lp) % 32 == 0; }
+constexpr int attn_threads(int lp) { return attn_split(lp) ? kThreadsSplit : kThreads; }
 
 // One M-tile: up to 128/G consecutive query tokens of one sequence x the G
 // heads of one KV group.
@@ -295,7 +304,7 @@ struct Params {
     int tm_o;                   // tensor-memory column of O (d2 columns)
     int tm_s, s_stride;         // column of score buffer 0, columns between buffers
     // shared-memory layout (byte offsets from a 1024-aligned base)
-    int off_q, q_bytes, off_ring, slot_bytes, off_bar, smem_bytes;
+    int off_q, q_bytes, off_ring, slot_bytes, off_bar, off_x, smem_bytes;
 };
 
 cudaError_t launch_plan(const Params& p, int max_words, cudaStream_t st);

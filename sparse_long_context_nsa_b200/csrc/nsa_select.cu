@@ -158,11 +158,14 @@ cudaError_t launch_plan(const Params& p, int max_words, cudaStream_t st) {
 // KV tile skips the exponentials and writes zero P.
 // ---------------------------------------------------------------------------
 template <typename T, int LP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(attn_threads(LP), 1)
 sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
     // BPT listed blocks side by side in one KV tile of NKV keys
     constexpr int BPT = blocks_per_tile(LP);
+    // a KV tile of several listed blocks splits between two softmax warps per lane quadrant
+    constexpr bool kSplit = attn_split(LP);
+    constexpr int kSoft = kSplit ? 8 : 4;   // softmax warps
     constexpr int NKV = BPT * LP;
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int kWarpTma = 4, kWarpMma = 5;
@@ -187,10 +190,10 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < kMaxSBuf; ++i) {
             mbar_init(bar(B_S_FULL0 + i), 1);
             mbar_init(bar(B_S_EMPTY0 + i), 1);
-            mbar_init(bar(B_P_FULL0 + i), 4);
+            mbar_init(bar(B_P_FULL0 + i), kSoft);
         }
         mbar_init(bar(B_O_FULL), 1);
-        mbar_init(bar(B_O_EMPTY), 4);
+        mbar_init(bar(B_O_EMPTY), kSoft);
         mbar_init(bar(B_MMA_DONE), 1);
         for (int s = 0; s < 8; ++s) {
             mbar_init(bar(B_SLOT_FULL0 + s), 1);
@@ -348,7 +351,9 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int ks = 0; ks < nks_pv; ++ks) {
                         const uint64_t bd = sdesc_sw128(vbase + ks * 2048, NKV * 128, 1024);
-                        umma_ts(tmem_o, tmem + s_col(sb) + ks * 8, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+                        // split tiles: the second half's P sits at the start of its own half
+                        const uint32_t pc = ks * 8 + ((kSplit && ks >= nks_pv / 2) ? NKV / 4 : 0);
+                        umma_ts(tmem_o, tmem + s_col(sb) + pc, bd, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(bar(B_S_EMPTY0 + sb));     // the buffer is free, O holds P V_0..i
                     umma_commit(bar(B_SLOT_EMPTY0 + slot));
@@ -367,10 +372,19 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             umma_commit(bar(B_MMA_DONE));
             mbar_wait(bar(B_MMA_DONE), 0, abort_flag, nullptr, 0);
         }
-    } else if (warp < 4) {
-        // ============ softmax and output (128 thr, one row each) ============
-        const int row = warp * 32 + lane;          // tile row = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    } else if (warp < 4 || (kSplit && warp >= 6 && warp < 10)) {
+        // ===== softmax and output (one row per thread; split tiles: two warps per row) =====
+        // warps 0-3 take the first NKV/2 columns of a KV tile (all of it when the tile does
+        // not split), warps 6-9 the second, in lane quadrant warp % 4.  The two halves of a
+        // row exchange their maxima through shared memory every tile (both then move the
+        // reference maximum alike) and their sums once per M-tile.
+        constexpr int NH = kSplit ? NKV / 2 : NKV;   // columns per warp
+        const int quad = warp & 3, half = warp >= 6 ? 1 : 0;
+        const int col0 = half * NH;
+        const int row = quad * 32 + lane;          // tile row = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float* const xmax = reinterpret_cast<float*>(smem + p.off_x);        // [parity][half][128]
+        float* const xsum = xmax + 2 * 2 * 128;                               // [half][128]
         const float c2 = p.scale_log2;
         const int h = row % G;
         const int tok = row / G;
@@ -380,19 +394,30 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // is attended to iff k < lim[q]; the others become -inf.
         const bool pos_scale = c2 > 0.f;
         const float ce = pos_scale ? c2 : 1.f;
-        auto prep = [&](float (&s)[NKV], const int (&lim)[BPT]) {
+        auto prep = [&](float (&s)[NH], const int (&lim)[BPT]) {
             if (!pos_scale) {
 #pragma unroll
-                for (int c = 0; c < NKV; ++c) s[c] *= c2;
+                for (int c = 0; c < NH; ++c) s[c] *= c2;
             }
             bool full = true;
 #pragma unroll
             for (int q = 0; q < BPT; ++q) full = full && lim[q] == LP;
             if (!full) {
 #pragma unroll
-                for (int c = 0; c < NKV; ++c) s[c] = (c % LP < lim[c / LP]) ? s[c] : -INFINITY;
+                for (int c = 0; c < NH; ++c) {
+                    const int cg = col0 + c;   // column of the KV tile
+                    s[c] = (cg % LP < lim[cg / LP]) ? s[c] : -INFINITY;
+                }
             }
         };
+        // the two warps of a lane quadrant meet at named barrier 1 + quad
+        auto pair_sync = [&]() {
+            if constexpr (kSplit) named_bar_sync(1 + quad, 64);
+        };
+        // this warp's O columns: its half of the 16-column pieces
+        const int npc = p.d2 / 16;
+        const int oc0 = kSplit ? half * ((npc + 1) / 2) * 16 : 0;
+        const int oc1 = kSplit ? min(p.d2, (half + 1) * ((npc + 1) / 2) * 16) : p.d2;
         uint32_t scnt = 0, oc = 0;
 
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -405,8 +430,8 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (n == 0) {
                 // no listed block: nothing is attended to
                 if (valid) {
-                    p.lse[ridx] = -INFINITY;
-                    for (int c = 0; c < p.d2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
+                    if (half == 0) p.lse[ridx] = -INFINITY;
+                    for (int c = oc0; c < oc1; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
                 }
                 continue;
             }
@@ -427,7 +452,7 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 return lim > 0 ? lim : 0;
             };
 
-            float m = -INFINITY, L = 0.f;   // reference max (exponent units), sum of 2^(x - m)
+            float m = -INFINITY, L = 0.f;   // reference max (exponent units), this half's sum of 2^(x - m)
             const int nkv = (n + BPT - 1) / BPT;
             int lim[BPT], nb[BPT];
             uint32_t nw[BPT];
@@ -441,69 +466,81 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             for (int i = 0; i < nkv; ++i) {
                 const uint32_t sb = scnt % nsbuf;
-                const uint32_t ts = tmem + lane_off + s_col(sb);
+                const uint32_t ts = tmem + lane_off + s_col(sb) + col0;
                 int lim_next[BPT];
                 bool any = false;
 #pragma unroll
                 for (int q = 0; q < BPT; ++q) {
                     lim_next[q] = lim_of(nb[q], nw[q]);
                     fetch((i + 2) * BPT + q, nb[q], nw[q]);
-                    any = any || lim[q] > 0;
+                    const bool mine = !kSplit || (q * LP < col0 + NH && (q + 1) * LP > col0);
+                    any = any || (mine && lim[q] > 0);
                 }
                 const bool work = __any_sync(0xffffffffu, any);
                 mbar_wait(bar(B_S_FULL0 + sb), (scnt / nsbuf) & 1, abort_flag, p.err, kErrTimeoutBase + 10);
                 tc_fence_after();
-                uint32_t pw[NKV / 2];
+                uint32_t pw[NH / 2];
+                float s[NH];
+                float mx = -INFINITY;
                 if (work) {
-                    float s[NKV];
                     {
-                        uint32_t r[NKV];
-                        tmem_ld_cols<NKV>(ts, r);
-                        tmem_wait_ld_regs<NKV>(r);
+                        uint32_t r[NH];
+                        tmem_ld_cols<NH>(ts, r);
+                        tmem_wait_ld_regs<NH>(r);
 #pragma unroll
-                        for (int c = 0; c < NKV; ++c) s[c] = __uint_as_float(r[c]);
+                        for (int c = 0; c < NH; ++c) s[c] = __uint_as_float(r[c]);
                     }
                     prep(s, lim);
                     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < NKV; c += 8) {
+                    for (int c = 0; c < NH; c += 8) {
                         mx4[0] = fmax3(mx4[0], s[c + 0], s[c + 1]);
                         mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
                         mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
                         mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
                     }
-                    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
-                    // move the reference up only by more than 8: P <= 2^8 in between
-                    const bool raise = mx > m + 8.f;            // from -inf: any finite maximum
-                    const bool resc = raise && (m != -INFINITY); // O holds earlier blocks' P V
-                    float corr = 1.f;
-                    if (raise) {
-                        corr = ex2(m - mx);                     // 0 from -inf
-                        L *= corr;
-                        m = mx;
-                    }
-                    if (__any_sync(0xffffffffu, resc)) {
-                        // O rows of this warp times corr, after P V of the previous block
-                        const uint32_t pg = scnt - 1;
-                        mbar_wait(bar(B_S_EMPTY0 + pg % nsbuf), (pg / nsbuf) & 1, abort_flag, p.err,
-                                  kErrTimeoutBase + 11);
-                        tc_fence_after();
-                        const float f = resc ? corr : 1.f;
-                        for (int c = 0; c < p.d2; c += 16) {
-                            uint32_t r[16];
-                            tmem_ld16(tmem_o + lane_off + c, r);
-                            tmem_wait_ld_regs<16>(r);
+                    mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * ce;
+                }
+                if constexpr (kSplit) {
+                    // the row's maximum over both halves (buffers alternate by tile, so a
+                    // write never meets the other warp's read of the tile before)
+                    float* xm = xmax + (scnt & 1) * 256;
+                    xm[half * 128 + row] = mx;
+                    pair_sync();
+                    mx = fmaxf(mx, xm[(half ^ 1) * 128 + row]);
+                }
+                // move the reference up only by more than 8: P <= 2^8 in between
+                const bool raise = mx > m + 8.f;            // from -inf: any finite maximum
+                const bool resc = raise && (m != -INFINITY); // O holds earlier blocks' P V
+                float corr = 1.f;
+                if (raise) {
+                    corr = ex2(m - mx);                     // 0 from -inf
+                    L *= corr;
+                    m = mx;
+                }
+                if (__any_sync(0xffffffffu, resc)) {
+                    // this warp's O columns times corr, after P V of the previous block
+                    const uint32_t pg = scnt - 1;
+                    mbar_wait(bar(B_S_EMPTY0 + pg % nsbuf), (pg / nsbuf) & 1, abort_flag, p.err,
+                              kErrTimeoutBase + 11);
+                    tc_fence_after();
+                    const float f = resc ? corr : 1.f;
+                    for (int c = oc0; c < oc1; c += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(tmem_o + lane_off + c, r);
+                        tmem_wait_ld_regs<16>(r);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-                            tmem_st16(tmem_o + lane_off + c, r);
-                        }
+                        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+                        tmem_st16(tmem_o + lane_off + c, r);
                     }
+                }
+                if (work) {
                     const float mref = (m == -INFINITY) ? 0.f : m;
                     const float2 ce2 = make_float2(ce, ce), nm2 = make_float2(-mref, -mref);
                     float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                      make_float2(0.f, 0.f)};
 #pragma unroll
-                    for (int c = 0; c < NKV; c += 2) {
+                    for (int c = 0; c < NH; c += 2) {
                         const float2 x = ffma2(make_float2(s[c], s[c + 1]), ce2, nm2);
                         const float2 e2 = make_float2(ex2(x.x), ex2(x.y));
                         acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e2);
@@ -513,15 +550,16 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     L += (t01.x + t01.y) + (t23.x + t23.y);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < NKV / 2; ++c) pw[c] = 0u;
+                    for (int c = 0; c < NH / 2; ++c) pw[c] = 0u;
                 }
-                // P in the storage dtype over the first NKV/2 columns of the buffer
-                if constexpr ((NKV / 2) % 16 == 0) {
+                // P in the storage dtype over the first NH/2 columns of this warp's part of
+                // the buffer (columns it has read)
+                if constexpr ((NH / 2) % 16 == 0) {
 #pragma unroll
-                    for (int c = 0; c < NKV / 32; ++c) tmem_st16(ts + c * 16, pw + c * 16);
+                    for (int c = 0; c < NH / 32; ++c) tmem_st16(ts + c * 16, pw + c * 16);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < NKV / 16; ++c) tmem_st8(ts + c * 8, pw + c * 8);
+                    for (int c = 0; c < NH / 16; ++c) tmem_st8(ts + c * 8, pw + c * 8);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -531,13 +569,20 @@ sel_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int q = 0; q < BPT; ++q) lim[q] = lim_next[q];
             }
+            if constexpr (kSplit) {
+                // the row's sum over both halves
+                xsum[half * 128 + row] = L;
+                pair_sync();
+                L += xsum[(half ^ 1) * 128 + row];
+                pair_sync();   // both have read before the next M-tile writes again
+            }
 
             // ------------- O / L -> attention_out, log-sum-exp -------------
             mbar_wait(bar(B_O_FULL), oc & 1, abort_flag, p.err, kErrTimeoutBase + 12);
             tc_fence_after();
-            if (valid) p.lse[ridx] = (L > 0.f) ? (m + lg2(L)) * 0.69314718055994530942f : -INFINITY;
+            if (valid && half == 0) p.lse[ridx] = (L > 0.f) ? (m + lg2(L)) * 0.69314718055994530942f : -INFINITY;
             const float inv = (L > 0.f) ? 1.f / L : 0.f;
-            for (int c = 0; c < p.d2; c += 16) {
+            for (int c = oc0; c < oc1; c += 16) {
                 uint32_t r[16];
                 tmem_ld16(tmem_o + lane_off + c, r);
                 tmem_wait_ld_regs<16>(r);
@@ -583,7 +628,7 @@ static cudaError_t launch_t(const Params& p, const CUtensorMap& tq, const CUtens
     auto kern = sel_attn_kernel<T, LP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, p.smem_bytes, st>>>(tq, tk, tv, p);
+    kern<<<grid, attn_threads(LP), p.smem_bytes, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
